@@ -1,0 +1,208 @@
+"""Seeded synthetic workloads for the MTFM masked-attention path.
+
+This module only draws inputs: jagged user lengths, R-token timestamps, T-token
+exposure times and bf16 activations.  It holds none of the attention, mask or
+normalisation arithmetic, so both the fp64 oracle (``oracle/``) and the CUDA
+path (``hybrid_masked_attention_b200``) can consume the very same arrays
+without sharing any of the method's code.
+
+Workload shapes follow the pages:
+  * user-level samples [H | R | T] with history lengths in the hundreds to
+    thousands ("MTFM: Meituan unified recommendation foundation model ..."
+    tech blog, section 3.3.1, and section 7.1 for the 400-2000 length range);
+  * several exposure targets per user, spread over scenarios (same blog,
+    section 4.1, user-level samples);
+  * R tokens sorted by their action timestamps, T tokens carrying the
+    exposure time of their request (same blog, section 3.1 and 3.2).
+The proprietary logs the pages train on are not available; these seeded
+draws stand in for them.
+
+Every tensor gets its own numpy ``SeedSequence`` stream ``[seed, stream_id]``
+so that adding a tensor never changes the values of the others.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+
+# Stream ids (one independent generator per drawn quantity).
+S_LEN, S_TS, S_EXP, S_SCEN, S_Q, S_K, S_V, S_U, S_DY, S_GAMMA, S_BETA, S_W = range(12)
+
+
+def rng_for(seed: int, stream: int) -> np.random.Generator:
+    return np.random.default_rng(np.random.SeedSequence([int(seed), int(stream)]))
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (round to nearest, ties to even); return the raw uint16 bits."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounding = ((u >> 16) & 1) + 0x7FFF
+    out = ((u + rounding) >> 16).astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        out[nan] = 0x7FC0
+    return out
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32."""
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def normal_bf16(seed: int, stream: int, shape, std: float = 1.0) -> np.ndarray:
+    """N(0, std^2) draws rounded to bf16; returns uint16 bit patterns."""
+    g = rng_for(seed, stream)
+    x = (g.standard_normal(size=shape) * std).astype(np.float32)
+    return f32_to_bf16_bits(x)
+
+
+@dataclass
+class JaggedBatch:
+    """Per-user lengths and timestamps of one jagged batch of user-level samples."""
+    L_H: np.ndarray            # int32 [B]
+    L_R: np.ndarray            # int32 [B]
+    L_T: np.ndarray            # int32 [B]
+    r_ts: np.ndarray           # int64 [sum L_R], sorted ascending within each user
+    t_exp: np.ndarray          # int64 [sum L_T], exposure time of each T token
+    scenario: np.ndarray       # int32 [sum L_T], scenario id (metadata only)
+    v2_subtokens: int = 1      # 1: one token per target; 4: V2 target scale-up
+
+    @property
+    def B(self) -> int:
+        return int(self.L_H.shape[0])
+
+    @property
+    def N(self) -> np.ndarray:
+        return (self.L_H.astype(np.int64) + self.L_R + self.L_T)
+
+    @property
+    def total_tokens(self) -> int:
+        return int(self.N.sum())
+
+    @property
+    def total_t(self) -> int:
+        return int(self.L_T.sum())
+
+    @property
+    def total_r(self) -> int:
+        return int(self.L_R.sum())
+
+
+def _draw_times(seed, lens_r, lens_t_targets, v2):
+    g_ts = rng_for(seed, S_TS)
+    g_ex = rng_for(seed, S_EXP)
+    g_sc = rng_for(seed, S_SCEN)
+    r_parts, e_parts, s_parts = [], [], []
+    for lr, nt in zip(lens_r, lens_t_targets):
+        r_parts.append(np.sort(g_ts.integers(0, 1000, size=int(lr), dtype=np.int64)))
+        e = g_ex.integers(0, 1000, size=int(nt), dtype=np.int64)
+        s = g_sc.integers(0, 3, size=int(nt), dtype=np.int64).astype(np.int32)
+        e_parts.append(np.repeat(e, v2))
+        s_parts.append(np.repeat(s, v2))
+    cat = lambda parts, dt: (np.concatenate(parts).astype(dt) if parts else np.zeros(0, dt))
+    return cat(r_parts, np.int64), cat(e_parts, np.int64), cat(s_parts, np.int32)
+
+
+def fixed_batch(L_H, L_R, L_T, seed: int, v2_subtokens: int = 1) -> JaggedBatch:
+    """A batch with given per-user lengths; timestamps drawn uniformly in [0, 1000)."""
+    L_H = np.asarray(L_H, dtype=np.int32)
+    L_R = np.asarray(L_R, dtype=np.int32)
+    L_T = np.asarray(L_T, dtype=np.int32)
+    assert np.all(L_T % v2_subtokens == 0)
+    r_ts, t_exp, scen = _draw_times(seed, L_R, L_T // v2_subtokens, v2_subtokens)
+    return JaggedBatch(L_H, L_R, L_T, r_ts, t_exp, scen, v2_subtokens)
+
+
+def tiny_batch(seed: int = 1000) -> JaggedBatch:
+    """2 users of 32 H + 16 R + 8 T tokens."""
+    return fixed_batch([32, 32], [16, 16], [8, 8], seed)
+
+
+def pair_batch(B: int = 32, seed: int = 1001) -> JaggedBatch:
+    """Production-shape jagged batch: L_H ~ U[256,1024], L_R ~ U[32,256], L_T ~ U[16,128]."""
+    g = rng_for(seed, S_LEN)
+    L_H = g.integers(256, 1025, size=B).astype(np.int32)
+    L_R = g.integers(32, 257, size=B).astype(np.int32)
+    L_T = g.integers(16, 129, size=B).astype(np.int32)
+    return fixed_batch(L_H, L_R, L_T, seed)
+
+
+def sweep_batch(N: int, v2: bool = False, total_tokens: int = 1 << 21, B: Optional[int] = None,
+                seed: int = 1003) -> JaggedBatch:
+    """Sequence-length sweep: every user has N tokens split H:R:T ~ 70:15:15.
+
+    V1: L_H = round(0.7 N), L_R = round(0.15 N), L_T = N - L_H - L_R.
+    V2: n_targets = round(0.15 N / 4) targets of 4 sub-tokens each; H absorbs the rounding.
+    """
+    if B is None:
+        B = max(1, total_tokens // N)
+    L_R = int(round(0.15 * N))
+    if v2:
+        nt = int(round(0.15 * N / 4))
+        L_T = 4 * nt
+        L_H = N - L_R - L_T
+        sub = 4
+    else:
+        L_H = int(round(0.7 * N))
+        L_T = N - L_H - L_R
+        sub = 1
+    return fixed_batch([L_H] * B, [L_R] * B, [L_T] * B, seed, v2_subtokens=sub)
+
+
+@dataclass
+class Heads:
+    hq: int
+    hkv: int
+    dh: int
+
+    @property
+    def dq(self) -> int:
+        return self.hq * self.dh
+
+    @property
+    def dkv(self) -> int:
+        return self.hkv * self.dh
+
+
+TINY_HEADS = Heads(2, 1, 32)
+PAIR_HEADS = Heads(8, 2, 64)
+
+
+@dataclass
+class LayerInputs:
+    """bf16 bit patterns (uint16) of one attention layer's inputs."""
+    q: np.ndarray      # [rows_q, hq*dh]
+    k: np.ndarray      # [sum N, hkv*dh]
+    v: np.ndarray      # [sum N, hkv*dh]
+    u: np.ndarray      # [rows_q, hq*dh]
+    gamma: Optional[np.ndarray] = None   # float32 [3, hq*dh]
+    beta: Optional[np.ndarray] = None    # float32 [3, hq*dh]
+    dy: Optional[np.ndarray] = None      # bf16 bits [rows_q, hq*dh]
+
+
+def layer_inputs(batch: JaggedBatch, heads: Heads, target: bool, seed: int,
+                 gln: bool = True, with_dy: bool = False, random_affine: bool = True) -> LayerInputs:
+    """Q, K, V, U ~ N(0,1) in bf16; GLN gamma/beta per token type (H, R, T).
+
+    ``target`` selects the Target-Attention layout where Q and U exist only for T rows.
+    """
+    rows_q = batch.total_t if target else batch.total_tokens
+    off = 50 if target else 0
+    q = normal_bf16(seed, S_Q + off, (rows_q, heads.dq))
+    k = normal_bf16(seed, S_K + off, (batch.total_tokens, heads.dkv))
+    v = normal_bf16(seed, S_V + off, (batch.total_tokens, heads.dkv))
+    u = normal_bf16(seed, S_U + off, (rows_q, heads.dq))
+    gamma = beta = None
+    if gln:
+        if random_affine:
+            gamma = (1.0 + 0.25 * rng_for(seed, S_GAMMA + off).standard_normal((3, heads.dq))).astype(np.float32)
+            beta = (0.25 * rng_for(seed, S_BETA + off).standard_normal((3, heads.dq))).astype(np.float32)
+        else:
+            gamma = np.ones((3, heads.dq), np.float32)
+            beta = np.zeros((3, heads.dq), np.float32)
+    dy = normal_bf16(seed, S_DY + off, (rows_q, heads.dq)) if with_dy else None
+    return LayerInputs(q, k, v, u, gamma, beta, dy)
