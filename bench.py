@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark of the MTFM hybrid masked-attention hot path on B200.
+
+One step = one pass of the whole hot path over one jagged batch of the
+production-shape workload "hybrid pair": 32 users, L_H ~ U[256,1024],
+L_R ~ U[32,256] (sorted timestamps), L_T ~ U[16,128]; Hq 8 / Hkv 2, head_dim 64:
+    pack (metadata + work lists) -> Full-layer attention -> Full gate (GLN)
+    -> Target-layer attention -> Target gate.
+Inputs are resident in HBM, rotated over several copies so that no step reads
+data left in L2 by the previous one.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mtfm|reference]
+
+Prints one JSON line (rank 0).  ``value`` = unmasked attention TFLOP/s of the
+whole step (4 * head_dim * Hq FLOPs per visible query/key pair, both layers),
+summed over ranks and divided by the slowest rank's time.  Multi-GPU runs are
+replicas: each rank packs and runs its own batch of users (no collective on the
+data path), so scaling is weak.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (the
+only other place this script runs oracle code, besides the cpu_baseline leg).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mtfm_synth as syn  # noqa: E402
+
+METRIC = "masked-attn TFLOP/s (unmasked) & user-samples/s per layer; % BF16/HBM roofline"
+WORKLOAD = ("hybrid pair: 32 users jagged, L_H~U[256,1024], L_R~U[32,256] sorted ts, "
+            "L_T~U[16,128] over 3 scenarios; Hq 8 / Hkv 2, head_dim 64; pack + Full fwd + Target fwd "
+            "(attention + GLN gate)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["hybrid_masked_attention_b200/csrc/attn_mma.cu",
+                  "hybrid_masked_attention_b200/csrc/mma_util.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_full_fwd_pair.md")
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def visible_pairs(b: syn.JaggedBatch, target: bool) -> int:
+    """Number of visible (query, key) pairs: H rows see L_H keys, R row a sees L_H + a + 1,
+    a T row sees L_H + #{R : ts < exposure} keys plus its sibling block (itself, or the
+    4 sub-tokens of its target in V2)."""
+    ro = np.concatenate([[0], np.cumsum(b.L_R)])
+    to = np.concatenate([[0], np.cumsum(b.L_T)])
+    total = 0
+    for u in range(b.B):
+        LH, LR, LT = int(b.L_H[u]), int(b.L_R[u]), int(b.L_T[u])
+        ts = b.r_ts[ro[u]:ro[u + 1]]
+        ex = b.t_exp[to[u]:to[u + 1]]
+        k = np.searchsorted(ts, ex, side="left") if LT else np.zeros(0)
+        t_pairs = int(LT * LH + k.sum() + LT * b.v2_subtokens)
+        if target:
+            total += t_pairs
+        else:
+            total += LH * LH + LR * LH + LR * (LR + 1) // 2 + t_pairs
+    return total
+
+
+def attn_flops(b, heads, target) -> float:
+    return 4.0 * heads.dh * heads.hq * visible_pairs(b, target)
+
+
+def target_attn_bytes(b, heads) -> float:
+    """Algorithmic bytes of Target attention: K, V of every row (bf16), Q_T (bf16), A_T (fp32)."""
+    return b.total_tokens * 2 * heads.dkv * 2 + b.total_t * heads.dq * (2 + 4)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the Full attention kernel from the committed ncu summary,
+    or None when the kernel source changed since the capture."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not sha or not val or sha.group(1) != kernel_source_sha():
+        return None
+    return float(val.group(1))
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, interval_ms: int = 50):
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={interval_ms}", f"-i={device_index}"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [l.strip().split(",") for l in self.out.read().splitlines() if l.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_mtfm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import hybrid_masked_attention_b200 as M
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    heads = syn.PAIR_HEADS
+    b = syn.pair_batch(args.users, seed=1001 + 7919 * rank)
+    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh)
+    to_dev = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
+    bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    lens = (to_dev(b.L_H, np.int32), to_dev(b.L_R, np.int32), to_dev(b.L_T, np.int32),
+            to_dev(b.r_ts, np.int64), to_dev(b.t_exp, np.int64))
+    sets = []
+    for r in range(args.sets):
+        fi = syn.layer_inputs(b, heads, target=False, seed=11 + r)
+        ti = syn.layer_inputs(b, heads, target=True, seed=111 + r)
+        sets.append(dict(q=bf(fi.q), k=bf(fi.k), v=bf(fi.v), u=bf(fi.u),
+                         g=to_dev(fi.gamma, np.float32), bt=to_dev(fi.beta, np.float32),
+                         tq=bf(ti.q), tk=bf(ti.k), tv=bf(ti.v), tu=bf(ti.u),
+                         tg=to_dev(ti.gamma, np.float32), tbt=to_dev(ti.beta, np.float32)))
+    meta = M.alloc_meta(cfg, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    A_f = torch.empty(b.total_tokens, heads.dq, **f32)
+    Y_f = torch.empty(b.total_tokens, heads.dq, **f32)
+    S_f = torch.empty(b.total_tokens, 2, **f32)
+    A_t = torch.empty(b.total_t, heads.dq, **f32)
+    Y_t = torch.empty(b.total_t, heads.dq, **f32)
+    S_t = torch.empty(b.total_t, 2, **f32)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 6   # pack (2 kernels), Full attention, Full gate, Target attention, Target gate
+
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_ev)]
+
+    def step(i, record=None):
+        s = sets[i % len(sets)]
+        e = record
+        if e: e[0].record(stream)
+        M.pack(cfg, *lens, meta, stream)
+        if e: e[1].record(stream)
+        M.attn_full(cfg, meta, s["q"], s["k"], s["v"], A_f, stream)
+        if e: e[2].record(stream)
+        M.gate_fwd(cfg, meta, False, A_f, s["u"], s["g"], s["bt"], Y_f, S_f, stream)
+        if e: e[3].record(stream)
+        M.attn_target(cfg, meta, s["tq"], s["tk"], s["tv"], A_t, stream)
+        if e: e[4].record(stream)
+        M.gate_fwd(cfg, meta, True, A_t, s["tu"], s["tg"], s["tbt"], Y_t, S_t, stream)
+        if e: e[5].record(stream)
+
+    # correctness gate before timing: the metadata must be valid
+    step(0)
+    M.pack_check(meta, stream)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+
+    def avg(a, z):
+        return sum(ev[i][a].elapsed_time(ev[i][z]) for i in range(args.steps)) / args.steps
+
+    ms_parts = {"pack": avg(0, 1), "full_attn": avg(1, 2), "full_gate": avg(2, 3),
+                "target_attn": avg(3, 4), "target_gate": avg(4, 5)}
+    fl_full = attn_flops(b, heads, False)
+    fl_tgt = attn_flops(b, heads, True)
+    flops_step = fl_full + fl_tgt
+
+    # aggregate over ranks: time = max, work = sum
+    tot = [ms_total, flops_step, float(b.B)]
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        w = torch.tensor([flops_step, float(b.B)], dtype=torch.float64, device=dev)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+        tot = [float(t[0]), float(w[0]), float(w[1])]
+    ms_max, flops_all, users_all = tot
+    ms_per_step = ms_max / args.steps
+    value = flops_all / (ms_per_step * 1e-3) / 1e12
+
+    # end-to-end through the public API with host buffers
+    e2e = run_e2e(args, M, cfg, b, heads, dev, stream, world)
+
+    result = None
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        full_tf = fl_full / (ms_parts["full_attn"] * 1e-3) / 1e12
+        tgt_gbs = target_attn_bytes(b, heads) / (ms_parts["target_attn"] * 1e-3) / 1e9
+        traffic = recorded_traffic()
+        result = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; stands in for the pages' proprietary logs)",
+            "config": {"workload": WORKLOAD, "users_per_gpu": b.B, "total_tokens": b.total_tokens,
+                       "total_t": b.total_t, "flops_per_step_per_gpu": flops_step,
+                       "l2": f"inputs rotated over {args.sets} resident copies "
+                             f"({args.sets * 89} MB of inputs > 126 MB L2)",
+                       "parallelism": f"replicas x{world} (users sharded, no collective)"},
+            "users_per_s": round(users_all * args.steps / (ms_max * 1e-3), 1),
+            "per_layer": {
+                "full": {"ms": round(ms_parts["full_attn"] + ms_parts["full_gate"], 5),
+                         "attn_tflops": round(full_tf, 2),
+                         "users_per_s": round(b.B / ((ms_parts["full_attn"] + ms_parts["full_gate"]) * 1e-3), 1)},
+                "target": {"ms": round(ms_parts["target_attn"] + ms_parts["target_gate"], 5),
+                           "attn_tflops": round(fl_tgt / (ms_parts["target_attn"] * 1e-3) / 1e12, 2),
+                           "attn_gbs": round(tgt_gbs, 1), "attn_hbm_frac": round(tgt_gbs / hbm, 4),
+                           "users_per_s": round(b.B / ((ms_parts["target_attn"] + ms_parts["target_gate"]) * 1e-3), 1)},
+                "ms_parts": {k: round(v, 5) for k, v in ms_parts.items()},
+            },
+            "roofline": {"kernel": "Full-layer attention (attn_fwd_mma_kernel)", "bound": "tensor",
+                         "achieved": round(full_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": round(full_tf / peak_tf, 4), "traffic": traffic,
+                         "peak_source": f"{src} bf16 dense (burst)",
+                         "flops_per_launch": fl_full, "launch_ms": round(ms_parts["full_attn"], 5)},
+            "e2e": e2e,
+            "clocks": clocks,
+            "gpu_launches": launches_per_step * args.steps,
+        }
+    return result, b, heads
+
+
+def run_e2e(args, M, cfg, b, heads, dev, stream, world):
+    """Same metric through the public layer calls, with inputs in pinned host memory and the
+    host<->device copies of each step's inputs and outputs inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    fi = syn.layer_inputs(b, heads, target=False, seed=11)
+    ti = syn.layer_inputs(b, heads, target=True, seed=111)
+    pin = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).pin_memory()
+    pbf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+    host = [pin(b.L_H, np.int32), pin(b.L_R, np.int32), pin(b.L_T, np.int32), pin(b.r_ts, np.int64),
+            pin(b.t_exp, np.int64), pbf(fi.q), pbf(fi.k), pbf(fi.v), pbf(fi.u),
+            pin(fi.gamma, np.float32), pin(fi.beta, np.float32), pbf(ti.q), pbf(ti.k), pbf(ti.v),
+            pbf(ti.u), pin(ti.gamma, np.float32), pin(ti.beta, np.float32)]
+    devb = [torch.empty_like(h, device=dev) for h in host]
+    meta = M.alloc_meta(cfg, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    Y_f, A_f, S_f = (torch.empty(b.total_tokens, heads.dq, **f32), torch.empty(b.total_tokens, heads.dq, **f32),
+                     torch.empty(b.total_tokens, 2, **f32))
+    Y_t, A_t, S_t = (torch.empty(b.total_t, heads.dq, **f32), torch.empty(b.total_t, heads.dq, **f32),
+                     torch.empty(b.total_t, 2, **f32))
+    out_f = torch.empty(Y_f.shape, dtype=torch.float32).pin_memory()
+    out_t = torch.empty(Y_t.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h in host)
+    d2h = out_f.numel() * 4 + out_t.numel() * 4
+
+    def step():
+        for h, d in zip(host, devb):
+            d.copy_(h, non_blocking=True)
+        lh, lr, lt, rts, tex, q, k, v, u, g, bt, tq, tk, tv, tu, tg, tbt = devb
+        M.pack(cfg, lh, lr, lt, rts, tex, meta, stream)
+        M.attn_full_fwd(cfg, meta, q, k, v, u, g, bt, Y_f, A_f, S_f, stream)
+        M.attn_target_fwd(cfg, meta, tq, tk, tv, tu, tg, tbt, Y_t, A_t, S_t, stream)
+        out_f.copy_(Y_f, non_blocking=True)
+        out_t.copy_(Y_t, non_blocking=True)
+
+    steps = max(3, min(args.steps, args.e2e_steps))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1)
+    fl = attn_flops(b, heads, False) + attn_flops(b, heads, True)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        w = torch.tensor([fl], dtype=torch.float64, device=dev)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+        ms, fl = float(t[0]), float(w[0])
+    return {"value": round(fl / (ms / steps * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": round(ms / steps, 4)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_time(b, heads, users, seeds=(11, 111)):
+    """Time the fp64 oracle's Full + Target forward on the given users; returns (seconds, flops)."""
+    from oracle import mtfm_oracle as O  # the CPU-baseline leg is allowed to run the oracle
+    fi = syn.layer_inputs(b, heads, target=False, seed=seeds[0])
+    ti = syn.layer_inputs(b, heads, target=True, seed=seeds[1])
+    t = time.perf_counter()
+    O.full_fwd(b, heads, fi, users=set(users))
+    O.target_fwd(b, heads, ti, users=set(users))
+    dt = time.perf_counter() - t
+    sub = syn.JaggedBatch(b.L_H[users], b.L_R[users], b.L_T[users],
+                          np.concatenate([b.r_ts[int(np.sum(b.L_R[:u])):int(np.sum(b.L_R[:u + 1]))] for u in users]),
+                          np.concatenate([b.t_exp[int(np.sum(b.L_T[:u])):int(np.sum(b.L_T[:u + 1]))] for u in users]),
+                          b.scenario, b.v2_subtokens)
+    return dt, attn_flops(sub, heads, False) + attn_flops(sub, heads, True)
+
+
+def cpu_baseline(b, heads, budget_s=20.0):
+    """The oracle as it stands on the host cores, on a bounded sample of the same workload."""
+    users, spent, fl = [], 0.0, 0.0
+    order = list(range(b.B))
+    for u in order:
+        dt, f = oracle_time(b, heads, [u])
+        users.append(u)
+        spent += dt
+        fl += f
+        if spent >= budget_s:
+            break
+    return {"value": round(fl / spent / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle, Full + Target forward of {len(users)} of {b.B} users "
+                      f"of the same batch ({spent:.1f} s of CPU work)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    heads = syn.PAIR_HEADS
+    b = syn.pair_batch(args.users, seed=1001)
+    # each step: the oracle on one user of the batch (users in turn); bounded so the run ends in minutes
+    per_user = oracle_time(b, heads, [0])[0]
+    budget = 150.0
+    steps = max(1, min(args.steps, int(budget / max(per_user, 1e-3)) - args.warmup))
+    warm = min(args.warmup, 3)
+    for i in range(warm):
+        oracle_time(b, heads, [i % b.B])
+    spent, fl = 0.0, 0.0
+    for i in range(steps):
+        dt, f = oracle_time(b, heads, [i % b.B])
+        spent += dt
+        fl += f
+    value = fl / spent / 1e12
+    cores = blas_threads()
+    sample = (f"fp64 numpy oracle; each step = Full + Target forward of one user of the "
+              f"{b.B}-user batch (users in turn); {steps} steps timed")
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": steps, "steps_requested": args.steps, "warmup": warm,
+            "ms_per_step": round(spent / steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "users_per_gpu": b.B},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["mtfm", "reference"], default="mtfm")
+    ap.add_argument("--users", type=int, default=32)
+    ap.add_argument("--sets", type=int, default=4, help="resident input copies rotated across steps")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res, b, heads = run_mtfm(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(b, heads)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,297 @@
+"""Python binding of libmtfm, the B200 (sm_100a) MTFM hybrid masked-attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/mtfm.h``.  PyTorch supplies
+device memory and streams.  There is no fallback: if ``libmtfm.so`` is missing
+this import fails; build it with ``python hybrid_masked_attention_b200/build.py``.
+
+Function names mirror the C entry points:
+    meta_bytes, max_items, pack, pack_check, meta_read,
+    attn_full_fwd, attn_target_fwd, attn_full, attn_target, gate_fwd,
+    bwd_workspace_bytes, attn_full_bwd, attn_target_bwd
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmtfm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libmtfm.so not found at {LIB_PATH}; build it with "
+        "`python hybrid_masked_attention_b200/build.py` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MTFM_OK = 0
+STATUS_NAMES = {
+    0: "MTFM_OK", 1: "MTFM_ERR_INVALID_ARG", 2: "MTFM_ERR_UNSORTED_TS", 3: "MTFM_ERR_UNSUPPORTED",
+    4: "MTFM_ERR_WORKSPACE_TOO_SMALL", 5: "MTFM_ERR_CUDA", 6: "MTFM_ERR_TIMEOUT",
+    7: "MTFM_ERR_BAD_LENGTHS",
+}
+
+
+class MtfmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.mtfm_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({msg})")
+
+
+class CCfg(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
+                ("total_r", ctypes.c_int32), ("total_t", ctypes.c_int32),
+                ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("v2_subtokens", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("gln_eps", ctypes.c_float)]
+
+
+@dataclass
+class Config:
+    """Problem description (mirrors ``mtfm_cfg``)."""
+    batch: int
+    total_tokens: int
+    total_r: int
+    total_t: int
+    hq: int
+    hkv: int
+    head_dim: int
+    v2_subtokens: int = 1
+    alpha: float = 0.0      # <= 0: 1/sqrt(head_dim)
+    gln_eps: float = 0.0    # <= 0: 1e-5
+
+    def c(self) -> CCfg:
+        return CCfg(self.batch, self.total_tokens, self.total_r, self.total_t, self.hq, self.hkv,
+                    self.head_dim, self.v2_subtokens, self.alpha, self.gln_eps)
+
+    @property
+    def D(self) -> int:
+        return self.hq * self.head_dim
+
+    @property
+    def Dkv(self) -> int:
+        return self.hkv * self.head_dim
+
+    @property
+    def alpha_eff(self) -> float:
+        return self.alpha if self.alpha > 0 else 1.0 / math.sqrt(self.head_dim)
+
+
+_P = ctypes.c_void_p
+_CP = ctypes.POINTER(CCfg)
+_sigs = {
+    "mtfm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mtfm_meta_bytes": (ctypes.c_size_t, [_CP]),
+    "mtfm_pack": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "mtfm_pack_check": (ctypes.c_int, [_P, _P]),
+    "mtfm_meta_read": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "mtfm_max_items": (ctypes.c_int32, [_CP, ctypes.c_int]),
+    "mtfm_attn_full_fwd": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "mtfm_attn_target_fwd": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "mtfm_attn_full": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
+    "mtfm_attn_target": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
+    "mtfm_gate_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]),
+    "mtfm_bwd_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int]),
+    "mtfm_attn_full_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
+    "mtfm_attn_target_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
+}
+for _name, (_res, _args) in _sigs.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_sigs)
+
+
+def _check(status: int, where: str):
+    if status != MTFM_OK:
+        raise MtfmError(status, where)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, shape=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr() if t.numel() else (t.data_ptr() or None)
+
+
+def meta_bytes(cfg: Config) -> int:
+    c = cfg.c()
+    n = _lib.mtfm_meta_bytes(ctypes.byref(c))
+    if n == 0:
+        raise MtfmError(1, "mtfm_meta_bytes")
+    return n
+
+
+def max_items(cfg: Config, target: bool) -> int:
+    """Capacity of the Full or Target work list of the metadata block."""
+    c = cfg.c()
+    n = _lib.mtfm_max_items(ctypes.byref(c), int(bool(target)))
+    if n < 0:
+        raise MtfmError(1, "mtfm_max_items")
+    return n
+
+
+def alloc_meta(cfg: Config, device="cuda") -> torch.Tensor:
+    """A metadata block of the right size (torch's allocator aligns to >= 256 bytes)."""
+    return torch.empty(meta_bytes(cfg), dtype=torch.uint8, device=device)
+
+
+def pack(cfg: Config, lh, lr, lt, r_ts, t_exp, meta: torch.Tensor, stream=None):
+    c = cfg.c()
+    B = cfg.batch
+    st = _lib.mtfm_pack(ctypes.byref(c),
+                        _ptr(lh, torch.int32, (B,), "lh"), _ptr(lr, torch.int32, (B,), "lr"),
+                        _ptr(lt, torch.int32, (B,), "lt"),
+                        _ptr(r_ts, torch.int64, (cfg.total_r,), "r_ts"),
+                        _ptr(t_exp, torch.int64, (cfg.total_t,), "t_exp"),
+                        _ptr(meta, torch.uint8, None, "meta"), meta.numel(), _stream(stream))
+    _check(st, "mtfm_pack")
+
+
+def pack_check(meta: torch.Tensor, stream=None):
+    _check(_lib.mtfm_pack_check(_ptr(meta, torch.uint8, None, "meta"), _stream(stream)), "mtfm_pack_check")
+
+
+def meta_read(cfg: Config, meta: torch.Tensor, stream=None) -> dict:
+    B, T = cfg.batch, cfg.total_tokens
+    out = {"seq_off": np.zeros(B + 1, np.int32), "r_off": np.zeros(B + 1, np.int32),
+           "t_off": np.zeros(B + 1, np.int32), "kv_end": np.zeros(max(T, 1), np.int32),
+           "row_type": np.zeros(max(T, 1), np.uint8)}
+    nf = ctypes.c_int32()
+    nt = ctypes.c_int32()
+    c = cfg.c()
+    mf = max_items(cfg, False)
+    mt = max_items(cfg, True)
+    out["items_full"] = np.zeros((max(mf, 1), 4), np.int32)
+    out["items_target"] = np.zeros((max(mt, 1), 4), np.int32)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    st = _lib.mtfm_meta_read(ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"), p(out["seq_off"]),
+                             p(out["r_off"]), p(out["t_off"]), p(out["kv_end"]), p(out["row_type"]),
+                             ctypes.byref(nf), ctypes.byref(nt), p(out["items_full"]),
+                             p(out["items_target"]), _stream(stream))
+    _check(st, "mtfm_meta_read")
+    out["kv_end"] = out["kv_end"][:T]
+    out["row_type"] = out["row_type"][:T]
+    out["n_items_full"] = nf.value
+    out["n_items_target"] = nt.value
+    out["items_full"] = out["items_full"][:nf.value]
+    out["items_target"] = out["items_target"][:nt.value]
+    return out
+
+
+def _fwd(fn, where, cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream, rows):
+    c = cfg.c()
+    D, Dkv, N = cfg.D, cfg.Dkv, cfg.total_tokens
+    bf = torch.bfloat16
+    st = fn(ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"),
+            _ptr(q, bf, (rows, D), "q"), _ptr(k, bf, (N, Dkv), "k"), _ptr(v, bf, (N, Dkv), "v"),
+            _ptr(u, bf, (rows, D), "u"),
+            _ptr(gamma, torch.float32, (3, D), "gamma"), _ptr(beta, torch.float32, (3, D), "beta"),
+            _ptr(y, torch.float32, (rows, D), "y"), _ptr(a, torch.float32, (rows, D), "a"),
+            _ptr(stats, torch.float32, (rows, 2), "stats"), _stream(stream))
+    _check(st, where)
+
+
+def attn_full_fwd(cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream=None):
+    """Full-Attention layer forward: writes y, a (and stats when gamma is given)."""
+    _fwd(_lib.mtfm_attn_full_fwd, "mtfm_attn_full_fwd", cfg, meta, q, k, v, u, gamma, beta, y, a,
+         stats, stream, cfg.total_tokens)
+
+
+def attn_target_fwd(cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream=None):
+    """Target-Attention layer forward (T rows only)."""
+    _fwd(_lib.mtfm_attn_target_fwd, "mtfm_attn_target_fwd", cfg, meta, q, k, v, u, gamma, beta, y,
+         a, stats, stream, cfg.total_t)
+
+
+def _attn_only(fn, where, cfg, meta, q, k, v, a, stream, rows):
+    c = cfg.c()
+    D, Dkv, N = cfg.D, cfg.Dkv, cfg.total_tokens
+    bf = torch.bfloat16
+    st = fn(ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"), _ptr(q, bf, (rows, D), "q"),
+            _ptr(k, bf, (N, Dkv), "k"), _ptr(v, bf, (N, Dkv), "v"),
+            _ptr(a, torch.float32, (rows, D), "a"), _stream(stream))
+    _check(st, where)
+
+
+def attn_full(cfg, meta, q, k, v, a, stream=None):
+    """Full-layer attention only (A, fp32)."""
+    _attn_only(_lib.mtfm_attn_full, "mtfm_attn_full", cfg, meta, q, k, v, a, stream, cfg.total_tokens)
+
+
+def attn_target(cfg, meta, q, k, v, a, stream=None):
+    """Target-layer attention only (A of the T rows, fp32)."""
+    _attn_only(_lib.mtfm_attn_target, "mtfm_attn_target", cfg, meta, q, k, v, a, stream, cfg.total_t)
+
+
+def gate_fwd(cfg, meta, target: bool, a, u, gamma, beta, y, stats, stream=None):
+    """Y = GLN(A) (*) U for the Full or Target layout."""
+    c = cfg.c()
+    rows = cfg.total_t if target else cfg.total_tokens
+    D = cfg.D
+    f32 = torch.float32
+    st = _lib.mtfm_gate_fwd(ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"), int(bool(target)),
+                            _ptr(a, f32, (rows, D), "a"), _ptr(u, torch.bfloat16, (rows, D), "u"),
+                            _ptr(gamma, f32, (3, D), "gamma"), _ptr(beta, f32, (3, D), "beta"),
+                            _ptr(y, f32, (rows, D), "y"), _ptr(stats, f32, (rows, 2), "stats"),
+                            _stream(stream))
+    _check(st, "mtfm_gate_fwd")
+
+
+def bwd_workspace_bytes(cfg: Config, target: bool) -> int:
+    c = cfg.c()
+    n = _lib.mtfm_bwd_workspace_bytes(ctypes.byref(c), int(bool(target)))
+    if n == 0:
+        raise MtfmError(1, "mtfm_bwd_workspace_bytes")
+    return n
+
+
+def _bwd(fn, where, cfg, meta, q, k, v, u, gamma, beta, a, stats, dy, dq, dk, dv, du, dgamma,
+         dbeta, ws, stream, rows):
+    c = cfg.c()
+    D, Dkv, N = cfg.D, cfg.Dkv, cfg.total_tokens
+    bf, f32 = torch.bfloat16, torch.float32
+    st = fn(ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"),
+            _ptr(q, bf, (rows, D), "q"), _ptr(k, bf, (N, Dkv), "k"), _ptr(v, bf, (N, Dkv), "v"),
+            _ptr(u, bf, (rows, D), "u"), _ptr(gamma, f32, (3, D), "gamma"),
+            _ptr(beta, f32, (3, D), "beta"), _ptr(a, f32, (rows, D), "a"),
+            _ptr(stats, f32, (rows, 2), "stats"), _ptr(dy, bf, (rows, D), "dy"),
+            _ptr(dq, f32, (rows, D), "dq"), _ptr(dk, f32, (N, Dkv), "dk"),
+            _ptr(dv, f32, (N, Dkv), "dv"), _ptr(du, f32, (rows, D), "du"),
+            _ptr(dgamma, f32, (3, D), "dgamma"), _ptr(dbeta, f32, (3, D), "dbeta"),
+            _ptr(ws, torch.uint8, None, "ws"), ws.numel(), _stream(stream))
+    _check(st, where)
+
+
+def attn_full_bwd(cfg, meta, q, k, v, u, gamma, beta, a, stats, dy, dq, dk, dv, du, dgamma, dbeta,
+                  ws, stream=None):
+    _bwd(_lib.mtfm_attn_full_bwd, "mtfm_attn_full_bwd", cfg, meta, q, k, v, u, gamma, beta, a,
+         stats, dy, dq, dk, dv, du, dgamma, dbeta, ws, stream, cfg.total_tokens)
+
+
+def attn_target_bwd(cfg, meta, q, k, v, u, gamma, beta, a, stats, dy, dq, dk, dv, du, dgamma,
+                    dbeta, ws, stream=None):
+    _bwd(_lib.mtfm_attn_target_bwd, "mtfm_attn_target_bwd", cfg, meta, q, k, v, u, gamma, beta, a,
+         stats, dy, dq, dk, dv, du, dgamma, dbeta, ws, stream, cfg.total_t)

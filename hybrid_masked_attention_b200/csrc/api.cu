@@ -1,0 +1,339 @@
+// extern "C" entry points of libmtfm: host-side argument checks, then launches.
+// No allocation, no synchronisation (except mtfm_pack_check / mtfm_meta_read,
+// which synchronise on purpose).  See include/mtfm.h for the contract.
+#include <math.h>
+#include <string.h>
+
+#include "mtfm_internal.cuh"
+
+using namespace mtfm;
+
+namespace {
+
+struct Resolved {
+  int B, total_tokens, total_r, total_t, hq, hkv, dh, v2, D, Dkv;
+  float alpha, eps;
+};
+
+mtfm_status resolve(const mtfm_cfg* c, Resolved* r) {
+  if (!c) return MTFM_ERR_INVALID_ARG;
+  if (c->batch < 0 || c->total_tokens < 0 || c->total_r < 0 || c->total_t < 0)
+    return MTFM_ERR_INVALID_ARG;
+  if (c->total_r + c->total_t > c->total_tokens) return MTFM_ERR_INVALID_ARG;
+  if (c->hq <= 0 || c->hkv <= 0 || c->head_dim <= 0) return MTFM_ERR_INVALID_ARG;
+  if (c->hq % c->hkv != 0) return MTFM_ERR_INVALID_ARG;
+  if (c->v2_subtokens != 1 && c->v2_subtokens != 4) return MTFM_ERR_INVALID_ARG;
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return MTFM_ERR_UNSUPPORTED;
+  if (c->hq / c->hkv > 8) return MTFM_ERR_UNSUPPORTED;
+  const long long D = (long long)c->hq * c->head_dim;
+  if (D > 1024 || D % 32 != 0) return MTFM_ERR_UNSUPPORTED;
+  // Row offsets are int32 inside the kernels; element offsets are size_t.
+  if ((long long)c->total_tokens * D > (1ll << 40)) return MTFM_ERR_UNSUPPORTED;
+  r->B = c->batch;
+  r->total_tokens = c->total_tokens;
+  r->total_r = c->total_r;
+  r->total_t = c->total_t;
+  r->hq = c->hq;
+  r->hkv = c->hkv;
+  r->dh = c->head_dim;
+  r->v2 = c->v2_subtokens;
+  r->D = (int)D;
+  r->Dkv = c->hkv * c->head_dim;
+  r->alpha = c->alpha > 0.f ? c->alpha : 1.0f / sqrtf((float)c->head_dim);
+  r->eps = c->gln_eps > 0.f ? c->gln_eps : 1e-5f;
+  return MTFM_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline mtfm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MTFM_OK : MTFM_ERR_CUDA; }
+
+mtfm_status check_meta(const void* d_meta, const Resolved& r) {
+  if (!d_meta) return MTFM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_meta) & 255u) != 0) return MTFM_ERR_INVALID_ARG;
+  return MTFM_OK;
+}
+
+// Attention only: A (fp32) for the Full or Target layout.
+mtfm_status attn_only(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                      const uint16_t* d_k, const uint16_t* d_v, float* d_a, void* stream,
+                      bool target) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  const int rows = target ? r.total_t : r.total_tokens;
+  if (r.total_tokens == 0) return MTFM_OK;
+  if (!d_k || !d_v) return MTFM_ERR_INVALID_ARG;
+  if (rows > 0 && (!d_q || !d_a)) return MTFM_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_v) || !aligned16(d_a))
+    return MTFM_ERR_INVALID_ARG;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  const MetaView m = meta_view(const_cast<void*>(d_meta), L);
+  AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
+  const int max_items = target ? L.max_items_target : L.max_items_full;
+  return cuda_status(launch_attn_fwd_mma(shape, m, max_items,
+                                         reinterpret_cast<const __nv_bfloat16*>(d_q),
+                                         reinterpret_cast<const __nv_bfloat16*>(d_k),
+                                         reinterpret_cast<const __nv_bfloat16*>(d_v), d_a,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+mtfm_status gate_fwd(const mtfm_cfg* cfg, const void* d_meta, bool target, const float* d_a,
+                     const uint16_t* d_u, const float* d_gamma, const float* d_beta, float* d_y,
+                     float* d_stats, void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  const int rows = target ? r.total_t : r.total_tokens;
+  if (rows == 0) return MTFM_OK;
+  if (!d_a || !d_u || !d_y) return MTFM_ERR_INVALID_ARG;
+  if ((d_gamma == nullptr) != (d_beta == nullptr)) return MTFM_ERR_INVALID_ARG;
+  if (d_gamma && !d_stats) return MTFM_ERR_INVALID_ARG;
+  if (!aligned16(d_a) || !aligned16(d_u) || !aligned16(d_y) ||
+      (d_gamma && (!aligned16(d_gamma) || !aligned16(d_beta))) ||
+      (d_stats && (reinterpret_cast<uintptr_t>(d_stats) & 7u)))
+    return MTFM_ERR_INVALID_ARG;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  const MetaView m = meta_view(const_cast<void*>(d_meta), L);
+  return cuda_status(launch_gate_fwd(m, target, rows, r.D, r.eps, d_a,
+                                     reinterpret_cast<const __nv_bfloat16*>(d_u), d_gamma, d_beta,
+                                     d_y, d_stats, static_cast<cudaStream_t>(stream)));
+}
+
+mtfm_status attn_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                     const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                     const float* d_gamma, const float* d_beta, float* d_y, float* d_a,
+                     float* d_stats, void* stream, bool target) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  const int rows = target ? r.total_t : r.total_tokens;
+  // validate both halves before launching either
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  if (r.total_tokens == 0) return MTFM_OK;
+  if (rows > 0 && (!d_u || !d_y)) return MTFM_ERR_INVALID_ARG;
+  if ((d_gamma == nullptr) != (d_beta == nullptr)) return MTFM_ERR_INVALID_ARG;
+  if (d_gamma && rows > 0 && !d_stats) return MTFM_ERR_INVALID_ARG;
+  if (!aligned16(d_u) || !aligned16(d_y) || (d_gamma && (!aligned16(d_gamma) || !aligned16(d_beta))) ||
+      (d_stats && (reinterpret_cast<uintptr_t>(d_stats) & 7u)))
+    return MTFM_ERR_INVALID_ARG;
+  s = attn_only(cfg, d_meta, d_q, d_k, d_v, d_a, stream, target);
+  if (s != MTFM_OK) return s;
+  return gate_fwd(cfg, d_meta, target, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream);
+}
+
+// Scratch of the backward: dA in bf16 [rows, D], then the dgamma/dbeta partials.
+struct BwdWs {
+  size_t da, partials, total;
+};
+BwdWs bwd_ws(const Resolved& r, bool target) {
+  BwdWs w;
+  const int rows = target ? r.total_t : r.total_tokens;
+  w.da = 0;
+  w.partials = align256(sizeof(uint16_t) * (size_t)rows * r.D);
+  w.total = align256(w.partials + sizeof(float) * 6 * (size_t)r.D * kGateBwdBlocks);
+  return w;
+}
+
+mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                     const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                     const float* d_gamma, const float* d_beta, const float* d_a,
+                     const float* d_stats, const uint16_t* d_dy, float* d_dq, float* d_dk,
+                     float* d_dv, float* d_du, float* d_dgamma, float* d_dbeta, void* d_ws,
+                     size_t ws_bytes, void* stream, bool target) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  if (r.total_tokens == 0) return MTFM_OK;
+  const int rows = target ? r.total_t : r.total_tokens;
+  if (!d_k || !d_v || !d_dk || !d_dv || !d_ws) return MTFM_ERR_INVALID_ARG;
+  if (rows > 0 && (!d_q || !d_u || !d_a || !d_dy || !d_dq || !d_du)) return MTFM_ERR_INVALID_ARG;
+  const bool gln = d_gamma != nullptr;
+  if ((d_beta != nullptr) != gln || (d_dgamma != nullptr) != gln || (d_dbeta != nullptr) != gln)
+    return MTFM_ERR_INVALID_ARG;
+  if (gln && rows > 0 && !d_stats) return MTFM_ERR_INVALID_ARG;
+  const void* ptrs[] = {d_q, d_k, d_v, d_u, d_a, d_dy, d_dq, d_dk, d_dv, d_du, d_ws};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MTFM_ERR_INVALID_ARG;
+  const BwdWs w = bwd_ws(r, target);
+  if (ws_bytes < w.total) return MTFM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  const MetaView m = meta_view(const_cast<void*>(d_meta), L);
+  char* ws = static_cast<char*>(d_ws);
+  __nv_bfloat16* da = reinterpret_cast<__nv_bfloat16*>(ws + w.da);
+  float* partials = reinterpret_cast<float*>(ws + w.partials);
+  cudaError_t e = cudaSuccess;
+  if (rows > 0) {
+    e = cudaMemsetAsync(d_dq, 0, sizeof(float) * (size_t)rows * r.D, st);
+    if (e != cudaSuccess) return MTFM_ERR_CUDA;
+  }
+  e = launch_gate_bwd(m, target, rows, r.D, r.eps, d_a, d_stats,
+                      reinterpret_cast<const __nv_bfloat16*>(d_u),
+                      reinterpret_cast<const __nv_bfloat16*>(d_dy), d_gamma, d_beta, d_du, da,
+                      partials, kGateBwdBlocks, d_dgamma, d_dbeta, st);
+  if (e != cudaSuccess) return MTFM_ERR_CUDA;
+  AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
+  e = launch_attn_bwd_mma(shape, m, L.max_items_full, reinterpret_cast<const __nv_bfloat16*>(d_q),
+                          reinterpret_cast<const __nv_bfloat16*>(d_k),
+                          reinterpret_cast<const __nv_bfloat16*>(d_v), da, d_dq, d_dk, d_dv, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mtfm_status_string(mtfm_status s) {
+  switch (s) {
+    case MTFM_OK: return "ok";
+    case MTFM_ERR_INVALID_ARG: return "invalid argument";
+    case MTFM_ERR_UNSORTED_TS: return "R timestamps not ascending within a user";
+    case MTFM_ERR_UNSUPPORTED: return "unsupported shape";
+    case MTFM_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MTFM_ERR_CUDA: return "CUDA runtime error";
+    case MTFM_ERR_TIMEOUT: return "device wait timed out";
+    case MTFM_ERR_BAD_LENGTHS: return "lengths negative, inconsistent with totals, or L_T not a multiple of v2_subtokens";
+  }
+  return "unknown status";
+}
+
+size_t mtfm_meta_bytes(const mtfm_cfg* cfg) {
+  Resolved r;
+  if (resolve(cfg, &r) != MTFM_OK) return 0;
+  return meta_layout(r.B, r.total_tokens, r.total_t).total;
+}
+
+mtfm_status mtfm_pack(const mtfm_cfg* cfg, const int32_t* d_lh, const int32_t* d_lr,
+                      const int32_t* d_lt, const int64_t* d_r_ts, const int64_t* d_t_exp,
+                      void* d_meta, size_t meta_bytes, void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  if (meta_bytes < L.total) return MTFM_ERR_WORKSPACE_TOO_SMALL;
+  if (r.B > 0 && (!d_lh || !d_lr || !d_lt)) return MTFM_ERR_INVALID_ARG;
+  if (r.total_r > 0 && !d_r_ts) return MTFM_ERR_INVALID_ARG;
+  if (r.total_t > 0 && !d_t_exp) return MTFM_ERR_INVALID_ARG;
+  const MetaView m = meta_view(d_meta, L);
+  return cuda_status(launch_pack(*cfg, m, d_lh, d_lr, d_lt, d_r_ts, d_t_exp,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+mtfm_status mtfm_pack_check(const void* d_meta, void* stream) {
+  if (!d_meta) return MTFM_ERR_INVALID_ARG;
+  MetaHeader h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, d_meta, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MTFM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MTFM_ERR_CUDA;
+  if (h.magic != kMetaMagic) return MTFM_ERR_INVALID_ARG;
+  if (h.error & kErrBadLengths) return MTFM_ERR_BAD_LENGTHS;
+  if (h.error & kErrUnsorted) return MTFM_ERR_UNSORTED_TS;
+  if (h.error & kErrTimeout) return MTFM_ERR_TIMEOUT;
+  return MTFM_OK;
+}
+
+mtfm_status mtfm_meta_read(const mtfm_cfg* cfg, const void* d_meta, int32_t* seq_off,
+                           int32_t* r_off, int32_t* t_off, int32_t* kv_end, uint8_t* row_type,
+                           int32_t* n_items_full, int32_t* n_items_target, int32_t* items_full,
+                           int32_t* items_target, void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const char* b = static_cast<const char*>(d_meta);
+  MetaHeader h;
+  struct Cp { void* dst; size_t off, bytes; } cps[] = {
+      {&h, 0, sizeof(h)},
+      {seq_off, L.seq_off, sizeof(int32_t) * (size_t)(r.B + 1)},
+      {r_off, L.r_off, sizeof(int32_t) * (size_t)(r.B + 1)},
+      {t_off, L.t_off, sizeof(int32_t) * (size_t)(r.B + 1)},
+      {kv_end, L.kv_end, sizeof(int32_t) * (size_t)r.total_tokens},
+      {row_type, L.row_type, (size_t)r.total_tokens},
+      {items_full, L.items_full, sizeof(WorkItem) * (size_t)L.max_items_full},
+      {items_target, L.items_target, sizeof(WorkItem) * (size_t)L.max_items_target},
+  };
+  for (const Cp& c : cps) {
+    if (!c.dst || c.bytes == 0) continue;
+    if (cudaMemcpyAsync(c.dst, b + c.off, c.bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return MTFM_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MTFM_ERR_CUDA;
+  if (n_items_full) *n_items_full = h.n_items_full;
+  if (n_items_target) *n_items_target = h.n_items_target;
+  return MTFM_OK;
+}
+
+mtfm_status mtfm_attn_full_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                               const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                               const float* d_gamma, const float* d_beta, float* d_y, float* d_a,
+                               float* d_stats, void* stream) {
+  return attn_fwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_y, d_a, d_stats, stream,
+                  false);
+}
+
+mtfm_status mtfm_attn_target_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                 const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                 const float* d_gamma, const float* d_beta, float* d_y,
+                                 float* d_a, float* d_stats, void* stream) {
+  return attn_fwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_y, d_a, d_stats, stream,
+                  true);
+}
+
+int32_t mtfm_max_items(const mtfm_cfg* cfg, int is_target) {
+  Resolved r;
+  if (resolve(cfg, &r) != MTFM_OK) return -1;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  return is_target ? L.max_items_target : L.max_items_full;
+}
+
+mtfm_status mtfm_attn_full(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                           const uint16_t* d_k, const uint16_t* d_v, float* d_a, void* stream) {
+  return attn_only(cfg, d_meta, d_q, d_k, d_v, d_a, stream, false);
+}
+
+mtfm_status mtfm_attn_target(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                             const uint16_t* d_k, const uint16_t* d_v, float* d_a, void* stream) {
+  return attn_only(cfg, d_meta, d_q, d_k, d_v, d_a, stream, true);
+}
+
+mtfm_status mtfm_gate_fwd(const mtfm_cfg* cfg, const void* d_meta, int is_target, const float* d_a,
+                          const uint16_t* d_u, const float* d_gamma, const float* d_beta,
+                          float* d_y, float* d_stats, void* stream) {
+  return gate_fwd(cfg, d_meta, is_target != 0, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream);
+}
+
+size_t mtfm_bwd_workspace_bytes(const mtfm_cfg* cfg, int is_target) {
+  Resolved r;
+  if (resolve(cfg, &r) != MTFM_OK) return 0;
+  return bwd_ws(r, is_target != 0).total;
+}
+
+mtfm_status mtfm_attn_full_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                               const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                               const float* d_gamma, const float* d_beta, const float* d_a,
+                               const float* d_stats, const uint16_t* d_dy, float* d_dq,
+                               float* d_dk, float* d_dv, float* d_du, float* d_dgamma,
+                               float* d_dbeta, void* d_ws, size_t ws_bytes, void* stream) {
+  return attn_bwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_a, d_stats, d_dy, d_dq,
+                  d_dk, d_dv, d_du, d_dgamma, d_dbeta, d_ws, ws_bytes, stream, false);
+}
+
+mtfm_status mtfm_attn_target_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                 const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                 const float* d_gamma, const float* d_beta, const float* d_a,
+                                 const float* d_stats, const uint16_t* d_dy, float* d_dq,
+                                 float* d_dk, float* d_dv, float* d_du, float* d_dgamma,
+                                 float* d_dbeta, void* d_ws, size_t ws_bytes, void* stream) {
+  return attn_bwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_a, d_stats, d_dy, d_dq,
+                  d_dk, d_dv, d_du, d_dgamma, d_dbeta, d_ws, ws_bytes, stream, true);
+}
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+// Internal definitions shared by the CUDA translation units of libmtfm.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/mtfm.h"
+
+namespace mtfm {
+
+// Query rows per work item (one item = one 128-row query tile of one user).
+constexpr int kTileM = 128;
+constexpr int kRowH = 0, kRowR = 1, kRowT = 2;
+
+// Device error bits recorded in MetaHeader::error.
+constexpr int kErrBadLengths = 1;
+constexpr int kErrUnsorted = 2;
+constexpr int kErrTimeout = 4;
+
+constexpr int kMetaMagic = 0x4d54464d;  // "MTFM"
+
+// Layout of the caller-owned metadata block written by mtfm_pack.
+struct MetaHeader {
+  int32_t magic;
+  int32_t batch;
+  int32_t total_tokens;
+  int32_t total_r;
+  int32_t total_t;
+  int32_t v2;
+  int32_t n_items_full;
+  int32_t n_items_target;
+  int32_t error;
+  int32_t max_items_full;
+  int32_t max_items_target;
+  int32_t pad[5];
+};
+
+// One work item: a 128-row query tile of one user and the range of prefix
+// ends (kv_end) over its rows.  Keys at or beyond kv_max are never read for
+// the prefix part; key blocks entirely below kv_min need no mask test.
+struct WorkItem {
+  int32_t user;
+  int32_t tile;
+  int32_t kv_min;
+  int32_t kv_max;
+};
+
+struct MetaLayout {
+  size_t seq_off, r_off, t_off, lh, lr, lt, kv_end, row_type, items_full, items_target, total;
+  int32_t max_items_full, max_items_target;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline MetaLayout meta_layout(int B, int total_tokens, int total_t) {
+  MetaLayout L;
+  size_t o = align256(sizeof(MetaHeader));
+  L.seq_off = o; o = align256(o + sizeof(int32_t) * (B + 1));
+  L.r_off = o;   o = align256(o + sizeof(int32_t) * (B + 1));
+  L.t_off = o;   o = align256(o + sizeof(int32_t) * (B + 1));
+  L.lh = o;      o = align256(o + sizeof(int32_t) * B);
+  L.lr = o;      o = align256(o + sizeof(int32_t) * B);
+  L.lt = o;      o = align256(o + sizeof(int32_t) * B);
+  L.kv_end = o;  o = align256(o + sizeof(int32_t) * (size_t)total_tokens);
+  L.row_type = o; o = align256(o + (size_t)total_tokens);
+  L.max_items_full = (total_tokens + kTileM - 1) / kTileM + B;
+  L.max_items_target = (total_t + kTileM - 1) / kTileM + B;
+  L.items_full = o;   o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_full);
+  L.items_target = o; o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_target);
+  L.total = o;
+  return L;
+}
+
+// Device view of the metadata block.
+struct MetaView {
+  MetaHeader* hdr;
+  int32_t* seq_off;
+  int32_t* r_off;
+  int32_t* t_off;
+  int32_t* lh;
+  int32_t* lr;
+  int32_t* lt;
+  int32_t* kv_end;
+  uint8_t* row_type;
+  WorkItem* items_full;
+  WorkItem* items_target;
+};
+
+inline MetaView meta_view(void* base, const MetaLayout& L) {
+  char* b = static_cast<char*>(base);
+  MetaView v;
+  v.hdr = reinterpret_cast<MetaHeader*>(b);
+  v.seq_off = reinterpret_cast<int32_t*>(b + L.seq_off);
+  v.r_off = reinterpret_cast<int32_t*>(b + L.r_off);
+  v.t_off = reinterpret_cast<int32_t*>(b + L.t_off);
+  v.lh = reinterpret_cast<int32_t*>(b + L.lh);
+  v.lr = reinterpret_cast<int32_t*>(b + L.lr);
+  v.lt = reinterpret_cast<int32_t*>(b + L.lt);
+  v.kv_end = reinterpret_cast<int32_t*>(b + L.kv_end);
+  v.row_type = reinterpret_cast<uint8_t*>(b + L.row_type);
+  v.items_full = reinterpret_cast<WorkItem*>(b + L.items_full);
+  v.items_target = reinterpret_cast<WorkItem*>(b + L.items_target);
+  return v;
+}
+
+// Everything an attention launch needs besides the tensors.
+struct AttnShape {
+  int hq, hkv, dh, v2;
+  float alpha;
+  bool target;  // Target-Attention layer: queries are T rows only
+};
+
+// Launchers implemented in the .cu files (return cudaGetLastError()).
+cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* lh,
+                        const int32_t* lr, const int32_t* lt, const int64_t* r_ts,
+                        const int64_t* t_exp, cudaStream_t st);
+cudaError_t launch_attn_fwd_mma(const AttnShape& s, const MetaView& m, int max_items,
+                                const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                const __nv_bfloat16* v, float* a, cudaStream_t st);
+cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, float eps,
+                            const float* a, const __nv_bfloat16* u, const float* gamma,
+                            const float* beta, float* y, float* stats, cudaStream_t st);
+cudaError_t launch_gate_bwd(const MetaView& m, bool target, int rows, int D, float eps,
+                            const float* a, const float* stats, const __nv_bfloat16* u,
+                            const __nv_bfloat16* dy, const float* gamma, const float* beta,
+                            float* du, __nv_bfloat16* da, float* partials, int n_part_blocks,
+                            float* dgamma, float* dbeta, cudaStream_t st);
+cudaError_t launch_attn_bwd_mma(const AttnShape& s, const MetaView& m, int max_items_full,
+                                const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                const __nv_bfloat16* v, const __nv_bfloat16* da, float* dq,
+                                float* dk, float* dv, cudaStream_t st);
+
+constexpr int kGateBwdBlocks = 296;  // 2 per SM on a 148-SM part; partial dgamma/dbeta slots
+
+}  // namespace mtfm

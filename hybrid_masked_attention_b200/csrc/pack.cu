@@ -1,0 +1,292 @@
+// Jagged-batch packer and mask-metadata builder.
+//
+// Turns per-user lengths (L_H, L_R, L_T), sorted R timestamps and T exposure
+// times into the "1-D jagged mask" form that the attention kernels read
+// (Meituan tech blog "MTFM：美团统一推荐基座大模型...", §6.1: the
+// multi-dimensional mask is pre-processed into a 1-D jagged mask): one prefix
+// end kv_end per row, plus the T rows' own sibling block, which follows from the
+// row's position.  The visibility rules are those of §3.2 of the same blog:
+//   H row          : keys [0, L_H)
+//   R row a        : keys [0, L_H + a + 1)           (causal, self included)
+//   T row t        : keys [0, L_H + k_t) + itself     k_t = #{R : ts < exposure_t}
+// k_t is a lower_bound over the user's ascending R timestamps.
+//
+// Two launches, no host synchronisation:
+//   pack_users_kernel (1 CTA): validates lengths, scans offsets, orders users
+//     longest first and writes the work lists of 128-row query tiles;
+//   pack_rows_kernel (1 CTA per work item): per-row kv_end / row type, the
+//     sortedness check, and each tile's [kv_min, kv_max] used for block skipping.
+#include "mtfm_internal.cuh"
+
+namespace mtfm {
+namespace {
+
+constexpr int kPackThreads = 1024;
+constexpr int kSortMax = 8192;  // users sorted by length when B <= this; natural order beyond
+
+// Block-wide exclusive scan of one int64 value per thread; returns the prefix and the total.
+__device__ long long block_exclusive_scan(long long v, long long* total, long long* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      long long y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;  // inclusive prefix over warps
+  }
+  __syncthreads();
+  long long before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+  *total = s_warp[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+__global__ void __launch_bounds__(kPackThreads)
+pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t, int v2,
+                  int max_if, int max_it, int sort_n, const int32_t* __restrict__ lh,
+                  const int32_t* __restrict__ lr, const int32_t* __restrict__ lt) {
+  extern __shared__ unsigned long long s_keys[];  // [sort_n] (0 when not sorting)
+  __shared__ long long s_warp[32];
+  __shared__ int s_err;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_err = 0;
+  __syncthreads();
+
+  const int chunk = (B + kPackThreads - 1) / kPackThreads;
+  const int b0 = min(B, tid * chunk), b1 = min(B, b0 + chunk);
+
+  // 1. validate lengths, local sums
+  long long sN = 0, sR = 0, sT = 0;
+  int err = 0;
+  for (int b = b0; b < b1; ++b) {
+    int a = lh[b], r = lr[b], t = lt[b];
+    if (a < 0 || r < 0 || t < 0 || (t % v2) != 0) err = 1;
+    sN += (long long)a + r + t;
+    sR += r;
+    sT += t;
+  }
+  if (err) atomicOr(&s_err, kErrBadLengths);
+
+  // 2. offsets
+  long long totN, totR, totT;
+  long long pN = block_exclusive_scan(sN, &totN, s_warp);
+  long long pR = block_exclusive_scan(sR, &totR, s_warp);
+  long long pT = block_exclusive_scan(sT, &totT, s_warp);
+  if (tid == 0 && (totN != total_tokens || totR != total_r || totT != total_t))
+    atomicOr(&s_err, kErrBadLengths);
+  __syncthreads();
+  if (s_err) {
+    if (tid == 0) {
+      m.hdr->magic = kMetaMagic;
+      m.hdr->batch = B;
+      m.hdr->total_tokens = total_tokens;
+      m.hdr->total_r = total_r;
+      m.hdr->total_t = total_t;
+      m.hdr->v2 = v2;
+      m.hdr->n_items_full = 0;
+      m.hdr->n_items_target = 0;
+      m.hdr->error = s_err;
+      m.hdr->max_items_full = max_if;
+      m.hdr->max_items_target = max_it;
+    }
+    return;
+  }
+  for (int b = b0; b < b1; ++b) {
+    int a = lh[b], r = lr[b], t = lt[b];
+    m.seq_off[b] = (int)pN;
+    m.r_off[b] = (int)pR;
+    m.t_off[b] = (int)pT;
+    m.lh[b] = a;
+    m.lr[b] = r;
+    m.lt[b] = t;
+    pN += a + r + t;
+    pR += r;
+    pT += t;
+  }
+  if (tid == 0) {
+    m.seq_off[B] = total_tokens;
+    m.r_off[B] = total_r;
+    m.t_off[B] = total_t;
+  }
+
+  // 3. longest-first order (bitonic sort, descending key = N_u << 32 | ~index)
+  if (sort_n > 0) {
+    for (int i = tid; i < sort_n; i += kPackThreads) {
+      unsigned long long key = 0;
+      if (i < B) {
+        unsigned long long n = (unsigned long long)(lh[i] + lr[i] + lt[i]);
+        key = (n << 32) | (unsigned long long)(0xffffffffu - (unsigned)i);
+      }
+      s_keys[i] = key;
+    }
+    __syncthreads();
+    for (int size = 2; size <= sort_n; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < sort_n; i += kPackThreads) {
+          int j = i ^ stride;
+          if (j > i) {
+            bool desc = (i & size) == 0;
+            unsigned long long a = s_keys[i], b = s_keys[j];
+            if ((a < b) == desc) {
+              s_keys[i] = b;
+              s_keys[j] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+  auto user_at = [&](int p) -> int {
+    return sort_n > 0 ? (int)(0xffffffffu - (unsigned)(s_keys[p] & 0xffffffffull)) : p;
+  };
+
+  // 4. work lists: tiles of each user, last tile first (later rows see more keys)
+  long long cF = 0, cT = 0;
+  for (int p = b0; p < b1; ++p) {
+    int u = user_at(p);
+    int n = lh[u] + lr[u] + lt[u];
+    cF += (n + kTileM - 1) / kTileM;
+    cT += (lt[u] + kTileM - 1) / kTileM;
+  }
+  long long totF, totTT;
+  long long oF = block_exclusive_scan(cF, &totF, s_warp);
+  long long oT = block_exclusive_scan(cT, &totTT, s_warp);
+  for (int p = b0; p < b1; ++p) {
+    int u = user_at(p);
+    int n = lh[u] + lr[u] + lt[u];
+    int nf = (n + kTileM - 1) / kTileM, nt = (lt[u] + kTileM - 1) / kTileM;
+    for (int k = 0; k < nf; ++k) m.items_full[oF + k] = WorkItem{u, nf - 1 - k, 0, 0};
+    for (int k = 0; k < nt; ++k) m.items_target[oT + k] = WorkItem{u, nt - 1 - k, 0, 0};
+    oF += nf;
+    oT += nt;
+  }
+  if (tid == 0) {
+    m.hdr->magic = kMetaMagic;
+    m.hdr->batch = B;
+    m.hdr->total_tokens = total_tokens;
+    m.hdr->total_r = total_r;
+    m.hdr->total_t = total_t;
+    m.hdr->v2 = v2;
+    m.hdr->n_items_full = (int)totF;
+    m.hdr->n_items_target = (int)totTT;
+    m.hdr->error = 0;
+    m.hdr->max_items_full = max_if;
+    m.hdr->max_items_target = max_it;
+  }
+}
+
+// Number of R timestamps strictly below `x` in the ascending array ts[0, n).
+__device__ __forceinline__ int count_below(const int64_t* __restrict__ ts, int n, int64_t x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (ts[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kTileM)
+pack_rows_kernel(MetaView m, int max_if, const int64_t* __restrict__ r_ts,
+                 const int64_t* __restrict__ t_exp) {
+  __shared__ int s_min[kTileM / 32], s_max[kTileM / 32];
+  const MetaHeader* hdr = m.hdr;
+  if (hdr->error & kErrBadLengths) return;
+  const bool tgt = (int)blockIdx.x >= max_if;
+  const int idx = tgt ? blockIdx.x - max_if : blockIdx.x;
+  if (idx >= (tgt ? hdr->n_items_target : hdr->n_items_full)) return;
+  WorkItem* it = (tgt ? m.items_target : m.items_full) + idx;
+  const int u = it->user, tile = it->tile;
+  const int LH = m.lh[u], LR = m.lr[u], LT = m.lt[u];
+  const int N = LH + LR + LT, so = m.seq_off[u];
+  const int nq = tgt ? LT : N;
+  const int r = tile * kTileM + threadIdx.x;
+  int kmin = 0x7fffffff, kmax = 0;
+  if (r < nq) {
+    const int i = tgt ? LH + LR + r : r;
+    int kve, type;
+    if (i < LH) {
+      type = kRowH;
+      kve = LH;
+    } else if (i < LH + LR) {
+      type = kRowR;
+      kve = i + 1;
+      const int a = i - LH;
+      if (!tgt && a > 0 && r_ts[m.r_off[u] + a - 1] > r_ts[m.r_off[u] + a])
+        atomicOr(&m.hdr->error, kErrUnsorted);
+    } else {
+      type = kRowT;
+      kve = LH + count_below(r_ts + m.r_off[u], LR, t_exp[m.t_off[u] + (i - LH - LR)]);
+    }
+    if (!tgt) {
+      m.kv_end[so + i] = kve;
+      m.row_type[so + i] = (uint8_t)type;
+    }
+    kmin = kve;
+    kmax = kve;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_min[threadIdx.x >> 5] = kmin;
+    s_max[threadIdx.x >> 5] = kmax;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kTileM / 32; ++w) {
+      kmin = min(kmin, s_min[w]);
+      kmax = max(kmax, s_max[w]);
+    }
+    it->kv_min = kmin;
+    it->kv_max = kmax;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* lh,
+                        const int32_t* lr, const int32_t* lt, const int64_t* r_ts,
+                        const int64_t* t_exp, cudaStream_t st) {
+  const MetaLayout L = meta_layout(cfg.batch, cfg.total_tokens, cfg.total_t);
+  int sort_n = 0;
+  if (cfg.batch > 0 && cfg.batch <= kSortMax) {
+    sort_n = 1;
+    while (sort_n < cfg.batch) sort_n <<= 1;
+  }
+  const size_t smem = sizeof(unsigned long long) * (size_t)sort_n;
+  static bool attr_set = false;  // idempotent attribute; a race only repeats the same call
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(pack_users_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(unsigned long long) * kSortMax));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  pack_users_kernel<<<1, kPackThreads, smem, st>>>(m, cfg.batch, cfg.total_tokens, cfg.total_r,
+                                                   cfg.total_t, cfg.v2_subtokens,
+                                                   L.max_items_full, L.max_items_target, sort_n,
+                                                   lh, lr, lt);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int blocks = L.max_items_full + L.max_items_target;
+  if (blocks > 0) {
+    pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, r_ts, t_exp);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace mtfm

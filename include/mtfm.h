@@ -1,0 +1,197 @@
+/*
+ * mtfm.h -- C ABI of the B200 (sm_100a) library for MTFM's hybrid masked
+ * attention: HSTU-style pointwise-SiLU attention over jagged user-level
+ * samples [H | R | T] with the dynamic H/R/T mask, in Full-Attention layers
+ * (every token queries) and Target-Attention layers (only T tokens query),
+ * with grouped-query attention and the GLN gate.
+ *
+ * Sources (web pages on MTFM):
+ *   [DY] "美团推荐大模型 MTFM 深度硬核解析" (dingyadong.top), §4.1 Full Attention
+ *        layer equations, §4.1.1 and §8.2 dynamic mask, §4.2 Target Attention.
+ *   [MT] "MTFM：美团统一推荐基座大模型在外卖多业务场景的落地实践" (Meituan tech
+ *        blog), §3.2 mask rules, §3.3 hybrid architecture and V2 target
+ *        scale-up, §6.1 kernels (1-D jagged mask, SiLU fusion, GLN [G, D]).
+ *
+ * What every attention call computes, for user u with N_u = L_H + L_R + L_T
+ * tokens, query row i, query head h and KV group g = h / (hq / hkv):
+ *
+ *     A[i, h] = (1 / N_u) * sum_{j visible from i} SiLU(alpha * q[i,h] . k[j,g]) * v[j,g]
+ *     Y[i]    = GLN_type(i)(A[i]) (*) U[i]      (GLN over the whole row of hq*head_dim)
+ *
+ * Visibility ([MT] §3.2): H keys are visible to every query; R keys are causal
+ * within R (self included) and visible to a T query only when the R action's
+ * timestamp is strictly earlier than that target's exposure; a T key is
+ * visible only to itself (V2: to the sub-tokens of its own target).  H rows
+ * see only H.  Since SiLU(0) = 0, masking the scores before phi_2 ([DY] §4.1)
+ * is the same as dropping invisible keys.
+ *
+ * Conventions for every call below:
+ *   - Pointers named d_* are DEVICE pointers; all memory is owned by the
+ *     caller.  The library never allocates, frees or synchronises, except
+ *     mtfm_pack_check(), which synchronises the given stream on purpose.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *     Every call is asynchronous on that stream.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  Activation layout is
+ *     jagged row-major: the rows of user 0, then user 1, ...; within a user
+ *     the H rows, then R rows, then T rows.  Q/U/Y/A of a Full layer are
+ *     [sum N, hq*head_dim]; of a Target layer [sum L_T, hq*head_dim] (T rows
+ *     only, same user order); K/V are always [sum N, hkv*head_dim].  Head h
+ *     occupies columns [h*head_dim, (h+1)*head_dim).
+ *   - Host-side argument checks run before any launch; a call that returns
+ *     an error launched nothing.  Errors found on the device (lengths that do
+ *     not add up to the totals, unsorted timestamps) are recorded in the
+ *     metadata block; every later kernel that reads that block does nothing,
+ *     and mtfm_pack_check() reports them.
+ *   - Supported: head_dim in {32, 64, 128}; hq % hkv == 0; hq/hkv <= 8;
+ *     hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
+ *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
+ *   - No exceptions cross this boundary; no global state is kept.
+ */
+#ifndef MTFM_H_
+#define MTFM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MTFM_OK = 0,
+  MTFM_ERR_INVALID_ARG = 1,         /* null pointer, negative size, hq % hkv != 0, ... */
+  MTFM_ERR_UNSORTED_TS = 2,         /* R timestamps of some user not ascending (device check) */
+  MTFM_ERR_UNSUPPORTED = 3,         /* valid but unsupported shape (head_dim, widths) */
+  MTFM_ERR_WORKSPACE_TOO_SMALL = 4, /* meta or workspace buffer smaller than the size query */
+  MTFM_ERR_CUDA = 5,                /* a CUDA runtime call failed (launch error etc.) */
+  MTFM_ERR_TIMEOUT = 6,             /* a bounded device wait gave up (kernel returned early) */
+  MTFM_ERR_BAD_LENGTHS = 7          /* device lengths negative, not summing to the totals, or
+                                       L_T not a multiple of v2_subtokens */
+} mtfm_status;
+
+/* Problem description shared by all calls (host memory, read only). */
+typedef struct {
+  int32_t batch;          /* B: number of users (jagged samples) */
+  int32_t total_tokens;   /* sum over users of N_u = L_H + L_R + L_T */
+  int32_t total_r;        /* sum of L_R */
+  int32_t total_t;        /* sum of L_T */
+  int32_t hq;             /* query heads H */
+  int32_t hkv;            /* KV heads G (GQA groups); r = hq / hkv query heads share one */
+  int32_t head_dim;       /* per-head width */
+  int32_t v2_subtokens;   /* 1: one token per target; 4: V2 target scale-up ([MT] §3.3.2) */
+  float alpha;            /* score scale inside SiLU; <= 0 selects 1/sqrt(head_dim) */
+  float gln_eps;          /* GLN epsilon; <= 0 selects 1e-5 */
+} mtfm_cfg;
+
+/* Human-readable text of a status (static string, never NULL). */
+const char* mtfm_status_string(mtfm_status s);
+
+/* ---------------------------------------------------------------------------
+ * Jagged pack + mask metadata ("1-D jagged mask" of [MT] §6.1; mask rules of
+ * [MT] §3.2).  Builds, in the caller's d_meta block: per-user offsets, per-row
+ * token type and prefix end kv_end (H row: L_H; R row a: L_H + a + 1; T row:
+ * L_H + #{R : ts < exposure}), and the work lists of 128-row query tiles with
+ * their key bounds, users ordered longest first.  Fully masked key blocks are
+ * never visited by the attention kernels: they read only keys below the
+ * tile's largest kv_end plus the T tile's own sibling block.
+ *
+ *   d_lh, d_lr, d_lt : int32 [batch] device arrays of per-user lengths.
+ *   d_r_ts           : int64 [total_r] R-token timestamps, ascending per user.
+ *   d_t_exp          : int64 [total_t] exposure time of every T token (V2:
+ *                      the 4 sub-tokens of one target carry the same value).
+ *   d_meta           : device block of at least mtfm_meta_bytes(cfg) bytes,
+ *                      256-byte aligned; fully rewritten by this call.
+ * ------------------------------------------------------------------------- */
+size_t mtfm_meta_bytes(const mtfm_cfg* cfg);
+mtfm_status mtfm_pack(const mtfm_cfg* cfg, const int32_t* d_lh, const int32_t* d_lr,
+                      const int32_t* d_lt, const int64_t* d_r_ts, const int64_t* d_t_exp,
+                      void* d_meta, size_t meta_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device-side verdict of the last
+ * mtfm_pack on d_meta (MTFM_OK, MTFM_ERR_BAD_LENGTHS, MTFM_ERR_UNSORTED_TS)
+ * or MTFM_ERR_TIMEOUT if an attention kernel recorded a timeout there.
+ * Optional: the hot path never needs it. */
+mtfm_status mtfm_pack_check(const void* d_meta, void* stream);
+
+/* Copies the metadata block's arrays into caller host buffers (synchronous;
+ * any pointer may be NULL).  seq_off/r_off/t_off are int32 [batch+1],
+ * kv_end int32 [total_tokens], row_type uint8 [total_tokens] (0 H, 1 R, 2 T).
+ * items_full / items_target receive the work lists as int32 [n][4] rows
+ * (user, tile, kv_min, kv_max) and must hold mtfm_max_items(cfg, 0 / 1) rows.
+ * For tests and debugging. */
+mtfm_status mtfm_meta_read(const mtfm_cfg* cfg, const void* d_meta, int32_t* seq_off,
+                           int32_t* r_off, int32_t* t_off, int32_t* kv_end, uint8_t* row_type,
+                           int32_t* n_items_full, int32_t* n_items_target, int32_t* items_full,
+                           int32_t* items_target, void* stream);
+
+/* Capacity of the Full (is_target = 0) or Target (1) work list: the upper bound
+ * sum(ceil(rows_u / 128)) <= ceil(rows / 128) + batch. */
+int32_t mtfm_max_items(const mtfm_cfg* cfg, int is_target);
+
+/* ---------------------------------------------------------------------------
+ * Full-Attention layer forward ([DY] §4.1): every token of every user is a query.
+ *   d_q, d_u : bf16 [total_tokens, hq*head_dim];   d_k, d_v : bf16 [total_tokens, hkv*head_dim]
+ *   d_gamma, d_beta : fp32 [3, hq*head_dim] GLN affine rows for H, R, T tokens
+ *                     ([MT] §6.1, one [G, D] matrix indexed by token type), or
+ *                     both NULL for the plain gate Y = A (*) U.
+ *   d_y       : fp32 [total_tokens, hq*head_dim] output Y.
+ *   d_a       : fp32 [total_tokens, hq*head_dim] output A (attention before the
+ *               gate; saved for the backward pass).  Required.
+ *   d_stats   : fp32 [total_tokens, 2] output (mean, rstd) of each row's GLN;
+ *               ignored (may be NULL) when d_gamma is NULL.
+ * ------------------------------------------------------------------------- */
+mtfm_status mtfm_attn_full_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                               const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                               const float* d_gamma, const float* d_beta, float* d_y, float* d_a,
+                               float* d_stats, void* stream);
+
+/* Target-Attention layer forward ([DY] §4.2): only T rows query; K/V span the
+ * whole sequence of each user.  As mtfm_attn_full_fwd except that d_q, d_u,
+ * d_y, d_a are [total_t, hq*head_dim] and d_stats is [total_t, 2]; all rows use
+ * the T row of gamma/beta.  H/R rows are not touched (the shortcut of [DY] §4.2). */
+mtfm_status mtfm_attn_target_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                 const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                 const float* d_gamma, const float* d_beta, float* d_y,
+                                 float* d_a, float* d_stats, void* stream);
+
+/* The two halves of a layer forward, for callers that schedule them apart
+ * (the layer calls above are exactly attention followed by the gate).
+ *   mtfm_attn_full / mtfm_attn_target : writes A only (fp32, shapes as above).
+ *   mtfm_gate_fwd : Y = GLN(A) (*) U (plain A (*) U when d_gamma is NULL) for the
+ *                   Full (is_target = 0, GLN row picked by token type) or Target
+ *                   (is_target = 1, T row of gamma/beta) layout; writes d_y and,
+ *                   with GLN, d_stats.  [DY] §4.1 gate; [MT] §6.1 GLN kernel. */
+mtfm_status mtfm_attn_full(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                           const uint16_t* d_k, const uint16_t* d_v, float* d_a, void* stream);
+mtfm_status mtfm_attn_target(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                             const uint16_t* d_k, const uint16_t* d_v, float* d_a, void* stream);
+mtfm_status mtfm_gate_fwd(const mtfm_cfg* cfg, const void* d_meta, int is_target, const float* d_a,
+                          const uint16_t* d_u, const float* d_gamma, const float* d_beta,
+                          float* d_y, float* d_stats, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Backward passes (training step).  Inputs are the forward's inputs, its saved
+ * A (d_a) and stats, and the upstream gradient d_dy (bf16, same shape as Y).
+ * Outputs (fp32, fully overwritten):
+ *   d_dq, d_du : same rows as Q/U;   d_dk, d_dv : [total_tokens, hkv*head_dim]
+ *   d_dgamma, d_dbeta : [3, hq*head_dim] (NULL iff d_gamma is NULL)
+ * d_ws is scratch of at least mtfm_bwd_workspace_bytes(cfg, is_target) bytes.
+ * ------------------------------------------------------------------------- */
+size_t mtfm_bwd_workspace_bytes(const mtfm_cfg* cfg, int is_target);
+mtfm_status mtfm_attn_full_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                               const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                               const float* d_gamma, const float* d_beta, const float* d_a,
+                               const float* d_stats, const uint16_t* d_dy, float* d_dq,
+                               float* d_dk, float* d_dv, float* d_du, float* d_dgamma,
+                               float* d_dbeta, void* d_ws, size_t ws_bytes, void* stream);
+mtfm_status mtfm_attn_target_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                 const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                 const float* d_gamma, const float* d_beta, const float* d_a,
+                                 const float* d_stats, const uint16_t* d_dy, float* d_dq,
+                                 float* d_dk, float* d_dv, float* d_du, float* d_dgamma,
+                                 float* d_dbeta, void* d_ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MTFM_H_ */

@@ -1,0 +1,106 @@
+"""The C-ABI library builds, loads and exports every symbol include/mtfm.h declares;
+host-side argument checks reject bad input before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _build():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_mtfm_build", os.path.join(ROOT, "hybrid_masked_attention_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = _build()
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "mtfm.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mtfm_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    for s in syms:
+        assert hasattr(lib, s), f"{s} missing from libmtfm.so"
+
+
+def test_binding_wraps_every_symbol(lib):
+    import hybrid_masked_attention_b200 as m
+    assert set(declared_symbols()) == set(m.EXPORTED)
+
+
+def _cfg(**kw):
+    import hybrid_masked_attention_b200 as m
+    base = dict(batch=2, total_tokens=20, total_r=4, total_t=4, hq=8, hkv=2, head_dim=64)
+    base.update(kw)
+    return m.Config(**base).c()
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(hq=6, hkv=4), 1),           # hq % hkv != 0
+    (dict(head_dim=48), 3),           # unsupported head_dim
+    (dict(hq=16, hkv=1, head_dim=32), 3),   # r > 8
+    (dict(batch=-1), 1),
+    (dict(total_r=30), 1),            # R + T exceed the token total
+    (dict(v2_subtokens=3), 1),
+])
+def test_invalid_config_rejected_before_launch(lib, kw, status):
+    import hybrid_masked_attention_b200 as m
+    c = _cfg(**kw)
+    assert m._lib.mtfm_meta_bytes(ctypes.byref(c)) == 0
+    st = m._lib.mtfm_pack(ctypes.byref(c), None, None, None, None, None, None, 0, None)
+    assert st == status
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    import hybrid_masked_attention_b200 as m
+    c = _cfg()
+    # null metadata block
+    assert m._lib.mtfm_pack(ctypes.byref(c), 1024, 1024, 1024, 1024, 1024, None, 1 << 20, None) == 1
+    # metadata block not 256-byte aligned
+    assert m._lib.mtfm_pack(ctypes.byref(c), 1024, 1024, 1024, 1024, 1024, 4096 + 16, 1 << 20, None) == 1
+    # too small
+    need = m._lib.mtfm_meta_bytes(ctypes.byref(c))
+    assert m._lib.mtfm_pack(ctypes.byref(c), 1024, 1024, 1024, 1024, 1024, 4096, need - 1, None) == 4
+    # attention with missing K
+    assert m._lib.mtfm_attn_full_fwd(ctypes.byref(c), 4096, 4096, None, 4096, 4096, None, None,
+                                     4096, 4096, None, None) == 1
+    # misaligned Q
+    assert m._lib.mtfm_attn_full_fwd(ctypes.byref(c), 4096, 4096 + 2, 4096, 4096, 4096, None, None,
+                                     4096, 4096, None, None) == 1
+    # gamma without beta
+    assert m._lib.mtfm_attn_target_fwd(ctypes.byref(c), 4096, 4096, 4096, 4096, 4096, 4096, None,
+                                       4096, 4096, 4096, None) == 1
+    # backward workspace too small
+    ws = m._lib.mtfm_bwd_workspace_bytes(ctypes.byref(c), 0)
+    assert ws > 0
+    args = [4096] * 17
+    args[5], args[6], args[14], args[15] = None, None, None, None   # no GLN
+    assert m._lib.mtfm_attn_full_bwd(ctypes.byref(c), *args, ws - 1, None) == 4
+
+
+def test_status_strings(lib):
+    import hybrid_masked_attention_b200 as m
+    for s in range(8):
+        assert m._lib.mtfm_status_string(s)
+    assert b"unknown" in m._lib.mtfm_status_string(99)
+
+
+def test_meta_capacity_bounds(lib):
+    import hybrid_masked_attention_b200 as m
+    c = _cfg(batch=3, total_tokens=300, total_r=10, total_t=129)
+    assert m._lib.mtfm_max_items(ctypes.byref(c), 0) == (300 + 127) // 128 + 3
+    assert m._lib.mtfm_max_items(ctypes.byref(c), 1) == (129 + 127) // 128 + 3

@@ -1,0 +1,67 @@
+"""Full and Target forward on the GPU (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import mtfm_synth as syn
+from gpu_cases import BATCHES, HEADS
+from gpu_helpers import assert_close, packed, upload_layer
+from oracle import mtfm_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("tiny", "tiny", True), ("tiny", "tiny", False),
+    ("pair", "pair", True), ("pair", "pair", False),
+    ("edge", "pair", True), ("edge", "dh128", True), ("edge", "r8", True),
+    ("v2_n512", "pair", True), ("v2_n1024", "pair", True), ("v1_n2048", "pair", True),
+]
+
+
+def _run(batch, heads, target, gln, seed=11):
+    inp = syn.layer_inputs(batch, heads, target=target, seed=seed, gln=gln)
+    s = packed(batch, heads)
+    d = upload_layer(inp)
+    f = s.target_fwd if target else s.full_fwd
+    y, a, st = f(d["q"], d["k"], d["v"], d["u"], d["gamma"], d["beta"])
+    torch.cuda.synchronize()
+    ref = (O.target_fwd if target else O.full_fwd)(batch, heads, inp)
+    return y.cpu().numpy(), a.cpu().numpy(), (None if st is None else st.cpu().numpy()), ref
+
+
+@pytest.mark.parametrize("bname,hname,gln", CASES)
+@pytest.mark.parametrize("target", [False, True], ids=["full", "target"])
+def test_fwd_parity(bname, hname, gln, target, cuda_ok):
+    b, hd = BATCHES[bname](), HEADS[hname]
+    y, a, st, ref = _run(b, hd, target, gln)
+    assert_close(a, ref["A"], "A")
+    assert_close(y, ref["Y"], "Y")
+    if gln and len(st):
+        assert_close(st[:, 0], ref["mean"], "mean")
+        assert_close(st[:, 1], ref["rstd"], "rstd")
+
+
+def test_target_equals_full_t_rows_on_gpu(cuda_ok):
+    """Target layer == T rows of a Full layer fed the same Q/U rows (GPU vs GPU)."""
+    b, hd = BATCHES["pair"](), HEADS["pair"]
+    full = syn.layer_inputs(b, hd, target=False, seed=21)
+    so = O.offsets(b.N)
+    trows = np.concatenate([np.arange(so[u] + b.L_H[u] + b.L_R[u], so[u + 1]) for u in range(b.B)])
+    tgt = syn.LayerInputs(full.q[trows], full.k, full.v, full.u[trows], full.gamma, full.beta)
+    s = packed(b, hd)
+    df, dt = upload_layer(full), upload_layer(tgt)
+    yf, af, _ = s.full_fwd(df["q"], df["k"], df["v"], df["u"], df["gamma"], df["beta"])
+    yt, at, _ = s.target_fwd(dt["q"], dt["k"], dt["v"], dt["u"], dt["gamma"], dt["beta"])
+    torch.cuda.synchronize()
+    assert_close(at.cpu().numpy(), af.cpu().numpy()[trows], "A_T vs A_full[T]")
+    assert_close(yt.cpu().numpy(), yf.cpu().numpy()[trows], "Y_T vs Y_full[T]")
+
+
+def test_fwd_deterministic(cuda_ok):
+    b, hd = BATCHES["pair"](), HEADS["pair"]
+    inp = upload_layer(syn.layer_inputs(b, hd, target=False, seed=3))
+    s = packed(b, hd)
+    y1, a1, _ = s.full_fwd(inp["q"], inp["k"], inp["v"], inp["u"], inp["gamma"], inp["beta"])
+    y2, a2, _ = s.full_fwd(inp["q"], inp["k"], inp["v"], inp["u"], inp["gamma"], inp["beta"])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(a1, a2)
