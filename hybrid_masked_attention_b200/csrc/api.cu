@@ -2,6 +2,7 @@
 // No allocation, no synchronisation (except mtfm_pack_check / mtfm_meta_read,
 // which synchronise on purpose).  See include/mtfm.h for the contract.
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "mtfm_internal.cuh"
@@ -72,11 +73,18 @@ mtfm_status attn_only(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d
   const MetaView m = meta_view(const_cast<void*>(d_meta), L);
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
   const int max_items = target ? L.max_items_target : L.max_items_full;
-  return cuda_status(launch_attn_fwd_mma(shape, m, max_items,
-                                         reinterpret_cast<const __nv_bfloat16*>(d_q),
-                                         reinterpret_cast<const __nv_bfloat16*>(d_k),
-                                         reinterpret_cast<const __nv_bfloat16*>(d_v), d_a,
-                                         static_cast<cudaStream_t>(stream)));
+  const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(d_q);
+  const __nv_bfloat16* k = reinterpret_cast<const __nv_bfloat16*>(d_k);
+  const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(d_v);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // tcgen05/TMEM kernel where its TMEM plan fits (head_dim 64, r in {1, 2, 4});
+  // the mma.sync kernel covers the other head shapes.  MTFM_FWD_KERNEL=mma
+  // selects the mma.sync kernel for every shape (for comparisons).
+  const char* force = getenv("MTFM_FWD_KERNEL");
+  const bool force_mma = force && strcmp(force, "mma") == 0;
+  if (!force_mma && attn_fwd_tc_supported(shape))
+    return cuda_status(launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, d_a, st));
+  return cuda_status(launch_attn_fwd_mma(shape, m, max_items, q, k, v, d_a, st));
 }
 
 mtfm_status gate_fwd(const mtfm_cfg* cfg, const void* d_meta, bool target, const float* d_a,
@@ -124,15 +132,17 @@ mtfm_status attn_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   return gate_fwd(cfg, d_meta, target, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream);
 }
 
-// Scratch of the backward: dA in bf16 [rows, D], then the dgamma/dbeta partials.
+// Scratch of the backward: dA as bf16 hi and lo parts [rows, D] each, then the
+// per-block dgamma/dbeta partials.
 struct BwdWs {
-  size_t da, partials, total;
+  size_t da_hi, da_lo, partials, total;
 };
 BwdWs bwd_ws(const Resolved& r, bool target) {
   BwdWs w;
   const int rows = target ? r.total_t : r.total_tokens;
-  w.da = 0;
-  w.partials = align256(sizeof(uint16_t) * (size_t)rows * r.D);
+  w.da_hi = 0;
+  w.da_lo = align256(sizeof(uint16_t) * (size_t)rows * r.D);
+  w.partials = w.da_lo + align256(sizeof(uint16_t) * (size_t)rows * r.D);
   w.total = align256(w.partials + sizeof(float) * 6 * (size_t)r.D * kGateBwdBlocks);
   return w;
 }
@@ -164,7 +174,8 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
   const MetaView m = meta_view(const_cast<void*>(d_meta), L);
   char* ws = static_cast<char*>(d_ws);
-  __nv_bfloat16* da = reinterpret_cast<__nv_bfloat16*>(ws + w.da);
+  __nv_bfloat16* da_hi = reinterpret_cast<__nv_bfloat16*>(ws + w.da_hi);
+  __nv_bfloat16* da_lo = reinterpret_cast<__nv_bfloat16*>(ws + w.da_lo);
   float* partials = reinterpret_cast<float*>(ws + w.partials);
   cudaError_t e = cudaSuccess;
   if (rows > 0) {
@@ -173,13 +184,14 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   }
   e = launch_gate_bwd(m, target, rows, r.D, r.eps, d_a, d_stats,
                       reinterpret_cast<const __nv_bfloat16*>(d_u),
-                      reinterpret_cast<const __nv_bfloat16*>(d_dy), d_gamma, d_beta, d_du, da,
-                      partials, kGateBwdBlocks, d_dgamma, d_dbeta, st);
+                      reinterpret_cast<const __nv_bfloat16*>(d_dy), d_gamma, d_beta, d_du, da_hi,
+                      da_lo, partials, kGateBwdBlocks, d_dgamma, d_dbeta, st);
   if (e != cudaSuccess) return MTFM_ERR_CUDA;
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
   e = launch_attn_bwd_mma(shape, m, L.max_items_full, reinterpret_cast<const __nv_bfloat16*>(d_q),
                           reinterpret_cast<const __nv_bfloat16*>(d_k),
-                          reinterpret_cast<const __nv_bfloat16*>(d_v), da, d_dq, d_dk, d_dv, st);
+                          reinterpret_cast<const __nv_bfloat16*>(d_v), da_hi, da_lo, d_dq, d_dk,
+                          d_dv, st);
   return cuda_status(e);
 }
 

@@ -14,6 +14,8 @@
 // Backward: one CTA = one 64-key block of one user x one KV group; loops over
 // the r query heads of the group and every query tile that can see the block;
 // dK/dV accumulate in registers, dQ is added with fp32 atomics.
+// Operands formed from fp32 intermediates (P, dS, dA) enter the bf16 MMAs as
+// hi + lo pairs, which keeps the products accurate to ~16 bits.
 #include "mtfm_internal.cuh"
 #include "mma_util.cuh"
 
@@ -198,7 +200,8 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
     }
     // P = mask * SiLU(alpha S), packed to bf16 A fragments
     const bool full = (blk < nb_pre) && (j0 + kBN <= it.kv_min);
-    uint32_t pa[4][4];
+    // P = P_hi + P_lo (two bf16 parts): the PV product keeps ~16 bits of P.
+    uint32_t pa[4][4], pl[4][4];
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const int jc = j0 + n * 8 + 2 * (lane & 3);
@@ -212,10 +215,10 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
         if (!mb.visible(jc)) x2 = 0.f;
         if (!mb.visible(jc + 1)) x3 = 0.f;
       }
-      pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(x0, x1);
-      pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(x2, x3);
+      split_bf16x2(x0, x1, pa[n >> 1][(n & 1) * 2 + 0], pl[n >> 1][(n & 1) * 2 + 0]);
+      split_bf16x2(x2, x3, pa[n >> 1][(n & 1) * 2 + 1], pl[n >> 1][(n & 1) * 2 + 1]);
     }
-    // O += P V
+    // O += (P_hi + P_lo) V
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
@@ -227,6 +230,8 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
         ldsm_x4_t(smem_u32(cV + key * S::kStride + col), b0, b1, b2, b3);
         mma_bf16(o[2 * dp], pa[kk], b0, b1);
         mma_bf16(o[2 * dp + 1], pa[kk], b2, b3);
+        mma_bf16(o[2 * dp], pl[kk], b0, b1);
+        mma_bf16(o[2 * dp + 1], pl[kk], b2, b3);
       }
     }
     __syncthreads();
@@ -255,8 +260,9 @@ struct BwdArgs {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
-  const __nv_bfloat16* da;  // bf16 gradient of A (from the gate backward)
-  float* dq;                // fp32, zeroed before the launch; atomically accumulated
+  const __nv_bfloat16* da_hi;  // gradient of A from the gate backward, dA = da_hi + da_lo (bf16 parts)
+  const __nv_bfloat16* da_lo;
+  float* dq;                   // fp32, zeroed before the launch; atomically accumulated
   float* dk;
   float* dv;
   int hq, hkv, v2;
@@ -272,10 +278,13 @@ struct BwdSmem {
   static constexpr int kStride = DH + 8;
   static constexpr int kDSStride = kBwdQ + 8;
   static constexpr int kTile = 64 * kStride;
+  static constexpr int kDS = kBwdKeys * kDSStride;
   static constexpr size_t kBytes =
-      sizeof(__nv_bfloat16) * (size_t)(4 * kTile + kBwdKeys * kDSStride) + sizeof(int) * 3 * kBwdQ;
+      sizeof(__nv_bfloat16) * (size_t)(5 * kTile + 2 * kDS) + sizeof(int) * 3 * kBwdQ;
 };
 
+// Every bf16 operand built from an fp32 intermediate (P, dS, dA) is split into
+// hi + lo bf16 parts and multiplied twice, so the products keep ~16 bits.
 template <int DH>
 __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
   using S = BwdSmem<DH>;
@@ -283,9 +292,11 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   __nv_bfloat16* sV = sK + S::kTile;
   __nv_bfloat16* sQ = sV + S::kTile;
-  __nv_bfloat16* sA = sQ + S::kTile;  // dA tile
-  __nv_bfloat16* sDS = sA + S::kTile; // [keys][queries] dS^T
-  int* sKv = reinterpret_cast<int*>(sDS + kBwdKeys * S::kDSStride);
+  __nv_bfloat16* sAh = sQ + S::kTile;   // dA hi tile [query][dh]
+  __nv_bfloat16* sAl = sAh + S::kTile;  // dA lo tile
+  __nv_bfloat16* sDh = sAl + S::kTile;  // dS^T hi [keys][queries]
+  __nv_bfloat16* sDl = sDh + S::kDS;    // dS^T lo
+  int* sKv = reinterpret_cast<int*>(sDl + S::kDS);
   int* sLo = sKv + kBwdQ;
   int* sHi = sLo + kBwdQ;
 
@@ -344,24 +355,24 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
 
   const float alpha = p.alpha;
   const float inv_n = 1.f / (float)max(ui.N, 1);
-  const float cP = inv_n;           // P = SiLU(x) / N
   const float cD = alpha * inv_n;   // dS = dP * SiLU'(x) * alpha / N
 
-  // keys owned by this thread in S^T rows: ka = warp*16 + lane/4, kb = ka + 8
+  // keys owned by this thread in S^T rows: ka = j0 + warp*16 + lane/4, kb = ka + 8
   const int ka = j0 + warp * 16 + (lane >> 2), kb2 = ka + 8;
 
   for (int hh = 0; hh < r; ++hh) {
     const int h = g * r + hh;
     for (int qt = (qi_lo / kBwdQ) * kBwdQ; qt < qi_hi; qt += kBwdQ) {
-      // load Q and dA tiles (head h) + per-query masks
-      for (int c = tid; c < 2 * kBwdQ * kChunks; c += 128) {
+      // load Q and dA (hi, lo) tiles of head h + per-query masks
+      for (int c = tid; c < 3 * kBwdQ * kChunks; c += 128) {
         const int which = c / (kBwdQ * kChunks);
         const int rem = c % (kBwdQ * kChunks);
         const int rr = rem / kChunks, cc = rem % kChunks;
         const int qi = qt + rr;
         const bool ok = qi < nq;
-        const __nv_bfloat16* base = which ? p.da : p.q;
-        cp_async16(smem_u32((which ? sA : sQ) + rr * S::kStride + cc * 8),
+        const __nv_bfloat16* base = which == 0 ? p.q : (which == 1 ? p.da_hi : p.da_lo);
+        __nv_bfloat16* dst = which == 0 ? sQ : (which == 1 ? sAh : sAl);
+        cp_async16(smem_u32(dst + rr * S::kStride + cc * 8),
                    base + (size_t)(qrow0 + (ok ? qi : 0)) * ldq + h * DH + cc * 8, ok ? 16 : 0);
       }
       cp_async_commit();
@@ -375,7 +386,7 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
       cp_async_wait<0>();
       __syncthreads();
 
-      // S^T = K Q^T and dP^T = V dA^T  (16 keys x 64 queries per warp)
+      // S^T = K Q^T and dP^T = V (dA_hi + dA_lo)^T  (16 keys x 64 queries per warp)
       float st[8][4], dpt[8][4];
 #pragma unroll
       for (int n = 0; n < 8; ++n)
@@ -396,75 +407,89 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
           ldsm_x4(smem_u32(sQ + qq * S::kStride + cq), b0, b1, b2, b3);
           mma_bf16(st[2 * np], ak, b0, b1);
           mma_bf16(st[2 * np + 1], ak, b2, b3);
-          ldsm_x4(smem_u32(sA + qq * S::kStride + cq), b0, b1, b2, b3);
+          ldsm_x4(smem_u32(sAh + qq * S::kStride + cq), b0, b1, b2, b3);
+          mma_bf16(dpt[2 * np], av, b0, b1);
+          mma_bf16(dpt[2 * np + 1], av, b2, b3);
+          ldsm_x4(smem_u32(sAl + qq * S::kStride + cq), b0, b1, b2, b3);
           mma_bf16(dpt[2 * np], av, b0, b1);
           mma_bf16(dpt[2 * np + 1], av, b2, b3);
         }
       }
-      // P^T and dS^T
-      uint32_t pt[4][4], dst[4][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        float pv[4], dv4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = (e < 2) ? ka : kb2;
-          const int ql = n * 8 + 2 * (lane & 3) + (e & 1);
-          const bool vis = key < ui.N && (key < sKv[ql] || (key >= sLo[ql] && key < sHi[ql]));
-          const float x = alpha * st[n][e];
-          const float sg = sigmoid_fast(x);
-          pv[e] = vis ? x * sg * cP : 0.f;
-          dv4[e] = vis ? dpt[n][e] * sg * fmaf(x, 1.f - sg, 1.f) * cD : 0.f;
-        }
-        pt[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
-        pt[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-        dst[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(dv4[0], dv4[1]);
-        dst[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(dv4[2], dv4[3]);
-        // stash dS^T (keys x queries) for the dQ product
-        const int ql = n * 8 + 2 * (lane & 3);
-        const int kr = warp * 16 + (lane >> 2);
-        *reinterpret_cast<uint32_t*>(sDS + kr * S::kDSStride + ql) = dst[n >> 1][(n & 1) * 2 + 0];
-        *reinterpret_cast<uint32_t*>(sDS + (kr + 8) * S::kDSStride + ql) =
-            dst[n >> 1][(n & 1) * 2 + 1];
-      }
-      // dV += P^T dA ; dK += dS^T Q   (B operands [query][dh] row-major -> trans loads)
+      // Per 16-query step: P^T, dS^T (hi/lo), then dV += P^T dA and dK += dS^T Q.
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
+        uint32_t ph[4], pl[4], dh_[4], dl_[4];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int n = 2 * kk + half;
+          float pv[4], ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = (e < 2) ? ka : kb2;
+            const int ql = n * 8 + 2 * (lane & 3) + (e & 1);
+            const bool vis = key < ui.N && (key < sKv[ql] || (key >= sLo[ql] && key < sHi[ql]));
+            const float x = alpha * st[n][e];
+            const float sg = sigmoid_fast(x);
+            pv[e] = vis ? x * sg * inv_n : 0.f;
+            ds[e] = vis ? dpt[n][e] * sg * fmaf(x, 1.f - sg, 1.f) * cD : 0.f;
+          }
+          split_bf16x2(pv[0], pv[1], ph[half * 2 + 0], pl[half * 2 + 0]);
+          split_bf16x2(pv[2], pv[3], ph[half * 2 + 1], pl[half * 2 + 1]);
+          split_bf16x2(ds[0], ds[1], dh_[half * 2 + 0], dl_[half * 2 + 0]);
+          split_bf16x2(ds[2], ds[3], dh_[half * 2 + 1], dl_[half * 2 + 1]);
+          // stash dS^T (keys x queries) for the dQ product
+          const int ql = n * 8 + 2 * (lane & 3);
+          const int kr = warp * 16 + (lane >> 2);
+          *reinterpret_cast<uint32_t*>(sDh + kr * S::kDSStride + ql) = dh_[half * 2 + 0];
+          *reinterpret_cast<uint32_t*>(sDh + (kr + 8) * S::kDSStride + ql) = dh_[half * 2 + 1];
+          *reinterpret_cast<uint32_t*>(sDl + kr * S::kDSStride + ql) = dl_[half * 2 + 0];
+          *reinterpret_cast<uint32_t*>(sDl + (kr + 8) * S::kDSStride + ql) = dl_[half * 2 + 1];
+        }
 #pragma unroll
         for (int dp = 0; dp < DH / 16; ++dp) {
           uint32_t b0, b1, b2, b3;
           const int mi = lane >> 3;
           const int qq = kk * 16 + (lane & 7) + (mi & 1) * 8;
           const int col = dp * 16 + (mi >> 1) * 8;
-          ldsm_x4_t(smem_u32(sA + qq * S::kStride + col), b0, b1, b2, b3);
-          mma_bf16(dv[2 * dp], pt[kk], b0, b1);
-          mma_bf16(dv[2 * dp + 1], pt[kk], b2, b3);
+          ldsm_x4_t(smem_u32(sAh + qq * S::kStride + col), b0, b1, b2, b3);
+          mma_bf16(dv[2 * dp], ph, b0, b1);
+          mma_bf16(dv[2 * dp + 1], ph, b2, b3);
+          mma_bf16(dv[2 * dp], pl, b0, b1);
+          mma_bf16(dv[2 * dp + 1], pl, b2, b3);
+          ldsm_x4_t(smem_u32(sAl + qq * S::kStride + col), b0, b1, b2, b3);
+          mma_bf16(dv[2 * dp], ph, b0, b1);
+          mma_bf16(dv[2 * dp + 1], ph, b2, b3);
           ldsm_x4_t(smem_u32(sQ + qq * S::kStride + col), b0, b1, b2, b3);
-          mma_bf16(dk[2 * dp], dst[kk], b0, b1);
-          mma_bf16(dk[2 * dp + 1], dst[kk], b2, b3);
+          mma_bf16(dk[2 * dp], dh_, b0, b1);
+          mma_bf16(dk[2 * dp + 1], dh_, b2, b3);
+          mma_bf16(dk[2 * dp], dl_, b0, b1);
+          mma_bf16(dk[2 * dp + 1], dl_, b2, b3);
         }
       }
       __syncthreads();
-      // dQ[16 queries of this warp] += dS (queries x keys) K  -> fp32 atomics
+      // dQ[16 queries of this warp] += (dS_hi + dS_lo) K  -> fp32 atomics
       {
         float dq[DH / 8][4];
 #pragma unroll
         for (int i = 0; i < DH / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < kBwdKeys / 16; ++kk) {
-          uint32_t a[4];
+          uint32_t ah[4], al[4];
           const int mi = lane >> 3;
           const int key = kk * 16 + (lane & 7) + (mi >> 1) * 8;
           const int qq = warp * 16 + (mi & 1) * 8;
-          ldsm_x4_t(smem_u32(sDS + key * S::kDSStride + qq), a[0], a[1], a[2], a[3]);
+          ldsm_x4_t(smem_u32(sDh + key * S::kDSStride + qq), ah[0], ah[1], ah[2], ah[3]);
+          ldsm_x4_t(smem_u32(sDl + key * S::kDSStride + qq), al[0], al[1], al[2], al[3]);
 #pragma unroll
           for (int dp = 0; dp < DH / 16; ++dp) {
             uint32_t b0, b1, b2, b3;
             const int key2 = kk * 16 + (lane & 7) + (mi & 1) * 8;
             const int col = dp * 16 + (mi >> 1) * 8;
             ldsm_x4_t(smem_u32(sK + key2 * S::kStride + col), b0, b1, b2, b3);
-            mma_bf16(dq[2 * dp], a, b0, b1);
-            mma_bf16(dq[2 * dp + 1], a, b2, b3);
+            mma_bf16(dq[2 * dp], ah, b0, b1);
+            mma_bf16(dq[2 * dp + 1], ah, b2, b3);
+            mma_bf16(dq[2 * dp], al, b0, b1);
+            mma_bf16(dq[2 * dp + 1], al, b2, b3);
           }
         }
         const int qa_ = qt + warp * 16 + (lane >> 2), qb_ = qa_ + 8;
@@ -543,10 +568,11 @@ cudaError_t launch_attn_fwd_mma(const AttnShape& s, const MetaView& m, int max_i
 
 cudaError_t launch_attn_bwd_mma(const AttnShape& s, const MetaView& m, int max_items_full,
                                 const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                const __nv_bfloat16* v, const __nv_bfloat16* da, float* dq,
-                                float* dk, float* dv, cudaStream_t st) {
+                                const __nv_bfloat16* v, const __nv_bfloat16* da_hi,
+                                const __nv_bfloat16* da_lo, float* dq, float* dk, float* dv,
+                                cudaStream_t st) {
   if (max_items_full <= 0) return cudaSuccess;
-  BwdArgs args{m, q, k, v, da, dq, dk, dv, s.hq, s.hkv, s.v2, s.alpha, s.target};
+  BwdArgs args{m, q, k, v, da_hi, da_lo, dq, dk, dv, s.hq, s.hkv, s.v2, s.alpha, s.target};
   switch (s.dh) {
     case 32: return bwd_dispatch<32>(args, max_items_full, st);
     case 64: return bwd_dispatch<64>(args, max_items_full, st);

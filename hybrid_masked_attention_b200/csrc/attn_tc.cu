@@ -1,0 +1,392 @@
+// sm_100a forward kernel of the masked SiLU attention: tcgen05 MMAs with TMEM
+// accumulators, operands staged by TMA (128-byte swizzle), K/V blocks shared
+// by the r query heads of one GQA group.
+//
+// Computes, per query row i of a 128-row tile of user u and head h of KV group g
+// (page "美团推荐大模型 MTFM 深度硬核解析", §4.1 attention equation and §4.2
+// Target Attention; visibility from the Meituan tech blog §3.2):
+//     A[i, h] = (1/N_u) sum_{j visible from i} SiLU(alpha q[i,h].k[j,g]) v[j,g]
+// with "visible" = the row's key prefix [0, kv_end) plus, for T rows, the
+// sibling block (itself, or the 4 sub-tokens of its target in V2).
+//
+// One CTA = one work item (user, 128-row query tile) x one KV group:
+//   warp 0      : TMA producer (Q tiles of the r heads once, then K/V blocks of
+//                 128 keys through a 3-stage ring);
+//   warp 1      : TMEM allocation and the single MMA-issuing thread;
+//   warps 4..11 : two "SiLU" warpgroups.  Warpgroup b owns S buffer b: it reads
+//                 S = Q K^T (fp32) from TMEM, applies mask + SiLU, writes P as
+//                 two bf16 parts P_hi + P_lo (~16 significant bits) back into
+//                 the same TMEM columns, and signals the MMA thread, which
+//                 issues O_h += P_hi V + P_lo V with P read from TMEM.
+// TMEM (512 columns): O_h at columns [64h, 64h+64) for h < r (<= 4), S buffer b
+// at [256 + 128b, 384 + 128b).  The MMA thread keeps one score block in flight
+// ahead: S(n+1) is issued before O += P(n) V, so the tensor pipe works while a
+// warpgroup runs the SiLU of the other buffer.
+// Key blocks above the tile's largest kv_end are never loaded; blocks entirely
+// below its smallest kv_end skip the per-element mask test.
+//
+// Every wait is bounded (about one second); a wait that gives up raises a
+// CTA-wide abort flag, every role drains its in-flight copies/MMAs with a
+// bounded wait, TMEM is freed, and MetaHeader::error gets the timeout bit.
+#include <cuda.h>
+
+#include "mtfm_internal.cuh"
+#include "mma_util.cuh"
+#include "sm100.cuh"
+
+namespace mtfm {
+namespace {
+
+using namespace sm100;
+
+constexpr int kDH = 64;
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kStages = 3;
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = kBM * kDH * 2;  // 16 KB: one 128 x 64 bf16 tile
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCol0 = 256;  // first column of S buffer 0
+
+struct TcArgs {
+  MetaView m;
+  float* a;
+  int hq, hkv, v2;
+  float alpha;
+};
+
+template <int R>
+constexpr size_t tc_smem_bytes() {
+  return (size_t)(R + 2 * kStages) * kTileBytes + 1024;
+}
+
+template <int R, bool TARGET>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, TcArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_q, bar_o, bar_drain;
+  __shared__ __align__(8) uint64_t bar_kv_full[kStages], bar_kv_empty[kStages];
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const MetaView& m = p.m;
+  MetaHeader* hdr = m.hdr;
+  if (hdr->error) return;
+  const int n_items = TARGET ? hdr->n_items_target : hdr->n_items_full;
+  if ((int)blockIdx.x >= n_items) return;
+  const WorkItem it = (TARGET ? m.items_target : m.items_full)[blockIdx.x];
+  const int u = it.user;
+  const int LH = m.lh[u], LR = m.lr[u], LT = m.lt[u];
+  const int N = LH + LR + LT, so = m.seq_off[u];
+  const int nq = TARGET ? LT : N;
+  const int q0 = it.tile * kBM;
+  const int qrow0 = TARGET ? m.t_off[u] : so;
+  const int pos0 = TARGET ? LH + LR : 0;
+  const int g = blockIdx.y;
+  const int ldq = p.hq * kDH;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // key blocks: prefix [0, kv_max) then the sibling span of the tile's T rows
+  const int t0pos = LH + LR;
+  const int nb_pre = (it.kv_max + kBN - 1) / kBN;
+  int sb_lo = 0, sb_hi = 0;
+  {
+    const int first = max(pos0 + q0, t0pos);
+    const int last = pos0 + min(q0 + kBM, nq) - 1;
+    if (first <= last) {
+      const int lo = t0pos + ((first - t0pos) / p.v2) * p.v2;
+      const int hi = t0pos + ((last - t0pos) / p.v2 + 1) * p.v2;
+      sb_lo = max(lo / kBN, nb_pre);
+      sb_hi = (hi + kBN - 1) / kBN;
+    }
+  }
+  const int n_blocks = nb_pre + max(0, sb_hi - sb_lo);
+  const int total = n_blocks * R;  // (key block, head) steps
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_addr(smem);
+  const uint32_t sK = sQ + R * kTileBytes;
+  const uint32_t sV = sK + kStages * kTileBytes;
+
+  const uint32_t b_q = smem_addr(&bar_q), b_o = smem_addr(&bar_o), b_drain = smem_addr(&bar_drain);
+  auto b_kvf = [&](int s) { return smem_addr(&bar_kv_full[s]); };
+  auto b_kve = [&](int s) { return smem_addr(&bar_kv_empty[s]); };
+  auto b_sf = [&](int b) { return smem_addr(&bar_s_full[b]); };
+  auto b_pf = [&](int b) { return smem_addr(&bar_p_full[b]); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q, 1);
+    mbar_init(b_o, 1);
+    mbar_init(b_drain, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(b_kvf(s), 1);
+      mbar_init(b_kve(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(b_sf(b), 1);
+      mbar_init(b_pf(b), 128);
+    }
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&s_tmem), kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+
+  auto block_of = [&](int bi) { return bi < nb_pre ? bi : sb_lo + (bi - nb_pre); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(b_q, R * kTileBytes);
+      for (int hh = 0; hh < R; ++hh)
+        tma_load_2d(sQ + hh * kTileBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
+      int issued = 0;
+      for (int bi = 0; bi < n_blocks; ++bi) {
+        const int s = bi % kStages;
+        if (bi >= kStages && !mbar_wait(b_kve(s), ((bi / kStages) - 1) & 1, abort_flag)) break;
+        const int row = so + block_of(bi) * kBN;
+        mbar_expect_tx(b_kvf(s), 2 * kTileBytes);
+        tma_load_2d(sK + s * kTileBytes, &tm_k, b_kvf(s), g * kDH, row);
+        tma_load_2d(sV + s * kTileBytes, &tm_v, b_kvf(s), g * kDH, row);
+        ++issued;
+      }
+      // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
+      // no TMA write may land after this CTA leaves.
+      const long long t0 = clock64();
+      auto drain_wait = [&](uint32_t bar, uint32_t par) {
+        while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
+        }
+      };
+      drain_wait(b_q, 0);
+      for (int bi = max(0, issued - kStages); bi < issued; ++bi)
+        drain_wait(b_kvf(bi % kStages), (bi / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDH, true);
+      bool ok = mbar_wait(b_q, 0, abort_flag);
+      auto issue_s = [&](int n) -> bool {
+        const int bi = n / R, hh = n % R, s = bi % kStages;
+        if (hh == 0 && !mbar_wait(b_kvf(s), (bi / kStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + kSCol0 + (n & 1) * kBN;
+#pragma unroll
+        for (int kk = 0; kk < kDH / 16; ++kk) {
+          const uint64_t ad = sw128_desc(sQ + hh * kTileBytes + kk * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(sK + s * kTileBytes + kk * 32, 16, 1024);
+          mma_ss(d, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(b_sf(n & 1));
+        return true;
+      };
+      if (ok && total > 0) ok = issue_s(0);
+      for (int n = 0; ok && n < total; ++n) {
+        if (n + 1 < total && !issue_s(n + 1)) {
+          ok = false;
+          break;
+        }
+        const int b = n & 1;
+        if (!mbar_wait(b_pf(b), (n >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int bi = n / R, hh = n % R, s = bi % kStages;
+        const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo, bf16 pairs
+        const uint32_t o = tmem + hh * kDH;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = sw128_desc(sV + s * kTileBytes + kk * 2048, 16, 1024);
+          const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
+          mma_ts(o, pt + col, bd, idesc_pv, (bi > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(o, pt + col + 16, bd, idesc_pv, 1u);
+        }
+        if (hh == R - 1) mma_commit(b_kve(s));
+      }
+      if (ok) {
+        mma_commit(b_o);
+      } else {
+        // drain every MMA issued so far before TMEM is released
+        mma_commit(b_drain);
+        const long long t0 = clock64();
+        while (!mbar_try(b_drain, 0) && clock64() - t0 < kWaitCycles) {
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- SiLU warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int qi = q0 + row;
+    const bool valid = qi < nq;
+    int kv_end = 0, sib_lo = 0, sib_hi = 0;
+    if (valid) {
+      const int pos = pos0 + qi;
+      kv_end = m.kv_end[so + pos];
+      if (pos >= t0pos) {
+        sib_lo = t0pos + ((pos - t0pos) / p.v2) * p.v2;
+        sib_hi = sib_lo + p.v2;
+      }
+    }
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const float alpha = p.alpha;
+    bool ok = true;
+    for (int n = wg; n < total; n += 2) {
+      ok = __all_sync(0xffffffffu, mbar_wait(b_sf(wg), (n >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int bi = n / R;
+      const int j0 = block_of(bi) * kBN;
+      const bool full = (bi < nb_pre) && (j0 + kBN <= it.kv_min);
+      const uint32_t sb = lane_base + kSCol0 + wg * kBN;
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(sb + c * 32, raw);
+        tmem_ld_wait();
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float x0 = silu_fast(alpha * __uint_as_float(raw[2 * e]));
+          float x1 = silu_fast(alpha * __uint_as_float(raw[2 * e + 1]));
+          if (!full) {
+            const int key = j0 + c * 32 + 2 * e;
+            if (!(key < kv_end || (key >= sib_lo && key < sib_hi))) x0 = 0.f;
+            if (!(key + 1 < kv_end || (key + 1 >= sib_lo && key + 1 < sib_hi))) x1 = 0.f;
+          }
+          split_bf16x2(x0, x1, ph[e], pl[e]);
+        }
+        // keys [32c, 32c+32): P_hi in columns [32c, 32c+16), P_lo in [32c+16, 32c+32),
+        // i.e. over the S columns of this chunk, which were read above.
+        tmem_st16(sb + c * 32, ph);
+        tmem_st16(sb + c * 32 + 16, pl);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(b_pf(wg));
+    }
+    // ------------------------------------------------------------- epilogue: A = O / N_u
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, 0, abort_flag));
+    if (ok && total == 0) {
+      // no visible key at all (cannot happen for a non-empty tile): A = 0
+      for (int hh = wg; hh < R && valid; hh += 2)
+        for (int c = 0; c < kDH; c += 4)
+          *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+    } else if (ok) {
+      tc_fence_after();
+      const float inv_n = 1.f / (float)N;
+      for (int hh = wg; hh < R; hh += 2) {
+#pragma unroll
+        for (int c = 0; c < kDH / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(lane_base + hh * kDH + c * 32, raw);
+          tmem_ld_wait();
+          if (valid) {
+            float* dst = p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c * 32;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              reinterpret_cast<float4*>(dst)[e] =
+                  make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
+                              __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && s_abort) atomicOr(&hdr->error, kErrTimeout);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols]; 128 x 64 boxes with the 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kDH, (cuuint32_t)kBM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R, bool TARGET>
+cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const TcArgs& a, int max_items, cudaStream_t st) {
+  const size_t smem = tc_smem_bytes<R>();
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R, TARGET>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(max_items, a.hkv);
+  attn_fwd_tc_kernel<R, TARGET><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_fwd_tc_supported(const AttnShape& s) {
+  const int r = s.hq / s.hkv;
+  return s.dh == kDH && (r == 1 || r == 2 || r == 4);
+}
+
+cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
+                               int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                               const __nv_bfloat16* v, float* a, cudaStream_t st) {
+  if (max_items <= 0 || rows_q <= 0 || total_tokens <= 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, rows_q, s.hq * kDH) || !make_map(&mk, k, total_tokens, s.hkv * kDH) ||
+      !make_map(&mv, v, total_tokens, s.hkv * kDH))
+    return cudaErrorInvalidValue;
+  TcArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha};
+  const int r = s.hq / s.hkv;
+  if (s.target) {
+    if (r == 1) return tc_launch<1, true>(mq, mk, mv, args, max_items, st);
+    if (r == 2) return tc_launch<2, true>(mq, mk, mv, args, max_items, st);
+    return tc_launch<4, true>(mq, mk, mv, args, max_items, st);
+  }
+  if (r == 1) return tc_launch<1, false>(mq, mk, mv, args, max_items, st);
+  if (r == 2) return tc_launch<2, false>(mq, mk, mv, args, max_items, st);
+  return tc_launch<4, false>(mq, mk, mv, args, max_items, st);
+}
+
+}  // namespace mtfm

@@ -28,13 +28,20 @@ __device__ __forceinline__ float4 load_bf16x4(const __nv_bfloat16* p) {
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
-__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, float4 v) {
-  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
-  uint2 raw;
-  raw.x = *reinterpret_cast<uint32_t*>(&lo);
-  raw.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(p) = raw;
+// Stores v as two bf16 parts, hi = bf16(v) and lo = bf16(v - hi).
+__device__ __forceinline__ void store_split_bf16x4(__nv_bfloat16* hi_p, __nv_bfloat16* lo_p, float4 v) {
+  __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 h1 = __floats2bfloat162_rn(v.z, v.w);
+  const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+  __nv_bfloat162 l0 = __floats2bfloat162_rn(v.x - f0.x, v.y - f0.y);
+  __nv_bfloat162 l1 = __floats2bfloat162_rn(v.z - f1.x, v.w - f1.y);
+  uint2 rh, rl;
+  rh.x = *reinterpret_cast<uint32_t*>(&h0);
+  rh.y = *reinterpret_cast<uint32_t*>(&h1);
+  rl.x = *reinterpret_cast<uint32_t*>(&l0);
+  rl.y = *reinterpret_cast<uint32_t*>(&l1);
+  *reinterpret_cast<uint2*>(hi_p) = rh;
+  *reinterpret_cast<uint2*>(lo_p) = rl;
 }
 
 __global__ void __launch_bounds__(256)
@@ -105,15 +112,16 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
   if (lane == 0) *reinterpret_cast<float2*>(stats + 2 * (size_t)row) = make_float2(mean, rstd);
 }
 
-// Backward of the gate.  dU = GLN(A) (*) dY; dA (bf16, the attention backward's
-// MMA operand) through the LayerNorm; per-block partial dgamma/dbeta sums.
+// Backward of the gate.  dU = GLN(A) (*) dY; dA through the LayerNorm, stored as
+// bf16 hi + lo parts (the attention backward's MMA operands); per-block partial
+// dgamma/dbeta sums.
 __global__ void __launch_bounds__(256)
 gate_bwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, bool target, int rows,
                 int D, const float* __restrict__ a, const float* __restrict__ stats,
                 const __nv_bfloat16* __restrict__ u, const __nv_bfloat16* __restrict__ dy,
                 const float* __restrict__ gamma, const float* __restrict__ beta,
-                float* __restrict__ du, __nv_bfloat16* __restrict__ da,
-                float* __restrict__ partials) {
+                float* __restrict__ du, __nv_bfloat16* __restrict__ da_hi,
+                __nv_bfloat16* __restrict__ da_lo, float* __restrict__ partials) {
   extern __shared__ float s_acc[];  // [2][3][D] (dgamma, dbeta) when gamma != NULL
   if (hdr->error) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,14 +136,16 @@ gate_bwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
     const __nv_bfloat16* ur = u + (size_t)row * D;
     const __nv_bfloat16* dyr = dy + (size_t)row * D;
     float* dur = du + (size_t)row * D;
-    __nv_bfloat16* dar = da + (size_t)row * D;
+    __nv_bfloat16* dhr = da_hi + (size_t)row * D;
+    __nv_bfloat16* dlr = da_lo + (size_t)row * D;
     if (!gln) {
       for (int c = lane; c < nch; c += 32) {
         const float4 x = *reinterpret_cast<const float4*>(ar + 4 * c);
         const float4 uu = load_bf16x4(ur + 4 * c);
         const float4 g = load_bf16x4(dyr + 4 * c);
         *reinterpret_cast<float4*>(dur + 4 * c) = make_float4(g.x * x.x, g.y * x.y, g.z * x.z, g.w * x.w);
-        store_bf16x4(dar + 4 * c, make_float4(g.x * uu.x, g.y * uu.y, g.z * uu.z, g.w * uu.w));
+        store_split_bf16x4(dhr + 4 * c, dlr + 4 * c,
+                           make_float4(g.x * uu.x, g.y * uu.y, g.z * uu.z, g.w * uu.w));
       }
       continue;
     }
@@ -187,7 +197,7 @@ gate_bwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
         o.y = rstd * (dz[i].y - m1 - z[i].y * m2);
         o.z = rstd * (dz[i].z - m1 - z[i].z * m2);
         o.w = rstd * (dz[i].w - m1 - z[i].w * m2);
-        store_bf16x4(dar + 4 * c, o);
+        store_split_bf16x4(dhr + 4 * c, dlr + 4 * c, o);
       }
     }
   }
@@ -224,8 +234,9 @@ cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, flo
 cudaError_t launch_gate_bwd(const MetaView& m, bool target, int rows, int D, float eps,
                             const float* a, const float* stats, const __nv_bfloat16* u,
                             const __nv_bfloat16* dy, const float* gamma, const float* beta,
-                            float* du, __nv_bfloat16* da, float* partials, int n_part_blocks,
-                            float* dgamma, float* dbeta, cudaStream_t st) {
+                            float* du, __nv_bfloat16* da_hi, __nv_bfloat16* da_lo,
+                            float* partials, int n_part_blocks, float* dgamma, float* dbeta,
+                            cudaStream_t st) {
   (void)eps;
   const bool gln = gamma != nullptr;
   const size_t smem = gln ? sizeof(float) * 6 * (size_t)D : 0;
@@ -236,7 +247,7 @@ cudaError_t launch_gate_bwd(const MetaView& m, bool target, int rows, int D, flo
   }
   if (rows > 0 || gln) {
     gate_bwd_kernel<<<n_part_blocks, 256, smem, st>>>(m.hdr, m.row_type, target, rows, D, a, stats,
-                                                      u, dy, gamma, beta, du, da, partials);
+                                                      u, dy, gamma, beta, du, da_hi, da_lo, partials);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -48,6 +48,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi): two bf16 MMAs on (hi, lo)
+// carry ~16 significant bits of x instead of 8.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 // Hardware tanh approximation (MUFU); relative error well below bf16 resolution.
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;

@@ -117,18 +117,24 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
 cudaError_t launch_attn_fwd_mma(const AttnShape& s, const MetaView& m, int max_items,
                                 const __nv_bfloat16* q, const __nv_bfloat16* k,
                                 const __nv_bfloat16* v, float* a, cudaStream_t st);
+bool attn_fwd_tc_supported(const AttnShape& s);
+cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
+                               int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                               const __nv_bfloat16* v, float* a, cudaStream_t st);
 cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, float eps,
                             const float* a, const __nv_bfloat16* u, const float* gamma,
                             const float* beta, float* y, float* stats, cudaStream_t st);
 cudaError_t launch_gate_bwd(const MetaView& m, bool target, int rows, int D, float eps,
                             const float* a, const float* stats, const __nv_bfloat16* u,
                             const __nv_bfloat16* dy, const float* gamma, const float* beta,
-                            float* du, __nv_bfloat16* da, float* partials, int n_part_blocks,
+                            float* du, __nv_bfloat16* da_hi, __nv_bfloat16* da_lo,
+                            float* partials, int n_part_blocks,
                             float* dgamma, float* dbeta, cudaStream_t st);
 cudaError_t launch_attn_bwd_mma(const AttnShape& s, const MetaView& m, int max_items_full,
                                 const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                const __nv_bfloat16* v, const __nv_bfloat16* da, float* dq,
-                                float* dk, float* dv, cudaStream_t st);
+                                const __nv_bfloat16* v, const __nv_bfloat16* da_hi,
+                                const __nv_bfloat16* da_lo, float* dq, float* dk, float* dv,
+                                cudaStream_t st);
 
 constexpr int kGateBwdBlocks = 296;  // 2 per SM on a 148-SM part; partial dgamma/dbeta slots
 

@@ -45,7 +45,11 @@
  *   - Supported: head_dim in {32, 64, 128}; hq % hkv == 0; hq/hkv <= 8;
  *     hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
- *   - No exceptions cross this boundary; no global state is kept.
+ *   - No exceptions cross this boundary; no global state is kept.  The
+ *     forward attention runs the tcgen05/TMEM kernel for head_dim 64 with
+ *     hq/hkv in {1, 2, 4} and the portable mma.sync kernel otherwise; the
+ *     environment variable MTFM_FWD_KERNEL=mma selects the portable kernel for
+ *     every shape (used to compare the two).
  */
 #ifndef MTFM_H_
 #define MTFM_H_
