@@ -9,19 +9,22 @@
 // with "visible" = the row's key prefix [0, kv_end) plus, for T rows, the
 // sibling block (itself, or the 4 sub-tokens of its target in V2).
 //
-// One CTA = one work item (user, 128-row query tile) x one KV group:
+// One CTA = one work item (user, 128-row query tile) x one KV group; a step is
+// one (128-key block, query head) pair:
 //   warp 0      : TMA producer (Q tiles of the r heads once, then K/V blocks of
 //                 128 keys through a 3-stage ring);
-//   warp 1      : TMEM allocation and the single MMA-issuing thread;
-//   warps 4..11 : two "SiLU" warpgroups.  Warpgroup b owns S buffer b: it reads
-//                 S = Q K^T (fp32) from TMEM, applies mask + SiLU, writes P as
-//                 two bf16 parts P_hi + P_lo (~16 significant bits) back into
-//                 the same TMEM columns, and signals the MMA thread, which
-//                 issues O_h += P_hi V + P_lo V with P read from TMEM.
-// TMEM (512 columns): O_h at columns [64h, 64h+64) for h < r (<= 4), S buffer b
-// at [256 + 128b, 384 + 128b).  The MMA thread keeps one score block in flight
-// ahead: S(n+1) is issued before O += P(n) V, so the tensor pipe works while a
-// warpgroup runs the SiLU of the other buffer.
+//   warp 1      : TMEM allocation and the MMA issue (whole warp runs the
+//                 control flow, one elected lane issues);
+//   warps 4..19 : four "SiLU" warpgroups that share every step, each on 32 of
+//                 its 128 key columns: read S = Q K^T (fp32) from TMEM, apply
+//                 mask + SiLU, write P as two bf16 parts P_hi + P_lo (~16
+//                 significant bits) back into the same TMEM columns, and signal
+//                 the MMA warp, which issues O_h += P_hi V + P_lo V with P read
+//                 from TMEM.
+// TMEM (512 columns): O_h at columns [64h, 64h+64) for h < r (<= 4), S buffers
+// b = 0, 1 at [256 + 128b, 384 + 128b).  While the warpgroups run the SiLU of
+// step n, the tensor pipe runs O += P(n-1) V and S(n+1) = Q K^T: the tanh
+// throughput (16 per clock per SM) and the MMA time per step are about equal.
 // Key blocks above the tile's largest kv_end are never loaded; blocks entirely
 // below its smallest kv_end skip the per-element mask test.
 //
@@ -40,13 +43,21 @@ namespace {
 using namespace sm100;
 
 constexpr int kDH = 64;
-constexpr int kBM = 128;
-constexpr int kBN = 128;
-constexpr int kStages = 3;
-constexpr int kThreads = 384;
-constexpr uint32_t kTileBytes = kBM * kDH * 2;  // 16 KB: one 128 x 64 bf16 tile
+constexpr int kBM = 128;          // query rows per tile (TMEM lanes)
+constexpr int kBN = 128;          // keys per block
+constexpr int kStages = 3;        // K/V ring depth
+constexpr int kSBuf = 2;          // S/P buffers in TMEM
+constexpr int kSiluWG = 4;        // SiLU warpgroups
+constexpr int kWGPerBuf = 4;      // warpgroups sharing one step (split by key columns)
+constexpr int kTeams = kSiluWG / kWGPerBuf;         // teams take steps n = team (mod kTeams)
+constexpr int kChunksPerWG = kBN / 32 / kWGPerBuf;  // 32-key chunks per warpgroup and step
+constexpr int kThreads = 128 + 128 * kSiluWG;
+constexpr uint32_t kQBytes = kBM * kDH * 2;   // 16 KB
+constexpr uint32_t kKVBytes = kBN * kDH * 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol0 = 256;  // first column of S buffer 0
+constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
+static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
+static_assert(kSiluWG % kWGPerBuf == 0 && kChunksPerWG >= 1 && kSBuf % kTeams == 0, "warpgroup split");
 
 struct TcArgs {
   MetaView m;
@@ -57,7 +68,27 @@ struct TcArgs {
 
 template <int R>
 constexpr size_t tc_smem_bytes() {
-  return (size_t)(R + 2 * kStages) * kTileBytes + 1024;
+  return (size_t)R * kQBytes + 2 * kStages * kKVBytes + 1024;
+}
+
+// SiLU of 32 scores of one row (one TMEM chunk), masked, split into bf16 hi/lo
+// pairs: P = SiLU(alpha s) = h + h tanh(h), h = alpha s / 2.  Scalar fp32 math:
+// the packed f32x2 forms measured slower here (extra register moves).
+template <bool MASKED>
+__device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half_alpha, uint32_t vis,
+                                           uint32_t (&ph)[16], uint32_t (&pl)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float h0 = half_alpha * __uint_as_float(raw[2 * e]);
+    const float h1 = half_alpha * __uint_as_float(raw[2 * e + 1]);
+    float p0 = fmaf(h0, tanh_approx(h0), h0);
+    float p1 = fmaf(h1, tanh_approx(h1), h1);
+    if (MASKED) {
+      p0 = (vis & (1u << (2 * e))) ? p0 : 0.f;
+      p1 = (vis & (2u << (2 * e))) ? p1 : 0.f;
+    }
+    split_trunc_bf16x2(p0, p1, ph[e], pl[e]);
+  }
 }
 
 template <int R, bool TARGET>
@@ -67,7 +98,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q, bar_o, bar_drain;
   __shared__ __align__(8) uint64_t bar_kv_full[kStages], bar_kv_empty[kStages];
-  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2];
+  __shared__ __align__(8) uint64_t bar_s_full[kSBuf], bar_p_full[kSBuf];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -103,12 +134,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   }
   const int n_blocks = nb_pre + max(0, sb_hi - sb_lo);
-  const int total = n_blocks * R;  // (key block, head) steps
+  const int total = n_blocks * R;  // steps n = (key block n / R, head n % R)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_addr(smem);
-  const uint32_t sK = sQ + R * kTileBytes;
-  const uint32_t sV = sK + kStages * kTileBytes;
+  const uint32_t sK = sQ + R * kQBytes;
+  const uint32_t sV = sK + kStages * kKVBytes;
 
   const uint32_t b_q = smem_addr(&bar_q), b_o = smem_addr(&bar_o), b_drain = smem_addr(&bar_drain);
   auto b_kvf = [&](int s) { return smem_addr(&bar_kv_full[s]); };
@@ -124,9 +155,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(b_kvf(s), 1);
       mbar_init(b_kve(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSBuf; ++b) {
       mbar_init(b_sf(b), 1);
-      mbar_init(b_pf(b), 128);
+      mbar_init(b_pf(b), 128 * kWGPerBuf);
     }
     s_abort = 0;
     fence_barrier_init();
@@ -149,17 +180,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_expect_tx(b_q, R * kTileBytes);
+      mbar_expect_tx(b_q, R * kQBytes);
       for (int hh = 0; hh < R; ++hh)
-        tma_load_2d(sQ + hh * kTileBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
+        tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
       int issued = 0;
       for (int bi = 0; bi < n_blocks; ++bi) {
         const int s = bi % kStages;
         if (bi >= kStages && !mbar_wait(b_kve(s), ((bi / kStages) - 1) & 1, abort_flag)) break;
         const int row = so + block_of(bi) * kBN;
-        mbar_expect_tx(b_kvf(s), 2 * kTileBytes);
-        tma_load_2d(sK + s * kTileBytes, &tm_k, b_kvf(s), g * kDH, row);
-        tma_load_2d(sV + s * kTileBytes, &tm_v, b_kvf(s), g * kDH, row);
+        mbar_expect_tx(b_kvf(s), 2 * kKVBytes);
+        tma_load_2d(sK + s * kKVBytes, &tm_k, b_kvf(s), g * kDH, row);
+        tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
         ++issued;
       }
       // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
@@ -175,61 +206,75 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDH, true);
-      bool ok = mbar_wait(b_q, 0, abort_flag);
-      auto issue_s = [&](int n) -> bool {
-        const int bi = n / R, hh = n % R, s = bi % kStages;
-        if (hh == 0 && !mbar_wait(b_kvf(s), (bi / kStages) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + kSCol0 + (n & 1) * kBN;
+    // Order: S(0); then for every step n: S(n+1), [P(n) ready] O_h += P(n) V.
+    // S(n+1) reuses the buffer of step n-1, whose PV was issued before it.
+    // The whole warp runs the control flow (so operands stay warp-uniform) and
+    // one elected lane issues the MMAs and commits.
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDH, true);
+    // descriptor words: the high word is shared; low words step by (bytes >> 4)
+    const uint32_t dhi = sw128_desc_hi(1024);
+    const uint32_t q_lo = sw128_desc_lo(sQ, 16), k_lo = sw128_desc_lo(sK, 16), v_lo = sw128_desc_lo(sV, 16);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(b_q, 0, abort_flag));
+    auto issue_s = [&](int n) -> bool {
+      const int bi = n / R, hh = n % R, s = bi % kStages;
+      if (hh == 0 && !__all_sync(0xffffffffu, mbar_wait(b_kvf(s), (bi / kStages) & 1, abort_flag)))
+        return false;
+      tc_fence_after();
+      const uint32_t d = tmem + kSCol0 + (n % kSBuf) * kBN;
+      const uint32_t a0 = q_lo + hh * (kQBytes >> 4), b0 = k_lo + s * (kKVBytes >> 4);
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kDH / 16; ++kk) {
-          const uint64_t ad = sw128_desc(sQ + hh * kTileBytes + kk * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(sK + s * kTileBytes + kk * 32, 16, 1024);
-          mma_ss(d, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(b_sf(n & 1));
-        return true;
-      };
-      if (ok && total > 0) ok = issue_s(0);
-      for (int n = 0; ok && n < total; ++n) {
-        if (n + 1 < total && !issue_s(n + 1)) {
-          ok = false;
-          break;
-        }
-        const int b = n & 1;
-        if (!mbar_wait(b_pf(b), (n >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int bi = n / R, hh = n % R, s = bi % kStages;
-        const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo, bf16 pairs
-        const uint32_t o = tmem + hh * kDH;
+        for (int kk = 0; kk < kDH / 16; ++kk)
+          mma_ss2(d, a0 + kk * 2, dhi, b0 + kk * 2, dhi, idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(b_sf(n % kSBuf));
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int n = 0; ok && n < min(total, kSBuf - 1); ++n) ok = issue_s(n);
+    for (int n = 0; ok && n < total; ++n) {
+      if (n + kSBuf - 1 < total && !issue_s(n + kSBuf - 1)) {
+        ok = false;
+        break;
+      }
+      const int b = n % kSBuf;
+      if (!__all_sync(0xffffffffu, mbar_wait(b_pf(b), (n / kSBuf) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int bi = n / R, hh = n % R, s = bi % kStages;
+      const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo, bf16 pairs
+      const uint32_t o = tmem + hh * kDH;
+      const uint32_t vb = v_lo + s * (kKVBytes >> 4);  // V rows (keys): 16 per k-step = 2048 B
+      const uint32_t acc0 = bi > 0 ? 1u : 0u;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = sw128_desc(sV + s * kTileBytes + kk * 2048, 16, 1024);
           const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
-          mma_ts(o, pt + col, bd, idesc_pv, (bi > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(o, pt + col + 16, bd, idesc_pv, 1u);
+          mma_ts2(o, pt + col, vb + kk * (2048 >> 4), dhi, idesc_pv, kk > 0 ? 1u : acc0);
+          mma_ts2(o, pt + col + 16, vb + kk * (2048 >> 4), dhi, idesc_pv, 1u);
         }
         if (hh == R - 1) mma_commit(b_kve(s));
       }
-      if (ok) {
-        mma_commit(b_o);
-      } else {
-        // drain every MMA issued so far before TMEM is released
-        mma_commit(b_drain);
-        const long long t0 = clock64();
-        while (!mbar_try(b_drain, 0) && clock64() - t0 < kWaitCycles) {
-        }
+      __syncwarp();
+    }
+    if (elect_one()) {
+      // on failure, drain every MMA issued so far before TMEM is released
+      mma_commit(ok ? b_o : b_drain);
+    }
+    __syncwarp();
+    if (!ok) {
+      const long long t0 = clock64();
+      while (!mbar_try(b_drain, 0) && clock64() - t0 < kWaitCycles) {
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- SiLU warpgroups
-    const int wg = (warp - 4) >> 2;
+    const int wg = (warp - 4) >> 2;   // warpgroup 0..3
+    const int team = wg % kTeams;      // steps n = team (mod kTeams)
+    const int cpart = wg / kTeams;     // part of the key columns of a step this warpgroup handles
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const int qi = q0 + row;
@@ -244,32 +289,27 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
     }
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const float alpha = p.alpha;
+    const float half_alpha = 0.5f * p.alpha;
     bool ok = true;
-    for (int n = wg; n < total; n += 2) {
-      ok = __all_sync(0xffffffffu, mbar_wait(b_sf(wg), (n >> 1) & 1, abort_flag));
+    for (int n = team; n < total; n += kTeams) {
+      const int buf = n % kSBuf;
+      ok = __all_sync(0xffffffffu, mbar_wait(b_sf(buf), (n / kSBuf) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int bi = n / R;
       const int j0 = block_of(bi) * kBN;
       const bool full = (bi < nb_pre) && (j0 + kBN <= it.kv_min);
-      const uint32_t sb = lane_base + kSCol0 + wg * kBN;
+      const uint32_t sb = lane_base + kSCol0 + buf * kBN;
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = cpart * kChunksPerWG; c < (cpart + 1) * kChunksPerWG; ++c) {
         uint32_t raw[32];
         tmem_ld32(sb + c * 32, raw);
         tmem_ld_wait();
         uint32_t ph[16], pl[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float x0 = silu_fast(alpha * __uint_as_float(raw[2 * e]));
-          float x1 = silu_fast(alpha * __uint_as_float(raw[2 * e + 1]));
-          if (!full) {
-            const int key = j0 + c * 32 + 2 * e;
-            if (!(key < kv_end || (key >= sib_lo && key < sib_hi))) x0 = 0.f;
-            if (!(key + 1 < kv_end || (key + 1 >= sib_lo && key + 1 < sib_hi))) x1 = 0.f;
-          }
-          split_bf16x2(x0, x1, ph[e], pl[e]);
+        if (full) {
+          silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
+        } else {
+          silu_chunk<true>(raw, half_alpha, vis_bits(j0 + 32 * c, kv_end, sib_lo, sib_hi), ph, pl);
         }
         // keys [32c, 32c+32): P_hi in columns [32c, 32c+16), P_lo in [32c+16, 32c+32),
         // i.e. over the S columns of this chunk, which were read above.
@@ -278,20 +318,20 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(b_pf(wg));
+      mbar_arrive(b_pf(buf));
     }
     // ------------------------------------------------------------- epilogue: A = O / N_u
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, 0, abort_flag));
     if (ok && total == 0) {
       // no visible key at all (cannot happen for a non-empty tile): A = 0
-      for (int hh = wg; hh < R && valid; hh += 2)
+      for (int hh = wg; hh < R && valid; hh += kSiluWG)
         for (int c = 0; c < kDH; c += 4)
           *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
               make_float4(0.f, 0.f, 0.f, 0.f);
     } else if (ok) {
       tc_fence_after();
       const float inv_n = 1.f / (float)N;
-      for (int hh = wg; hh < R; hh += 2) {
+      for (int hh = wg; hh < R; hh += kSiluWG) {
 #pragma unroll
         for (int c = 0; c < kDH / 32; ++c) {
           uint32_t raw[32];
@@ -337,13 +377,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows, cols]; 128 x 64 boxes with the 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int rows, int cols) {
+// Row-major bf16 matrix [rows, cols]; box_rows x 64 boxes with the 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kDH, (cuuint32_t)kBM};
+  cuuint32_t box[2] = {(cuuint32_t)kDH, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -374,8 +414,8 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
                                const __nv_bfloat16* v, float* a, cudaStream_t st) {
   if (max_items <= 0 || rows_q <= 0 || total_tokens <= 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, rows_q, s.hq * kDH) || !make_map(&mk, k, total_tokens, s.hkv * kDH) ||
-      !make_map(&mv, v, total_tokens, s.hkv * kDH))
+  if (!make_map(&mq, q, rows_q, s.hq * kDH, kBM) || !make_map(&mk, k, total_tokens, s.hkv * kDH, kBN) ||
+      !make_map(&mv, v, total_tokens, s.hkv * kDH, kBN))
     return cudaErrorInvalidValue;
   TcArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha};
   const int r = s.hq / s.hkv;

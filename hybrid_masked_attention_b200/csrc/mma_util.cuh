@@ -58,6 +58,27 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
+// Same split with a truncated hi part: hi takes the upper 16 bits of each float
+// (one byte permute for the pair), lo = bf16(x - hi) with x - hi exact in fp32.
+// |x - hi| < 2^-7 |x|, so hi + lo carries x to within 2^-15 relative.
+__device__ __forceinline__ void split_trunc_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+  hi = __byte_perm(b0, b1, 0x7632);
+  const float r0 = x0 - __uint_as_float(b0 & 0xffff0000u);
+  const float r1 = x1 - __uint_as_float(b1 & 0xffff0000u);
+  lo = pack_bf16x2(r0, r1);
+}
+
+// Visibility bits of the 32 keys [j, j + 32) for a row that sees the prefix
+// [0, kv_end) and the sibling block [sib_lo, sib_hi): bit e <=> key j + e visible.
+__device__ __forceinline__ uint32_t low_bits(int n) {
+  n = min(max(n, 0), 32);
+  return n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+}
+__device__ __forceinline__ uint32_t vis_bits(int j, int kv_end, int sib_lo, int sib_hi) {
+  return low_bits(kv_end - j) | (low_bits(sib_hi - j) & ~low_bits(sib_lo - j));
+}
+
 // Hardware tanh approximation (MUFU); relative error well below bf16 resolution.
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;

@@ -46,17 +46,28 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Returns false when
 // the CTA-wide abort flag is raised or the wait exceeds kWaitCycles (which
 // raises the flag): the caller then stops its work and heads for the exit.
+// (try_wait itself suspends the thread for a short hardware-defined window; the
+// abort flag and the clock are checked only every 64 polls.)
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      *abort_flag = 1;
-      return false;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
+}
+
+// One lane of the (converged) warp returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{ .reg .pred p; elect.sync _|p, 0xffffffff; selp.u32 %0, 1, 0, p; }" : "=r"(pred));
+  return pred != 0;
 }
 
 // ---------------------------------------------------------------- TMA
@@ -159,6 +170,35 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// The same descriptor as two 32-bit words, so that stepping the start address
+// inside the hot loop is one 32-bit add on the low word ((addr + off) >> 4 ==
+// (addr >> 4) + (off >> 4) for 16-byte aligned addresses below 256 KB).
+__device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFF) | (((lbo >> 4) & 0x3FFF) << 16);
+}
+__device__ __forceinline__ uint32_t sw128_desc_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFF) | (1u << 14) | (2u << 29);
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc], descriptors given as (lo, hi) words
+__device__ __forceinline__ void mma_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                        uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; .reg .b64 da, db; mov.b64 da, {%1, %2}; mov.b64 db, {%3, %4};"
+      " setp.ne.b32 p, %6, 0;"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p; }" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc (lo, hi)]
+__device__ __forceinline__ void mma_ts2(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; .reg .b64 db; mov.b64 db, {%2, %3}; setp.ne.b32 p, %5, 0;"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
