@@ -102,6 +102,7 @@ _sigs = {
     "mtfm_bwd_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int]),
     "mtfm_attn_full_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
     "mtfm_attn_target_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
+    "mtfm_attn_target_bwd_static": (ctypes.c_int, [_CP] + [_P] * 17),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -295,3 +296,23 @@ def attn_target_bwd(cfg, meta, q, k, v, u, gamma, beta, a, stats, dy, dq, dk, dv
                     dbeta, ws, stream=None):
     _bwd(_lib.mtfm_attn_target_bwd, "mtfm_attn_target_bwd", cfg, meta, q, k, v, u, gamma, beta, a,
          stats, dy, dq, dk, dv, du, dgamma, dbeta, ws, stream, cfg.total_t)
+
+
+def attn_target_bwd_static(cfg, meta, q, k, v, u, gamma, beta, a, stats, dy, dq, dk, dv, du, dgamma,
+                           dbeta, stream=None):
+    """Target-layer backward without a caller scratch block: the library's fixed
+    24 MiB device array is used instead (for callers that cannot allocate).
+    Calls that may overlap on the GPU must be serialised by the caller."""
+    c = cfg.c()
+    D, Dkv, N, rows = cfg.D, cfg.Dkv, cfg.total_tokens, cfg.total_t
+    bf, f32 = torch.bfloat16, torch.float32
+    st = _lib.mtfm_attn_target_bwd_static(
+        ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"),
+        _ptr(q, bf, (rows, D), "q"), _ptr(k, bf, (N, Dkv), "k"), _ptr(v, bf, (N, Dkv), "v"),
+        _ptr(u, bf, (rows, D), "u"), _ptr(gamma, f32, (3, D), "gamma"),
+        _ptr(beta, f32, (3, D), "beta"), _ptr(a, f32, (rows, D), "a"),
+        _ptr(stats, f32, (rows, 2), "stats"), _ptr(dy, bf, (rows, D), "dy"),
+        _ptr(dq, f32, (rows, D), "dq"), _ptr(dk, f32, (N, Dkv), "dk"),
+        _ptr(dv, f32, (N, Dkv), "dv"), _ptr(du, f32, (rows, D), "du"),
+        _ptr(dgamma, f32, (3, D), "dgamma"), _ptr(dbeta, f32, (3, D), "dbeta"), _stream(stream))
+    _check(st, "mtfm_attn_target_bwd_static")

@@ -195,6 +195,36 @@ mtfm_status mtfm_attn_target_bwd(const mtfm_cfg* cfg, const void* d_meta, const 
                                  float* d_dk, float* d_dv, float* d_du, float* d_dgamma,
                                  float* d_dbeta, void* d_ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Allocation-free Target-layer backward.  No passage of the pages corresponds
+ * to this call: it exists for callers that cannot allocate device memory (code
+ * running inside someone else's memory pool or allocator, or a process that
+ * reserved all of its device memory up front) and so cannot provide the
+ * scratch block mtfm_attn_target_bwd asks for.
+ *
+ * Same arguments and results as mtfm_attn_target_bwd, minus d_ws / ws_bytes:
+ * the scratch is a fixed 24 MiB array inside the library, held on every GPU
+ * that loads the library until the process exits.  Returns
+ * MTFM_ERR_WORKSPACE_TOO_SMALL, launching nothing, when the problem needs
+ * more scratch than that (mtfm_bwd_workspace_bytes(cfg, 1) > 24 MiB; at
+ * hq * head_dim = 512 that is about 10,000 T rows).
+ *
+ * The library allocates nothing here.  The first call on a device looks up the
+ * array's device address (make that first call before any stream capture).
+ * All calls share the one array: calls whose GPU work can overlap (other
+ * streams, or unordered host threads) race on it and must be serialised by
+ * the caller.  Its contents are left over from the previous call; none of
+ * them is read before this call rewrites it.
+ * ------------------------------------------------------------------------- */
+mtfm_status mtfm_attn_target_bwd_static(const mtfm_cfg* cfg, const void* d_meta,
+                                        const uint16_t* d_q, const uint16_t* d_k,
+                                        const uint16_t* d_v, const uint16_t* d_u,
+                                        const float* d_gamma, const float* d_beta,
+                                        const float* d_a, const float* d_stats,
+                                        const uint16_t* d_dy, float* d_dq, float* d_dk,
+                                        float* d_dv, float* d_du, float* d_dgamma,
+                                        float* d_dbeta, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
