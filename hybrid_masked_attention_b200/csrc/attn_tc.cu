@@ -9,8 +9,12 @@
 // with "visible" = the row's key prefix [0, kv_end) plus, for T rows, the
 // sibling block (itself, or the 4 sub-tokens of its target in V2).
 //
-// One CTA = one work item (user, 128-row query tile) x one KV group; a step is
-// one (128-key block, query head) pair:
+// Persistent CTAs (one per SM) stride over work units x KV groups.  A Full-layer
+// unit is one work item (user, 128-row query tile) with all its key blocks; a
+// Target-layer unit is a chunk of kTargetUnitBlocks key blocks of one item (the
+// packer splits each Target tile's key range so that short Target layers still
+// fill the GPU), and its partial O is added into A (zeroed first) with fp32
+// vector atomics.  A step is one (128-key block, query head) pair:
 //   warp 0      : TMA producer (Q tiles of the r heads once, then K/V blocks of
 //                 128 keys through a 3-stage ring);
 //   warp 1      : TMEM allocation and the MMA issue (whole warp runs the
@@ -32,6 +36,8 @@
 // CTA-wide abort flag, every role drains its in-flight copies/MMAs with a
 // bounded wait, TMEM is freed, and MetaHeader::error gets the timeout bit.
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "mtfm_internal.cuh"
 #include "mma_util.cuh"
@@ -57,6 +63,7 @@ constexpr uint32_t kKVBytes = kBN * kDH * 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
+static_assert(kBN == kKeyBlock, "the packer sizes Target units in blocks of kKeyBlock keys");
 static_assert(kSiluWG % kWGPerBuf == 0 && kChunksPerWG >= 1 && kSBuf % kTeams == 0, "warpgroup split");
 
 struct TcArgs {
@@ -105,36 +112,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const MetaView& m = p.m;
   MetaHeader* hdr = m.hdr;
   if (hdr->error) return;
-  const int n_items = TARGET ? hdr->n_items_target : hdr->n_items_full;
-  if ((int)blockIdx.x >= n_items) return;
-  const WorkItem it = (TARGET ? m.items_target : m.items_full)[blockIdx.x];
-  const int u = it.user;
-  const int LH = m.lh[u], LR = m.lr[u], LT = m.lt[u];
-  const int N = LH + LR + LT, so = m.seq_off[u];
-  const int nq = TARGET ? LT : N;
-  const int q0 = it.tile * kBM;
-  const int qrow0 = TARGET ? m.t_off[u] : so;
-  const int pos0 = TARGET ? LH + LR : 0;
-  const int g = blockIdx.y;
+  // Work units: Full layer = one work item (all its key blocks); Target layer =
+  // one chunk of kTargetUnitBlocks key blocks of a work item.  Each unit runs
+  // for every KV group; the CTAs stride over (unit, group) pairs.
+  const int n_units = TARGET ? hdr->n_units_target : hdr->n_items_full;
+  const int n_work = n_units * p.hkv;
+  if ((int)blockIdx.x >= n_work) return;
   const int ldq = p.hq * kDH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // key blocks: prefix [0, kv_max) then the sibling span of the tile's T rows
-  const int t0pos = LH + LR;
-  const int nb_pre = (it.kv_max + kBN - 1) / kBN;
-  int sb_lo = 0, sb_hi = 0;
-  {
-    const int first = max(pos0 + q0, t0pos);
-    const int last = pos0 + min(q0 + kBM, nq) - 1;
-    if (first <= last) {
-      const int lo = t0pos + ((first - t0pos) / p.v2) * p.v2;
-      const int hi = t0pos + ((last - t0pos) / p.v2 + 1) * p.v2;
-      sb_lo = max(lo / kBN, nb_pre);
-      sb_hi = (hi + kBN - 1) / kBN;
-    }
-  }
-  const int n_blocks = nb_pre + max(0, sb_hi - sb_lo);
-  const int total = n_blocks * R;  // steps n = (key block n / R, head n % R)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_addr(smem);
@@ -148,6 +133,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto b_pf = [&](int b) { return smem_addr(&bar_p_full[b]); };
 
   if (threadIdx.x == 0) {
+    s_abort = 0;
     mbar_init(b_q, 1);
     mbar_init(b_o, 1);
     mbar_init(b_drain, 1);
@@ -159,7 +145,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(b_sf(b), 1);
       mbar_init(b_pf(b), 128 * kWGPerBuf);
     }
-    s_abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -167,190 +152,230 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tmem_relinquish();
     tc_fence_before();
   }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
 
-  auto block_of = [&](int bi) { return bi < nb_pre ? bi : sb_lo + (bi - nb_pre); };
+  // Barrier phases run on across units: K/V stages count key blocks, S/P
+  // buffers count steps, Q and O count units, all from the start of the CTA.
+  int blk_base = 0, step_base = 0, unit_iter = 0;
+  for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+    const int unit = w / p.hkv, g = w % p.hkv;
+    int item = unit, chunk = 0;
+    if (TARGET) {  // last item whose first unit is <= unit
+      int lo = 0, hi = hdr->n_items_target - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (m.unit_off[mid] <= unit) lo = mid; else hi = mid - 1;
+      }
+      item = lo;
+      chunk = unit - m.unit_off[lo];
+    }
+    const WorkItem it = (TARGET ? m.items_target : m.items_full)[item];
+    const int u = it.user;
+    const int LH = m.lh[u], LR = m.lr[u], LT = m.lt[u];
+    const int N = LH + LR + LT, so = m.seq_off[u];
+    const int nq = TARGET ? LT : N;
+    const int q0 = it.tile * kBM;
+    const int qrow0 = TARGET ? m.t_off[u] : so;
+    const int pos0 = TARGET ? LH + LR : 0;
+    const int t0pos = LH + LR;
+    const KeyBlocks kb = key_blocks(it.kv_max, LH, LR, nq, pos0, q0, p.v2);
+    const int bi0 = TARGET ? chunk * kTargetUnitBlocks : 0;
+    const int bi1 = TARGET ? min(bi0 + kTargetUnitBlocks, kb.n_blocks) : kb.n_blocks;
+    const int n_blocks = max(0, bi1 - bi0);
+    const int total = n_blocks * R;  // steps n = (key block bi0 + n / R, head n % R)
+    auto block_of = [&](int bi) { return kb.block(bi0 + bi); };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_expect_tx(b_q, R * kQBytes);
-      for (int hh = 0; hh < R; ++hh)
-        tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
-      int issued = 0;
-      for (int bi = 0; bi < n_blocks; ++bi) {
-        const int s = bi % kStages;
-        if (bi >= kStages && !mbar_wait(b_kve(s), ((bi / kStages) - 1) & 1, abort_flag)) break;
-        const int row = so + block_of(bi) * kBN;
-        mbar_expect_tx(b_kvf(s), 2 * kKVBytes);
-        tma_load_2d(sK + s * kKVBytes, &tm_k, b_kvf(s), g * kDH, row);
-        tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
-        ++issued;
-      }
-      // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
-      // no TMA write may land after this CTA leaves.
-      const long long t0 = clock64();
-      auto drain_wait = [&](uint32_t bar, uint32_t par) {
-        while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
+    if (warp == 0) {
+      // ----------------------------------------------------------- producer
+      if (lane == 0) {
+        mbar_expect_tx(b_q, R * kQBytes);  // Q of the previous unit was consumed before the unit barrier
+        for (int hh = 0; hh < R; ++hh)
+          tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
+        int issued = 0;
+        for (int bi = 0; bi < n_blocks; ++bi) {
+          const int G = blk_base + bi, s = G % kStages;
+          if (G >= kStages && !mbar_wait(b_kve(s), ((G / kStages) - 1) & 1, abort_flag)) break;
+          const int row = so + block_of(bi) * kBN;
+          mbar_expect_tx(b_kvf(s), 2 * kKVBytes);
+          tma_load_2d(sK + s * kKVBytes, &tm_k, b_kvf(s), g * kDH, row);
+          tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
+          ++issued;
         }
+        // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
+        // no TMA write may land after this unit's barriers are re-armed or the CTA leaves.
+        const long long t0 = clock64();
+        auto drain_wait = [&](uint32_t bar, uint32_t par) {
+          while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
+          }
+        };
+        drain_wait(b_q, unit_iter & 1);
+        for (int bi = max(0, issued - kStages); bi < issued; ++bi)
+          drain_wait(b_kvf((blk_base + bi) % kStages), ((blk_base + bi) / kStages) & 1);
+      }
+    } else if (warp == 1) {
+      // ----------------------------------------------------------- MMA issuer
+      // Order: S(0); then for every step n: S(n+1), [P(n) ready] O_h += P(n) V.
+      // S(n+1) reuses the buffer of step n-1, whose PV was issued before it.
+      // The whole warp runs the control flow (so operands stay warp-uniform) and
+      // one elected lane issues the MMAs and commits.
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDH, true);
+      // descriptor words: the high word is shared; low words step by (bytes >> 4)
+      const uint32_t dhi = sw128_desc_hi(1024);
+      const uint32_t q_lo = sw128_desc_lo(sQ, 16), k_lo = sw128_desc_lo(sK, 16), v_lo = sw128_desc_lo(sV, 16);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(b_q, unit_iter & 1, abort_flag));
+      auto issue_s = [&](int n) -> bool {
+        const int G = blk_base + n / R, hh = n % R, s = G % kStages;
+        if (hh == 0 && !__all_sync(0xffffffffu, mbar_wait(b_kvf(s), (G / kStages) & 1, abort_flag)))
+          return false;
+        tc_fence_after();
+        const int gb = (step_base + n) % kSBuf;
+        const uint32_t d = tmem + kSCol0 + gb * kBN;
+        const uint32_t a0 = q_lo + hh * (kQBytes >> 4), b0 = k_lo + s * (kKVBytes >> 4);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kDH / 16; ++kk)
+            mma_ss2(d, a0 + kk * 2, dhi, b0 + kk * 2, dhi, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_commit(b_sf(gb));
+        }
+        __syncwarp();
+        return true;
       };
-      drain_wait(b_q, 0);
-      for (int bi = max(0, issued - kStages); bi < issued; ++bi)
-        drain_wait(b_kvf(bi % kStages), (bi / kStages) & 1);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
-    // Order: S(0); then for every step n: S(n+1), [P(n) ready] O_h += P(n) V.
-    // S(n+1) reuses the buffer of step n-1, whose PV was issued before it.
-    // The whole warp runs the control flow (so operands stay warp-uniform) and
-    // one elected lane issues the MMAs and commits.
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
-    constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDH, true);
-    // descriptor words: the high word is shared; low words step by (bytes >> 4)
-    const uint32_t dhi = sw128_desc_hi(1024);
-    const uint32_t q_lo = sw128_desc_lo(sQ, 16), k_lo = sw128_desc_lo(sK, 16), v_lo = sw128_desc_lo(sV, 16);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(b_q, 0, abort_flag));
-    auto issue_s = [&](int n) -> bool {
-      const int bi = n / R, hh = n % R, s = bi % kStages;
-      if (hh == 0 && !__all_sync(0xffffffffu, mbar_wait(b_kvf(s), (bi / kStages) & 1, abort_flag)))
-        return false;
-      tc_fence_after();
-      const uint32_t d = tmem + kSCol0 + (n % kSBuf) * kBN;
-      const uint32_t a0 = q_lo + hh * (kQBytes >> 4), b0 = k_lo + s * (kKVBytes >> 4);
-      if (elect_one()) {
+      for (int n = 0; ok && n < min(total, kSBuf - 1); ++n) ok = issue_s(n);
+      for (int n = 0; ok && n < total; ++n) {
+        if (n + kSBuf - 1 < total && !issue_s(n + kSBuf - 1)) {
+          ok = false;
+          break;
+        }
+        const int b = (step_base + n) % kSBuf;
+        if (!__all_sync(0xffffffffu, mbar_wait(b_pf(b), ((step_base + n) / kSBuf) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int bi = n / R, hh = n % R, s = (blk_base + bi) % kStages;
+        const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo, bf16 pairs
+        const uint32_t o = tmem + hh * kDH;
+        const uint32_t vb = v_lo + s * (kKVBytes >> 4);  // V rows (keys): 16 per k-step = 2048 B
+        const uint32_t acc0 = bi > 0 ? 1u : 0u;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kDH / 16; ++kk)
-          mma_ss2(d, a0 + kk * 2, dhi, b0 + kk * 2, dhi, idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(b_sf(n % kSBuf));
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
+            mma_ts2(o, pt + col, vb + kk * (2048 >> 4), dhi, idesc_pv, kk > 0 ? 1u : acc0);
+            mma_ts2(o, pt + col + 16, vb + kk * (2048 >> 4), dhi, idesc_pv, 1u);
+          }
+          if (hh == R - 1) mma_commit(b_kve(s));
+        }
+        __syncwarp();
+      }
+      if (elect_one()) {
+        // on failure, drain every MMA issued so far before TMEM is reused or released
+        mma_commit(ok ? b_o : b_drain);
       }
       __syncwarp();
-      return true;
-    };
-    for (int n = 0; ok && n < min(total, kSBuf - 1); ++n) ok = issue_s(n);
-    for (int n = 0; ok && n < total; ++n) {
-      if (n + kSBuf - 1 < total && !issue_s(n + kSBuf - 1)) {
-        ok = false;
-        break;
-      }
-      const int b = n % kSBuf;
-      if (!__all_sync(0xffffffffu, mbar_wait(b_pf(b), (n / kSBuf) & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int bi = n / R, hh = n % R, s = bi % kStages;
-      const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo, bf16 pairs
-      const uint32_t o = tmem + hh * kDH;
-      const uint32_t vb = v_lo + s * (kKVBytes >> 4);  // V rows (keys): 16 per k-step = 2048 B
-      const uint32_t acc0 = bi > 0 ? 1u : 0u;
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
-          mma_ts2(o, pt + col, vb + kk * (2048 >> 4), dhi, idesc_pv, kk > 0 ? 1u : acc0);
-          mma_ts2(o, pt + col + 16, vb + kk * (2048 >> 4), dhi, idesc_pv, 1u);
+      if (!ok) {
+        const long long t0 = clock64();
+        while (!mbar_try(b_drain, 0) && clock64() - t0 < kWaitCycles) {
         }
-        if (hh == R - 1) mma_commit(b_kve(s));
       }
-      __syncwarp();
-    }
-    if (elect_one()) {
-      // on failure, drain every MMA issued so far before TMEM is released
-      mma_commit(ok ? b_o : b_drain);
-    }
-    __syncwarp();
-    if (!ok) {
-      const long long t0 = clock64();
-      while (!mbar_try(b_drain, 0) && clock64() - t0 < kWaitCycles) {
-      }
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------- SiLU warpgroups
-    const int wg = (warp - 4) >> 2;   // warpgroup 0..3
-    const int team = wg % kTeams;      // steps n = team (mod kTeams)
-    const int cpart = wg / kTeams;     // part of the key columns of a step this warpgroup handles
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const int qi = q0 + row;
-    const bool valid = qi < nq;
-    int kv_end = 0, sib_lo = 0, sib_hi = 0;
-    if (valid) {
-      const int pos = pos0 + qi;
-      kv_end = m.kv_end[so + pos];
-      if (pos >= t0pos) {
-        sib_lo = t0pos + ((pos - t0pos) / p.v2) * p.v2;
-        sib_hi = sib_lo + p.v2;
-      }
-    }
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const float half_alpha = 0.5f * p.alpha;
-    bool ok = true;
-    for (int n = team; n < total; n += kTeams) {
-      const int buf = n % kSBuf;
-      ok = __all_sync(0xffffffffu, mbar_wait(b_sf(buf), (n / kSBuf) & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const int bi = n / R;
-      const int j0 = block_of(bi) * kBN;
-      const bool full = (bi < nb_pre) && (j0 + kBN <= it.kv_min);
-      const uint32_t sb = lane_base + kSCol0 + buf * kBN;
-#pragma unroll
-      for (int c = cpart * kChunksPerWG; c < (cpart + 1) * kChunksPerWG; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(sb + c * 32, raw);
-        tmem_ld_wait();
-        uint32_t ph[16], pl[16];
-        if (full) {
-          silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
-        } else {
-          silu_chunk<true>(raw, half_alpha, vis_bits(j0 + 32 * c, kv_end, sib_lo, sib_hi), ph, pl);
+    } else if (warp >= 4) {
+      // ----------------------------------------------------------- SiLU warpgroups
+      const int wg = (warp - 4) >> 2;   // warpgroup 0..3
+      const int team = wg % kTeams;      // steps n = team (mod kTeams)
+      const int cpart = wg / kTeams;     // part of the key columns of a step this warpgroup handles
+      const int quad = warp & 3;
+      const int row = quad * 32 + lane;
+      const int qi = q0 + row;
+      const bool valid = qi < nq;
+      int kv_end = 0, sib_lo = 0, sib_hi = 0;
+      if (valid) {
+        const int pos = pos0 + qi;
+        kv_end = m.kv_end[so + pos];
+        if (pos >= t0pos) {
+          sib_lo = t0pos + ((pos - t0pos) / p.v2) * p.v2;
+          sib_hi = sib_lo + p.v2;
         }
-        // keys [32c, 32c+32): P_hi in columns [32c, 32c+16), P_lo in [32c+16, 32c+32),
-        // i.e. over the S columns of this chunk, which were read above.
-        tmem_st16(sb + c * 32, ph);
-        tmem_st16(sb + c * 32 + 16, pl);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(b_pf(buf));
-    }
-    // ------------------------------------------------------------- epilogue: A = O / N_u
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, 0, abort_flag));
-    if (ok && total == 0) {
-      // no visible key at all (cannot happen for a non-empty tile): A = 0
-      for (int hh = wg; hh < R && valid; hh += kSiluWG)
-        for (int c = 0; c < kDH; c += 4)
-          *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
-              make_float4(0.f, 0.f, 0.f, 0.f);
-    } else if (ok) {
-      tc_fence_after();
-      const float inv_n = 1.f / (float)N;
-      for (int hh = wg; hh < R; hh += kSiluWG) {
+      const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+      const float half_alpha = 0.5f * p.alpha;
+      bool ok = true;
+      for (int n = team; n < total; n += kTeams) {
+        const int buf = (step_base + n) % kSBuf;
+        ok = __all_sync(0xffffffffu, mbar_wait(b_sf(buf), ((step_base + n) / kSBuf) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int gbi = bi0 + n / R;  // block index within the item
+        const int j0 = kb.block(gbi) * kBN;
+        const bool full = (gbi < kb.nb_pre) && (j0 + kBN <= it.kv_min);
+        const uint32_t sb = lane_base + kSCol0 + buf * kBN;
 #pragma unroll
-        for (int c = 0; c < kDH / 32; ++c) {
+        for (int c = cpart * kChunksPerWG; c < (cpart + 1) * kChunksPerWG; ++c) {
           uint32_t raw[32];
-          tmem_ld32(lane_base + hh * kDH + c * 32, raw);
+          tmem_ld32(sb + c * 32, raw);
           tmem_ld_wait();
-          if (valid) {
-            float* dst = p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c * 32;
+          uint32_t ph[16], pl[16];
+          if (full) {
+            silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
+          } else {
+            silu_chunk<true>(raw, half_alpha, vis_bits(j0 + 32 * c, kv_end, sib_lo, sib_hi), ph, pl);
+          }
+          // keys [32c, 32c+32): P_hi in columns [32c, 32c+16), P_lo in [32c+16, 32c+32),
+          // i.e. over the S columns of this chunk, which were read above.
+          tmem_st16(sb + c * 32, ph);
+          tmem_st16(sb + c * 32 + 16, pl);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(b_pf(buf));
+      }
+      // ----------------------------------------------------------- epilogue: A (+)= O / N_u
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, unit_iter & 1, abort_flag));
+      if (ok && total == 0) {
+        // no visible key at all (cannot happen for a non-empty Full tile): A = 0
+        if (!TARGET)
+          for (int hh = wg; hh < R && valid; hh += kSiluWG)
+            for (int c = 0; c < kDH; c += 4)
+              *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
+                  make_float4(0.f, 0.f, 0.f, 0.f);
+      } else if (ok) {
+        tc_fence_after();
+        const float inv_n = 1.f / (float)N;
+        for (int hh = wg; hh < R; hh += kSiluWG) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              reinterpret_cast<float4*>(dst)[e] =
-                  make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
-                              __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
+          for (int c = 0; c < kDH / 32; ++c) {
+            uint32_t raw[32];
+            tmem_ld32(lane_base + hh * kDH + c * 32, raw);
+            tmem_ld_wait();
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float4 v = make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
+                                             __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
+                if (TARGET) atomicAdd(dst + e, v);  // partial over this unit's key chunk; A zeroed first
+                else dst[e] = v;
+              }
+            }
           }
         }
       }
     }
+    tc_fence_before();
+    __syncthreads();
+    if (s_abort) break;  // uniform: read after the barrier
+    blk_base += n_blocks;
+    step_base += total;
+    ++unit_iter;
   }
-  tc_fence_before();
-  __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -390,6 +415,19 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+// One CTA per SM (TMEM and shared memory allow no more); the CTAs stride over
+// the (work unit, KV group) pairs, whose count the kernel reads from the metadata.
 template <int R, bool TARGET>
 cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const TcArgs& a, int max_items, cudaStream_t st) {
@@ -397,7 +435,8 @@ cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R, TARGET>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(max_items, a.hkv);
+  int grid = sm_count();
+  if (!TARGET) grid = std::min(grid, max_items * a.hkv);
   attn_fwd_tc_kernel<R, TARGET><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
@@ -419,6 +458,11 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
     return cudaErrorInvalidValue;
   TcArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha};
   const int r = s.hq / s.hkv;
+  if (s.target) {
+    // Target units add partial sums over key chunks into A
+    cudaError_t e = cudaMemsetAsync(a, 0, sizeof(float) * (size_t)rows_q * s.hq * kDH, st);
+    if (e != cudaSuccess) return e;
+  }
   if (s.target) {
     if (r == 1) return tc_launch<1, true>(mq, mk, mv, args, max_items, st);
     if (r == 2) return tc_launch<2, true>(mq, mk, mv, args, max_items, st);

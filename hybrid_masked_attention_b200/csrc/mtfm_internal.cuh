@@ -32,7 +32,8 @@ struct MetaHeader {
   int32_t error;
   int32_t max_items_full;
   int32_t max_items_target;
-  int32_t pad[5];
+  int32_t n_units_target;  // key-range chunks of the Target work list (sum of unit_count)
+  int32_t pad[4];
 };
 
 // One work item: a 128-row query tile of one user and the range of prefix
@@ -46,7 +47,8 @@ struct WorkItem {
 };
 
 struct MetaLayout {
-  size_t seq_off, r_off, t_off, lh, lr, lt, kv_end, row_type, items_full, items_target, total;
+  size_t seq_off, r_off, t_off, lh, lr, lt, kv_end, row_type, items_full, items_target, unit_off,
+      total;
   int32_t max_items_full, max_items_target;
 };
 
@@ -67,6 +69,7 @@ inline MetaLayout meta_layout(int B, int total_tokens, int total_t) {
   L.max_items_target = (total_t + kTileM - 1) / kTileM + B;
   L.items_full = o;   o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_full);
   L.items_target = o; o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_target);
+  L.unit_off = o;     o = align256(o + sizeof(int32_t) * ((size_t)L.max_items_target + 1));
   L.total = o;
   return L;
 }
@@ -84,6 +87,7 @@ struct MetaView {
   uint8_t* row_type;
   WorkItem* items_full;
   WorkItem* items_target;
+  int32_t* unit_off;  // [max_items_target + 1]: first unit of each Target item (prefix sums)
 };
 
 inline MetaView meta_view(void* base, const MetaLayout& L) {
@@ -100,7 +104,39 @@ inline MetaView meta_view(void* base, const MetaLayout& L) {
   v.row_type = reinterpret_cast<uint8_t*>(b + L.row_type);
   v.items_full = reinterpret_cast<WorkItem*>(b + L.items_full);
   v.items_target = reinterpret_cast<WorkItem*>(b + L.items_target);
+  v.unit_off = reinterpret_cast<int32_t*>(b + L.unit_off);
   return v;
+}
+
+// Key blocks visited by the tensor-core forward for one work item: the prefix
+// [0, kv_max) in blocks of kKeyBlock keys, then the blocks of the sibling span of
+// the item's T rows that the prefix does not cover.  Shared by the packer (to
+// size the Target split) and the kernel (to walk the blocks).
+constexpr int kKeyBlock = 128;
+constexpr int kTargetUnitBlocks = 2;  // key blocks per Target work unit (split of the key range)
+
+struct KeyBlocks {
+  int nb_pre, sb_lo, n_blocks;
+  __host__ __device__ int block(int bi) const { return bi < nb_pre ? bi : sb_lo + (bi - nb_pre); }
+};
+
+__host__ __device__ inline KeyBlocks key_blocks(int kv_max, int LH, int LR, int nq, int pos0, int q0,
+                                                int v2) {
+  KeyBlocks kb;
+  const int t0pos = LH + LR;
+  kb.nb_pre = (kv_max + kKeyBlock - 1) / kKeyBlock;
+  int sb_lo = 0, sb_hi = 0;
+  const int first = pos0 + q0 > t0pos ? pos0 + q0 : t0pos;
+  const int last = pos0 + (q0 + kTileM < nq ? q0 + kTileM : nq) - 1;
+  if (first <= last) {
+    const int lo = t0pos + ((first - t0pos) / v2) * v2;
+    const int hi = t0pos + ((last - t0pos) / v2 + 1) * v2;
+    sb_lo = lo / kKeyBlock > kb.nb_pre ? lo / kKeyBlock : kb.nb_pre;
+    sb_hi = (hi + kKeyBlock - 1) / kKeyBlock;
+  }
+  kb.sb_lo = sb_lo;
+  kb.n_blocks = kb.nb_pre + (sb_hi > sb_lo ? sb_hi - sb_lo : 0);
+  return kb;
 }
 
 // Everything an attention launch needs besides the tensors.

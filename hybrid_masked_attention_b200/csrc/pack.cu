@@ -11,11 +11,14 @@
 //   T row t        : keys [0, L_H + k_t) + itself     k_t = #{R : ts < exposure_t}
 // k_t is a lower_bound over the user's ascending R timestamps.
 //
-// Two launches, no host synchronisation:
+// Three launches, no host synchronisation:
 //   pack_users_kernel (1 CTA): validates lengths, scans offsets, orders users
 //     longest first and writes the work lists of 128-row query tiles;
 //   pack_rows_kernel (1 CTA per work item): per-row kv_end / row type, the
-//     sortedness check, and each tile's [kv_min, kv_max] used for block skipping.
+//     sortedness check, and each tile's [kv_min, kv_max] used for block skipping;
+//   pack_units_kernel (1 CTA): prefix sums of the Target tiles' key-range units
+//     (each Target tile's keys are split into chunks of kTargetUnitBlocks blocks,
+//     so that short Target layers still fill every SM).
 #include "mtfm_internal.cuh"
 
 namespace mtfm {
@@ -98,6 +101,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->error = s_err;
       m.hdr->max_items_full = max_if;
       m.hdr->max_items_target = max_it;
+      m.hdr->n_units_target = 0;
     }
     return;
   }
@@ -183,6 +187,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->error = 0;
     m.hdr->max_items_full = max_if;
     m.hdr->max_items_target = max_it;
+    m.hdr->n_units_target = 0;
   }
 }
 
@@ -252,6 +257,35 @@ pack_rows_kernel(MetaView m, int max_if, const int64_t* __restrict__ r_ts,
     }
     it->kv_min = kmin;
     it->kv_max = kmax;
+    if (tgt) {
+      // number of key-range units this Target tile is split into (scanned by pack_units_kernel)
+      const KeyBlocks kb = key_blocks(kmax, LH, LR, LT, LH + LR, tile * kTileM, hdr->v2);
+      m.unit_off[idx + 1] = (kb.n_blocks + kTargetUnitBlocks - 1) / kTargetUnitBlocks;
+      if (idx == 0) m.unit_off[0] = 0;
+    }
+  }
+}
+
+// In-place inclusive scan of the Target units per item: unit_off[i] becomes the
+// first unit of item i; n_units_target the total.
+__global__ void __launch_bounds__(kPackThreads) pack_units_kernel(MetaView m) {
+  __shared__ long long s_warp[32];
+  MetaHeader* hdr = m.hdr;
+  if (hdr->error & kErrBadLengths) return;
+  const int n = hdr->n_items_target;
+  const int chunk = (n + kPackThreads - 1) / kPackThreads;
+  const int a = min(n, (int)threadIdx.x * chunk), b = min(n, a + chunk);
+  long long local = 0;
+  for (int i = a; i < b; ++i) local += m.unit_off[i + 1];
+  long long total;
+  long long run = block_exclusive_scan(local, &total, s_warp);
+  for (int i = a; i < b; ++i) {
+    run += m.unit_off[i + 1];
+    m.unit_off[i + 1] = (int)run;
+  }
+  if (threadIdx.x == 0) {
+    m.unit_off[0] = 0;
+    hdr->n_units_target = (int)total;
   }
 }
 
@@ -284,6 +318,9 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
   const int blocks = L.max_items_full + L.max_items_target;
   if (blocks > 0) {
     pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, r_ts, t_exp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    pack_units_kernel<<<1, kPackThreads, 0, st>>>(m);
     e = cudaGetLastError();
   }
   return e;
