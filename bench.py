@@ -47,8 +47,10 @@ WORKLOAD = ("hybrid pair: 32 users jagged, L_H~U[256,1024], L_R~U[32,256] sorted
             "L_T~U[16,128] over 3 scenarios; Hq 8 / Hkv 2, head_dim 64; pack + Full fwd + Target fwd "
             "(attention + GLN gate)")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["hybrid_masked_attention_b200/csrc/attn_mma.cu",
-                  "hybrid_masked_attention_b200/csrc/mma_util.cuh"]
+KERNEL_SOURCES = ["hybrid_masked_attention_b200/csrc/attn_tc.cu",
+                  "hybrid_masked_attention_b200/csrc/sm100.cuh",
+                  "hybrid_masked_attention_b200/csrc/mma_util.cuh",
+                  "hybrid_masked_attention_b200/csrc/mtfm_internal.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_full_fwd_pair.md")
 
 
@@ -295,7 +297,7 @@ def run_mtfm(args, rank, world, local_rank):
                            "users_per_s": round(b.B / ((ms_parts["target_attn"] + ms_parts["target_gate"]) * 1e-3), 1)},
                 "ms_parts": {k: round(v, 5) for k, v in ms_parts.items()},
             },
-            "roofline": {"kernel": "Full-layer attention (attn_fwd_mma_kernel)", "bound": "tensor",
+            "roofline": {"kernel": "Full-layer attention (attn_fwd_tc_kernel, tcgen05)", "bound": "tensor",
                          "achieved": round(full_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(full_tf / peak_tf, 4), "traffic": traffic,
                          "peak_source": f"{src} bf16 dense (burst)",
