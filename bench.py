@@ -447,6 +447,103 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------- other workloads
+
+def run_extra(args):
+    """Per-kernel timings of the other configurations (one JSON line; not the headline metric):
+    ``sweep``: per-user length N (H:R:T ~ 70:15:15, V2 with --v2), 2^21 / N users;
+    ``train``: forward + backward of one Full and one Target layer, --users users of the
+    production-shape distributions.  Activations are seeded device-side normals (bf16)."""
+    import torch
+    import hybrid_masked_attention_b200 as M
+    from hybrid_masked_attention_b200.session import HybridAttention
+    dev = torch.device("cuda", 0)
+    heads = syn.PAIR_HEADS
+    if args.workload == "sweep":
+        b = syn.sweep_batch(args.seqlen, v2=args.v2, seed=1003)
+        name = f"sweep N={args.seqlen}{' V2' if args.v2 else ''}: {b.B} users x {args.seqlen} tokens"
+    else:
+        b = syn.pair_batch(args.users, seed=1005)
+        name = f"training step: {b.B} users, production-shape lengths"
+    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh,
+                   b.v2_subtokens)
+    s = HybridAttention(cfg, dev)
+    it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
+    lens = (it(b.L_H, np.int32), it(b.L_R, np.int32), it(b.L_T, np.int32), it(b.r_ts, np.int64),
+            it(b.t_exp, np.int64))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    rnd = lambda *shape: torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    N, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
+    gam = torch.ones(3, D, device=dev)
+    bet = torch.zeros(3, D, device=dev)
+    F = dict(q=rnd(N, D), k=rnd(N, Dkv), v=rnd(N, Dkv), u=rnd(N, D), dy=rnd(N, D))
+    Tg = dict(q=rnd(T, D), k=rnd(N, Dkv), v=rnd(N, Dkv), u=rnd(T, D), dy=rnd(T, D))
+    s.pack(*lens, check=True)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    res = {}
+
+    def timed(label, fn, steps):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a, z = ev(), ev()
+        a.record()
+        for _ in range(steps):
+            fn()
+        z.record()
+        torch.cuda.synchronize()
+        res[label] = a.elapsed_time(z) / steps
+
+    out_f = s._fwd_out(N, True)
+    out_t = s._fwd_out(T, True)
+    steps = max(1, args.steps)
+    timed("pack", lambda: s.pack(*lens), steps)
+    timed("full_attn", lambda: M.attn_full(cfg, s.meta, F["q"], F["k"], F["v"], out_f[1]), steps)
+    timed("full_fwd", lambda: s.full_fwd(F["q"], F["k"], F["v"], F["u"], gam, bet, out=out_f), steps)
+    timed("target_attn", lambda: M.attn_target(cfg, s.meta, Tg["q"], Tg["k"], Tg["v"], out_t[1]), steps)
+    timed("target_fwd", lambda: s.target_fwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, out=out_t), steps)
+    if args.workload == "train":
+        yf, af, sf = s.full_fwd(F["q"], F["k"], F["v"], F["u"], gam, bet)
+        yt, at, st_ = s.target_fwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet)
+        timed("full_bwd", lambda: s.full_bwd(F["q"], F["k"], F["v"], F["u"], gam, bet, af, sf, F["dy"]), steps)
+        timed("target_bwd", lambda: s.target_bwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, at, st_, Tg["dy"]), steps)
+    M.pack_check(s.meta)
+    peaks, src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ff, ft = attn_flops(b, heads, False), attn_flops(b, heads, True)
+    tf = lambda fl, ms: fl / (ms * 1e-3) / 1e12
+    layers = {
+        "full_attn": {"ms": res["full_attn"], "tflops": tf(ff, res["full_attn"]),
+                      "frac_tensor_peak": tf(ff, res["full_attn"]) / peak_tf},
+        "full_fwd": {"ms": res["full_fwd"], "tflops": tf(ff, res["full_fwd"]),
+                     "users_per_s": b.B / (res["full_fwd"] * 1e-3)},
+        "target_attn": {"ms": res["target_attn"], "tflops": tf(ft, res["target_attn"]),
+                        "gbs": target_attn_bytes(b, heads) / (res["target_attn"] * 1e-3) / 1e9,
+                        "frac_tensor_peak": tf(ft, res["target_attn"]) / peak_tf},
+        "target_fwd": {"ms": res["target_fwd"], "tflops": tf(ft, res["target_fwd"]),
+                       "users_per_s": b.B / (res["target_fwd"] * 1e-3)},
+        "pack": {"ms": res["pack"]},
+    }
+    layers["target_attn"]["frac_hbm"] = layers["target_attn"]["gbs"] / hbm
+    if args.workload == "train":
+        for k, fl in (("full_bwd", ff), ("target_bwd", ft)):
+            layers[k] = {"ms": res[k], "tflops": tf(2.5 * fl, res[k]),
+                         "users_per_s": b.B / (res[k] * 1e-3)}
+    total_ms = res["pack"] + res["full_fwd"] + res["target_fwd"] + res.get("full_bwd", 0) + res.get("target_bwd", 0)
+    total_fl = ff + ft + (2.5 * (ff + ft) if args.workload == "train" else 0.0)
+    out = {"metric": METRIC, "value": round(total_fl / (total_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(total_ms, 5),
+           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": name, "users": b.B, "total_tokens": N, "total_t": T,
+                      "flops_fwd_full": ff, "flops_fwd_target": ft,
+                      "peak": f"{src} bf16 {peak_tf} TF/s, HBM {hbm} GB/s"},
+           "per_kernel": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                          for k, v in layers.items()}}
+    print(json.dumps(out), flush=True)
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -459,6 +556,10 @@ def main():
     ap.add_argument("--sets", type=int, default=4, help="resident input copies rotated across steps")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["pair", "sweep", "train"], default="pair",
+                    help="pair: the headline step; sweep/train: per-kernel timings of the other configs")
+    ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
+    ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -469,6 +570,9 @@ def main():
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
 
+    if args.workload != "pair":
+        run_extra(args)
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:
