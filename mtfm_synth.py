@@ -206,3 +206,62 @@ def layer_inputs(batch: JaggedBatch, heads: Heads, target: bool, seed: int,
             beta = np.zeros((3, heads.dq), np.float32)
     dy = normal_bf16(seed, S_DY + off, (rows_q, heads.dq)) if with_dy else None
     return LayerInputs(q, k, v, u, gamma, beta, dy)
+
+
+# ----------------------------------------------------------------------------
+# Backbone stack (4 blocks of one Full-Attention layer and three Target-Attention
+# layers; page "美团推荐大模型 MTFM 深度硬核解析" §4.1-4.2): projection weights
+# and the input token matrix.
+# ----------------------------------------------------------------------------
+
+STACK_KINDS = ("F", "T", "T", "T") * 4
+S_X0, S_WIN, S_WKV, S_WO, S_RMS = 20, 21, 22, 23, 24
+
+
+@dataclass
+class LayerWeights:
+    """One layer's parameters.  Projection matrices are bf16 bit patterns in the
+    [out_features, in_features] layout; norms' parameters are float32."""
+    kind: str                     # "F" (Full) or "T" (Target)
+    rms_w: np.ndarray             # [d_model] RMSNorm weight
+    w_in: np.ndarray              # F: W_uqkv [2*dq + 2*dkv, d_model]; T: W_uq [2*dq, d_model]
+    w_kv: Optional[np.ndarray]    # T: W_kv [2*dkv, d_model]; F: None
+    w_o: np.ndarray               # [d_model, dq]
+    gamma: np.ndarray             # [3, dq] GLN affine rows (H, R, T)
+    beta: np.ndarray              # [3, dq]
+
+
+def stack_weights(heads: Heads, d_model: int, seed: int, kinds=STACK_KINDS, std: float = 0.02,
+                  std_o: Optional[float] = None, random_norms: bool = False) -> list:
+    """Weights ~ N(0, std) (std 0.02), output projections ~ N(0, std_o) with the
+    depth-scaled std_o = 0.02 / sqrt(layers).  Norm parameters are the identity
+    (RMSNorm weight 1, GLN gamma 1 and beta 0) unless ``random_norms``."""
+    if std_o is None:
+        std_o = std / np.sqrt(len(kinds))
+    dq, dkv = heads.dq, heads.dkv
+    out = []
+    for l, kind in enumerate(kinds):
+        s = seed * 1000 + l
+        if kind == "F":
+            w_in = normal_bf16(s, S_WIN, (2 * dq + 2 * dkv, d_model), std)
+            w_kv = None
+        else:
+            w_in = normal_bf16(s, S_WIN, (2 * dq, d_model), std)
+            w_kv = normal_bf16(s, S_WKV, (2 * dkv, d_model), std)
+        w_o = normal_bf16(s, S_WO, (d_model, dq), std_o)
+        if random_norms:
+            g = rng_for(s, S_RMS)
+            rms_w = (1.0 + 0.25 * g.standard_normal(d_model)).astype(np.float32)
+            gamma = (1.0 + 0.25 * g.standard_normal((3, dq))).astype(np.float32)
+            beta = (0.25 * g.standard_normal((3, dq))).astype(np.float32)
+        else:
+            rms_w = np.ones(d_model, np.float32)
+            gamma = np.ones((3, dq), np.float32)
+            beta = np.zeros((3, dq), np.float32)
+        out.append(LayerWeights(kind, rms_w, w_in, w_kv, w_o, gamma, beta))
+    return out
+
+
+def stack_input(batch: JaggedBatch, d_model: int, seed: int) -> np.ndarray:
+    """Token matrix X0 [sum N, d_model] ~ N(0, 1), bf16 bit patterns."""
+    return normal_bf16(seed, S_X0, (batch.total_tokens, d_model))

@@ -392,3 +392,78 @@ def target_bwd(batch, heads, inp, alpha=None, eps: float = GLN_EPS, users=None):
             dbeta += db
         dq[ts], dk[ks], dv[ks] = attention_user_bwd(q[ts], k[ks], v[ks], M, dA, hq, hkv, dh, alpha, N)
     return {"dq": dq, "dk": dk, "dv": dv, "du": dU, "dgamma": dgamma, "dbeta": dbeta}
+
+
+# ----------------------------------------------------------------------------
+# Backbone stack: layers of the form of [DY] §4.1 (Full) and §4.2 (Target),
+# interleaved 1 Full : 3 Target ([DY] §4.1 block structure; [MT] §3.3).
+# ----------------------------------------------------------------------------
+
+RMS_EPS = 1e-6
+
+
+def rmsnorm(X, w, eps: float = RMS_EPS):
+    """Pre-norm X~ = X / sqrt(mean_j X_ij^2 + eps) * w, row by row.
+
+    The pages call X~ "the normalised feature matrix" ([DY] §4.2) without naming
+    the norm; RMSNorm with eps = 1e-6 is the reading taken here.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    ms = (X * X).mean(axis=1, keepdims=True)
+    return X / np.sqrt(ms + eps) * np.asarray(w, dtype=np.float64)
+
+
+def t_row_index(batch) -> np.ndarray:
+    """Global row of every T token, in the Target layout order (user by user)."""
+    out = []
+    for u, LH, LR, LT, s0, _, _ in _users(batch):
+        out.append(np.arange(s0 + LH + LR, s0 + LH + LR + LT))
+    return np.concatenate(out) if out else np.zeros(0, np.int64)
+
+
+class _Proj:
+    """Attention inputs handed to full_fwd / target_fwd (float64 arrays)."""
+
+    def __init__(self, q, k, v, u, gamma, beta):
+        self.q, self.k, self.v, self.u, self.gamma, self.beta = q, k, v, u, gamma, beta
+
+
+def full_layer(batch, heads, X, lw, alpha=None):
+    """X' = f2(GLN(A) o U) + X with U, Q, K, V = Split(SiLU(f1(RMSNorm(X)))) ([DY] §4.1).
+
+    f1 = X~ W_in^T, W_in = [W_u; W_q; W_k; W_v] (heads contiguous inside each
+    part); phi_1 = SiLU; f2 = Y W_o^T; no biases.  X: [sum N, d_model] float64.
+    """
+    dq, dkv = heads.dq, heads.dkv
+    Xn = rmsnorm(X, lw.rms_w)
+    Z = silu(Xn @ _f64(lw.w_in).T)
+    U, Q, K, V = Z[:, :dq], Z[:, dq:2 * dq], Z[:, 2 * dq:2 * dq + dkv], Z[:, 2 * dq + dkv:]
+    out = full_fwd(batch, heads, _Proj(Q, K, V, U, _f64(lw.gamma), _f64(lw.beta)), alpha)
+    return X + out["Y"] @ _f64(lw.w_o).T
+
+
+def target_layer(batch, heads, X, lw, alpha=None):
+    """Target-Attention layer ([DY] §4.2): U_T, Q_T = Split(SiLU(X~_T W_uq^T)),
+    K, V = Split(SiLU(X~ W_kv^T)); only T rows are updated,
+    X'_T = f2(GLN(A_T) o U_T) + X_T, and the H / R rows pass through unchanged."""
+    dq, dkv = heads.dq, heads.dkv
+    Xn = rmsnorm(X, lw.rms_w)
+    trow = t_row_index(batch)
+    ZT = silu(Xn[trow] @ _f64(lw.w_in).T)
+    Zkv = silu(Xn @ _f64(lw.w_kv).T)
+    inp = _Proj(ZT[:, dq:], Zkv[:, :dkv], Zkv[:, dkv:], ZT[:, :dq], _f64(lw.gamma), _f64(lw.beta))
+    out = target_fwd(batch, heads, inp, alpha)
+    Xo = np.array(X, dtype=np.float64, copy=True)
+    Xo[trow] = Xo[trow] + out["Y"] @ _f64(lw.w_o).T
+    return Xo
+
+
+def stack_fwd(batch, heads, weights, X0, alpha=None, record: bool = False):
+    """Run the layers in order (kind "F" = Full, "T" = Target).  Returns X_L, or
+    the list [X_0, ..., X_L] when ``record``."""
+    X = _f64(X0)
+    xs = [X]
+    for lw in weights:
+        X = (full_layer if lw.kind == "F" else target_layer)(batch, heads, X, lw, alpha)
+        xs.append(X)
+    return xs if record else X

@@ -7,6 +7,7 @@ import numpy as np
 import pytest
 
 import oracle_pins as P
+import stack_pins as S
 from oracle import mtfm_oracle as O
 
 
@@ -106,6 +107,58 @@ def _gate_bwd_no_mean_term(A, U, types, gamma, beta, dY, eps=O.GLN_EPS):
     return rstd[:, None] * dz, dU, dg, db
 
 
+def _rms_no_sqrt(X, w, eps=O.RMS_EPS):
+    X = np.asarray(X, dtype=np.float64)
+    return X / ((X * X).mean(axis=1, keepdims=True) + eps) * w
+
+
+def _rms_no_weight(X, w, eps=O.RMS_EPS):
+    return O.rmsnorm.__wrapped__(X, np.ones_like(np.asarray(w, dtype=np.float64)), eps)
+
+
+def _full_layer_variant(phi1=True, split_q_first=False, residual=True, gln=True, w_o_t=False):
+    def layer(batch, heads, X, lw, alpha=None):
+        dq, dkv = heads.dq, heads.dkv
+        Xn = O.rmsnorm(X, lw.rms_w)
+        Z = Xn @ O._f64(lw.w_in).T
+        if phi1:
+            Z = O.silu(Z)
+        U, Q = Z[:, :dq], Z[:, dq:2 * dq]
+        if split_q_first:
+            U, Q = Q, U
+        K, V = Z[:, 2 * dq:2 * dq + dkv], Z[:, 2 * dq + dkv:]
+        g = O._f64(lw.gamma) if gln else None
+        out = O.full_fwd(batch, heads, O._Proj(Q, K, V, U, g, O._f64(lw.beta)), alpha)
+        Wo = O._f64(lw.w_o)
+        upd = out["Y"] @ (Wo if w_o_t else Wo.T)
+        return X + upd if residual else upd
+    return layer
+
+
+def _target_layer_kv_from_t_rows(batch, heads, X, lw, alpha=None):
+    dq, dkv = heads.dq, heads.dkv
+    Xn = O.rmsnorm(X, lw.rms_w)
+    trow = O.t_row_index(batch)
+    ZT = O.silu(Xn[trow] @ O._f64(lw.w_in).T)
+    Xk = np.zeros_like(Xn)
+    Xk[trow] = Xn[trow]                     # keys and values from T rows only
+    Zkv = O.silu(Xk @ O._f64(lw.w_kv).T)
+    inp = O._Proj(ZT[:, dq:], Zkv[:, :dkv], Zkv[:, dkv:], ZT[:, :dq], O._f64(lw.gamma), O._f64(lw.beta))
+    out = O.target_fwd(batch, heads, inp, alpha)
+    Xo = np.array(X, dtype=np.float64, copy=True)
+    Xo[trow] = Xo[trow] + out["Y"] @ O._f64(lw.w_o).T
+    return Xo
+
+
+def _target_layer_updates_all_rows(batch, heads, X, lw, alpha=None):
+    Xo = O.target_layer.__wrapped__(batch, heads, X, lw, alpha)
+    return Xo + 1e-3 * O.rmsnorm(X, lw.rms_w)
+
+
+def _t_rows_shifted(batch):
+    return O.t_row_index.__wrapped__(batch) - 1
+
+
 MUTATIONS = {
     "t_rows_do_not_see_self": ("dense_mask_fast", _mask_no_self_t),
     "tie_visible": ("dense_mask_fast", _mask_fast_ties_visible),
@@ -121,6 +174,16 @@ MUTATIONS = {
     "bwd_wrong_sign": ("attention_user_bwd", _bwd_sign),
     "bwd_dk_rows_reversed": ("attention_user_bwd", _bwd_dk_transposed),
     "gate_bwd_dropped_mean_terms": ("gate_bwd", _gate_bwd_no_mean_term),
+    "rmsnorm_no_sqrt": ("rmsnorm", _rms_no_sqrt),
+    "rmsnorm_ignores_weight": ("rmsnorm", _rms_no_weight),
+    "stack_phi1_dropped": ("full_layer", _full_layer_variant(phi1=False)),
+    "stack_u_q_swapped": ("full_layer", _full_layer_variant(split_q_first=True)),
+    "stack_residual_dropped": ("full_layer", _full_layer_variant(residual=False)),
+    "stack_gate_without_gln": ("full_layer", _full_layer_variant(gln=False)),
+    "stack_w_o_transposed": ("full_layer", _full_layer_variant(w_o_t=True)),
+    "target_kv_from_t_rows": ("target_layer", _target_layer_kv_from_t_rows),
+    "target_updates_hr_rows": ("target_layer", _target_layer_updates_all_rows),
+    "t_rows_shifted": ("t_row_index", _t_rows_shifted),
 }
 
 
@@ -136,7 +199,7 @@ def test_pins_catch_mutation(name, monkeypatch):
     fn.__wrapped__ = orig
     monkeypatch.setattr(O, attr, fn)
     caught = []
-    for check in P.ALL_CHECKS:
+    for check in P.ALL_CHECKS + S.STACK_CHECKS:
         try:
             check()
         except AssertionError:
