@@ -9,7 +9,7 @@
 // with "visible" = the row's key prefix [0, kv_end) plus, for T rows, the
 // sibling block (itself, or the 4 sub-tokens of its target in V2).
 //
-// Persistent CTAs (one per SM) stride over work units x KV groups.  A Full-layer
+// Persistent CTAs (one per SM) take work units x KV groups from a counter.  A Full-layer
 // unit is one work item (user, 128-row query tile) with all its key blocks; a
 // Target-layer unit is a chunk of kTargetUnitBlocks key blocks of one item (the
 // packer splits each Target tile's key range so that short Target layers still
@@ -108,16 +108,22 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __shared__ __align__(8) uint64_t bar_s_full[kSBuf], bar_p_full[kSBuf];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ int s_ticket[2];  // this unit's and the next unit's (unit, group) index
 
   const MetaView& m = p.m;
   MetaHeader* hdr = m.hdr;
   if (hdr->error) return;
   // Work units: Full layer = one work item (all its key blocks); Target layer =
   // one chunk of kTargetUnitBlocks key blocks of a work item.  Each unit runs
-  // for every KV group; the CTAs stride over (unit, group) pairs.
+  // for every KV group.  The CTAs take (unit, group) pairs from a counter in the
+  // metadata header, in work-list order (longest users first), so that a CTA
+  // that finishes early takes the next pair: greedy list scheduling.
   const int n_units = TARGET ? hdr->n_units_target : hdr->n_items_full;
   const int n_work = n_units * p.hkv;
   if ((int)blockIdx.x >= n_work) return;
+  const int participants = min((int)gridDim.x, n_work);
+  uint32_t* ticket_ctr = &hdr->sched[TARGET ? 2 : 0];
+  uint32_t* done_ctr = &hdr->sched[TARGET ? 3 : 1];
   const int ldq = p.hq * kDH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -134,6 +140,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (threadIdx.x == 0) {
     s_abort = 0;
+    s_ticket[0] = (int)atomicAdd(ticket_ctr, 1u);
     mbar_init(b_q, 1);
     mbar_init(b_o, 1);
     mbar_init(b_drain, 1);
@@ -165,7 +172,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // Barrier phases run on across units: K/V stages count key blocks, S/P
   // buffers count steps, Q and O count units, all from the start of the CTA.
   int blk_base = 0, step_base = 0, unit_iter = 0;
-  for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
+  for (;;) {
+    const int w = s_ticket[unit_iter & 1];  // written before the last block-wide barrier
+    if (w >= n_work) break;
     const int unit = w / p.hkv, g = w % p.hkv;
     int item = unit, chunk = 0;
     if (TARGET) {  // last item whose first unit is <= unit
@@ -209,6 +218,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
           ++issued;
         }
+        // the next pair, read by every role after this unit's closing barrier
+        s_ticket[(unit_iter + 1) & 1] = (int)atomicAdd(ticket_ctr, 1u);
         // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
         // no TMA write may land after this unit's barriers are re-armed or the CTA leaves.
         const long long t0 = clock64();
@@ -381,7 +392,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && s_abort) atomicOr(&hdr->error, kErrTimeout);
+  if (threadIdx.x == 0) {
+    if (s_abort) atomicOr(&hdr->error, kErrTimeout);
+    // Every CTA has drawn its last ticket before it counts itself finished, so the
+    // last one to finish may rewind both counters for the next launch on this block.
+    __threadfence();
+    if (atomicAdd(done_ctr, 1u) == (uint32_t)participants - 1) {
+      atomicExch(ticket_ctr, 0u);
+      atomicExch(done_ctr, 0u);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side

@@ -58,15 +58,16 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
-// Same split with a truncated hi part: hi takes the upper 16 bits of each float
-// (one byte permute for the pair), lo = bf16(x - hi) with x - hi exact in fp32.
-// |x - hi| < 2^-7 |x|, so hi + lo carries x to within 2^-15 relative.
+// Split by truncation, integer and fp32-add work only (no conversion
+// instruction): hi = the upper 16 bits of each float (one byte permute for the
+// pair); r = x - hi is exact in fp32 with |r| < 2^-7 |x|; lo = the upper 16 bits
+// of r.  hi + lo carries x to within 2^-14 relative.
 __device__ __forceinline__ void split_trunc_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
   hi = __byte_perm(b0, b1, 0x7632);
   const float r0 = x0 - __uint_as_float(b0 & 0xffff0000u);
   const float r1 = x1 - __uint_as_float(b1 & 0xffff0000u);
-  lo = pack_bf16x2(r0, r1);
+  lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
 }
 
 // Visibility bits of the 32 keys [j, j + 32) for a row that sees the prefix

@@ -33,7 +33,10 @@ struct MetaHeader {
   int32_t max_items_full;
   int32_t max_items_target;
   int32_t n_units_target;  // key-range chunks of the Target work list (sum of unit_count)
-  int32_t pad[4];
+  // Work counters of the persistent forward kernels: [0] next Full unit, [1] Full CTAs
+  // finished, [2] next Target unit, [3] Target CTAs finished.  Zeroed by the packer; the
+  // last CTA of a launch to finish sets its pair back to zero for the next launch.
+  uint32_t sched[4];
 };
 
 // One work item: a 128-row query tile of one user and the range of prefix

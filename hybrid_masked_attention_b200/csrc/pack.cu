@@ -102,6 +102,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->max_items_full = max_if;
       m.hdr->max_items_target = max_it;
       m.hdr->n_units_target = 0;
+      for (int i = 0; i < 4; ++i) m.hdr->sched[i] = 0;
     }
     return;
   }
@@ -188,6 +189,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->max_items_full = max_if;
     m.hdr->max_items_target = max_it;
     m.hdr->n_units_target = 0;
+    for (int i = 0; i < 4; ++i) m.hdr->sched[i] = 0;
   }
 }
 

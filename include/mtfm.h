@@ -42,6 +42,12 @@
  *     not add up to the totals, unsorted timestamps) are recorded in the
  *     metadata block; every later kernel that reads that block does nothing,
  *     and mtfm_pack_check() reports them.
+ *   - The metadata block is read-only for every call but mtfm_pack, except
+ *     for 16 bytes of work counters in its header: the persistent forward
+ *     attention kernels draw their work from them and set them back to zero
+ *     when they finish.  Hence two Full-layer (or two Target-layer) forward
+ *     calls on one metadata block must be ordered (same stream, or an event);
+ *     a Full and a Target call may overlap, and so may calls on different blocks.
  *   - Supported: head_dim in {32, 64, 128}; hq % hkv == 0; hq/hkv <= 8;
  *     hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).

@@ -65,3 +65,31 @@ def test_fwd_deterministic(cuda_ok):
     y2, a2, _ = s.full_fwd(inp["q"], inp["k"], inp["v"], inp["u"], inp["gamma"], inp["beta"])
     torch.cuda.synchronize()
     assert torch.equal(y1, y2) and torch.equal(a1, a2)
+
+
+def test_work_counters_rewind(cuda_ok):
+    """The persistent forward kernels draw work from counters in the metadata
+    header and set them back to zero: repeated and interleaved Full / Target
+    calls on one block all cover every tile."""
+    b, hd = BATCHES["pair"](), HEADS["pair"]
+    s = packed(b, hd)
+    full = upload_layer(syn.layer_inputs(b, hd, target=False, seed=5))
+    tgt = upload_layer(syn.layer_inputs(b, hd, target=True, seed=6))
+    outs = []
+    for _ in range(3):
+        outs.append((s.full_fwd(full["q"], full["k"], full["v"], full["u"], full["gamma"], full["beta"]),
+                     s.target_fwd(tgt["q"], tgt["k"], tgt["v"], tgt["u"], tgt["gamma"], tgt["beta"])))
+    torch.cuda.synchronize()
+    hdr = s.meta[:64].view(torch.int32).cpu().numpy()
+    assert hdr[8] == 0, "error flag"
+    assert (hdr[12:16] == 0).all(), f"work counters not rewound: {hdr[12:16]}"
+    (yf0, af0, _), (yt0, at0, _) = outs[0]
+    for (yf, af, _), (yt, at, _) in outs[1:]:
+        assert torch.equal(af, af0) and torch.equal(yf, yf0)
+        # Target A sums key-range partials with atomics: equal up to summation order
+        assert_close(at.cpu().numpy(), at0.cpu().numpy(), "A_T repeat")
+    ref_f = O.full_fwd(b, hd, syn.layer_inputs(b, hd, target=False, seed=5))
+    ref_t = O.target_fwd(b, hd, syn.layer_inputs(b, hd, target=True, seed=6))
+    for (yf, af, _), (yt, at, _) in outs:
+        assert_close(af.cpu().numpy(), ref_f["A"], "A full")
+        assert_close(at.cpu().numpy(), ref_t["A"], "A target")
