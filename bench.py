@@ -544,6 +544,100 @@ def run_extra(args):
     print(json.dumps(out), flush=True)
 
 
+def run_stack(args):
+    """The 16-layer backbone stack (4 x (Full, Target, Target, Target)) forward on --users
+    users (default 64) of the production-shape distributions, d_model 512, Hq 8 / Hkv 2,
+    head_dim 64; seeded device-side weights N(0, 0.02), output projections N(0, 0.005),
+    X ~ N(0, 1) rounded to bf16.  One JSON line: the stack's time, users/s, and the
+    unmasked attention FLOP plus projection GEMM FLOP rates, with per-layer timings."""
+    import torch
+    import hybrid_masked_attention_b200 as M
+    dev = torch.device("cuda", 0)
+    heads, d = syn.PAIR_HEADS, 512
+    B = args.users if args.users is not None else 64
+    b = syn.pair_batch(B, seed=1002)
+    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh, 1)
+    meta = M.alloc_meta(cfg, dev)
+    it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
+    M.pack(cfg, it(b.L_H, np.int32), it(b.L_R, np.int32), it(b.L_T, np.int32), it(b.r_ts, np.int64),
+           it(b.t_exp, np.int64), meta)
+    M.pack_check(meta)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1002)
+    rnd = lambda std, *shape: (std * torch.randn(*shape, generator=gen, device=dev)).to(torch.bfloat16)
+    N, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
+    kinds = syn.STACK_KINDS
+    layers = []
+    for k in kinds:
+        w_in = rnd(0.02, 2 * D + 2 * Dkv, d) if k == "F" else rnd(0.02, 2 * D, d)
+        w_kv = rnd(0.02, 2 * Dkv, d) if k == "T" else None
+        layers.append(M.LayerWeights(k, torch.ones(d, device=dev), w_in, w_kv,
+                                     rnd(0.02 / np.sqrt(len(kinds)), d, D),
+                                     torch.ones(3, D, device=dev), torch.zeros(3, D, device=dev)))
+    x = rnd(1.0, N, d).float()
+    ws = torch.empty(M.stack_workspace_bytes(cfg, d), dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    res = {}
+
+    def timed(label, fn, steps):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a, z = ev(), ev()
+        a.record()
+        for _ in range(steps):
+            fn()
+        z.record()
+        torch.cuda.synchronize()
+        res[label] = a.elapsed_time(z) / steps
+
+    steps = max(1, args.steps)
+    clocks = ClockSampler(0)
+    timed("stack", lambda: M.stack_fwd(cfg, meta, d, layers, x, ws), steps)
+    clk = clocks.stop()
+    timed("full_layer", lambda: M.layer_fwd(cfg, meta, d, layers[0], x, ws), steps)
+    timed("target_layer", lambda: M.layer_fwd(cfg, meta, d, layers[1], x, ws), steps)
+    q, kk, vv = rnd(1.0, N, D), rnd(1.0, N, Dkv), rnd(1.0, N, Dkv)
+    a_buf = torch.empty(N, D, device=dev)
+    timed("full_attn", lambda: M.attn_full(cfg, meta, q, kk, vv, a_buf), steps)
+    timed("target_attn", lambda: M.attn_target(cfg, meta, q[:T], kk, vv, a_buf[:T]), steps)
+    M.pack_check(meta)
+    assert torch.isfinite(x).all().item()
+    peaks, src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops"]))
+    ff, ft = attn_flops(b, heads, False), attn_flops(b, heads, True)
+    g_full = 2.0 * N * d * (2 * D + 2 * Dkv) + 2.0 * N * D * d
+    g_tgt = 2.0 * T * d * 2 * D + 2.0 * N * d * 2 * Dkv + 2.0 * T * D * d
+    n_f = sum(k == "F" for k in kinds)
+    n_t = len(kinds) - n_f
+    attn_fl = n_f * ff + n_t * ft
+    gemm_fl = n_f * g_full + n_t * g_tgt
+    tf = lambda fl, ms: fl / (ms * 1e-3) / 1e12
+    ms = res["stack"]
+    out = {"metric": METRIC, "value": round(tf(attn_fl + gemm_fl, ms), 3), "unit": "TFLOP/s",
+           "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
+           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"16-layer backbone stack, 4 x (Full, Target, Target, Target): {b.B} users, "
+                                  f"production-shape lengths, d_model {d}, Hq 8 / Hkv 2, head_dim 64",
+                      "users": b.B, "total_tokens": N, "total_t": T, "attn_flops": attn_fl,
+                      "gemm_flops": gemm_fl,
+                      "l2": "per-layer working set (X fp32 + scratch) larger than the 126 MB L2",
+                      "peak": f"{src} bf16 sustained {peak_tf} TF/s"},
+           "users_per_s": round(b.B / (ms * 1e-3), 1),
+           "per_layer_users_per_s": round(b.B * len(kinds) / (ms * 1e-3), 1),
+           "per_kernel": {
+               "full_layer": {"ms": round(res["full_layer"], 5),
+                              "tflops": round(tf(ff + g_full, res["full_layer"]), 2)},
+               "target_layer": {"ms": round(res["target_layer"], 5),
+                                "tflops": round(tf(ft + g_tgt, res["target_layer"]), 2)},
+               "full_attn": {"ms": round(res["full_attn"], 5), "tflops": round(tf(ff, res["full_attn"]), 2)},
+               "target_attn": {"ms": round(res["target_attn"], 5), "tflops": round(tf(ft, res["target_attn"]), 2)},
+               "full_gemm_and_rest_ms": round(res["full_layer"] - res["full_attn"], 5),
+               "target_gemm_and_rest_ms": round(res["target_layer"] - res["target_attn"], 5)},
+           "clocks": clk}
+    print(json.dumps(out), flush=True)
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -552,12 +646,12 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["mtfm", "reference"], default="mtfm")
-    ap.add_argument("--users", type=int, default=32)
+    ap.add_argument("--users", type=int, default=None, help="users (default 32; 64 for --workload stack)")
     ap.add_argument("--sets", type=int, default=4, help="resident input copies rotated across steps")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["pair", "sweep", "train"], default="pair",
-                    help="pair: the headline step; sweep/train: per-kernel timings of the other configs")
+    ap.add_argument("--workload", choices=["pair", "sweep", "train", "stack"], default="pair",
+                    help="pair: the headline step; sweep/train/stack: timings of the other configs")
     ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
     ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")
     args = ap.parse_args()
@@ -570,6 +664,11 @@ def main():
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
 
+    if args.workload == "stack":
+        run_stack(args)
+        return
+    if args.users is None:
+        args.users = 32
     if args.workload != "pair":
         run_extra(args)
         return

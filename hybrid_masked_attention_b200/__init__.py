@@ -8,7 +8,8 @@ this import fails; build it with ``python hybrid_masked_attention_b200/build.py`
 Function names mirror the C entry points:
     meta_bytes, max_items, pack, pack_check, meta_read,
     attn_full_fwd, attn_target_fwd, attn_full, attn_target, gate_fwd,
-    bwd_workspace_bytes, attn_full_bwd, attn_target_bwd
+    bwd_workspace_bytes, attn_full_bwd, attn_target_bwd, attn_target_bwd_static,
+    stack_workspace_bytes, layer_fwd, stack_fwd
 """
 from __future__ import annotations
 
@@ -85,8 +86,14 @@ class Config:
         return self.alpha if self.alpha > 0 else 1.0 / math.sqrt(self.head_dim)
 
 
+class CLayerWeights(ctypes.Structure):
+    _fields_ = [("rms_w", ctypes.c_void_p), ("w_in", ctypes.c_void_p), ("w_kv", ctypes.c_void_p),
+                ("w_o", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _CP = ctypes.POINTER(CCfg)
+_LWP = ctypes.POINTER(CLayerWeights)
 _sigs = {
     "mtfm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mtfm_meta_bytes": (ctypes.c_size_t, [_CP]),
@@ -103,6 +110,10 @@ _sigs = {
     "mtfm_attn_full_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
     "mtfm_attn_target_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
     "mtfm_attn_target_bwd_static": (ctypes.c_int, [_CP] + [_P] * 17),
+    "mtfm_stack_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int32]),
+    "mtfm_layer_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int, _LWP, _P, _P, ctypes.c_size_t, _P]),
+    "mtfm_stack_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_char_p, _LWP, _P, _P,
+                                      ctypes.c_size_t, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -316,3 +327,72 @@ def attn_target_bwd_static(cfg, meta, q, k, v, u, gamma, beta, a, stats, dy, dq,
         _ptr(dv, f32, (N, Dkv), "dv"), _ptr(du, f32, (rows, D), "du"),
         _ptr(dgamma, f32, (3, D), "dgamma"), _ptr(dbeta, f32, (3, D), "dbeta"), _stream(stream))
     _check(st, "mtfm_attn_target_bwd_static")
+
+
+# ---------------------------------------------------------------------------- backbone stack
+
+@dataclass
+class LayerWeights:
+    """Device tensors of one backbone layer (see ``mtfm_layer_weights`` in mtfm.h).
+
+    rms_w fp32 [d_model]; w_in bf16 [out, d_model]; w_kv bf16 [2*Dkv, d_model] for a
+    Target layer (None for Full); w_o bf16 [d_model, D]; gamma, beta fp32 [3, D] or None.
+    """
+    kind: str
+    rms_w: torch.Tensor
+    w_in: torch.Tensor
+    w_kv: Optional[torch.Tensor]
+    w_o: torch.Tensor
+    gamma: Optional[torch.Tensor] = None
+    beta: Optional[torch.Tensor] = None
+
+
+def _layer_struct(cfg: Config, d_model: int, w: LayerWeights) -> CLayerWeights:
+    D, Dkv = cfg.D, cfg.Dkv
+    target = w.kind == "T"
+    out = 2 * D if target else 2 * D + 2 * Dkv
+    if w.kind not in ("F", "T"):
+        raise ValueError("layer kind must be 'F' or 'T'")
+    if target != (w.w_kv is not None):
+        raise ValueError("w_kv is required for a Target layer and must be None for a Full layer")
+    return CLayerWeights(
+        _ptr(w.rms_w, torch.float32, (d_model,), "rms_w"),
+        _ptr(w.w_in, torch.bfloat16, (out, d_model), "w_in"),
+        _ptr(w.w_kv, torch.bfloat16, (2 * Dkv, d_model), "w_kv"),
+        _ptr(w.w_o, torch.bfloat16, (d_model, D), "w_o"),
+        _ptr(w.gamma, torch.float32, (3, D), "gamma"),
+        _ptr(w.beta, torch.float32, (3, D), "beta"))
+
+
+def stack_workspace_bytes(cfg: Config, d_model: int) -> int:
+    c = cfg.c()
+    n = _lib.mtfm_stack_workspace_bytes(ctypes.byref(c), int(d_model))
+    if n == 0:
+        raise MtfmError(3, "mtfm_stack_workspace_bytes")
+    return n
+
+
+def layer_fwd(cfg: Config, meta: torch.Tensor, d_model: int, w: LayerWeights, x: torch.Tensor,
+              ws: torch.Tensor, stream=None):
+    """One backbone layer on X (fp32 [total_tokens, d_model], updated in place)."""
+    c = cfg.c()
+    lw = _layer_struct(cfg, d_model, w)
+    _check(_lib.mtfm_layer_fwd(ctypes.byref(c), _ptr(meta, torch.uint8, name="meta"), int(d_model),
+                               int(w.kind == "T"), ctypes.byref(lw),
+                               _ptr(x, torch.float32, (cfg.total_tokens, d_model), "x"),
+                               _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream)),
+           "mtfm_layer_fwd")
+
+
+def stack_fwd(cfg: Config, meta: torch.Tensor, d_model: int, layers, x: torch.Tensor, ws: torch.Tensor,
+              stream=None):
+    """Run ``layers`` (a list of LayerWeights) on X in place."""
+    c = cfg.c()
+    arr = (CLayerWeights * max(1, len(layers)))(*[_layer_struct(cfg, d_model, w) for w in layers])
+    kinds = "".join(w.kind for w in layers).encode()
+    _check(_lib.mtfm_stack_fwd(ctypes.byref(c), _ptr(meta, torch.uint8, name="meta"), int(d_model),
+                               len(layers), kinds, arr,
+                               _ptr(x, torch.float32, (cfg.total_tokens, d_model), "x"),
+                               _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream)),
+           "mtfm_stack_fwd")
+

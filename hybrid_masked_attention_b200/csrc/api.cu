@@ -55,6 +55,22 @@ mtfm_status check_meta(const void* d_meta, const Resolved& r) {
   return MTFM_OK;
 }
 
+// tcgen05/TMEM kernel where its TMEM plan fits (head_dim 64, r in {1, 2, 4});
+// the mma.sync kernel covers the other head shapes.  MTFM_FWD_KERNEL=mma
+// selects the mma.sync kernel for every shape (for comparisons).
+cudaError_t launch_attn(const Resolved& r, const MetaView& m, const MetaLayout& L, bool target,
+                        const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                        float* a, cudaStream_t st) {
+  AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
+  const int max_items = target ? L.max_items_target : L.max_items_full;
+  const int rows = target ? r.total_t : r.total_tokens;
+  const char* force = getenv("MTFM_FWD_KERNEL");
+  const bool force_mma = force && strcmp(force, "mma") == 0;
+  if (!force_mma && attn_fwd_tc_supported(shape))
+    return launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
+  return launch_attn_fwd_mma(shape, m, max_items, q, k, v, a, st);
+}
+
 // Attention only: A (fp32) for the Full or Target layout.
 mtfm_status attn_only(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
                       const uint16_t* d_k, const uint16_t* d_v, float* d_a, void* stream,
@@ -71,20 +87,10 @@ mtfm_status attn_only(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d
     return MTFM_ERR_INVALID_ARG;
   const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
   const MetaView m = meta_view(const_cast<void*>(d_meta), L);
-  AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
-  const int max_items = target ? L.max_items_target : L.max_items_full;
-  const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(d_q);
-  const __nv_bfloat16* k = reinterpret_cast<const __nv_bfloat16*>(d_k);
-  const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(d_v);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // tcgen05/TMEM kernel where its TMEM plan fits (head_dim 64, r in {1, 2, 4});
-  // the mma.sync kernel covers the other head shapes.  MTFM_FWD_KERNEL=mma
-  // selects the mma.sync kernel for every shape (for comparisons).
-  const char* force = getenv("MTFM_FWD_KERNEL");
-  const bool force_mma = force && strcmp(force, "mma") == 0;
-  if (!force_mma && attn_fwd_tc_supported(shape))
-    return cuda_status(launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, d_a, st));
-  return cuda_status(launch_attn_fwd_mma(shape, m, max_items, q, k, v, d_a, st));
+  return cuda_status(launch_attn(r, m, L, target, reinterpret_cast<const __nv_bfloat16*>(d_q),
+                                 reinterpret_cast<const __nv_bfloat16*>(d_k),
+                                 reinterpret_cast<const __nv_bfloat16*>(d_v), d_a,
+                                 static_cast<cudaStream_t>(stream)));
 }
 
 mtfm_status gate_fwd(const mtfm_cfg* cfg, const void* d_meta, bool target, const float* d_a,
@@ -193,6 +199,116 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
                           reinterpret_cast<const __nv_bfloat16*>(d_v), da_hi, da_lo, d_dq, d_dk,
                           d_dv, st);
   return cuda_status(e);
+}
+
+
+// ------------------------------------------------------------------ backbone stack
+// Scratch of one layer, reused by every layer of a stack: X~ (all rows) and
+// X~_T (T rows) in bf16; U, Q (rows of the layer's queries), K, V in bf16; A in
+// fp32; Y in bf16; GLN row statistics.
+struct StackWs {
+  size_t xn, xnt, u, q, k, v, a, y, stats, total;
+};
+StackWs stack_ws(const Resolved& r, int d) {
+  StackWs w;
+  const size_t N = (size_t)r.total_tokens, T = (size_t)r.total_t;
+  size_t o = 0;
+  w.xn = o;    o = align256(o + N * d * 2);
+  w.xnt = o;   o = align256(o + T * d * 2);
+  w.u = o;     o = align256(o + N * r.D * 2);
+  w.q = o;     o = align256(o + N * r.D * 2);
+  w.k = o;     o = align256(o + N * r.Dkv * 2);
+  w.v = o;     o = align256(o + N * r.Dkv * 2);
+  w.a = o;     o = align256(o + N * r.D * 4);
+  w.y = o;     o = align256(o + N * r.D * 2);
+  w.stats = o; o = align256(o + N * 2 * 4);
+  w.total = o;
+  return w;
+}
+
+// Shapes the stack kernels take: d_model and hq*head_dim multiples of 64
+// (GEMM tiles), d_model <= 1024 (RMSNorm keeps a row in registers).
+mtfm_status check_stack_cfg(const Resolved& r, int d) {
+  if (d <= 0 || d % 64 != 0) return MTFM_ERR_INVALID_ARG;
+  if (d > 1024 || r.D % 64 != 0) return MTFM_ERR_UNSUPPORTED;
+  return MTFM_OK;
+}
+
+mtfm_status check_layer_weights(const Resolved& r, const mtfm_layer_weights* w, bool target) {
+  if (!w || !w->rms_w || !w->w_in || !w->w_o) return MTFM_ERR_INVALID_ARG;
+  if (target != (w->w_kv != nullptr)) return MTFM_ERR_INVALID_ARG;
+  if ((w->gamma == nullptr) != (w->beta == nullptr)) return MTFM_ERR_INVALID_ARG;
+  if (!aligned16(w->rms_w) || !aligned16(w->w_in) || !aligned16(w->w_o) ||
+      (w->w_kv && !aligned16(w->w_kv)) || (w->gamma && (!aligned16(w->gamma) || !aligned16(w->beta))))
+    return MTFM_ERR_INVALID_ARG;
+  return MTFM_OK;
+}
+
+// One layer, all launches on `st`; arguments already checked.
+cudaError_t layer_fwd(const Resolved& r, const MetaView& m, const MetaLayout& L, int d, bool target,
+                      const mtfm_layer_weights& w, float* x, char* ws, const StackWs& W,
+                      cudaStream_t st) {
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  auto wt = [](const uint16_t* p) { return reinterpret_cast<const __nv_bfloat16*>(p); };
+  const int N = r.total_tokens, T = r.total_t, D = r.D, Dkv = r.Dkv;
+  const int rows_q = target ? T : N;
+  cudaError_t e;
+  // X~ = RMSNorm(X) for every row (K, V read all rows); X~_T gathered for a Target layer
+  if ((e = launch_rmsnorm(m.hdr, x, N, d, nullptr, w.rms_w, kRmsEps, bf(W.xn), st)) != cudaSuccess) return e;
+  if (target && (e = launch_rmsnorm(m.hdr, x, T, d, m.t_rows, w.rms_w, kRmsEps, bf(W.xnt), st)) != cudaSuccess)
+    return e;
+  if (!target) {
+    // [U Q K V] = SiLU(X~ W_uqkv^T)
+    GemmEpi g{kEpiSiluSplit, 4, {0, D, 2 * D, 2 * D + Dkv, 2 * D + 2 * Dkv},
+              {bf(W.u), bf(W.q), bf(W.k), bf(W.v)}, {D, D, Dkv, Dkv}, nullptr, 0, nullptr};
+    if ((e = launch_gemm_tc(m.hdr, bf(W.xn), d, wt(w.w_in), N, 2 * D + 2 * Dkv, d, g, st)) != cudaSuccess)
+      return e;
+  } else {
+    // [U Q]_T = SiLU(X~_T W_uq^T), [K V] = SiLU(X~ W_kv^T)
+    GemmEpi guq{kEpiSiluSplit, 2, {0, D, 2 * D, 0, 0}, {bf(W.u), bf(W.q), nullptr, nullptr}, {D, D, 0, 0},
+                nullptr, 0, nullptr};
+    if ((e = launch_gemm_tc(m.hdr, bf(W.xnt), d, wt(w.w_in), T, 2 * D, d, guq, st)) != cudaSuccess) return e;
+    GemmEpi gkv{kEpiSiluSplit, 2, {0, Dkv, 2 * Dkv, 0, 0}, {bf(W.k), bf(W.v), nullptr, nullptr},
+                {Dkv, Dkv, 0, 0}, nullptr, 0, nullptr};
+    if ((e = launch_gemm_tc(m.hdr, bf(W.xn), d, wt(w.w_kv), N, 2 * Dkv, d, gkv, st)) != cudaSuccess) return e;
+  }
+  float* a = reinterpret_cast<float*>(ws + W.a);
+  if ((e = launch_attn(r, m, L, target, bf(W.q), bf(W.k), bf(W.v), a, st)) != cudaSuccess) return e;
+  if ((e = launch_gate_fwd_bf16(m, target, rows_q, D, r.eps, a, bf(W.u), w.gamma, w.beta, bf(W.y),
+                                reinterpret_cast<float*>(ws + W.stats), st)) != cudaSuccess)
+    return e;
+  // X (+)= Y W_o^T, scattered back to the T rows for a Target layer
+  GemmEpi go{kEpiResidual, 0, {0, 0, 0, 0, 0}, {nullptr, nullptr, nullptr, nullptr}, {0, 0, 0, 0}, x, d,
+             target ? m.t_rows : nullptr};
+  return launch_gemm_tc(m.hdr, bf(W.y), D, wt(w.w_o), rows_q, d, D, go, st);
+}
+
+mtfm_status stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int d, int n_layers, const char* kinds,
+                      const mtfm_layer_weights* layers, float* d_x, void* d_ws, size_t ws_bytes,
+                      void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  if ((s = check_stack_cfg(r, d)) != MTFM_OK) return s;
+  if (n_layers < 0 || (n_layers > 0 && (!kinds || !layers))) return MTFM_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    if (kinds[l] != 'F' && kinds[l] != 'T') return MTFM_ERR_INVALID_ARG;
+    if ((s = check_layer_weights(r, &layers[l], kinds[l] == 'T')) != MTFM_OK) return s;
+  }
+  if (n_layers == 0 || r.total_tokens == 0) return MTFM_OK;
+  const StackWs W = stack_ws(r, d);
+  if (!d_x || !aligned16(d_x)) return MTFM_ERR_INVALID_ARG;
+  if (!d_ws || (reinterpret_cast<uintptr_t>(d_ws) & 255u)) return MTFM_ERR_INVALID_ARG;
+  if (ws_bytes < W.total) return MTFM_ERR_WORKSPACE_TOO_SMALL;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  const MetaView m = meta_view(const_cast<void*>(d_meta), L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l = 0; l < n_layers; ++l) {
+    cudaError_t e = layer_fwd(r, m, L, d, kinds[l] == 'T', layers[l], d_x, static_cast<char*>(d_ws), W, st);
+    if (e != cudaSuccess) return MTFM_ERR_CUDA;
+  }
+  return MTFM_OK;
 }
 
 }  // namespace
@@ -346,6 +462,25 @@ mtfm_status mtfm_attn_target_bwd(const mtfm_cfg* cfg, const void* d_meta, const 
                                  float* d_dbeta, void* d_ws, size_t ws_bytes, void* stream) {
   return attn_bwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_a, d_stats, d_dy, d_dq,
                   d_dk, d_dv, d_du, d_dgamma, d_dbeta, d_ws, ws_bytes, stream, true);
+}
+
+size_t mtfm_stack_workspace_bytes(const mtfm_cfg* cfg, int32_t d_model) {
+  Resolved r;
+  if (resolve(cfg, &r) != MTFM_OK || check_stack_cfg(r, d_model) != MTFM_OK) return 0;
+  return stack_ws(r, d_model).total;
+}
+
+mtfm_status mtfm_layer_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_model, int is_target,
+                           const mtfm_layer_weights* weights, float* d_x, void* d_ws, size_t ws_bytes,
+                           void* stream) {
+  const char kind = is_target ? 'T' : 'F';
+  return stack_fwd(cfg, d_meta, d_model, 1, &kind, weights, d_x, d_ws, ws_bytes, stream);
+}
+
+mtfm_status mtfm_stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_model, int32_t n_layers,
+                           const char* kinds, const mtfm_layer_weights* layers, float* d_x, void* d_ws,
+                           size_t ws_bytes, void* stream) {
+  return stack_fwd(cfg, d_meta, d_model, n_layers, kinds, layers, d_x, d_ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -9,7 +9,8 @@
 // with "visible" = the row's key prefix [0, kv_end) plus, for T rows, the
 // sibling block (itself, or the 4 sub-tokens of its target in V2).
 //
-// Persistent CTAs (one per SM) take work units x KV groups from a counter.  A Full-layer
+// Persistent CTAs (one per SM) take work units x KV groups from a counter (Full)
+// or stride over them (Target).  A Full-layer
 // unit is one work item (user, 128-row query tile) with all its key blocks; a
 // Target-layer unit is a chunk of kTargetUnitBlocks key blocks of one item (the
 // packer splits each Target tile's key range so that short Target layers still
@@ -42,6 +43,7 @@
 #include "mtfm_internal.cuh"
 #include "mma_util.cuh"
 #include "sm100.cuh"
+#include "tma_host.cuh"
 
 namespace mtfm {
 namespace {
@@ -115,15 +117,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   if (hdr->error) return;
   // Work units: Full layer = one work item (all its key blocks); Target layer =
   // one chunk of kTargetUnitBlocks key blocks of a work item.  Each unit runs
-  // for every KV group.  The CTAs take (unit, group) pairs from a counter in the
-  // metadata header, in work-list order (longest users first), so that a CTA
-  // that finishes early takes the next pair: greedy list scheduling.
+  // for every KV group.  Full layer: the CTAs take (unit, group) pairs from a
+  // counter in the metadata header, in work-list order (longest users first), so
+  // that a CTA that finishes early takes the next pair (greedy list scheduling;
+  // unit costs vary with the user's length).  Target layer: units cost about the
+  // same, and the CTAs stride over the pairs (measured faster than the counter).
   const int n_units = TARGET ? hdr->n_units_target : hdr->n_items_full;
   const int n_work = n_units * p.hkv;
   if ((int)blockIdx.x >= n_work) return;
   const int participants = min((int)gridDim.x, n_work);
-  uint32_t* ticket_ctr = &hdr->sched[TARGET ? 2 : 0];
-  uint32_t* done_ctr = &hdr->sched[TARGET ? 3 : 1];
+  uint32_t* ticket_ctr = &hdr->sched[0];
+  uint32_t* done_ctr = &hdr->sched[1];
   const int ldq = p.hq * kDH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -140,7 +144,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    s_ticket[0] = (int)atomicAdd(ticket_ctr, 1u);
+    s_ticket[0] = TARGET ? (int)blockIdx.x : (int)atomicAdd(ticket_ctr, 1u);
     mbar_init(b_q, 1);
     mbar_init(b_o, 1);
     mbar_init(b_drain, 1);
@@ -219,7 +223,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           ++issued;
         }
         // the next pair, read by every role after this unit's closing barrier
-        s_ticket[(unit_iter + 1) & 1] = (int)atomicAdd(ticket_ctr, 1u);
+        s_ticket[(unit_iter + 1) & 1] = TARGET ? w + (int)gridDim.x : (int)atomicAdd(ticket_ctr, 1u);
         // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
         // no TMA write may land after this unit's barriers are re-armed or the CTA leaves.
         const long long t0 = clock64();
@@ -396,54 +400,20 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (s_abort) atomicOr(&hdr->error, kErrTimeout);
     // Every CTA has drawn its last ticket before it counts itself finished, so the
     // last one to finish may rewind both counters for the next launch on this block.
-    __threadfence();
-    if (atomicAdd(done_ctr, 1u) == (uint32_t)participants - 1) {
-      atomicExch(ticket_ctr, 0u);
-      atomicExch(done_ctr, 0u);
+    if (!TARGET) {
+      __threadfence();
+      if (atomicAdd(done_ctr, 1u) == (uint32_t)participants - 1) {
+        atomicExch(ticket_ctr, 0u);
+        atomicExch(done_ctr, 0u);
+      }
     }
   }
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 // Row-major bf16 matrix [rows, cols]; box_rows x 64 boxes with the 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kDH, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  }
-  return n;
+  return make_map_bf16(map, base, (uint64_t)rows, (uint64_t)cols, (uint64_t)cols, (uint32_t)box_rows, kDH);
 }
 
 // One CTA per SM (TMEM and shared memory allow no more); the CTAs stride over

@@ -44,11 +44,23 @@ __device__ __forceinline__ void store_split_bf16x4(__nv_bfloat16* hi_p, __nv_bfl
   *reinterpret_cast<uint2*>(lo_p) = rl;
 }
 
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 r;
+  r.x = *reinterpret_cast<uint32_t*>(&lo);
+  r.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p) = r;
+}
+
+// Y is fp32 for the layer entry points, bf16 (round to nearest) where Y feeds
+// the output projection of the backbone stack.
+template <typename OutT>
 __global__ void __launch_bounds__(256)
 gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, bool target, int rows,
                 int D, float eps, const float* __restrict__ a, const __nv_bfloat16* __restrict__ u,
                 const float* __restrict__ gamma, const float* __restrict__ beta,
-                float* __restrict__ y, float* __restrict__ stats) {
+                OutT* __restrict__ y, float* __restrict__ stats) {
   if (hdr->error) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
@@ -65,7 +77,7 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
       s += x[i].x + x[i].y + x[i].z + x[i].w;
     }
   }
-  float* yr = y + (size_t)row * D;
+  OutT* yr = y + (size_t)row * D;
   const __nv_bfloat16* ur = u + (size_t)row * D;
   if (gamma == nullptr) {
 #pragma unroll
@@ -73,8 +85,7 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
       const int c = lane + 32 * i;
       if (c < nch) {
         float4 uu = load_bf16x4(ur + 4 * c);
-        *reinterpret_cast<float4*>(yr + 4 * c) =
-            make_float4(x[i].x * uu.x, x[i].y * uu.y, x[i].z * uu.z, x[i].w * uu.w);
+        store4(yr + 4 * c, make_float4(x[i].x * uu.x, x[i].y * uu.y, x[i].z * uu.z, x[i].w * uu.w));
       }
     }
     return;
@@ -106,7 +117,7 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
       o.y = fmaf((x[i].y - mean) * rstd, gg.y, bb.y) * uu.y;
       o.z = fmaf((x[i].z - mean) * rstd, gg.z, bb.z) * uu.z;
       o.w = fmaf((x[i].w - mean) * rstd, gg.w, bb.w) * uu.w;
-      *reinterpret_cast<float4*>(yr + 4 * c) = o;
+      store4(yr + 4 * c, o);
     }
   }
   if (lane == 0) *reinterpret_cast<float2*>(stats + 2 * (size_t)row) = make_float2(mean, rstd);
@@ -226,8 +237,17 @@ cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, flo
                             const float* a, const __nv_bfloat16* u, const float* gamma,
                             const float* beta, float* y, float* stats, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  gate_fwd_kernel<<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps, a, u,
-                                                  gamma, beta, y, stats);
+  gate_fwd_kernel<float><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps, a, u,
+                                                         gamma, beta, y, stats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_fwd_bf16(const MetaView& m, bool target, int rows, int D, float eps,
+                                 const float* a, const __nv_bfloat16* u, const float* gamma,
+                                 const float* beta, __nv_bfloat16* y, float* stats, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  gate_fwd_kernel<__nv_bfloat16><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D,
+                                                                 eps, a, u, gamma, beta, y, stats);
   return cudaGetLastError();
 }
 

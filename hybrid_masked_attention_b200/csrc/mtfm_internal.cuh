@@ -33,9 +33,9 @@ struct MetaHeader {
   int32_t max_items_full;
   int32_t max_items_target;
   int32_t n_units_target;  // key-range chunks of the Target work list (sum of unit_count)
-  // Work counters of the persistent forward kernels: [0] next Full unit, [1] Full CTAs
-  // finished, [2] next Target unit, [3] Target CTAs finished.  Zeroed by the packer; the
-  // last CTA of a launch to finish sets its pair back to zero for the next launch.
+  // Work counter of the persistent Full-layer forward kernel: [0] next unit, [1] CTAs
+  // finished ([2], [3] reserved).  Zeroed by the packer; the last CTA of a launch to
+  // finish sets both back to zero for the next launch.
   uint32_t sched[4];
 };
 
@@ -51,7 +51,7 @@ struct WorkItem {
 
 struct MetaLayout {
   size_t seq_off, r_off, t_off, lh, lr, lt, kv_end, row_type, items_full, items_target, unit_off,
-      total;
+      t_rows, total;
   int32_t max_items_full, max_items_target;
 };
 
@@ -73,6 +73,7 @@ inline MetaLayout meta_layout(int B, int total_tokens, int total_t) {
   L.items_full = o;   o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_full);
   L.items_target = o; o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_target);
   L.unit_off = o;     o = align256(o + sizeof(int32_t) * ((size_t)L.max_items_target + 1));
+  L.t_rows = o;       o = align256(o + sizeof(int32_t) * (size_t)total_t);
   L.total = o;
   return L;
 }
@@ -91,6 +92,7 @@ struct MetaView {
   WorkItem* items_full;
   WorkItem* items_target;
   int32_t* unit_off;  // [max_items_target + 1]: first unit of each Target item (prefix sums)
+  int32_t* t_rows;    // [total_t]: global row (in the [sum N] layout) of each T row
 };
 
 inline MetaView meta_view(void* base, const MetaLayout& L) {
@@ -108,6 +110,7 @@ inline MetaView meta_view(void* base, const MetaLayout& L) {
   v.items_full = reinterpret_cast<WorkItem*>(b + L.items_full);
   v.items_target = reinterpret_cast<WorkItem*>(b + L.items_target);
   v.unit_off = reinterpret_cast<int32_t*>(b + L.unit_off);
+  v.t_rows = reinterpret_cast<int32_t*>(b + L.t_rows);
   return v;
 }
 
@@ -174,6 +177,37 @@ cudaError_t launch_attn_bwd_mma(const AttnShape& s, const MetaView& m, int max_i
                                 const __nv_bfloat16* v, const __nv_bfloat16* da_hi,
                                 const __nv_bfloat16* da_lo, float* dq, float* dk, float* dv,
                                 cudaStream_t st);
+
+cudaError_t launch_gate_fwd_bf16(const MetaView& m, bool target, int rows, int D, float eps,
+                                 const float* a, const __nv_bfloat16* u, const float* gamma,
+                                 const float* beta, __nv_bfloat16* y, float* stats, cudaStream_t st);
+
+// Backbone-stack pieces.  Projection GEMM C[M, N] = A[M, K] B[N, K]^T (bf16
+// operands, fp32 accumulation) with one of two fused epilogues:
+//   kEpiSiluSplit : SiLU, rounded to bf16, written into up to four column
+//                   segments (e.g. U | Q | K | V), each its own row-major array;
+//   kEpiResidual  : X[row_map[i], :] += C[i, :] in fp32 (row_map NULL: identity).
+constexpr float kRmsEps = 1e-6f;  // RMSNorm epsilon of the pre-norm
+constexpr int kEpiSiluSplit = 0;
+constexpr int kEpiResidual = 1;
+struct GemmEpi {
+  int kind;
+  int n_seg;
+  int seg_begin[5];  // segment s covers columns [seg_begin[s], seg_begin[s + 1]); seg_begin[n_seg] = N
+  __nv_bfloat16* seg_ptr[4];
+  int seg_ld[4];
+  float* x;
+  int ldx;
+  const int32_t* row_map;
+};
+// M >= 0; N a multiple of 64 (and of 32 at segment borders); K a multiple of 64;
+// lda a multiple of 8.  A and B 16-byte aligned.
+cudaError_t launch_gemm_tc(MetaHeader* hdr, const __nv_bfloat16* a, int lda, const __nv_bfloat16* b,
+                           int M, int N, int K, const GemmEpi& epi, cudaStream_t st);
+// out[i, :] = bf16(RMSNorm(X[row_map ? row_map[i] : i, :]) * w), d a multiple of 4, d <= 1024.
+cudaError_t launch_rmsnorm(const MetaHeader* hdr, const float* x, int rows, int d,
+                           const int32_t* row_map, const float* w, float eps, __nv_bfloat16* out,
+                           cudaStream_t st);
 
 constexpr int kGateBwdBlocks = 296;  // 2 per SM on a 148-SM part; partial dgamma/dbeta slots
 

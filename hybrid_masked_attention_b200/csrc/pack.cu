@@ -238,6 +238,8 @@ pack_rows_kernel(MetaView m, int max_if, const int64_t* __restrict__ r_ts,
     if (!tgt) {
       m.kv_end[so + i] = kve;
       m.row_type[so + i] = (uint8_t)type;
+    } else {
+      m.t_rows[m.t_off[u] + r] = so + i;
     }
     kmin = kve;
     kmax = kve;

@@ -1,0 +1,66 @@
+// RMSNorm pre-norm of the backbone layers: X~ = X / sqrt(mean(X^2) + eps) * w,
+// rounded to bf16 as the projection GEMM's operand.  Page "美团推荐大模型 MTFM
+// 深度硬核解析" §4.2 feeds the projections a normalised X~ without naming the
+// norm; RMSNorm is the reading taken.  With a row map the kernel gathers rows
+// (the Target layer's X~_T = X~[L_H + L_R:] of every user, §4.2).
+//
+// One warp per row, 128-bit loads, the row held in registers (d <= 1024).
+#include "mtfm_internal.cuh"
+
+namespace mtfm {
+namespace {
+
+constexpr int kMaxChunks = 8;  // float4 chunks per lane: d <= 32 * 4 * 8 = 1024
+
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const MetaHeader* hdr, const float* __restrict__ x, int rows, int d,
+               const int32_t* __restrict__ row_map, const float* __restrict__ w, float eps,
+               __nv_bfloat16* __restrict__ out) {
+  if (hdr->error) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  const int src = row_map ? row_map[row] : row;
+  const float* xr = x + (size_t)src * d;
+  const int nch = d >> 2;
+  float4 v[kMaxChunks];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nch) {
+      v[i] = *reinterpret_cast<const float4*>(xr + 4 * c);
+      s += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float inv = rsqrtf(s / (float)d + eps);
+  __nv_bfloat16* orow = out + (size_t)row * d;
+#pragma unroll
+  for (int i = 0; i < kMaxChunks; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nch) {
+      const float4 ww = *reinterpret_cast<const float4*>(w + 4 * c);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v[i].x * inv * ww.x, v[i].y * inv * ww.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(v[i].z * inv * ww.z, v[i].w * inv * ww.w);
+      uint2 r;
+      r.x = *reinterpret_cast<uint32_t*>(&lo);
+      r.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(orow + 4 * c) = r;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const MetaHeader* hdr, const float* x, int rows, int d,
+                           const int32_t* row_map, const float* w, float eps, __nv_bfloat16* out,
+                           cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (d <= 0 || d % 4 != 0 || d > 4 * 32 * kMaxChunks) return cudaErrorInvalidValue;
+  rmsnorm_kernel<<<(rows + 7) / 8, 256, 0, st>>>(hdr, x, rows, d, row_map, w, eps, out);
+  return cudaGetLastError();
+}
+
+}  // namespace mtfm

@@ -43,11 +43,10 @@
  *     metadata block; every later kernel that reads that block does nothing,
  *     and mtfm_pack_check() reports them.
  *   - The metadata block is read-only for every call but mtfm_pack, except
- *     for 16 bytes of work counters in its header: the persistent forward
- *     attention kernels draw their work from them and set them back to zero
- *     when they finish.  Hence two Full-layer (or two Target-layer) forward
- *     calls on one metadata block must be ordered (same stream, or an event);
- *     a Full and a Target call may overlap, and so may calls on different blocks.
+ *     for a work counter in its header: the persistent Full-layer forward
+ *     attention kernel draws its work from it and sets it back to zero when it
+ *     finishes.  Hence two Full-layer forward calls on one metadata block must
+ *     be ordered (same stream, or an event); other calls may overlap.
  *   - Supported: head_dim in {32, 64, 128}; hq % hkv == 0; hq/hkv <= 8;
  *     hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
@@ -230,6 +229,53 @@ mtfm_status mtfm_attn_target_bwd_static(const mtfm_cfg* cfg, const void* d_meta,
                                         const uint16_t* d_dy, float* d_dq, float* d_dk,
                                         float* d_dv, float* d_du, float* d_dgamma,
                                         float* d_dbeta, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Backbone stack forward ([DY] §4.1 and §4.2; blocks of one Full-Attention
+ * layer followed by Target-Attention layers, [DY] §4.1 and [MT] §3.3).
+ * Each layer, on the token matrix X (fp32 [total_tokens, d_model], updated in
+ * place):
+ *   X~ = RMSNorm(X) * rms_w (eps 1e-6; the pages leave the pre-norm unnamed),
+ *   Full  : [U Q K V] = SiLU(X~ W_in^T)            (phi_1 = SiLU, no biases)
+ *   Target: [U Q]_T = SiLU(X~_T W_in^T), [K V] = SiLU(X~ W_kv^T)
+ *   A = masked SiLU attention (as mtfm_attn_full / mtfm_attn_target),
+ *   Y = GLN(A) (*) U (plain A (*) U when gamma is NULL),
+ *   Full  : X <- X + Y W_o^T;  Target: X_T <- X_T + Y_T W_o^T, H/R rows unchanged.
+ * Precision: X~, U, Q, K, V and Y are rounded to bf16 (round to nearest) as
+ * the tensor-core operands; accumulation and X are fp32.
+ *
+ * mtfm_layer_weights holds device pointers (the struct itself is host memory):
+ *   rms_w : fp32 [d_model] RMSNorm weight
+ *   w_in  : bf16 [out, d_model] ("out x in", like a linear layer's weight);
+ *           Full: out = 2*hq*head_dim + 2*hkv*head_dim, rows ordered U, Q, K, V
+ *           (heads contiguous inside each part); Target: out = 2*hq*head_dim (U, Q)
+ *   w_kv  : Target only (NULL for Full): bf16 [2*hkv*head_dim, d_model] (K, V)
+ *   w_o   : bf16 [d_model, hq*head_dim]
+ *   gamma, beta : fp32 [3, hq*head_dim] GLN rows for H, R, T tokens, or both NULL.
+ * Shapes: d_model a multiple of 64 and <= 1024; hq*head_dim a multiple of 64.
+ * d_ws: scratch of at least mtfm_stack_workspace_bytes(cfg, d_model) bytes,
+ * 256-byte aligned, owned by the caller (reused by every layer; its contents
+ * are not needed between calls).  mtfm_stack_workspace_bytes returns 0 for an
+ * unsupported configuration.
+ * mtfm_stack_fwd runs n_layers layers; kinds[l] is 'F' (Full) or 'T' (Target).
+ * All layers' arguments are checked before the first launch.
+ * ------------------------------------------------------------------------- */
+typedef struct mtfm_layer_weights {
+  const float* rms_w;
+  const uint16_t* w_in;
+  const uint16_t* w_kv;
+  const uint16_t* w_o;
+  const float* gamma;
+  const float* beta;
+} mtfm_layer_weights;
+
+size_t mtfm_stack_workspace_bytes(const mtfm_cfg* cfg, int32_t d_model);
+mtfm_status mtfm_layer_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_model, int is_target,
+                           const mtfm_layer_weights* weights, float* d_x, void* d_ws,
+                           size_t ws_bytes, void* stream);
+mtfm_status mtfm_stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_model,
+                           int32_t n_layers, const char* kinds, const mtfm_layer_weights* layers,
+                           float* d_x, void* d_ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

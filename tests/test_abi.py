@@ -104,3 +104,32 @@ def test_meta_capacity_bounds(lib):
     c = _cfg(batch=3, total_tokens=300, total_r=10, total_t=129)
     assert m._lib.mtfm_max_items(ctypes.byref(c), 0) == (300 + 127) // 128 + 3
     assert m._lib.mtfm_max_items(ctypes.byref(c), 1) == (129 + 127) // 128 + 3
+
+
+def test_stack_arguments_rejected_before_launch(lib):
+    import hybrid_masked_attention_b200 as m
+    c = _cfg()
+    W = m.CLayerWeights
+    assert m._lib.mtfm_stack_workspace_bytes(ctypes.byref(c), 512) > 0
+    assert m._lib.mtfm_stack_workspace_bytes(ctypes.byref(c), 96) == 0     # d_model not a multiple of 64
+    assert m._lib.mtfm_stack_workspace_bytes(ctypes.byref(c), 2048) == 0   # d_model above 1024
+    ws = m._lib.mtfm_stack_workspace_bytes(ctypes.byref(c), 512)
+    full = W(4096, 4096, None, 4096, 4096, 4096)
+    tgt = W(4096, 4096, 4096, 4096, None, None)
+    # Full layer given a w_kv, Target layer without one
+    assert m._lib.mtfm_layer_fwd(ctypes.byref(c), 4096, 512, 0, ctypes.byref(tgt), 4096, 4096, ws, None) == 1
+    assert m._lib.mtfm_layer_fwd(ctypes.byref(c), 4096, 512, 1, ctypes.byref(full), 4096, 4096, ws, None) == 1
+    # gamma without beta
+    bad = W(4096, 4096, None, 4096, 4096, None)
+    assert m._lib.mtfm_layer_fwd(ctypes.byref(c), 4096, 512, 0, ctypes.byref(bad), 4096, 4096, ws, None) == 1
+    # misaligned X, workspace too small or misaligned
+    assert m._lib.mtfm_layer_fwd(ctypes.byref(c), 4096, 512, 0, ctypes.byref(full), 4096 + 4, 4096, ws, None) == 1
+    assert m._lib.mtfm_layer_fwd(ctypes.byref(c), 4096, 512, 0, ctypes.byref(full), 4096, 4096, ws - 1, None) == 4
+    assert m._lib.mtfm_layer_fwd(ctypes.byref(c), 4096, 512, 0, ctypes.byref(full), 4096, 4096 + 16, ws, None) == 1
+    # unknown layer kind; one bad layer among good ones stops the whole stack
+    arr = (W * 2)(full, tgt)
+    assert m._lib.mtfm_stack_fwd(ctypes.byref(c), 4096, 512, 2, b"FX", arr, 4096, 4096, ws, None) == 1
+    arr2 = (W * 2)(full, full)
+    assert m._lib.mtfm_stack_fwd(ctypes.byref(c), 4096, 512, 2, b"FT", arr2, 4096, 4096, ws, None) == 1
+    # no layers: nothing to do
+    assert m._lib.mtfm_stack_fwd(ctypes.byref(c), 4096, 512, 0, None, None, 4096, 4096, ws, None) == 0

@@ -1,0 +1,142 @@
+"""Backbone stack (RMSNorm, SiLU projections, attention, gate, output projection,
+residual; 4 x (Full, Target, Target, Target)) on the GPU through the C ABI,
+against the fp64 oracle.
+
+Tolerances.  The stack's output X is held to the standard bar (rel-L2 <= 1e-2,
+max-abs <= 2e-2 x RMS).  The layer increments X_out - X_in are checked too, at
+rel-L2 <= 1e-2 and max-abs <= 0.15 x RMS: the GPU rounds X~, U, Q, K, V and Y to
+bf16 as tensor-core operands (exact in the oracle), and replaying those roundings
+in numpy on the oracle puts the increments' max-abs error at 3e-2 .. 1e-1 x RMS
+(the GLN of rows with a small spread of A amplifies them), their rel-L2 at
+4e-3 .. 7e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mtfm_synth as syn
+from gpu_helpers import assert_close, bf16_tensor, close_report, config_for, f32_tensor, upload_batch
+from oracle import mtfm_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+INC_REL_L2 = 1e-2
+INC_MAX_ABS_RMS = 0.15
+
+
+def assert_increment_close(got, ref, name):
+    rel, mx, rms = close_report(got, ref)
+    assert rel <= INC_REL_L2, f"{name}: rel-L2 {rel:.3e} > {INC_REL_L2}"
+    assert mx <= INC_MAX_ABS_RMS * rms, f"{name}: max-abs {mx:.3e} > {INC_MAX_ABS_RMS} x RMS {rms:.3e}"
+
+
+def _device_layers(weights):
+    import hybrid_masked_attention_b200 as M
+    out = []
+    for lw in weights:
+        out.append(M.LayerWeights(
+            lw.kind, f32_tensor(lw.rms_w), bf16_tensor(lw.w_in),
+            bf16_tensor(lw.w_kv) if lw.w_kv is not None else None, bf16_tensor(lw.w_o),
+            f32_tensor(lw.gamma), f32_tensor(lw.beta)))
+    return out
+
+
+def _session(batch, heads, d_model):
+    import hybrid_masked_attention_b200 as M
+    cfg = config_for(batch, heads)
+    meta = M.alloc_meta(cfg)
+    M.pack(cfg, *upload_batch(batch), meta)
+    M.pack_check(meta)
+    ws = torch.empty(M.stack_workspace_bytes(cfg, d_model), dtype=torch.uint8, device="cuda")
+    return cfg, meta, ws
+
+
+def _x0(batch, d_model, seed):
+    return syn.bf16_bits_to_f32(syn.stack_input(batch, d_model, seed)).astype(np.float64)
+
+
+WEIGHTS = {
+    "spec": dict(std=0.02, std_o=None, random_norms=False),     # N(0, 0.02), W_o std 0.02 / sqrt(16)
+    "signal": dict(std=0.05, std_o=0.05, random_norms=True),    # larger updates, random norm parameters
+}
+
+
+@pytest.mark.parametrize("wname", sorted(WEIGHTS))
+@pytest.mark.parametrize("kind", ["F", "T"])
+def test_single_layer(kind, wname, cuda_ok):
+    import hybrid_masked_attention_b200 as M
+    b, hd, d = syn.pair_batch(4, 1002), syn.PAIR_HEADS, 512
+    lw = syn.stack_weights(hd, d, 71, kinds=(kind,), **WEIGHTS[wname])[0]
+    X0 = _x0(b, d, 71)
+    cfg, meta, ws = _session(b, hd, d)
+    x = torch.from_numpy(X0.astype(np.float32)).cuda()
+    M.layer_fwd(cfg, meta, d, _device_layers([lw])[0], x, ws)
+    M.pack_check(meta)
+    got = x.cpu().numpy().astype(np.float64)
+    ref = (O.full_layer if kind == "F" else O.target_layer)(b, hd, X0, lw)
+    assert_close(got, ref, f"X' {kind}")
+    assert_increment_close(got - X0, ref - X0, f"X' - X {kind}")
+    if kind == "T":
+        hr = np.setdiff1d(np.arange(b.total_tokens), O.t_row_index(b))
+        assert np.array_equal(got[hr], X0[hr]), "Target layer changed H/R rows"
+
+
+@pytest.mark.parametrize("wname", sorted(WEIGHTS))
+def test_stack_16_layers(wname, cuda_ok):
+    import hybrid_masked_attention_b200 as M
+    b, hd, d = syn.pair_batch(4, 1002), syn.PAIR_HEADS, 512
+    ws_ = syn.stack_weights(hd, d, 73, **WEIGHTS[wname])
+    X0 = _x0(b, d, 73)
+    cfg, meta, ws = _session(b, hd, d)
+    x = torch.from_numpy(X0.astype(np.float32)).cuda()
+    M.stack_fwd(cfg, meta, d, _device_layers(ws_), x, ws)
+    M.pack_check(meta)
+    got = x.cpu().numpy().astype(np.float64)
+    ref = O.stack_fwd(b, hd, ws_, X0)
+    if wname == "spec":
+        assert_close(got, ref, "X16")
+    assert_increment_close(got - X0, ref - X0, "X16 - X0")
+
+
+def test_stack_tiny_heads(cuda_ok):
+    """head_dim 32 (the mma.sync attention kernel), d_model 64, the 2-user batch."""
+    import hybrid_masked_attention_b200 as M
+    b, hd, d = syn.tiny_batch(), syn.TINY_HEADS, 64
+    ws_ = syn.stack_weights(hd, d, 75, std=0.1, std_o=0.1, random_norms=True)
+    X0 = _x0(b, d, 75)
+    cfg, meta, ws = _session(b, hd, d)
+    x = torch.from_numpy(X0.astype(np.float32)).cuda()
+    M.stack_fwd(cfg, meta, d, _device_layers(ws_), x, ws)
+    M.pack_check(meta)
+    got = x.cpu().numpy().astype(np.float64)
+    ref = O.stack_fwd(b, hd, ws_, X0)
+    assert_increment_close(got - X0, ref - X0, "X16 - X0 tiny")
+
+
+def _subset(batch, users):
+    ro, to = O.offsets(batch.L_R), O.offsets(batch.L_T)
+    idx = np.asarray(users)
+    return syn.JaggedBatch(batch.L_H[idx], batch.L_R[idx], batch.L_T[idx],
+                           np.concatenate([batch.r_ts[ro[u]:ro[u + 1]] for u in users]),
+                           np.concatenate([batch.t_exp[to[u]:to[u + 1]] for u in users]),
+                           np.zeros(int(batch.L_T[idx].sum()), np.int32), batch.v2_subtokens)
+
+
+def test_stack_full_size_sampled_users(cuda_ok):
+    """The 64-user batch through all 16 layers on the GPU; the oracle recomputes
+    three users from scratch (users never interact in the stack)."""
+    import hybrid_masked_attention_b200 as M
+    b, hd, d = syn.pair_batch(64, 1002), syn.PAIR_HEADS, 512
+    ws_ = syn.stack_weights(hd, d, 1002)
+    X0 = _x0(b, d, 1002)
+    cfg, meta, ws = _session(b, hd, d)
+    x = torch.from_numpy(X0.astype(np.float32)).cuda()
+    M.stack_fwd(cfg, meta, d, _device_layers(ws_), x, ws)
+    M.pack_check(meta)
+    got = x.cpu().numpy().astype(np.float64)
+    users = [0, 31, 63]
+    so = O.offsets(b.N)
+    rows = np.concatenate([np.arange(so[u], so[u + 1]) for u in users])
+    ref = O.stack_fwd(_subset(b, users), hd, ws_, X0[rows])
+    assert_close(got[rows], ref, "X16 sampled users")
+    assert_increment_close(got[rows] - X0[rows], ref - X0[rows], "X16 - X0 sampled users")
