@@ -405,8 +405,8 @@ RMS_EPS = 1e-6
 def rmsnorm(X, w, eps: float = RMS_EPS):
     """Pre-norm X~ = X / sqrt(mean_j X_ij^2 + eps) * w, row by row.
 
-    The pages call X~ "the normalised feature matrix" ([DY] §4.2) without naming
-    the norm; RMSNorm with eps = 1e-6 is the reading taken here.
+    [DY] §4.2 projects a normalised X~ but does not say which norm; RMSNorm
+    with eps = 1e-6 is the reading taken here.
     """
     X = np.asarray(X, dtype=np.float64)
     ms = (X * X).mean(axis=1, keepdims=True)
