@@ -9,7 +9,7 @@ Function names mirror the C entry points:
     meta_bytes, max_items, pack, pack_check, meta_read,
     attn_full_fwd, attn_target_fwd, attn_full, attn_target, gate_fwd,
     bwd_workspace_bytes, attn_full_bwd, attn_target_bwd, attn_target_bwd_static,
-    stack_workspace_bytes, layer_fwd, stack_fwd
+    stack_workspace_bytes, layer_fwd, stack_fwd, selftest_wait_timeout
 """
 from __future__ import annotations
 
@@ -110,6 +110,7 @@ _sigs = {
     "mtfm_attn_full_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
     "mtfm_attn_target_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
     "mtfm_attn_target_bwd_static": (ctypes.c_int, [_CP] + [_P] * 17),
+    "mtfm_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_int64, _P]),
     "mtfm_stack_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int32]),
     "mtfm_layer_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int, _LWP, _P, _P, ctypes.c_size_t, _P]),
     "mtfm_stack_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_char_p, _LWP, _P, _P,
@@ -395,4 +396,11 @@ def stack_fwd(cfg: Config, meta: torch.Tensor, d_model: int, layers, x: torch.Te
                                _ptr(x, torch.float32, (cfg.total_tokens, d_model), "x"),
                                _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream)),
            "mtfm_stack_fwd")
+
+
+def selftest_wait_timeout(meta: torch.Tensor, limit_cycles: int = 2_000_000, stream=None):
+    """Make one bounded wait run out on the GPU; the timeout is recorded in ``meta``
+    (``pack_check`` then raises MtfmError with MTFM_ERR_TIMEOUT)."""
+    _check(_lib.mtfm_selftest_wait_timeout(_ptr(meta, torch.uint8, name="meta"), int(limit_cycles),
+                                           _stream(stream)), "mtfm_selftest_wait_timeout")
 

@@ -483,4 +483,11 @@ mtfm_status mtfm_stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_mo
   return stack_fwd(cfg, d_meta, d_model, n_layers, kinds, layers, d_x, d_ws, ws_bytes, stream);
 }
 
+mtfm_status mtfm_selftest_wait_timeout(void* d_meta, int64_t limit_cycles, void* stream) {
+  if (!d_meta || (reinterpret_cast<uintptr_t>(d_meta) & 255u) != 0) return MTFM_ERR_INVALID_ARG;
+  if (limit_cycles <= 0 || limit_cycles > 4000000000ll) return MTFM_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_timeout(static_cast<MetaHeader*>(d_meta), (long long)limit_cycles,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -209,6 +209,10 @@ cudaError_t launch_rmsnorm(const MetaHeader* hdr, const float* x, int rows, int 
                            const int32_t* row_map, const float* w, float eps, __nv_bfloat16* out,
                            cudaStream_t st);
 
+// One CTA waits (bounded by `limit` SM cycles) on an mbarrier nothing arrives on and
+// sets the timeout bit in the header.
+cudaError_t launch_wait_timeout(MetaHeader* hdr, long long limit, cudaStream_t st);
+
 constexpr int kGateBwdBlocks = 296;  // 2 per SM on a 148-SM part; partial dgamma/dbeta slots
 
 }  // namespace mtfm

@@ -48,19 +48,23 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // raises the flag): the caller then stops its work and heads for the exit.
 // (try_wait itself suspends the thread for a short hardware-defined window; the
 // abort flag and the clock are checked only every 64 polls.)
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait_limit(bar, parity, abort_flag, kWaitCycles);
 }
 
 // One lane of the (converged) warp returns true.

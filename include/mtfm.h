@@ -277,6 +277,18 @@ mtfm_status mtfm_stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_mo
                            int32_t n_layers, const char* kinds, const mtfm_layer_weights* layers,
                            float* d_x, void* d_ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Self-test of failure detection (no counterpart on the pages).  Launches one
+ * CTA that waits, with the bounded mbarrier wait every tensor-core kernel of
+ * this library uses, on a barrier nothing arrives on; after limit_cycles SM
+ * clock cycles (1 .. 4e9; ~1.9e9 per second) it gives up and sets the timeout
+ * bit in d_meta's header, as an aborting kernel does.  mtfm_pack_check then
+ * returns MTFM_ERR_TIMEOUT and every later kernel on d_meta does nothing until
+ * the next mtfm_pack.  Nothing is left in flight; the context stays usable.
+ * d_meta: a metadata block written by mtfm_pack (256-byte aligned).
+ * ------------------------------------------------------------------------- */
+mtfm_status mtfm_selftest_wait_timeout(void* d_meta, int64_t limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

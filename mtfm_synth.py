@@ -234,7 +234,8 @@ class LayerWeights:
 def stack_weights(heads: Heads, d_model: int, seed: int, kinds=STACK_KINDS, std: float = 0.02,
                   std_o: Optional[float] = None, random_norms: bool = False) -> list:
     """Weights ~ N(0, std) (std 0.02), output projections ~ N(0, std_o) with the
-    depth-scaled std_o = 0.02 / sqrt(layers).  Norm parameters are the identity
+    depth-scaled std_o = 0.02 / sqrt(layers) (Meituan tech blog §5.1, depth-aware
+    initialisation; its formula is garbled, the standard deviation is the reading).  Norm parameters are the identity
     (RMSNorm weight 1, GLN gamma 1 and beta 0) unless ``random_norms``."""
     if std_o is None:
         std_o = std / np.sqrt(len(kinds))

@@ -133,3 +133,11 @@ def test_stack_arguments_rejected_before_launch(lib):
     assert m._lib.mtfm_stack_fwd(ctypes.byref(c), 4096, 512, 2, b"FT", arr2, 4096, 4096, ws, None) == 1
     # no layers: nothing to do
     assert m._lib.mtfm_stack_fwd(ctypes.byref(c), 4096, 512, 0, None, None, 4096, 4096, ws, None) == 0
+
+
+def test_selftest_arguments(lib):
+    import hybrid_masked_attention_b200 as m
+    assert m._lib.mtfm_selftest_wait_timeout(None, 1000, None) == 1
+    assert m._lib.mtfm_selftest_wait_timeout(4096 + 16, 1000, None) == 1
+    assert m._lib.mtfm_selftest_wait_timeout(4096, 0, None) == 1
+    assert m._lib.mtfm_selftest_wait_timeout(4096, 5_000_000_000, None) == 1
