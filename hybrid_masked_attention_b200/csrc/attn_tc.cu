@@ -66,6 +66,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
 static_assert(kBN == kKeyBlock, "the packer sizes Target units in blocks of kKeyBlock keys");
+static_assert(kBM * (4 * kDH + 4) * 4 <= 4 * kQBytes + 2 * kStages * kKVBytes, "O staging fits in the Q + K/V buffers");
 static_assert(kSiluWG % kWGPerBuf == 0 && kChunksPerWG >= 1 && kSBuf % kTeams == 0, "warpgroup split");
 
 struct TcArgs {
@@ -361,7 +362,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int c = 0; c < kDH; c += 4)
               *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
                   make_float4(0.f, 0.f, 0.f, 0.f);
-      } else if (ok) {
+      }
+      // O / N_u goes through shared memory (the Q and K/V buffers are idle once every
+      // MMA of the unit is done) so that each warp then writes whole rows of A:
+      // coalesced 512-byte stores (Target: vector atomics) instead of 16-byte pieces
+      // of 32 different rows.  The named barrier is reached by all 16 SiLU warps,
+      // also after an abort, so it cannot hang.
+      const bool have = ok && total > 0;
+      float* stage = reinterpret_cast<float*>(smem);
+      constexpr int kStageLd = R * kDH + 4;  // padded row: conflict-free float4 access
+      if (have) {
         tc_fence_after();
         const float inv_n = 1.f / (float)N;
         for (int hh = wg; hh < R; hh += kSiluWG) {
@@ -370,19 +380,29 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             uint32_t raw[32];
             tmem_ld32(lane_base + hh * kDH + c * 32, raw);
             tmem_ld_wait();
-            if (valid) {
-              float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c * 32);
+            float4* dst = reinterpret_cast<float4*>(stage + row * kStageLd + hh * kDH + c * 32);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float4 v = make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
-                                             __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
-                if (TARGET) atomicAdd(dst + e, v);  // partial over this unit's key chunk; A zeroed first
-                else dst[e] = v;
-              }
-            }
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
+                                   __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
           }
         }
       }
+      asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
+      if (have) {
+        const int sw = warp - 4;  // rows [8 sw, 8 sw + 8) of the tile
+#pragma unroll 1
+        for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
+          if (q0 + rr >= nq) break;
+          float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
+          const float4* src = reinterpret_cast<const float4*>(stage + rr * kStageLd);
+          for (int f = lane; f < R * kDH / 4; f += 32) {
+            if (TARGET) atomicAdd(dst + f, src[f]);  // partial over this unit's key chunk; A zeroed first
+            else dst[f] = src[f];
+          }
+        }
+      }
+      fence_proxy_async();  // the next unit's TMA writes overwrite the staged rows
     }
     tc_fence_before();
     __syncthreads();
