@@ -39,6 +39,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "mtfm_internal.cuh"
 #include "mma_util.cuh"
@@ -324,14 +325,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
       const float half_alpha = 0.5f * p.alpha;
       bool ok = true;
-      for (int n = team; n < total; n += kTeams) {
+      // Steps of the key blocks that lie inside every row's visible prefix (the prefix
+      // blocks below kv_min, which come first) run the unmasked code in a loop of their
+      // own; the rest run the masked loop, where a warp whose 32 rows see all or none of
+      // a chunk's keys takes the unmasked code or just writes zeros.
+      const int n_full = max(0, min(n_blocks, min(kb.nb_pre, it.kv_min / kBN) - bi0)) * R;
+      auto step = [&](int n, auto masked_tag) -> bool {
+        constexpr bool kMasked = decltype(masked_tag)::value;
         const int buf = (step_base + n) % kSBuf;
-        ok = __all_sync(0xffffffffu, mbar_wait(b_sf(buf), ((step_base + n) / kSBuf) & 1, abort_flag));
-        if (!ok) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(b_sf(buf), ((step_base + n) / kSBuf) & 1, abort_flag)))
+          return false;
         tc_fence_after();
-        const int gbi = bi0 + n / R;  // block index within the item
-        const int j0 = kb.block(gbi) * kBN;
-        const bool full = (gbi < kb.nb_pre) && (j0 + kBN <= it.kv_min);
         const uint32_t sb = lane_base + kSCol0 + buf * kBN;
 #pragma unroll
         for (int c = cpart * kChunksPerWG; c < (cpart + 1) * kChunksPerWG; ++c) {
@@ -339,10 +343,19 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tmem_ld32(sb + c * 32, raw);
           tmem_ld_wait();
           uint32_t ph[16], pl[16];
-          if (full) {
+          if (!kMasked) {
             silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
           } else {
-            silu_chunk<true>(raw, half_alpha, vis_bits(j0 + 32 * c, kv_end, sib_lo, sib_hi), ph, pl);
+            const int j0 = kb.block(bi0 + n / R) * kBN;
+            const uint32_t vis = vis_bits(j0 + 32 * c, kv_end, sib_lo, sib_hi);
+            if (__all_sync(0xffffffffu, vis == 0u)) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) ph[e] = pl[e] = 0u;
+            } else if (__all_sync(0xffffffffu, vis == 0xffffffffu)) {
+              silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
+            } else {
+              silu_chunk<true>(raw, half_alpha, vis, ph, pl);
+            }
           }
           // keys [32c, 32c+32): P_hi in columns [32c, 32c+16), P_lo in [32c+16, 32c+32),
           // i.e. over the S columns of this chunk, which were read above.
@@ -352,7 +365,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(b_pf(buf));
-      }
+        return true;
+      };
+      static_assert(kTeams == 1, "one team walks every step");
+      for (int n = 0; ok && n < n_full; ++n) ok = step(n, std::false_type{});
+      for (int n = n_full; ok && n < total; ++n) ok = step(n, std::true_type{});
       // ----------------------------------------------------------- epilogue: A (+)= O / N_u
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, unit_iter & 1, abort_flag));
       if (ok && total == 0) {
