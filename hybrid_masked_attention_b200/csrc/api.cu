@@ -55,7 +55,8 @@ mtfm_status check_meta(const void* d_meta, const Resolved& r) {
   return MTFM_OK;
 }
 
-// tcgen05/TMEM kernel where its TMEM plan fits (head_dim 64, r in {1, 2, 4});
+// tcgen05/TMEM kernels where their TMEM plans fit (head_dim 64, r in {1, 2, 4}; the
+// Target layer stacks the r heads of a group as MMA rows);
 // the mma.sync kernel covers the other head shapes.  MTFM_FWD_KERNEL=mma
 // selects the mma.sync kernel for every shape (for comparisons).
 cudaError_t launch_attn(const Resolved& r, const MetaView& m, const MetaLayout& L, bool target,
@@ -66,8 +67,10 @@ cudaError_t launch_attn(const Resolved& r, const MetaView& m, const MetaLayout& 
   const int rows = target ? r.total_t : r.total_tokens;
   const char* force = getenv("MTFM_FWD_KERNEL");
   const bool force_mma = force && strcmp(force, "mma") == 0;
-  if (!force_mma && attn_fwd_tc_supported(shape))
+  if (!force_mma && attn_fwd_tc_supported(shape)) {
+    if (target) return launch_attn_fwd_tgt(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
     return launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
+  }
   return launch_attn_fwd_mma(shape, m, max_items, q, k, v, a, st);
 }
 
@@ -363,6 +366,7 @@ mtfm_status mtfm_pack_check(const void* d_meta, void* stream) {
   if (h.error & kErrBadLengths) return MTFM_ERR_BAD_LENGTHS;
   if (h.error & kErrUnsorted) return MTFM_ERR_UNSORTED_TS;
   if (h.error & kErrTimeout) return MTFM_ERR_TIMEOUT;
+  if (h.error & kErrConfig) return MTFM_ERR_UNSUPPORTED;
   return MTFM_OK;
 }
 

@@ -1,23 +1,22 @@
-// sm_100a forward kernel of the masked SiLU attention: tcgen05 MMAs with TMEM
-// accumulators, operands staged by TMA (128-byte swizzle), K/V blocks shared
-// by the r query heads of one GQA group.
+// sm_100a forward kernel of the Full-Attention layer: tcgen05 MMAs with TMEM
+// accumulators, operands staged by TMA (128-byte swizzle), K/V blocks shared by
+// the r query heads of one GQA group.  (The Target layer has its own kernel,
+// attn_tgt.cu, which stacks the r heads as MMA rows.)
 //
 // Computes, per query row i of a 128-row tile of user u and head h of KV group g
-// (page "美团推荐大模型 MTFM 深度硬核解析", §4.1 attention equation and §4.2
-// Target Attention; visibility from the Meituan tech blog §3.2):
+// (page "美团推荐大模型 MTFM 深度硬核解析", §4.1 attention equation; visibility
+// from the Meituan tech blog §3.2):
 //     A[i, h] = (1/N_u) sum_{j visible from i} SiLU(alpha q[i,h].k[j,g]) v[j,g]
 // with "visible" = the row's key prefix [0, kv_end) plus, for T rows, the
 // sibling block (itself, or the 4 sub-tokens of its target in V2).
 //
-// Persistent CTAs (one per SM) take work units x KV groups from a counter (Full)
-// or stride over them (Target).  A Full-layer
-// unit is one work item (user, 128-row query tile) with all its key blocks; a
-// Target-layer unit is a chunk of kTargetUnitBlocks key blocks of one item (the
-// packer splits each Target tile's key range so that short Target layers still
-// fill the GPU), and its partial O is added into A (zeroed first) with fp32
-// vector atomics.  A step is one (128-key block, query head) pair:
-//   warp 0      : TMA producer (Q tiles of the r heads once, then K/V blocks of
-//                 128 keys through a 3-stage ring);
+// Persistent CTAs (one per SM) take (work item, KV group) pairs from a counter
+// in the metadata header, in work-list order (longest users first): greedy list
+// scheduling, since item costs vary with the user's length.  A work item is one
+// (user, 128-row query tile) with all its key blocks.  A step is one (128-key
+// block, query head) pair:
+//   warp 0      : TMA producer (Q tiles of the r heads once per item, then K/V
+//                 blocks of 128 keys through a 3-stage ring);
 //   warp 1      : TMEM allocation and the MMA issue (whole warp runs the
 //                 control flow, one elected lane issues);
 //   warps 4..19 : four "SiLU" warpgroups that share every step, each on 32 of
@@ -25,13 +24,13 @@
 //                 mask + SiLU, write P as two bf16 parts P_hi + P_lo (~16
 //                 significant bits) back into the same TMEM columns, and signal
 //                 the MMA warp, which issues O_h += P_hi V + P_lo V with P read
-//                 from TMEM.
+//                 from TMEM; at the end of the item they write O / N_u to A
+//                 through shared memory (whole rows per warp).
 // TMEM (512 columns): O_h at columns [64h, 64h+64) for h < r (<= 4), S buffers
 // b = 0, 1 at [256 + 128b, 384 + 128b).  While the warpgroups run the SiLU of
-// step n, the tensor pipe runs O += P(n-1) V and S(n+1) = Q K^T: the tanh
-// throughput (16 per clock per SM) and the MMA time per step are about equal.
+// step n, the tensor pipe runs O += P(n-1) V and S(n+1) = Q K^T.
 // Key blocks above the tile's largest kv_end are never loaded; blocks entirely
-// below its smallest kv_end skip the per-element mask test.
+// below its smallest kv_end come first and skip the per-element mask test.
 //
 // Every wait is bounded (about one second); a wait that gives up raises a
 // CTA-wide abort flag, every role drains its in-flight copies/MMAs with a
@@ -66,7 +65,7 @@ constexpr uint32_t kKVBytes = kBN * kDH * 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
-static_assert(kBN == kKeyBlock, "the packer sizes Target units in blocks of kKeyBlock keys");
+static_assert(kBN == kKeyBlock, "key blocks of the work lists");
 static_assert(kBM * (4 * kDH + 4) * 4 <= 4 * kQBytes + 2 * kStages * kKVBytes, "O staging fits in the Q + K/V buffers");
 static_assert(kSiluWG % kWGPerBuf == 0 && kChunksPerWG >= 1 && kSBuf % kTeams == 0, "warpgroup split");
 
@@ -102,7 +101,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half
   }
 }
 
-template <int R, bool TARGET>
+template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, TcArgs p) {
@@ -117,14 +116,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const MetaView& m = p.m;
   MetaHeader* hdr = m.hdr;
   if (hdr->error) return;
-  // Work units: Full layer = one work item (all its key blocks); Target layer =
-  // one chunk of kTargetUnitBlocks key blocks of a work item.  Each unit runs
-  // for every KV group.  Full layer: the CTAs take (unit, group) pairs from a
-  // counter in the metadata header, in work-list order (longest users first), so
-  // that a CTA that finishes early takes the next pair (greedy list scheduling;
-  // unit costs vary with the user's length).  Target layer: units cost about the
-  // same, and the CTAs stride over the pairs (measured faster than the counter).
-  const int n_units = TARGET ? hdr->n_units_target : hdr->n_items_full;
+  // (work item, KV group) pairs, taken from the counter (see the file comment)
+  const int n_units = hdr->n_items_full;
   const int n_work = n_units * p.hkv;
   if ((int)blockIdx.x >= n_work) return;
   const int participants = min((int)gridDim.x, n_work);
@@ -146,7 +139,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    s_ticket[0] = TARGET ? (int)blockIdx.x : (int)atomicAdd(ticket_ctr, 1u);
+    s_ticket[0] = (int)atomicAdd(ticket_ctr, 1u);
     mbar_init(b_q, 1);
     mbar_init(b_o, 1);
     mbar_init(b_drain, 1);
@@ -181,29 +174,19 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   for (;;) {
     const int w = s_ticket[unit_iter & 1];  // written before the last block-wide barrier
     if (w >= n_work) break;
-    const int unit = w / p.hkv, g = w % p.hkv;
-    int item = unit, chunk = 0;
-    if (TARGET) {  // last item whose first unit is <= unit
-      int lo = 0, hi = hdr->n_items_target - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (m.unit_off[mid] <= unit) lo = mid; else hi = mid - 1;
-      }
-      item = lo;
-      chunk = unit - m.unit_off[lo];
-    }
-    const WorkItem it = (TARGET ? m.items_target : m.items_full)[item];
+    const int item = w / p.hkv, g = w % p.hkv;
+    const WorkItem it = m.items_full[item];
     const int u = it.user;
     const int LH = m.lh[u], LR = m.lr[u], LT = m.lt[u];
     const int N = LH + LR + LT, so = m.seq_off[u];
-    const int nq = TARGET ? LT : N;
+    const int nq = N;
     const int q0 = it.tile * kBM;
-    const int qrow0 = TARGET ? m.t_off[u] : so;
-    const int pos0 = TARGET ? LH + LR : 0;
+    const int qrow0 = so;
+    const int pos0 = 0;
     const int t0pos = LH + LR;
     const KeyBlocks kb = key_blocks(it.kv_max, LH, LR, nq, pos0, q0, p.v2);
-    const int bi0 = TARGET ? chunk * kTargetUnitBlocks : 0;
-    const int bi1 = TARGET ? min(bi0 + kTargetUnitBlocks, kb.n_blocks) : kb.n_blocks;
+    const int bi0 = 0;
+    const int bi1 = kb.n_blocks;
     const int n_blocks = max(0, bi1 - bi0);
     const int total = n_blocks * R;  // steps n = (key block bi0 + n / R, head n % R)
     auto block_of = [&](int bi) { return kb.block(bi0 + bi); };
@@ -225,7 +208,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           ++issued;
         }
         // the next pair, read by every role after this unit's closing barrier
-        s_ticket[(unit_iter + 1) & 1] = TARGET ? w + (int)gridDim.x : (int)atomicAdd(ticket_ctr, 1u);
+        s_ticket[(unit_iter + 1) & 1] = (int)atomicAdd(ticket_ctr, 1u);
         // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
         // no TMA write may land after this unit's barriers are re-armed or the CTA leaves.
         const long long t0 = clock64();
@@ -374,15 +357,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, unit_iter & 1, abort_flag));
       if (ok && total == 0) {
         // no visible key at all (cannot happen for a non-empty Full tile): A = 0
-        if (!TARGET)
-          for (int hh = wg; hh < R && valid; hh += kSiluWG)
+        for (int hh = wg; hh < R && valid; hh += kSiluWG)
             for (int c = 0; c < kDH; c += 4)
               *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
                   make_float4(0.f, 0.f, 0.f, 0.f);
       }
       // O / N_u goes through shared memory (the Q and K/V buffers are idle once every
       // MMA of the unit is done) so that each warp then writes whole rows of A:
-      // coalesced 512-byte stores (Target: vector atomics) instead of 16-byte pieces
+      // coalesced 512-byte stores instead of 16-byte pieces
       // of 32 different rows.  The named barrier is reached by all 16 SiLU warps,
       // also after an abort, so it cannot hang.
       const bool have = ok && total > 0;
@@ -414,8 +396,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
           const float4* src = reinterpret_cast<const float4*>(stage + rr * kStageLd);
           for (int f = lane; f < R * kDH / 4; f += 32) {
-            if (TARGET) atomicAdd(dst + f, src[f]);  // partial over this unit's key chunk; A zeroed first
-            else dst[f] = src[f];
+            dst[f] = src[f];
           }
         }
       }
@@ -437,12 +418,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (s_abort) atomicOr(&hdr->error, kErrTimeout);
     // Every CTA has drawn its last ticket before it counts itself finished, so the
     // last one to finish may rewind both counters for the next launch on this block.
-    if (!TARGET) {
-      __threadfence();
-      if (atomicAdd(done_ctr, 1u) == (uint32_t)participants - 1) {
-        atomicExch(ticket_ctr, 0u);
-        atomicExch(done_ctr, 0u);
-      }
+    __threadfence();
+    if (atomicAdd(done_ctr, 1u) == (uint32_t)participants - 1) {
+      atomicExch(ticket_ctr, 0u);
+      atomicExch(done_ctr, 0u);
     }
   }
 }
@@ -455,16 +434,16 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
 
 // One CTA per SM (TMEM and shared memory allow no more); the CTAs stride over
 // the (work unit, KV group) pairs, whose count the kernel reads from the metadata.
-template <int R, bool TARGET>
+template <int R>
 cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const TcArgs& a, int max_items, cudaStream_t st) {
   const size_t smem = tc_smem_bytes<R>();
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R, TARGET>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
-  if (!TARGET) grid = std::min(grid, max_items * a.hkv);
-  attn_fwd_tc_kernel<R, TARGET><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  grid = std::min(grid, max_items * a.hkv);
+  attn_fwd_tc_kernel<R><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -478,6 +457,7 @@ bool attn_fwd_tc_supported(const AttnShape& s) {
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                const __nv_bfloat16* v, float* a, cudaStream_t st) {
+  if (s.target) return cudaErrorInvalidValue;  // the Target layer has its own kernel (attn_tgt.cu)
   if (max_items <= 0 || rows_q <= 0 || total_tokens <= 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, rows_q, s.hq * kDH, kBM) || !make_map(&mk, k, total_tokens, s.hkv * kDH, kBN) ||
@@ -485,19 +465,9 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
     return cudaErrorInvalidValue;
   TcArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha};
   const int r = s.hq / s.hkv;
-  if (s.target) {
-    // Target units add partial sums over key chunks into A
-    cudaError_t e = cudaMemsetAsync(a, 0, sizeof(float) * (size_t)rows_q * s.hq * kDH, st);
-    if (e != cudaSuccess) return e;
-  }
-  if (s.target) {
-    if (r == 1) return tc_launch<1, true>(mq, mk, mv, args, max_items, st);
-    if (r == 2) return tc_launch<2, true>(mq, mk, mv, args, max_items, st);
-    return tc_launch<4, true>(mq, mk, mv, args, max_items, st);
-  }
-  if (r == 1) return tc_launch<1, false>(mq, mk, mv, args, max_items, st);
-  if (r == 2) return tc_launch<2, false>(mq, mk, mv, args, max_items, st);
-  return tc_launch<4, false>(mq, mk, mv, args, max_items, st);
+  if (r == 1) return tc_launch<1>(mq, mk, mv, args, max_items, st);
+  if (r == 2) return tc_launch<2>(mq, mk, mv, args, max_items, st);
+  return tc_launch<4>(mq, mk, mv, args, max_items, st);
 }
 
 }  // namespace mtfm

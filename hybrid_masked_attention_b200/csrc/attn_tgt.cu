@@ -1,0 +1,524 @@
+// sm_100a forward kernel of the Target-Attention layer (page "美团推荐大模型 MTFM
+// 深度硬核解析" §4.2: only T rows query, keys and values span the whole sequence):
+//     A[i, h] = (1/N_u) sum_{j visible from i} SiLU(alpha q[i,h].k[j,g]) v[j,g]
+// for the T rows i of each user, visibility as in the Full layer (Meituan tech
+// blog §3.2: the H keys, the R keys with ts < exposure, the sibling block).
+//
+// The r = hq / hkv query heads of a KV group are stacked as MMA rows: a 128-row
+// tile holds TR = 128 / r T rows x r heads (row m = t r + h, which is exactly the
+// shared-memory order of a 3-D TMA box {64 dims, r heads, TR rows} of Q), so one
+// QK^T and one PV MMA chain per 128-key block serve all r heads and the few T rows
+// of a user fill the tile.  A work unit is one (sub-tile of TR T rows, chunk of
+// kTargetUnitBlocks key blocks, KV group); the CTAs (one per SM) stride over them.
+//
+// Roles and the pipeline across units (no block-wide barrier per unit):
+//   warp 0      : TMA producer.  Q tiles into two buffers (the next unit's Q
+//                 loads while this unit computes), K/V blocks through a 3-stage ring.
+//   warp 1      : TMEM allocation and MMA issue.  S = Q K^T into one of three
+//                 S buffers, issued up to two steps ahead (also into the next
+//                 unit), then O += P_hi V + P_lo V into one of two O buffers.
+//   warps 4..19 : SiLU warpgroups (as in the Full-layer kernel: each warpgroup
+//                 takes 32 of the 128 key columns of a step), then the unit's
+//                 epilogue: O / N_u from TMEM into a swizzled shared-memory tile
+//                 and one TMA reduce-add per 32 columns into A (fp32, zeroed
+//                 first), so chunks of the key range sum without atomics in the
+//                 kernel; rows past the user's last T row are staged as zeros.
+// TMEM: O buffers at columns [0, 64) and [64, 128), S buffers at [128 + 128b, +128).
+// Every mbarrier wait is bounded; after a timeout the roles stop issuing work and
+// drain (bounded), the SiLU warps still pass their named barriers the same
+// number of times, and MetaHeader::error gets the timeout bit.
+#include <cuda.h>
+
+#include <algorithm>
+#include <type_traits>
+
+#include "mma_util.cuh"
+#include "mtfm_internal.cuh"
+#include "sm100.cuh"
+#include "tma_host.cuh"
+
+namespace mtfm {
+namespace {
+
+using namespace sm100;
+
+constexpr int kDH = 64;
+constexpr int kBN = 128;     // keys per block
+constexpr int kStages = 3;   // K/V ring
+constexpr int kSBuf = 3;     // S/P buffers
+constexpr int kSiluWG = 4;
+constexpr int kThreads = 128 + 128 * kSiluWG;
+constexpr uint32_t kQBytes = 128 * kDH * 2;   // one stacked Q tile
+constexpr uint32_t kKVBytes = kBN * kDH * 2;
+constexpr uint32_t kStageBytes = 128 * kDH * 4;  // O tile in fp32: 2r boxes of TR x 32
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCol0 = 128;
+static_assert(kBN == kKeyBlock, "the packer sizes Target units in blocks of kKeyBlock keys");
+static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "TMEM plan");
+
+constexpr int kRing = 4;                 // decoded-unit descriptors in flight
+constexpr int kDescConsumers = 2 + 16;   // producer, MMA warp, 16 SiLU warps
+constexpr size_t tgt_smem_bytes() { return 2 * kQBytes + 2 * kStages * kKVBytes + kStageBytes + 1024; }
+
+struct TgtArgs {
+  MetaView m;
+  int hq, hkv, v2;
+  float alpha;
+};
+
+// One work unit of this kernel, decoded from the metadata.
+struct TgtUnit {
+  int u, so, LH, LR, LT, N, g;
+  int q_sub0;  // first T row (within the user's T rows) of the sub-tile
+  int bi0, nb, kv_min;
+  KeyBlocks kb;
+};
+
+template <int R>
+__device__ TgtUnit decode_unit(const MetaView& m, int w, int hkv, int v2) {
+  constexpr int TR = 128 / R;
+  TgtUnit U;
+  const int unit = w / hkv;
+  U.g = w % hkv;
+  int lo = 0, hi = m.hdr->n_items_target - 1;  // last item whose first unit is <= unit
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (m.unit_off[mid] <= unit) lo = mid; else hi = mid - 1;
+  }
+  const int local = unit - m.unit_off[lo];
+  const WorkItem it = m.items_target[lo];
+  U.u = it.user;
+  U.LH = m.lh[U.u];
+  U.LR = m.lr[U.u];
+  U.LT = m.lt[U.u];
+  U.N = U.LH + U.LR + U.LT;
+  U.so = m.seq_off[U.u];
+  const int q0 = it.tile * kTileM;
+  U.kb = key_blocks(it.kv_max, U.LH, U.LR, U.LT, U.LH + U.LR, q0, v2);
+  const int C = m.hdr->tgt_chunk_blocks;
+  const int nchunks = (U.kb.n_blocks + C - 1) / C;
+  const int sub = local / nchunks, chunk = local % nchunks;
+  U.q_sub0 = q0 + sub * TR;
+  U.bi0 = chunk * C;
+  U.nb = min(U.bi0 + C, U.kb.n_blocks) - U.bi0;
+  U.kv_min = it.kv_min;
+  return U;
+}
+
+// SiLU of 32 scores of one row, masked, split into bf16 hi/lo pairs (same
+// arithmetic as the Full-layer kernel: P = h + h tanh(h), h = alpha s / 2).
+template <bool MASKED>
+__device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half_alpha, uint32_t vis,
+                                           uint32_t (&ph)[16], uint32_t (&pl)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float h0 = half_alpha * __uint_as_float(raw[2 * e]);
+    const float h1 = half_alpha * __uint_as_float(raw[2 * e + 1]);
+    float p0 = fmaf(h0, tanh_approx(h0), h0);
+    float p1 = fmaf(h1, tanh_approx(h1), h1);
+    if (MASKED) {
+      p0 = (vis & (1u << (2 * e))) ? p0 : 0.f;
+      p1 = (vis & (2u << (2 * e))) ? p1 : 0.f;
+    }
+    split_trunc_bf16x2(p0, p1, ph[e], pl[e]);
+  }
+}
+
+__device__ __forceinline__ void silu_bar() { asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory"); }
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+                    TgtArgs p) {
+  constexpr int TR = 128 / R;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_qf[2], bar_qe[2], bar_of[2], bar_oe[2], bar_drain;
+  __shared__ __align__(8) uint64_t bar_kvf[kStages], bar_kve[kStages], bar_sf[kSBuf], bar_pf[kSBuf];
+  __shared__ __align__(8) uint64_t bar_df[kRing], bar_de[kRing];
+  __shared__ TgtUnit s_desc[kRing];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const MetaView& m = p.m;
+  MetaHeader* hdr = m.hdr;
+  if (hdr->error) return;
+  if (hdr->tgt_sub_rows != TR) {  // packed for another head configuration
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&hdr->error, kErrConfig);
+    return;
+  }
+  const int n_work = hdr->n_units_target * p.hkv;
+  if ((int)blockIdx.x >= n_work) return;
+  const int n_mine = (n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // units of this CTA
+  auto unit_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_addr(smem);
+  const uint32_t sK = sQ + 2 * kQBytes;
+  const uint32_t sV = sK + kStages * kKVBytes;
+  const uint32_t sO = sV + kStages * kKVBytes;
+  uint8_t* stage = smem + 2 * kQBytes + 2 * kStages * kKVBytes;
+
+  auto B = [&](uint64_t* b) { return smem_addr(b); };
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(B(&bar_qf[i]), 1);
+      mbar_init(B(&bar_qe[i]), 1);
+      mbar_init(B(&bar_of[i]), 1);
+      mbar_init(B(&bar_oe[i]), 128 * kSiluWG);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(B(&bar_kvf[s]), 1);
+      mbar_init(B(&bar_kve[s]), 1);
+    }
+    for (int b = 0; b < kSBuf; ++b) {
+      mbar_init(B(&bar_sf[b]), 1);
+      mbar_init(B(&bar_pf[b]), 128 * kSiluWG);
+    }
+    for (int j = 0; j < kRing; ++j) {
+      mbar_init(B(&bar_df[j]), 1);
+      mbar_init(B(&bar_de[j]), kDescConsumers);
+    }
+    mbar_init(B(&bar_drain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&s_tmem), kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_a);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+  // Unit descriptors come from warp 2 through a ring in shared memory, so that the
+  // dependent loads of the decode stay off the other roles' critical paths.
+  auto get_desc = [&](int k, TgtUnit& U) -> bool {
+    if (!mbar_wait(B(&bar_df[k % kRing]), (k / kRing) & 1, abort_flag)) return false;
+    U = s_desc[k % kRing];
+    return true;
+  };
+  auto release_desc = [&](int k) { mbar_arrive(B(&bar_de[k % kRing])); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      int G = 0, nq_loads = 0;
+      bool ok = true;
+      for (int k = 0; ok && k < n_mine; ++k) {
+        TgtUnit U;
+        if (!get_desc(k, U)) break;
+        release_desc(k);
+        const int qb = k & 1;
+        if (k >= 2 && !mbar_wait(B(&bar_qe[qb]), ((k - 2) >> 1) & 1, abort_flag)) break;
+        mbar_expect_tx(B(&bar_qf[qb]), kQBytes);
+        tma_load_3d(sQ + qb * kQBytes, &tm_q, B(&bar_qf[qb]), 0, U.g * R, m.t_off[U.u] + U.q_sub0);
+        ++nq_loads;
+        for (int i = 0; i < U.nb; ++i) {
+          const int s = G % kStages;
+          if (G >= kStages && !mbar_wait(B(&bar_kve[s]), ((G / kStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int row = U.so + U.kb.block(U.bi0 + i) * kBN;
+          mbar_expect_tx(B(&bar_kvf[s]), 2 * kKVBytes);
+          tma_load_2d(sK + s * kKVBytes, &tm_k, B(&bar_kvf[s]), U.g * kDH, row);
+          tma_load_2d(sV + s * kKVBytes, &tm_v, B(&bar_kvf[s]), U.g * kDH, row);
+          ++G;
+        }
+      }
+      // no TMA write may land after the CTA leaves: wait (bounded) for the last loads
+      const long long t0 = clock64();
+      auto drain = [&](uint32_t bar, uint32_t par) {
+        while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
+        }
+      };
+      for (int q = max(0, nq_loads - 2); q < nq_loads; ++q) drain(B(&bar_qf[q & 1]), (q >> 1) & 1);
+      for (int g2 = max(0, G - kStages); g2 < G; ++g2) drain(B(&bar_kvf[g2 % kStages]), (g2 / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBN, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kDH, true);
+    const uint32_t dhi = sw128_desc_hi(1024);
+    const uint32_t q_lo = sw128_desc_lo(sQ, 16), k_lo = sw128_desc_lo(sK, 16), v_lo = sw128_desc_lo(sV, 16);
+    bool ok = true;
+    // S cursor: unit ks, step is within it, global step gs
+    int ks = 0, is = 0, gs = 0, nb_s = 0;
+    auto issue_s = [&]() -> bool {
+      if (is == 0) {  // first S of unit ks: its descriptor (released after its PVs)
+        TgtUnit U;
+        if (!__all_sync(0xffffffffu, get_desc(ks, U))) return false;
+        nb_s = U.nb;
+      }
+      if (is == 0 && !__all_sync(0xffffffffu, mbar_wait(B(&bar_qf[ks & 1]), (ks >> 1) & 1, abort_flag)))
+        return false;
+      const int s = gs % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_kvf[s]), (gs / kStages) & 1, abort_flag))) return false;
+      tc_fence_after();
+      const uint32_t d = tmem + kSCol0 + (gs % kSBuf) * kBN;
+      const uint32_t a0 = q_lo + (ks & 1) * (kQBytes >> 4), b0 = k_lo + s * (kKVBytes >> 4);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kDH / 16; ++kk)
+          mma_ss2(d, a0 + kk * 2, dhi, b0 + kk * 2, dhi, idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(B(&bar_sf[gs % kSBuf]));
+        if (is == nb_s - 1) mma_commit(B(&bar_qe[ks & 1]));  // this Q tile is no longer read
+      }
+      __syncwarp();
+      ++gs;
+      if (++is == nb_s) {
+        is = 0;
+        ++ks;
+      }
+      return true;
+    };
+    int gp = 0;
+    for (int k = 0; ok && k < n_mine; ++k) {
+      // unit k's descriptor stays in the ring until this warp releases it below
+      TgtUnit Uk;
+      if (!__all_sync(0xffffffffu, get_desc(k, Uk))) {
+        ok = false;
+        break;
+      }
+      const int nb = Uk.nb;
+      const int ob = k & 1;
+      for (int i = 0; ok && i < nb; ++i, ++gp) {
+        while (ok && ks < n_mine && gs <= gp + (kSBuf - 1)) ok = issue_s();
+        if (!ok) break;
+        const int b = gp % kSBuf;
+        if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_pf[b]), (gp / kSBuf) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (i == 0 && k >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(B(&bar_oe[ob]), ((k >> 1) - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo
+        const uint32_t o = tmem + ob * kDH;
+        const uint32_t vb = v_lo + (gp % kStages) * (kKVBytes >> 4);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
+            mma_ts2(o, pt + col, vb + kk * (2048 >> 4), dhi, idesc_pv, (kk > 0 || i > 0) ? 1u : 0u);
+            mma_ts2(o, pt + col + 16, vb + kk * (2048 >> 4), dhi, idesc_pv, 1u);
+          }
+          mma_commit(B(&bar_kve[gp % kStages]));
+          if (i == nb - 1) mma_commit(B(&bar_of[ob]));
+        }
+        __syncwarp();
+      }
+      if (ok && lane == 0) release_desc(k);
+      __syncwarp();
+    }
+    if (!ok) {
+      // drain every MMA issued so far before TMEM is released
+      if (elect_one()) mma_commit(B(&bar_drain));
+      __syncwarp();
+      const long long t0 = clock64();
+      while (!mbar_try(B(&bar_drain), 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- unit scheduler
+    if (lane == 0) {
+      for (int k = 0; k < n_mine; ++k) {
+        const int j = k % kRing;
+        if (k >= kRing && !mbar_wait(B(&bar_de[j]), ((k / kRing) - 1) & 1, abort_flag)) break;
+        s_desc[j] = decode_unit<R>(m, unit_of(k), p.hkv, p.v2);
+        mbar_arrive(B(&bar_df[j]));  // release: the descriptor is visible to every waiter
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- SiLU warpgroups + epilogue
+    const int wg = (warp - 4) >> 2;  // key columns [32 wg, 32 wg + 32) of each step
+    const int quad = warp & 3;
+    const int mrow = quad * 32 + lane;  // TMEM lane = MMA row = t * R + h
+    const int t = mrow / R, hh = mrow % R;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const float half_alpha = 0.5f * p.alpha;
+    const bool issuer = threadIdx.x == 128;
+    bool ok = true;
+    int gp = 0;
+    // Epilogue of unit e.k: O / N_u -> swizzled staging tile -> TMA reduce-add into A.
+    // Each call passes the two named barriers, whatever e.ok says.
+    struct Prev {
+      int k, col, y;
+      bool ok;
+      float inv_n;
+    } prev{0, 0, 0, false, 0.f};
+    auto epilogue = [&](const Prev& e) {
+      const int ob = e.k & 1;
+      bool eok = e.ok && ok;
+      if (eok) eok = __all_sync(0xffffffffu, mbar_wait(B(&bar_of[ob]), (e.k >> 1) & 1, abort_flag));
+      if (!eok) ok = false;
+      if (issuer) bulk_wait_read<0>();  // the previous reduces have read the staging tile
+      silu_bar();
+      if (eok) {
+        tc_fence_after();
+        uint32_t raw[16];
+        tmem_ld16(lane_base + ob * kDH + wg * 16, raw);  // O columns [16 wg, 16 wg + 16)
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(B(&bar_oe[ob]));
+        const int box = hh * 2 + (wg >> 1);  // 32-column box of this head
+        uint8_t* rowp = stage + box * (TR * 128) + t * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int chunk = (wg & 1) * 4 + j;  // 16-byte chunk within the 128-byte row
+          *reinterpret_cast<float4*>(rowp + ((chunk ^ (t & 7)) << 4)) =
+              make_float4(__uint_as_float(raw[4 * j]) * e.inv_n, __uint_as_float(raw[4 * j + 1]) * e.inv_n,
+                          __uint_as_float(raw[4 * j + 2]) * e.inv_n, __uint_as_float(raw[4 * j + 3]) * e.inv_n);
+        }
+        fence_proxy_async();
+      }
+      silu_bar();
+      if (eok && issuer) {
+        for (int b = 0; b < 2 * R; ++b)
+          tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), e.col + (b >> 1) * kDH + (b & 1) * 32, e.y);
+        bulk_commit();
+      }
+    };
+    // Every SiLU warp walks all n_mine units, also after an abort, so that all of
+    // them pass the named barriers of each epilogue the same number of times.
+    for (int k = 0; k < n_mine; ++k) {
+      TgtUnit U;
+      if (ok) ok = __all_sync(0xffffffffu, get_desc(k, U));
+      __syncwarp();
+      if (ok && lane == 0) release_desc(k);
+      if (!ok) U = TgtUnit{};  // after an abort: no work, only the barriers below
+      const int qi = U.q_sub0 + t;  // T row within the user
+      const bool valid = qi < U.LT;
+      int kv_end = 0, sib_lo = 0, sib_hi = 0;
+      const int t0pos = U.LH + U.LR;
+      if (valid) {
+        const int pos = t0pos + qi;
+        kv_end = m.kv_end[U.so + pos];
+        sib_lo = t0pos + (qi / p.v2) * p.v2;
+        sib_hi = sib_lo + p.v2;
+      }
+      const int n_full = max(0, min(U.nb, min(U.kb.nb_pre, U.kv_min / kBN) - U.bi0));
+      auto step = [&](int i, auto masked_tag) -> bool {
+        constexpr bool kMasked = decltype(masked_tag)::value;
+        const int buf = (gp + i) % kSBuf;
+        if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_sf[buf]), ((gp + i) / kSBuf) & 1, abort_flag)))
+          return false;
+        tc_fence_after();
+        const uint32_t sb = lane_base + kSCol0 + buf * kBN + wg * 32;
+        uint32_t raw[32];
+        tmem_ld32(sb, raw);
+        tmem_ld_wait();
+        uint32_t ph[16], pl[16];
+        if (!kMasked) {
+          silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
+        } else {
+          const int j0 = U.kb.block(U.bi0 + i) * kBN + wg * 32;
+          const uint32_t vis = vis_bits(j0, kv_end, sib_lo, sib_hi);
+          if (__all_sync(0xffffffffu, vis == 0u)) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ph[e] = pl[e] = 0u;
+          } else if (__all_sync(0xffffffffu, vis == 0xffffffffu)) {
+            silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
+          } else {
+            silu_chunk<true>(raw, half_alpha, vis, ph, pl);
+          }
+        }
+        tmem_st16(sb, ph);       // P_hi over the first 16 columns of the chunk's S
+        tmem_st16(sb + 16, pl);  // P_lo over the next 16
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(B(&bar_pf[buf]));
+        return true;
+      };
+      auto run_steps = [&](int i0, int i1) {
+        for (int i = i0; ok && i < min(i1, n_full); ++i) ok = step(i, std::false_type{});
+        for (int i = max(i0, n_full); ok && i < i1; ++i) ok = step(i, std::true_type{});
+      };
+      // The epilogue of the previous unit runs after this unit's first step, so the
+      // wait for the previous unit's last PV overlaps that step's SiLU.
+      run_steps(0, 1);
+      if (k > 0) epilogue(prev);
+      run_steps(1, U.nb);
+      gp += U.nb;
+      prev.k = k;
+      prev.ok = ok;
+      prev.inv_n = valid && U.N > 0 ? 1.f / (float)U.N : 0.f;  // rows past the user's T rows add zeros
+      prev.col = U.g * R * kDH;
+      prev.y = ok ? m.t_off[U.u] + U.q_sub0 : 0;
+    }
+    if (n_mine > 0) epilogue(prev);
+    if (issuer) bulk_wait<0>();  // every reduce has completed before the CTA leaves
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && s_abort) atomicOr(&hdr->error, kErrTimeout);
+}
+
+}  // namespace
+
+// Q [total_t, hq * 64] as a 3-D tensor {64 dims, hq heads, total_t rows}: a box of
+// {64, r, 128 / r} is one stacked tile.  A [total_t, hq * 64] fp32 in boxes of 32 x TR.
+cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_items, int total_t,
+                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                const __nv_bfloat16* v, float* a, cudaStream_t st) {
+  if (max_items <= 0 || total_t <= 0 || total_tokens <= 0) return cudaSuccess;
+  const int r = s.hq / s.hkv;
+  const int TR = 128 / r;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, ma;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)kDH, (cuuint64_t)s.hq, (cuuint64_t)total_t};
+    cuuint64_t strides[2] = {(cuuint64_t)kDH * 2, (cuuint64_t)s.hq * kDH * 2};
+    cuuint32_t box[3] = {(cuuint32_t)kDH, (cuuint32_t)r, (cuuint32_t)TR};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  if (!make_map_bf16(&mk, k, (uint64_t)total_tokens, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH) ||
+      !make_map_bf16(&mv, v, (uint64_t)total_tokens, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH))
+    return cudaErrorInvalidValue;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)s.hq * kDH, (cuuint64_t)total_t};
+    cuuint64_t strides[1] = {(cuuint64_t)s.hq * kDH * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)TR};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaMemsetAsync(a, 0, sizeof(float) * (size_t)total_t * s.hq * kDH, st);  // units add partial sums
+  if (e != cudaSuccess) return e;
+  TgtArgs args{m, s.hq, s.hkv, s.v2, s.alpha};
+  const size_t smem = tgt_smem_bytes();
+  const int grid = sm_count();
+  auto launch = [&](auto kern) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e2 != cudaSuccess) return e2;
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, ma, args);
+    return cudaGetLastError();
+  };
+  if (r == 1) return launch(attn_fwd_tgt_kernel<1>);
+  if (r == 2) return launch(attn_fwd_tgt_kernel<2>);
+  return launch(attn_fwd_tgt_kernel<4>);
+}
+
+}  // namespace mtfm

@@ -16,6 +16,7 @@ constexpr int kRowH = 0, kRowR = 1, kRowT = 2;
 constexpr int kErrBadLengths = 1;
 constexpr int kErrUnsorted = 2;
 constexpr int kErrTimeout = 4;
+constexpr int kErrConfig = 8;  // a kernel's head configuration differs from the packed one
 
 constexpr int kMetaMagic = 0x4d54464d;  // "MTFM"
 
@@ -34,9 +35,15 @@ struct MetaHeader {
   int32_t max_items_target;
   int32_t n_units_target;  // key-range chunks of the Target work list (sum of unit_count)
   // Work counter of the persistent Full-layer forward kernel: [0] next unit, [1] CTAs
-  // finished ([2], [3] reserved).  Zeroed by the packer; the last CTA of a launch to
-  // finish sets both back to zero for the next launch.
-  uint32_t sched[4];
+  // finished.  Zeroed by the packer; the last CTA of a launch to finish sets both back
+  // to zero for the next launch.
+  uint32_t sched[2];
+  // T rows per sub-tile of the Target-layer units (128 / (hq / hkv) for r in {1, 2, 4},
+  // else 128): the packer sizes the Target units with it, the kernel checks it.
+  int32_t tgt_sub_rows;
+  // Key blocks per Target unit (>= kTargetUnitBlocks): the packer picks it so that the
+  // layer has a few units per SM, splitting long key ranges only as far as needed.
+  int32_t tgt_chunk_blocks;
 };
 
 // One work item: a 128-row query tile of one user and the range of prefix
@@ -119,7 +126,15 @@ inline MetaView meta_view(void* base, const MetaLayout& L) {
 // the item's T rows that the prefix does not cover.  Shared by the packer (to
 // size the Target split) and the kernel (to walk the blocks).
 constexpr int kKeyBlock = 128;
-constexpr int kTargetUnitBlocks = 2;  // key blocks per Target work unit (split of the key range)
+constexpr int kTargetUnitBlocks = 2;  // smallest key chunk of a Target work unit
+constexpr int kTargetUnitsPerSM = 8;  // the packer aims at about this many Target units per SM
+
+// T rows of a Target-layer sub-tile when the r = hq / hkv query heads of a KV group
+// are stacked as MMA rows (128 = rows x r); 128 when that kernel does not apply.
+__host__ __device__ inline int target_sub_rows(int hq, int hkv) {
+  const int r = hkv > 0 ? hq / hkv : 1;
+  return (r == 1 || r == 2 || r == 4) ? 128 / r : 128;
+}
 
 struct KeyBlocks {
   int nb_pre, sb_lo, n_blocks;
@@ -163,6 +178,10 @@ bool attn_fwd_tc_supported(const AttnShape& s);
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                const __nv_bfloat16* v, float* a, cudaStream_t st);
+// Target layer, heads stacked as MMA rows (head_dim 64, hq / hkv in {1, 2, 4}).
+cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_items, int total_t,
+                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                const __nv_bfloat16* v, float* a, cudaStream_t st);
 cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, float eps,
                             const float* a, const __nv_bfloat16* u, const float* gamma,
                             const float* beta, float* y, float* stats, cudaStream_t st);

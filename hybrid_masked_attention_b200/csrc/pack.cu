@@ -16,10 +16,11 @@
 //     longest first and writes the work lists of 128-row query tiles;
 //   pack_rows_kernel (1 CTA per work item): per-row kv_end / row type, the
 //     sortedness check, and each tile's [kv_min, kv_max] used for block skipping;
-//   pack_units_kernel (1 CTA): prefix sums of the Target tiles' key-range units
-//     (each Target tile's keys are split into chunks of kTargetUnitBlocks blocks,
-//     so that short Target layers still fill every SM).
+//   pack_units_kernel (1 CTA): the Target layer's work units (sub-tiles of T rows
+//     times chunks of the key range, the chunk sized so that short Target layers
+//     still fill every SM) and their prefix sums.
 #include "mtfm_internal.cuh"
+#include "tma_host.cuh"
 
 namespace mtfm {
 namespace {
@@ -55,7 +56,7 @@ __device__ long long block_exclusive_scan(long long v, long long* total, long lo
 }
 
 __global__ void __launch_bounds__(kPackThreads)
-pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t, int v2,
+pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t, int v2, int tgt_sub_rows,
                   int max_if, int max_it, int sort_n, const int32_t* __restrict__ lh,
                   const int32_t* __restrict__ lr, const int32_t* __restrict__ lt) {
   extern __shared__ unsigned long long s_keys[];  // [sort_n] (0 when not sorting)
@@ -102,7 +103,9 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->max_items_full = max_if;
       m.hdr->max_items_target = max_it;
       m.hdr->n_units_target = 0;
-      for (int i = 0; i < 4; ++i) m.hdr->sched[i] = 0;
+      m.hdr->sched[0] = m.hdr->sched[1] = 0;
+      m.hdr->tgt_sub_rows = tgt_sub_rows;
+      m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
     }
     return;
   }
@@ -189,7 +192,9 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->max_items_full = max_if;
     m.hdr->max_items_target = max_it;
     m.hdr->n_units_target = 0;
-    for (int i = 0; i < 4; ++i) m.hdr->sched[i] = 0;
+    m.hdr->sched[0] = m.hdr->sched[1] = 0;
+    m.hdr->tgt_sub_rows = tgt_sub_rows;
+    m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
   }
 }
 
@@ -204,7 +209,7 @@ __device__ __forceinline__ int count_below(const int64_t* __restrict__ ts, int n
 }
 
 __global__ void __launch_bounds__(kTileM)
-pack_rows_kernel(MetaView m, int max_if, const int64_t* __restrict__ r_ts,
+pack_rows_kernel(MetaView m, int max_if, int tgt_sub_rows, const int64_t* __restrict__ r_ts,
                  const int64_t* __restrict__ t_exp) {
   __shared__ int s_min[kTileM / 32], s_max[kTileM / 32];
   const MetaHeader* hdr = m.hdr;
@@ -262,34 +267,59 @@ pack_rows_kernel(MetaView m, int max_if, const int64_t* __restrict__ r_ts,
     it->kv_min = kmin;
     it->kv_max = kmax;
     if (tgt) {
-      // number of key-range units this Target tile is split into (scanned by pack_units_kernel)
+      // this Target tile's sub-tiles (of tgt_sub_rows T rows) and key blocks, packed
+      // as nsub * 65536 + blocks; pack_units_kernel turns them into unit counts
       const KeyBlocks kb = key_blocks(kmax, LH, LR, LT, LH + LR, tile * kTileM, hdr->v2);
-      m.unit_off[idx + 1] = (kb.n_blocks + kTargetUnitBlocks - 1) / kTargetUnitBlocks;
+      const int rows = min(kTileM, LT - tile * kTileM);
+      const int nsub = (rows + tgt_sub_rows - 1) / tgt_sub_rows;
+      m.unit_off[idx + 1] = nsub * 65536 + kb.n_blocks;
       if (idx == 0) m.unit_off[0] = 0;
     }
   }
 }
 
-// In-place inclusive scan of the Target units per item: unit_off[i] becomes the
-// first unit of item i; n_units_target the total.
-__global__ void __launch_bounds__(kPackThreads) pack_units_kernel(MetaView m) {
+// Target units: choose the key chunk C (blocks per unit) so that the layer has about
+// kTargetUnitsPerSM units per SM (C >= kTargetUnitBlocks; a tile is split only when
+// the layer is short), then units per item = sub-tiles * ceil(blocks / C), scanned in
+// place: unit_off[i] becomes the first unit of item i; n_units_target the total.
+__global__ void __launch_bounds__(kPackThreads) pack_units_kernel(MetaView m, int hkv, int n_sm) {
   __shared__ long long s_warp[32];
+  __shared__ int s_chunk;
   MetaHeader* hdr = m.hdr;
   if (hdr->error & kErrBadLengths) return;
   const int n = hdr->n_items_target;
-  const int chunk = (n + kPackThreads - 1) / kPackThreads;
-  const int a = min(n, (int)threadIdx.x * chunk), b = min(n, a + chunk);
+  const int per = (n + kPackThreads - 1) / kPackThreads;
+  const int a = min(n, (int)threadIdx.x * per), b = min(n, a + per);
+  long long steps = 0;  // sub-tile key blocks of my items
+  for (int i = a; i < b; ++i) {
+    const int v = m.unit_off[i + 1];
+    steps += (long long)(v >> 16) * (v & 0xffff);
+  }
+  long long total_steps;
+  block_exclusive_scan(steps, &total_steps, s_warp);
+  if (threadIdx.x == 0) {
+    const long long target_units = (long long)kTargetUnitsPerSM * n_sm;
+    const long long c = (total_steps * hkv + target_units - 1) / target_units;
+    s_chunk = (int)max((long long)kTargetUnitBlocks, min(c, (long long)1 << 20));
+  }
+  __syncthreads();
+  const int C = s_chunk;
   long long local = 0;
-  for (int i = a; i < b; ++i) local += m.unit_off[i + 1];
+  for (int i = a; i < b; ++i) {
+    const int v = m.unit_off[i + 1];
+    local += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
+  }
   long long total;
   long long run = block_exclusive_scan(local, &total, s_warp);
   for (int i = a; i < b; ++i) {
-    run += m.unit_off[i + 1];
+    const int v = m.unit_off[i + 1];
+    run += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
     m.unit_off[i + 1] = (int)run;
   }
   if (threadIdx.x == 0) {
     m.unit_off[0] = 0;
     hdr->n_units_target = (int)total;
+    hdr->tgt_chunk_blocks = C;
   }
 }
 
@@ -313,18 +343,19 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  const int tsr = target_sub_rows(cfg.hq, cfg.hkv);
   pack_users_kernel<<<1, kPackThreads, smem, st>>>(m, cfg.batch, cfg.total_tokens, cfg.total_r,
-                                                   cfg.total_t, cfg.v2_subtokens,
+                                                   cfg.total_t, cfg.v2_subtokens, tsr,
                                                    L.max_items_full, L.max_items_target, sort_n,
                                                    lh, lr, lt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int blocks = L.max_items_full + L.max_items_target;
   if (blocks > 0) {
-    pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, r_ts, t_exp);
+    pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, tsr, r_ts, t_exp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    pack_units_kernel<<<1, kPackThreads, 0, st>>>(m);
+    pack_units_kernel<<<1, kPackThreads, 0, st>>>(m, cfg.hkv > 0 ? cfg.hkv : 1, sm_count());
     e = cudaGetLastError();
   }
   return e;

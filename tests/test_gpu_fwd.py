@@ -82,7 +82,8 @@ def test_work_counters_rewind(cuda_ok):
     torch.cuda.synchronize()
     hdr = s.meta[:64].view(torch.int32).cpu().numpy()
     assert hdr[8] == 0, "error flag"
-    assert (hdr[12:16] == 0).all(), f"work counters not rewound: {hdr[12:16]}"
+    assert (hdr[12:14] == 0).all(), f"work counters not rewound: {hdr[12:14]}"
+    assert hdr[14] == 128 // (hd.hq // hd.hkv), "T rows per Target sub-tile"
     (yf0, af0, _), (yt0, at0, _) = outs[0]
     for (yf, af, _), (yt, at, _) in outs[1:]:
         assert torch.equal(af, af0) and torch.equal(yf, yf0)
