@@ -197,6 +197,15 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
                       da_lo, partials, kGateBwdBlocks, d_dgamma, d_dbeta, st);
   if (e != cudaSuccess) return MTFM_ERR_CUDA;
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
+  // tcgen05 kernel for head_dim 64; the mma.sync kernel for the other head sizes
+  // (MTFM_BWD_KERNEL=mma selects it for every shape, to compare the two).
+  const char* force = getenv("MTFM_BWD_KERNEL");
+  if (!(force && strcmp(force, "mma") == 0) && attn_bwd_tc_supported(shape)) {
+    e = launch_attn_bwd_tc(shape, m, L.max_items_full, rows, r.total_tokens,
+                           reinterpret_cast<const __nv_bfloat16*>(d_q), reinterpret_cast<const __nv_bfloat16*>(d_k),
+                           reinterpret_cast<const __nv_bfloat16*>(d_v), da_hi, da_lo, d_dq, d_dk, d_dv, st);
+    return cuda_status(e);
+  }
   e = launch_attn_bwd_mma(shape, m, L.max_items_full, reinterpret_cast<const __nv_bfloat16*>(d_q),
                           reinterpret_cast<const __nv_bfloat16*>(d_k),
                           reinterpret_cast<const __nv_bfloat16*>(d_v), da_hi, da_lo, d_dq, d_dk,

@@ -191,6 +191,12 @@ cudaError_t launch_gate_bwd(const MetaView& m, bool target, int rows, int D, flo
                             float* du, __nv_bfloat16* da_hi, __nv_bfloat16* da_lo,
                             float* partials, int n_part_blocks,
                             float* dgamma, float* dbeta, cudaStream_t st);
+// tcgen05 backward (head_dim 64): dQ (zeroed first, accumulated), dK, dV (written).
+bool attn_bwd_tc_supported(const AttnShape& s);
+cudaError_t launch_attn_bwd_tc(const AttnShape& s, const MetaView& m, int max_items_full, int rows_q,
+                               int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                               const __nv_bfloat16* v, const __nv_bfloat16* da_hi, const __nv_bfloat16* da_lo,
+                               float* dq, float* dk, float* dv, cudaStream_t st);
 cudaError_t launch_attn_bwd_mma(const AttnShape& s, const MetaView& m, int max_items_full,
                                 const __nv_bfloat16* q, const __nv_bfloat16* k,
                                 const __nv_bfloat16* v, const __nv_bfloat16* da_hi,
