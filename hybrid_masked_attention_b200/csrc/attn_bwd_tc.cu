@@ -23,22 +23,22 @@
 //   dK  += dS^T Q        (A operand from TMEM)
 // and after the second step of a super-tile
 //   dQ   = dS K          (M 128 queries: A = dS^T read MN-major from shared memory)
-// which goes to dQ (fp32, zeroed first) through a swizzled staging tile and TMA
-// reduce-add, since several key blocks add to the same query rows.  dK and dV
+// which goes to dQ (fp32, zeroed first) with fp32 vector atomics, since several
+// key blocks add to the same query rows.  dK and dV
 // stay in TMEM for the whole unit and are stored once (each key block belongs to
 // exactly one unit per group).
 //
-// Roles: warp 0 TMA (K/V block per unit, double-buffered; Q, dA_hi, dA_lo tiles
-// per step through a 2-stage ring), warp 1 TMEM allocation and MMA issue (one
+// Roles: warp 0 TMA (K/V block per unit; Q, dA_hi, dA_lo tiles per step through
+// a 2-stage ring), warp 1 TMEM allocation and MMA issue (one
 // elected lane; S^T/dP^T one step ahead), warps 4..19 the elementwise work and
 // the dQ / dK / dV epilogues.  TMEM: dV [0, 64), dK [64, 128), dQ buffers
 // [128, 192) and [192, 256), S^T / dP^T buffer b at [256 + 128 b, +64) / [+64, +128).
 // Every mbarrier wait is bounded; after a timeout the roles stop issuing work,
-// drain (bounded), the SiLU warps still pass their named barriers the same
-// number of times, and MetaHeader::error gets the timeout bit.
+// drain (bounded), and MetaHeader::error gets the timeout bit.
 #include <cuda.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "mma_util.cuh"
 #include "mtfm_internal.cuh"
@@ -59,16 +59,18 @@ constexpr uint32_t kKVTile = kKB * kDH * 2;   // 16 KB: one K or V block
 constexpr uint32_t kQTile = kQS * kDH * 2;    // 8 KB: Q, dA_hi or dA_lo tile of a step
 constexpr uint32_t kStepBytes = 3 * kQTile;   // one stage of the Q/dA ring
 constexpr uint32_t kDSHalf = kKB * kQS * 2;   // 16 KB: dS^T for 64 queries, one part
-constexpr uint32_t kDQStage = 128 * kDH * 4;  // 32 KB: dQ staging (2 boxes of 128 x 32 fp32)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDV = 0, kColDK = 64, kColDQ = 128, kColSP = 256;
 
 // shared memory map (offsets from the 1024-aligned base)
-constexpr uint32_t kOffKV = 0;                              // 2 x (K, V)
-constexpr uint32_t kOffStage = kOffKV + 4 * kKVTile;        // 2 x (Q, dA_hi, dA_lo)
-constexpr uint32_t kOffDS = kOffStage + 2 * kStepBytes;     // dS^T hi: 2 halves, then lo: 2 halves
-constexpr uint32_t kOffDQ = kOffDS + 4 * kDSHalf;           // dQ staging
-constexpr size_t kSmemBytes = kOffDQ + kDQStage + 1024;
+constexpr int kStages = 2;                                  // Q / dA ring
+constexpr uint32_t kOffKV = 0;                              // K, V of the unit
+constexpr uint32_t kOffStage = kOffKV + 2 * kKVTile;        // kStages x (Q, dA_hi, dA_lo)
+// dS^T of a super-tile: hi (2 query halves), then lo (2 halves); two buffers, so
+// that the SiLU warps fill one while the dQ MMA of the previous super-tile reads the other
+constexpr uint32_t kDSBuf = 4 * kDSHalf;
+constexpr uint32_t kOffDS = kOffStage + kStages * kStepBytes;
+constexpr size_t kSmemBytes = kOffDS + 2 * kDSBuf + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct BwdTcArgs {
@@ -80,7 +82,7 @@ struct BwdTcArgs {
 // One unit: key block [j0, j1) of user u, KV group g, and the query rows to visit.
 struct BwdUnit {
   int u, so, LH, LR, LT, N, g, j0, j1;
-  int q_begin, n_st;  // first query (position for Full, T-row index for Target), super-tiles
+  int q_begin, nq, n_st;  // first query (position for Full, T-row index for Target), count, super-tiles
   int qrow0;          // row of query q_begin in the Q / dA / dQ tensors
 };
 
@@ -119,11 +121,11 @@ __device__ BwdUnit decode_unit(const MetaView& m, int w, int hkv, int v2) {
     U.qrow0 = U.so + qb;
   }
   U.q_begin = qb;
-  U.n_st = qe > qb ? (qe - qb + 127) / 128 : 0;
+  U.nq = max(0, qe - qb);
+  U.n_st = (U.nq + 127) / 128;
   return U;
 }
 
-__device__ __forceinline__ void silu_bar() { asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory"); }
 
 // Per query column of a step: prefix end and sibling range (visibility of key j:
 // j < kve, or slo <= j < shi).  Columns past the unit's query rows see nothing.
@@ -150,11 +152,11 @@ template <bool TARGET>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dah,
-                   const __grid_constant__ CUtensorMap tm_dal, const __grid_constant__ CUtensorMap tm_dq,
+                   const __grid_constant__ CUtensorMap tm_dal, float* __restrict__ dq,
                    float* __restrict__ dk, float* __restrict__ dv, BwdTcArgs p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_kvf[2], bar_kve[2], bar_stf[2], bar_ste[2], bar_sdp[2], bar_pds[2];
-  __shared__ __align__(8) uint64_t bar_dqf[2], bar_dqe[2], bar_dsfree, bar_dkvf, bar_dkve, bar_drain;
+  __shared__ __align__(8) uint64_t bar_kvf, bar_kve, bar_stf[kStages], bar_ste[kStages], bar_sdp[2], bar_pds[2];
+  __shared__ __align__(8) uint64_t bar_dqf[2], bar_dqe[2], bar_dsfree[2], bar_dkvf, bar_dkve, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -166,33 +168,34 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   const int n_mine = (n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   auto unit_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
   const int r = p.hq / p.hkv;
-  const int ldkv = p.hkv * kDH;
+  const int ldkv = p.hkv * kDH, ldq = p.hq * kDH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
-  auto sK = [&](int b) { return sbase + kOffKV + b * 2 * kKVTile; };
-  auto sV = [&](int b) { return sbase + kOffKV + b * 2 * kKVTile + kKVTile; };
+  const uint32_t sKb = sbase + kOffKV, sVb = sbase + kOffKV + kKVTile;
   auto sQ = [&](int s) { return sbase + kOffStage + s * kStepBytes; };
   auto sDAh = [&](int s) { return sbase + kOffStage + s * kStepBytes + kQTile; };
   auto sDAl = [&](int s) { return sbase + kOffStage + s * kStepBytes + 2 * kQTile; };
   const uint32_t sDS = sbase + kOffDS;  // hi: halves at +0, +kDSHalf; lo: at +2 kDSHalf, +3 kDSHalf
-  const uint32_t sDQ = sbase + kOffDQ;
   auto B = [&](uint64_t* b) { return smem_addr(b); };
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(B(&bar_kvf[i]), 1);
-      mbar_init(B(&bar_kve[i]), 1);
+    mbar_init(B(&bar_kvf), 1);
+    mbar_init(B(&bar_kve), 1);
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(B(&bar_stf[i]), 1);
       mbar_init(B(&bar_ste[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(B(&bar_sdp[i]), 1);
       mbar_init(B(&bar_pds[i]), 128 * kSiluWG);
       mbar_init(B(&bar_dqf[i]), 1);
       mbar_init(B(&bar_dqe[i]), 128 * kSiluWG);
     }
-    mbar_init(B(&bar_dsfree), 1);
+    mbar_init(B(&bar_dsfree[0]), 1);
+    mbar_init(B(&bar_dsfree[1]), 1);
     mbar_init(B(&bar_dkvf), 1);
     mbar_init(B(&bar_dkve), 128 * kSiluWG);
     mbar_init(B(&bar_drain), 1);
@@ -209,7 +212,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_dah);
     tma_prefetch_desc(&tm_dal);
-    tma_prefetch_desc(&tm_dq);
   }
   __syncthreads();
   tc_fence_after();
@@ -226,15 +228,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const BwdUnit U = decode_unit<TARGET>(m, unit_of(k), p.hkv, p.v2);
         const int T = U.n_st * r * 2;
         if (T == 0) continue;
-        const int kb = nkv & 1;
-        if (nkv >= 2 && !mbar_wait(B(&bar_kve[kb]), ((nkv - 2) >> 1) & 1, abort_flag)) break;
-        mbar_expect_tx(B(&bar_kvf[kb]), 2 * kKVTile);
-        tma_load_2d(sK(kb), &tm_k, B(&bar_kvf[kb]), U.g * kDH, U.so + U.j0);
-        tma_load_2d(sV(kb), &tm_v, B(&bar_kvf[kb]), U.g * kDH, U.so + U.j0);
+        if (nkv >= 1 && !mbar_wait(B(&bar_kve), (nkv - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(B(&bar_kvf), 2 * kKVTile);
+        tma_load_2d(sKb, &tm_k, B(&bar_kvf), U.g * kDH, U.so + U.j0);
+        tma_load_2d(sVb, &tm_v, B(&bar_kvf), U.g * kDH, U.so + U.j0);
         ++nkv;
         for (int t = 0; t < T; ++t) {
-          const int s = G & 1;
-          if (G >= 2 && !mbar_wait(B(&bar_ste[s]), ((G >> 1) - 1) & 1, abort_flag)) {
+          const int s = G % kStages;
+          if (G >= kStages && !mbar_wait(B(&bar_ste[s]), ((G / kStages) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -253,8 +254,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
         }
       };
-      for (int q = max(0, nkv - 2); q < nkv; ++q) drain(B(&bar_kvf[q & 1]), (q >> 1) & 1);
-      for (int g2 = max(0, G - 2); g2 < G; ++g2) drain(B(&bar_stf[g2 & 1]), (g2 >> 1) & 1);
+      if (nkv > 0) drain(B(&bar_kvf), (nkv - 1) & 1);
+      for (int g2 = max(0, G - kStages); g2 < G; ++g2) drain(B(&bar_stf[g2 % kStages]), (g2 / kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -266,22 +267,22 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const uint32_t ds_lo = sw128_desc_lo(sDS, kDSHalf);  // MN-major A: query halves kDSHalf apart
     bool ok = true;
     int G = 0, ST = 0, kd = 0;
-    auto issue_sdp = [&](int gs, int kb) -> bool {
-      const int s = gs & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_stf[s]), (gs >> 1) & 1, abort_flag))) return false;
+    auto issue_sdp = [&](int gs) -> bool {
+      const int s = gs % kStages, b = gs & 1;  // Q / dA stage, S / dP buffer
+      if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_stf[s]), (gs / kStages) & 1, abort_flag))) return false;
       tc_fence_after();
-      const uint32_t dS_t = tmem + kColSP + s * 128, dP_t = dS_t + 64;
+      const uint32_t dS_t = tmem + kColSP + b * 128, dP_t = dS_t + 64;
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kDH / 16; ++kk)
-          mma_ss2(dS_t, lo(sK(kb)) + kk * 2, dhi, lo(sQ(s)) + kk * 2, dhi, id_sdp, kk > 0 ? 1u : 0u);
+          mma_ss2(dS_t, lo(sKb) + kk * 2, dhi, lo(sQ(s)) + kk * 2, dhi, id_sdp, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kDH / 16; ++kk)
-          mma_ss2(dP_t, lo(sV(kb)) + kk * 2, dhi, lo(sDAh(s)) + kk * 2, dhi, id_sdp, kk > 0 ? 1u : 0u);
+          mma_ss2(dP_t, lo(sVb) + kk * 2, dhi, lo(sDAh(s)) + kk * 2, dhi, id_sdp, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kDH / 16; ++kk)
-          mma_ss2(dP_t, lo(sV(kb)) + kk * 2, dhi, lo(sDAl(s)) + kk * 2, dhi, id_sdp, 1u);
-        mma_commit(B(&bar_sdp[s]));
+          mma_ss2(dP_t, lo(sVb) + kk * 2, dhi, lo(sDAl(s)) + kk * 2, dhi, id_sdp, 1u);
+        mma_commit(B(&bar_sdp[b]));
       }
       __syncwarp();
       return true;
@@ -290,16 +291,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       const BwdUnit U = decode_unit<TARGET>(m, unit_of(k), p.hkv, p.v2);
       const int T = U.n_st * r * 2;
       if (T == 0) continue;
-      const int kb = kd & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_kvf[kb]), (kd >> 1) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_kvf), kd & 1, abort_flag))) {
         ok = false;
         break;
       }
-      ok = issue_sdp(G, kb);
+      ok = issue_sdp(G);
       for (int t = 0; ok && t < T; ++t) {
-        const int gs = G + t, s = gs & 1;
-        if (t + 1 < T && !(ok = issue_sdp(gs + 1, kb))) break;
-        if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_pds[s]), (gs >> 1) & 1, abort_flag))) {
+        const int gs = G + t, s = gs % kStages, b = gs & 1;
+        if (t + 1 < T && !(ok = issue_sdp(gs + 1))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_pds[b]), (gs >> 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
@@ -309,7 +309,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           break;
         }
         tc_fence_after();
-        const uint32_t pT = tmem + kColSP + s * 128, dsT = pT + 64;
+        const uint32_t pT = tmem + kColSP + b * 128, dsT = pT + 64;
         if (elect_one()) {
 #pragma unroll
           for (int c = 0; c < kQS / 16; ++c) {  // 16 queries per MMA: TMEM columns [16c, 16c + 8) hi, [+8, +16) lo
@@ -332,15 +332,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           }
           tc_fence_after();
           if (elect_one()) {
+            const uint32_t dsb = ds_lo + db * (kDSBuf >> 4);  // dS buffer of this super-tile
 #pragma unroll
             for (int kk = 0; kk < kKB / 16; ++kk) {
-              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + kk * 128, dhi, lo(sK(kb)) + kk * 128, dhi, id_dq,
-                      kk > 0 ? 1u : 0u);
-              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + ((2 * kDSHalf) >> 4) + kk * 128, dhi, lo(sK(kb)) + kk * 128,
-                      dhi, id_dq, 1u);
+              mma_ss2(tmem + kColDQ + db * kDH, dsb + kk * 128, dhi, lo(sKb) + kk * 128, dhi, id_dq, kk > 0 ? 1u : 0u);
+              mma_ss2(tmem + kColDQ + db * kDH, dsb + ((2 * kDSHalf) >> 4) + kk * 128, dhi, lo(sKb) + kk * 128, dhi,
+                      id_dq, 1u);
             }
             mma_commit(B(&bar_dqf[db]));
-            mma_commit(B(&bar_dsfree));
+            mma_commit(B(&bar_dsfree[db]));
           }
           __syncwarp();
           ++ST;
@@ -349,7 +349,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       if (!ok) break;
       if (elect_one()) {
         mma_commit(B(&bar_dkvf));
-        mma_commit(B(&bar_kve[kb]));
+        mma_commit(B(&bar_kve));
       }
       __syncwarp();
       G += T;
@@ -368,45 +368,35 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int quad = warp & 3;
     const int mrow = quad * 32 + lane;  // TMEM lane: key row (steps) or query row (dQ)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const bool issuer = threadIdx.x == 128;
     const float half_alpha = 0.5f * p.alpha;
     bool ok = true;
     int G = 0, ST = 0, kd = 0;
-    // dQ of super-tile-head e waits for the next step before it is drained
+    // dQ of super-tile-head e (read from TMEM after the next step) goes to dq with
+    // fp32 vector atomics: several key blocks add to the same query rows.
     struct PendDQ {
-      int e, x, y;
+      int e, col, row0, nvalid;
       float sc;
       bool live;
-    } pend{0, 0, 0, 0.f, false};
-    auto dq_epilogue = [&](const PendDQ& e) {  // passes both named barriers whatever e says
+    } pend{0, 0, 0, 0, 0.f, false};
+    auto dq_epilogue = [&](const PendDQ& e) {
+      if (!(e.live && ok)) return;
       const int db = e.e & 1;
-      bool eok = e.live && ok;
-      if (eok) eok = __all_sync(0xffffffffu, mbar_wait(B(&bar_dqf[db]), (e.e >> 1) & 1, abort_flag));
-      if (e.live && !eok) ok = false;
-      if (issuer) bulk_wait_read<0>();  // the previous reduces have read the staging tile
-      silu_bar();
-      if (eok) {
-        tc_fence_after();
-        uint32_t raw[16];
-        tmem_ld16(lane_base + kColDQ + db * kDH + wg * 16, raw);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(B(&bar_dqe[db]));
-        uint8_t* rowp = smem + kOffDQ + (wg >> 1) * (128 * 128) + mrow * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int chunk = (wg & 1) * 4 + j;
-          *reinterpret_cast<float4*>(rowp + ((chunk ^ (mrow & 7)) << 4)) =
-              make_float4(__uint_as_float(raw[4 * j]) * e.sc, __uint_as_float(raw[4 * j + 1]) * e.sc,
-                          __uint_as_float(raw[4 * j + 2]) * e.sc, __uint_as_float(raw[4 * j + 3]) * e.sc);
-        }
-        fence_proxy_async();
+      if (!__all_sync(0xffffffffu, mbar_wait(B(&bar_dqf[db]), (e.e >> 1) & 1, abort_flag))) {
+        ok = false;
+        return;
       }
-      silu_bar();
-      if (eok && issuer) {
-        tma_reduce_add_2d(&tm_dq, sDQ, e.x, e.y);
-        tma_reduce_add_2d(&tm_dq, sDQ + 128 * 128, e.x + 32, e.y);
-        bulk_commit();
+      tc_fence_after();
+      uint32_t raw[16];
+      tmem_ld16(lane_base + kColDQ + db * kDH + wg * 16, raw);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(B(&bar_dqe[db]));
+      if (mrow < e.nvalid) {
+        float4* dst = reinterpret_cast<float4*>(dq + (size_t)(e.row0 + mrow) * ldq + e.col + wg * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          atomicAdd(dst + j, make_float4(__uint_as_float(raw[4 * j]) * e.sc, __uint_as_float(raw[4 * j + 1]) * e.sc,
+                                         __uint_as_float(raw[4 * j + 2]) * e.sc, __uint_as_float(raw[4 * j + 3]) * e.sc));
       }
     };
     for (int k = 0; k < n_mine; ++k) {
@@ -429,6 +419,35 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       const int t0pos = U.LH + U.LR;
       const bool sib_keys = U.j1 > t0pos;  // the block holds T keys: sibling visibility applies
       const int jw0 = U.j0 + quad * 32;     // this warp's 32 keys
+      // P^T, dS^T of 16 queries for this thread's key, as bf16 hi [0, 8) / lo [8, 16) pairs
+      auto elementwise = [&](const uint32_t (&sv)[16], const uint32_t (&dpv)[16], const ColInfo& ci, auto masked_tag,
+                             uint32_t (&pk)[16], uint32_t (&dk2)[16]) {
+        constexpr bool kMasked = decltype(masked_tag)::value;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float pr[2], dr[2];
+#pragma unroll
+          for (int u2 = 0; u2 < 2; ++u2) {
+            const int c = 2 * e + u2;
+            const float hh = half_alpha * __uint_as_float(sv[c]);
+            const float th = tanh_approx(hh);
+            pr[u2] = fmaf(hh, th, hh);                                                      // P = s sigma
+            dr[u2] = __uint_as_float(dpv[c]) * (fmaf(0.5f, th, 0.5f) * fmaf(-hh, th, hh + 1.f));  // dP SiLU'(s)
+            if (kMasked) {
+              const int kv = __shfl_sync(0xffffffffu, ci.kve, c);
+              bool vis = jrow < kv;
+              if (sib_keys) {
+                const int lo_ = __shfl_sync(0xffffffffu, ci.slo, c), hi_ = __shfl_sync(0xffffffffu, ci.shi, c);
+                vis = vis || (jrow >= lo_ && jrow < hi_);
+              }
+              pr[u2] = vis ? pr[u2] : 0.f;
+              dr[u2] = vis ? dr[u2] : 0.f;
+            }
+          }
+          split_trunc_bf16x2(pr[0], pr[1], pk[e], pk[8 + e]);
+          split_trunc_bf16x2(dr[0], dr[1], dk2[e], dk2[8 + e]);
+        }
+      };
       for (int t = 0; t < T; ++t) {
         const int gs = G + t, s = gs & 1;
         const int st = t / (2 * r), hf = t & 1, h = U.g * r + (t >> 1) % r;
@@ -444,49 +463,25 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (ok) {
           tc_fence_after();
           const uint32_t pT = lane_base + kColSP + s * 128 + wg * 16, dsT = pT + 64;
-          uint32_t sv[16], dpv[16];
-          tmem_ld16(pT, sv);
-          tmem_ld16(dsT, dpv);
-          tmem_ld_wait();
-          uint32_t pk[16], dk2[16];  // [0, 8): hi parts, [8, 16): lo parts (bf16 pairs)
+          uint32_t pk[16], dk2[16];
           if (none_vis) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = dk2[e] = 0u;
           } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float pr[2], dr[2];
-#pragma unroll
-              for (int u2 = 0; u2 < 2; ++u2) {
-                const int c = 2 * e + u2;
-                const float hh = half_alpha * __uint_as_float(sv[c]);
-                const float th = tanh_approx(hh);
-                const float pv = fmaf(hh, th, hh);                        // P = s sigma
-                const float uu = fmaf(-hh, th, hh + 1.f);                 // 1 + s - P
-                const float dsv = __uint_as_float(dpv[c]) * (fmaf(0.5f, th, 0.5f) * uu);  // dP SiLU'(s)
-                bool vis = true;
-                if (!all_vis) {
-                  const int kv = __shfl_sync(0xffffffffu, ci.kve, c);
-                  vis = jrow < kv;
-                  if (sib_keys) {
-                    const int lo_ = __shfl_sync(0xffffffffu, ci.slo, c), hi_ = __shfl_sync(0xffffffffu, ci.shi, c);
-                    vis = vis || (jrow >= lo_ && jrow < hi_);
-                  }
-                }
-                pr[u2] = vis ? pv : 0.f;
-                dr[u2] = vis ? dsv : 0.f;
-              }
-              split_trunc_bf16x2(pr[0], pr[1], pk[e], pk[8 + e]);
-              split_trunc_bf16x2(dr[0], dr[1], dk2[e], dk2[8 + e]);
-            }
+            uint32_t sv[16], dpv[16];
+            tmem_ld16(pT, sv);
+            tmem_ld16(dsT, dpv);
+            tmem_ld_wait();
+            if (all_vis) elementwise(sv, dpv, ci, std::false_type{}, pk, dk2);
+            else elementwise(sv, dpv, ci, std::true_type{}, pk, dk2);
           }
           tmem_st16(pT, pk);    // P^T over S^T: hi in 8 columns, lo in the next 8
           tmem_st16(dsT, dk2);  // dS^T over dP^T
           // dS^T into shared memory for the dQ MMA: half hf, key row mrow, queries [16 wg, +16)
-          if (hf == 0 && ST >= 1)
-            ok = __all_sync(0xffffffffu, mbar_wait(B(&bar_dsfree), (ST - 1) & 1, abort_flag));
+          if (hf == 0 && ST >= 2)  // the dQ MMA of super-tile ST - 2 has read this buffer
+            ok = __all_sync(0xffffffffu, mbar_wait(B(&bar_dsfree[ST & 1]), ((ST >> 1) - 1) & 1, abort_flag));
           if (ok) {
-            uint8_t* hrow = smem + kOffDS + hf * kDSHalf + mrow * 128;
+            uint8_t* hrow = smem + kOffDS + (ST & 1) * kDSBuf + hf * kDSHalf + mrow * 128;
             uint8_t* lrow = hrow + 2 * kDSHalf;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -507,7 +502,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           pend.live = false;
         }
         if (hf == 1) {
-          pend = PendDQ{ST, h * kDH, U.qrow0 + st * 128, p.alpha * inv_n, true};
+          pend = PendDQ{ST, h * kDH, U.qrow0 + st * 128, min(128, U.nq - st * 128), p.alpha * inv_n, true};
           ++ST;
         }
       }
@@ -541,7 +536,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       G += T;
       ++kd;
     }
-    if (issuer) bulk_wait<0>();  // every reduce has completed before the CTA leaves
   }
   __syncthreads();
   if (warp == 1) {
@@ -560,31 +554,19 @@ cudaError_t launch_attn_bwd_tc(const AttnShape& s, const MetaView& m, int max_it
                                const __nv_bfloat16* v, const __nv_bfloat16* da_hi, const __nv_bfloat16* da_lo,
                                float* dq, float* dk, float* dv, cudaStream_t st) {
   if (max_items_full <= 0 || total_tokens <= 0) return cudaSuccess;
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return cudaErrorInvalidValue;
   const uint64_t Dq = (uint64_t)s.hq * kDH, Dkv = (uint64_t)s.hkv * kDH;
   const uint64_t rq = rows_q > 0 ? (uint64_t)rows_q : 1;  // a valid map even without query rows
-  CUtensorMap mk, mv, mq, mdah, mdal, mdq;
+  CUtensorMap mk, mv, mq, mdah, mdal;
   if (!make_map_bf16(&mk, k, total_tokens, Dkv, Dkv, kKB, kDH) || !make_map_bf16(&mv, v, total_tokens, Dkv, Dkv, kKB, kDH) ||
       !make_map_bf16(&mq, q, rq, Dq, Dq, kQS, kDH) || !make_map_bf16(&mdah, da_hi, rq, Dq, Dq, kQS, kDH) ||
       !make_map_bf16(&mdal, da_lo, rq, Dq, Dq, kQS, kDH))
     return cudaErrorInvalidValue;
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)Dq, (cuuint64_t)rq};
-    cuuint64_t strides[1] = {(cuuint64_t)Dq * 4};
-    cuuint32_t box[2] = {32, 128};
-    cuuint32_t estr[2] = {1, 1};
-    if (fn(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dq, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
   BwdTcArgs args{m, s.hq, s.hkv, s.v2, s.alpha};
   const int grid = std::min(sm_count(), max_items_full * s.hkv);
   auto launch = [&](auto kern) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kSmemBytes, st>>>(mk, mv, mq, mdah, mdal, mdq, dk, dv, args);
+    kern<<<grid, kThreads, kSmemBytes, st>>>(mk, mv, mq, mdah, mdal, dq, dk, dv, args);
     return cudaGetLastError();
   };
   return s.target ? launch(attn_bwd_tc_kernel<true>) : launch(attn_bwd_tc_kernel<false>);

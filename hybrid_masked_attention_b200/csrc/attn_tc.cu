@@ -57,7 +57,6 @@ constexpr int kStages = 3;        // K/V ring depth
 constexpr int kSBuf = 2;          // S/P buffers in TMEM
 constexpr int kSiluWG = 4;        // SiLU warpgroups
 constexpr int kWGPerBuf = 4;      // warpgroups sharing one step (split by key columns)
-constexpr int kTeams = kSiluWG / kWGPerBuf;         // teams take steps n = team (mod kTeams)
 constexpr int kChunksPerWG = kBN / 32 / kWGPerBuf;  // 32-key chunks per warpgroup and step
 constexpr int kThreads = 128 + 128 * kSiluWG;
 constexpr uint32_t kQBytes = kBM * kDH * 2;   // 16 KB
@@ -67,7 +66,7 @@ constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kB
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
 static_assert(kBN == kKeyBlock, "key blocks of the work lists");
 static_assert(kBM * (4 * kDH + 4) * 4 <= 4 * kQBytes + 2 * kStages * kKVBytes, "O staging fits in the Q + K/V buffers");
-static_assert(kSiluWG % kWGPerBuf == 0 && kChunksPerWG >= 1 && kSBuf % kTeams == 0, "warpgroup split");
+static_assert(kSiluWG == kWGPerBuf && kChunksPerWG >= 1, "all warpgroups share every step");
 
 struct TcArgs {
   MetaView m;
@@ -290,8 +289,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     } else if (warp >= 4) {
       // ----------------------------------------------------------- SiLU warpgroups
       const int wg = (warp - 4) >> 2;   // warpgroup 0..3
-      const int team = wg % kTeams;      // steps n = team (mod kTeams)
-      const int cpart = wg / kTeams;     // part of the key columns of a step this warpgroup handles
+      const int cpart = wg;              // part of the key columns of a step this warpgroup handles
       const int quad = warp & 3;
       const int row = quad * 32 + lane;
       const int qi = q0 + row;
@@ -350,7 +348,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_arrive(b_pf(buf));
         return true;
       };
-      static_assert(kTeams == 1, "one team walks every step");
       for (int n = 0; ok && n < n_full; ++n) ok = step(n, std::false_type{});
       for (int n = n_full; ok && n < total; ++n) ok = step(n, std::true_type{});
       // ----------------------------------------------------------- epilogue: A (+)= O / N_u
