@@ -29,7 +29,7 @@
 // exactly one unit per group).
 //
 // Roles: warp 0 TMA (K/V block per unit; Q, dA_hi, dA_lo tiles per step through
-// a 2-stage ring), warp 1 TMEM allocation and MMA issue (one
+// a 4-stage ring), warp 1 TMEM allocation and MMA issue (one
 // elected lane; S^T/dP^T one step ahead), warps 4..19 the elementwise work and
 // the dQ / dK / dV epilogues.  TMEM: dV [0, 64), dK [64, 128), dQ buffers
 // [128, 192) and [192, 256), S^T / dP^T buffer b at [256 + 128 b, +64) / [+64, +128).
@@ -63,14 +63,15 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDV = 0, kColDK = 64, kColDQ = 128, kColSP = 256;
 
 // shared memory map (offsets from the 1024-aligned base)
-constexpr int kStages = 2;                                  // Q / dA ring
+constexpr int kStages = 4;                                  // Q / dA ring: loads run 3 steps ahead
 constexpr uint32_t kOffKV = 0;                              // K, V of the unit
 constexpr uint32_t kOffStage = kOffKV + 2 * kKVTile;        // kStages x (Q, dA_hi, dA_lo)
-// dS^T of a super-tile: hi (2 query halves), then lo (2 halves); two buffers, so
-// that the SiLU warps fill one while the dQ MMA of the previous super-tile reads the other
+// dS^T of a super-tile: hi (2 query halves), then lo (2 halves).  The dQ MMA that
+// reads it is issued as soon as the second half is written, ahead of that step's
+// dV/dK MMAs, so it has finished before the next super-tile's first half is written.
 constexpr uint32_t kDSBuf = 4 * kDSHalf;
 constexpr uint32_t kOffDS = kOffStage + kStages * kStepBytes;
-constexpr size_t kSmemBytes = kOffDS + 2 * kDSBuf + 1024;
+constexpr size_t kSmemBytes = kOffDS + kDSBuf + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct BwdTcArgs {
@@ -156,7 +157,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    float* __restrict__ dk, float* __restrict__ dv, BwdTcArgs p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_kvf, bar_kve, bar_stf[kStages], bar_ste[kStages], bar_sdp[2], bar_pds[2];
-  __shared__ __align__(8) uint64_t bar_dqf[2], bar_dqe[2], bar_dsfree[2], bar_dkvf, bar_dkve, bar_drain;
+  __shared__ __align__(8) uint64_t bar_dqf[2], bar_dqe[2], bar_dsfree, bar_dkvf, bar_dkve, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -194,8 +195,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       mbar_init(B(&bar_dqf[i]), 1);
       mbar_init(B(&bar_dqe[i]), 128 * kSiluWG);
     }
-    mbar_init(B(&bar_dsfree[0]), 1);
-    mbar_init(B(&bar_dsfree[1]), 1);
+    mbar_init(B(&bar_dsfree), 1);
     mbar_init(B(&bar_dkvf), 1);
     mbar_init(B(&bar_dkve), 128 * kSiluWG);
     mbar_init(B(&bar_drain), 1);
@@ -309,6 +309,26 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           break;
         }
         tc_fence_after();
+        if (t & 1) {  // second half of a super-tile: dQ = dS K over the 128 keys, first
+          const int db = ST & 1;
+          if (ST >= 2 && !__all_sync(0xffffffffu, mbar_wait(B(&bar_dqe[db]), ((ST >> 1) - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < kKB / 16; ++kk) {
+              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + kk * 128, dhi, lo(sKb) + kk * 128, dhi, id_dq, kk > 0 ? 1u : 0u);
+              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + ((2 * kDSHalf) >> 4) + kk * 128, dhi, lo(sKb) + kk * 128, dhi,
+                      id_dq, 1u);
+            }
+            mma_commit(B(&bar_dqf[db]));
+            mma_commit(B(&bar_dsfree));
+          }
+          __syncwarp();
+          ++ST;
+        }
         const uint32_t pT = tmem + kColSP + b * 128, dsT = pT + 64;
         if (elect_one()) {
 #pragma unroll
@@ -324,27 +344,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           mma_commit(B(&bar_ste[s]));  // the step's Q / dA tiles and S/dP buffer are free
         }
         __syncwarp();
-        if (t & 1) {  // second half of a super-tile: dQ = dS K over the 128 keys
-          const int db = ST & 1;
-          if (ST >= 2 && !__all_sync(0xffffffffu, mbar_wait(B(&bar_dqe[db]), ((ST >> 1) - 1) & 1, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (elect_one()) {
-            const uint32_t dsb = ds_lo + db * (kDSBuf >> 4);  // dS buffer of this super-tile
-#pragma unroll
-            for (int kk = 0; kk < kKB / 16; ++kk) {
-              mma_ss2(tmem + kColDQ + db * kDH, dsb + kk * 128, dhi, lo(sKb) + kk * 128, dhi, id_dq, kk > 0 ? 1u : 0u);
-              mma_ss2(tmem + kColDQ + db * kDH, dsb + ((2 * kDSHalf) >> 4) + kk * 128, dhi, lo(sKb) + kk * 128, dhi,
-                      id_dq, 1u);
-            }
-            mma_commit(B(&bar_dqf[db]));
-            mma_commit(B(&bar_dsfree[db]));
-          }
-          __syncwarp();
-          ++ST;
-        }
       }
       if (!ok) break;
       if (elect_one()) {
@@ -478,10 +477,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           tmem_st16(pT, pk);    // P^T over S^T: hi in 8 columns, lo in the next 8
           tmem_st16(dsT, dk2);  // dS^T over dP^T
           // dS^T into shared memory for the dQ MMA: half hf, key row mrow, queries [16 wg, +16)
-          if (hf == 0 && ST >= 2)  // the dQ MMA of super-tile ST - 2 has read this buffer
-            ok = __all_sync(0xffffffffu, mbar_wait(B(&bar_dsfree[ST & 1]), ((ST >> 1) - 1) & 1, abort_flag));
+          if (hf == 0 && ST >= 1)  // the dQ MMA of the previous super-tile has read the tile
+            ok = __all_sync(0xffffffffu, mbar_wait(B(&bar_dsfree), (ST - 1) & 1, abort_flag));
           if (ok) {
-            uint8_t* hrow = smem + kOffDS + (ST & 1) * kDSBuf + hf * kDSHalf + mrow * 128;
+            uint8_t* hrow = smem + kOffDS + hf * kDSHalf + mrow * 128;
             uint8_t* lrow = hrow + 2 * kDSHalf;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
