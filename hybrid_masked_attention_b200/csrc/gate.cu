@@ -54,8 +54,9 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 }
 
 // Y is fp32 for the layer entry points, bf16 (round to nearest) where Y feeds
-// the output projection of the backbone stack.
-template <typename OutT>
+// the output projection of the backbone stack.  NCH: float4 chunks per lane held
+// in registers (D <= 128 NCH); the smallest that fits keeps the occupancy up.
+template <typename OutT, int NCH>
 __global__ void __launch_bounds__(256)
 gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, bool target, int rows,
                 int D, float eps, const float* __restrict__ a, const __nv_bfloat16* __restrict__ u,
@@ -67,24 +68,34 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
   if (row >= rows) return;
   const int nch = D >> 2;  // float4 chunks in the row
   const float* ar = a + (size_t)row * D;
-  float4 x[kMaxChunks];
-  float s = 0.f;
+  const __nv_bfloat16* ur = u + (size_t)row * D;
+  // every load of the row (A and U) is issued before the reductions
+  float4 x[NCH];
+  uint2 uraw[NCH];
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NCH; ++i) {
     const int c = lane + 32 * i;
     if (c < nch) {
       x[i] = *reinterpret_cast<const float4*>(ar + 4 * c);
-      s += x[i].x + x[i].y + x[i].z + x[i].w;
+      uraw[i] = *reinterpret_cast<const uint2*>(ur + 4 * c);
     }
   }
+  auto u4 = [&](int i) {
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uraw[i].x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uraw[i].y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+  };
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i)
+    if (lane + 32 * i < nch) s += x[i].x + x[i].y + x[i].z + x[i].w;
   OutT* yr = y + (size_t)row * D;
-  const __nv_bfloat16* ur = u + (size_t)row * D;
   if (gamma == nullptr) {
 #pragma unroll
-    for (int i = 0; i < kMaxChunks; ++i) {
+    for (int i = 0; i < NCH; ++i) {
       const int c = lane + 32 * i;
       if (c < nch) {
-        float4 uu = load_bf16x4(ur + 4 * c);
+        const float4 uu = u4(i);
         store4(yr + 4 * c, make_float4(x[i].x * uu.x, x[i].y * uu.y, x[i].z * uu.z, x[i].w * uu.w));
       }
     }
@@ -93,7 +104,7 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
   const float mean = warp_sum(s) / (float)D;
   float s2 = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NCH; ++i) {
     const int c = lane + 32 * i;
     if (c < nch) {
       const float a0 = x[i].x - mean, a1 = x[i].y - mean, a2 = x[i].z - mean, a3 = x[i].w - mean;
@@ -106,12 +117,12 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
   const float* gr = gamma + (size_t)type * D;
   const float* br = beta + (size_t)type * D;
 #pragma unroll
-  for (int i = 0; i < kMaxChunks; ++i) {
+  for (int i = 0; i < NCH; ++i) {
     const int c = lane + 32 * i;
     if (c < nch) {
       const float4 gg = *reinterpret_cast<const float4*>(gr + 4 * c);
       const float4 bb = *reinterpret_cast<const float4*>(br + 4 * c);
-      const float4 uu = load_bf16x4(ur + 4 * c);
+      const float4 uu = u4(i);
       float4 o;
       o.x = fmaf((x[i].x - mean) * rstd, gg.x, bb.x) * uu.x;
       o.y = fmaf((x[i].y - mean) * rstd, gg.y, bb.y) * uu.y;
@@ -237,8 +248,12 @@ cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, flo
                             const float* a, const __nv_bfloat16* u, const float* gamma,
                             const float* beta, float* y, float* stats, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  gate_fwd_kernel<float><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps, a, u,
-                                                         gamma, beta, y, stats);
+  if (D <= 512)
+    gate_fwd_kernel<float, 4><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps, a, u,
+                                                              gamma, beta, y, stats);
+  else
+    gate_fwd_kernel<float, kMaxChunks><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps,
+                                                                       a, u, gamma, beta, y, stats);
   return cudaGetLastError();
 }
 
@@ -246,8 +261,12 @@ cudaError_t launch_gate_fwd_bf16(const MetaView& m, bool target, int rows, int D
                                  const float* a, const __nv_bfloat16* u, const float* gamma,
                                  const float* beta, __nv_bfloat16* y, float* stats, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  gate_fwd_kernel<__nv_bfloat16><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D,
-                                                                 eps, a, u, gamma, beta, y, stats);
+  if (D <= 512)
+    gate_fwd_kernel<__nv_bfloat16, 4><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps,
+                                                                      a, u, gamma, beta, y, stats);
+  else
+    gate_fwd_kernel<__nv_bfloat16, kMaxChunks><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows,
+                                                                               D, eps, a, u, gamma, beta, y, stats);
   return cudaGetLastError();
 }
 
