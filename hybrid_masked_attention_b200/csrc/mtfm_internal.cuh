@@ -44,6 +44,8 @@ struct MetaHeader {
   // Key blocks per Target unit (>= kTargetUnitBlocks): the packer picks it so that the
   // layer has a few units per SM, splitting long key ranges only as far as needed.
   int32_t tgt_chunk_blocks;
+  int32_t pack_done;  // CTAs of the packer's row pass that have finished (the last one scans)
+  int32_t pad[3];
 };
 
 // One work item: a 128-row query tile of one user and the range of prefix

@@ -11,14 +11,16 @@
 //   T row t        : keys [0, L_H + k_t) + itself     k_t = #{R : ts < exposure_t}
 // k_t is a lower_bound over the user's ascending R timestamps.
 //
-// Three launches, no host synchronisation:
+// Two launches, no host synchronisation:
 //   pack_users_kernel (1 CTA): validates lengths, scans offsets, orders users
 //     longest first and writes the work lists of 128-row query tiles;
 //   pack_rows_kernel (1 CTA per work item): per-row kv_end / row type, the
 //     sortedness check, and each tile's [kv_min, kv_max] used for block skipping;
-//   pack_units_kernel (1 CTA): the Target layer's work units (sub-tiles of T rows
-//     times chunks of the key range, the chunk sized so that short Target layers
-//     still fill every SM) and their prefix sums.
+//     the last CTA to finish builds the Target layer's work units (sub-tiles of T
+//     rows times chunks of the key range, the chunk sized so that short Target
+//     layers still fill every SM) and their prefix sums.
+#include <algorithm>
+
 #include "mtfm_internal.cuh"
 #include "tma_host.cuh"
 
@@ -66,7 +68,8 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
   if (tid == 0) s_err = 0;
   __syncthreads();
 
-  const int chunk = (B + kPackThreads - 1) / kPackThreads;
+  const int nthr = blockDim.x;
+  const int chunk = (B + nthr - 1) / nthr;
   const int b0 = min(B, tid * chunk), b1 = min(B, b0 + chunk);
 
   // 1. validate lengths, local sums
@@ -106,6 +109,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->sched[0] = m.hdr->sched[1] = 0;
       m.hdr->tgt_sub_rows = tgt_sub_rows;
       m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
+      m.hdr->pack_done = 0;
     }
     return;
   }
@@ -129,7 +133,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
 
   // 3. longest-first order (bitonic sort, descending key = N_u << 32 | ~index)
   if (sort_n > 0) {
-    for (int i = tid; i < sort_n; i += kPackThreads) {
+    for (int i = tid; i < sort_n; i += nthr) {
       unsigned long long key = 0;
       if (i < B) {
         unsigned long long n = (unsigned long long)(lh[i] + lr[i] + lt[i]);
@@ -140,7 +144,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     __syncthreads();
     for (int size = 2; size <= sort_n; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < sort_n; i += kPackThreads) {
+        for (int i = tid; i < sort_n; i += nthr) {
           int j = i ^ stride;
           if (j > i) {
             bool desc = (i & size) == 0;
@@ -195,6 +199,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->sched[0] = m.hdr->sched[1] = 0;
     m.hdr->tgt_sub_rows = tgt_sub_rows;
     m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
+    m.hdr->pack_done = 0;
   }
 }
 
@@ -208,15 +213,58 @@ __device__ __forceinline__ int count_below(const int64_t* __restrict__ ts, int n
   return lo;
 }
 
-__global__ void __launch_bounds__(kTileM)
-pack_rows_kernel(MetaView m, int max_if, int tgt_sub_rows, const int64_t* __restrict__ r_ts,
-                 const int64_t* __restrict__ t_exp) {
+// Target units: choose the key chunk C (blocks per unit) so that the layer has about
+// kTargetUnitsPerSM units per SM (C >= kTargetUnitBlocks; a tile is split only when
+// the layer is short), then units per item = sub-tiles * ceil(blocks / C), scanned in
+// place: unit_off[i] becomes the first unit of item i; n_units_target the total.
+// Run by one whole CTA (the last CTA of pack_rows_kernel to finish).
+__device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
+  __shared__ long long s_warp[32];
+  __shared__ int s_chunk;
+  MetaHeader* hdr = m.hdr;
+  const int n = hdr->n_items_target;
+  const int nthr = blockDim.x;
+  const int per = (n + nthr - 1) / nthr;
+  const int a = min(n, (int)threadIdx.x * per), b = min(n, a + per);
+  volatile int* uo = m.unit_off;  // written by other CTAs: read past L1
+  long long steps = 0;             // sub-tile key blocks of my items
+  for (int i = a; i < b; ++i) {
+    const int v = uo[i + 1];
+    steps += (long long)(v >> 16) * (v & 0xffff);
+  }
+  long long total_steps;
+  block_exclusive_scan(steps, &total_steps, s_warp);
+  if (threadIdx.x == 0) {
+    const long long target_units = (long long)kTargetUnitsPerSM * n_sm;
+    const long long c = (total_steps * hkv + target_units - 1) / target_units;
+    s_chunk = (int)max((long long)kTargetUnitBlocks, min(c, (long long)1 << 20));
+  }
+  __syncthreads();
+  const int C = s_chunk;
+  long long local = 0;
+  for (int i = a; i < b; ++i) {
+    const int v = uo[i + 1];
+    local += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
+  }
+  long long total;
+  long long run = block_exclusive_scan(local, &total, s_warp);
+  for (int i = a; i < b; ++i) {
+    const int v = uo[i + 1];
+    run += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
+    uo[i + 1] = (int)run;
+  }
+  if (threadIdx.x == 0) {
+    uo[0] = 0;
+    hdr->n_units_target = (int)total;
+    hdr->tgt_chunk_blocks = C;
+  }
+}
+
+// Per-row metadata of one work item (Full: all rows of a 128-row tile; Target: its T rows).
+__device__ void pack_item_rows(MetaView m, bool tgt, int idx, int tgt_sub_rows, const int64_t* __restrict__ r_ts,
+                               const int64_t* __restrict__ t_exp) {
   __shared__ int s_min[kTileM / 32], s_max[kTileM / 32];
   const MetaHeader* hdr = m.hdr;
-  if (hdr->error & kErrBadLengths) return;
-  const bool tgt = (int)blockIdx.x >= max_if;
-  const int idx = tgt ? blockIdx.x - max_if : blockIdx.x;
-  if (idx >= (tgt ? hdr->n_items_target : hdr->n_items_full)) return;
   WorkItem* it = (tgt ? m.items_target : m.items_full) + idx;
   const int u = it->user, tile = it->tile;
   const int LH = m.lh[u], LR = m.lr[u], LT = m.lt[u];
@@ -268,7 +316,7 @@ pack_rows_kernel(MetaView m, int max_if, int tgt_sub_rows, const int64_t* __rest
     it->kv_max = kmax;
     if (tgt) {
       // this Target tile's sub-tiles (of tgt_sub_rows T rows) and key blocks, packed
-      // as nsub * 65536 + blocks; pack_units_kernel turns them into unit counts
+      // as nsub * 65536 + blocks; scan_target_units turns them into unit counts
       const KeyBlocks kb = key_blocks(kmax, LH, LR, LT, LH + LR, tile * kTileM, hdr->v2);
       const int rows = min(kTileM, LT - tile * kTileM);
       const int nsub = (rows + tgt_sub_rows - 1) / tgt_sub_rows;
@@ -278,49 +326,24 @@ pack_rows_kernel(MetaView m, int max_if, int tgt_sub_rows, const int64_t* __rest
   }
 }
 
-// Target units: choose the key chunk C (blocks per unit) so that the layer has about
-// kTargetUnitsPerSM units per SM (C >= kTargetUnitBlocks; a tile is split only when
-// the layer is short), then units per item = sub-tiles * ceil(blocks / C), scanned in
-// place: unit_off[i] becomes the first unit of item i; n_units_target the total.
-__global__ void __launch_bounds__(kPackThreads) pack_units_kernel(MetaView m, int hkv, int n_sm) {
-  __shared__ long long s_warp[32];
-  __shared__ int s_chunk;
-  MetaHeader* hdr = m.hdr;
-  if (hdr->error & kErrBadLengths) return;
-  const int n = hdr->n_items_target;
-  const int per = (n + kPackThreads - 1) / kPackThreads;
-  const int a = min(n, (int)threadIdx.x * per), b = min(n, a + per);
-  long long steps = 0;  // sub-tile key blocks of my items
-  for (int i = a; i < b; ++i) {
-    const int v = m.unit_off[i + 1];
-    steps += (long long)(v >> 16) * (v & 0xffff);
-  }
-  long long total_steps;
-  block_exclusive_scan(steps, &total_steps, s_warp);
+__global__ void __launch_bounds__(kTileM)
+pack_rows_kernel(MetaView m, int max_if, int tgt_sub_rows, int hkv, int n_sm, const int64_t* __restrict__ r_ts,
+                 const int64_t* __restrict__ t_exp) {
+  const MetaHeader* hdr = m.hdr;
+  if (hdr->error & kErrBadLengths) return;  // uniform over the grid: nothing to scan either
+  const bool tgt = (int)blockIdx.x >= max_if;
+  const int idx = tgt ? blockIdx.x - max_if : blockIdx.x;
+  if (idx < (tgt ? hdr->n_items_target : hdr->n_items_full)) pack_item_rows(m, tgt, idx, tgt_sub_rows, r_ts, t_exp);
+  // The last CTA to finish turns the Target tiles' block counts into work units.
+  __shared__ bool s_last;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    const long long target_units = (long long)kTargetUnitsPerSM * n_sm;
-    const long long c = (total_steps * hkv + target_units - 1) / target_units;
-    s_chunk = (int)max((long long)kTargetUnitBlocks, min(c, (long long)1 << 20));
+    __threadfence();
+    s_last = atomicAdd(&m.hdr->pack_done, 1) == (int)gridDim.x - 1;
+    if (s_last) __threadfence();
   }
   __syncthreads();
-  const int C = s_chunk;
-  long long local = 0;
-  for (int i = a; i < b; ++i) {
-    const int v = m.unit_off[i + 1];
-    local += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
-  }
-  long long total;
-  long long run = block_exclusive_scan(local, &total, s_warp);
-  for (int i = a; i < b; ++i) {
-    const int v = m.unit_off[i + 1];
-    run += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
-    m.unit_off[i + 1] = (int)run;
-  }
-  if (threadIdx.x == 0) {
-    m.unit_off[0] = 0;
-    hdr->n_units_target = (int)total;
-    hdr->tgt_chunk_blocks = C;
-  }
+  if (s_last) scan_target_units(m, hkv, n_sm);
 }
 
 }  // namespace
@@ -344,7 +367,9 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
     attr_set = true;
   }
   const int tsr = target_sub_rows(cfg.hq, cfg.hkv);
-  pack_users_kernel<<<1, kPackThreads, smem, st>>>(m, cfg.batch, cfg.total_tokens, cfg.total_r,
+  // one thread per user up to kPackThreads (cheaper block barriers for small batches)
+  const int threads = std::min(kPackThreads, std::max(64, (cfg.batch + 31) / 32 * 32));
+  pack_users_kernel<<<1, threads, smem, st>>>(m, cfg.batch, cfg.total_tokens, cfg.total_r,
                                                    cfg.total_t, cfg.v2_subtokens, tsr,
                                                    L.max_items_full, L.max_items_target, sort_n,
                                                    lh, lr, lt);
@@ -352,10 +377,8 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
   if (e != cudaSuccess) return e;
   const int blocks = L.max_items_full + L.max_items_target;
   if (blocks > 0) {
-    pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, tsr, r_ts, t_exp);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    pack_units_kernel<<<1, kPackThreads, 0, st>>>(m, cfg.hkv > 0 ? cfg.hkv : 1, sm_count());
+    pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, tsr, cfg.hkv > 0 ? cfg.hkv : 1, sm_count(),
+                                                r_ts, t_exp);
     e = cudaGetLastError();
   }
   return e;
