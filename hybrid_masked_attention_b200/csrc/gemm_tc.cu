@@ -19,6 +19,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "mma_util.cuh"
 #include "mtfm_internal.cuh"
@@ -32,7 +33,9 @@ using namespace sm100;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of bf16
-constexpr int kStages = 4;
+constexpr int kStagesDirect = 4;  // K-slice ring; 3 when the epilogue stages tiles for TMA
+constexpr uint32_t kBoxBytes = 128 * 128;  // one staged box: 128 rows x 128 bytes
+constexpr uint32_t kStageWG = 2 * kBoxBytes;  // staging per epilogue warpgroup
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 128 + 32 * kEpiWarps;
 constexpr uint32_t kABytes = kBM * kBK * 2;
@@ -47,9 +50,27 @@ template <int BN>
 __host__ __device__ constexpr uint32_t stage_bytes() {
   return kABytes + (uint32_t)BN * kBK * 2;
 }
-template <int BN>
+template <bool TMA_EPI>
+__host__ __device__ constexpr int n_stages() {
+  return TMA_EPI ? 3 : kStagesDirect;
+}
+template <int BN, bool TMA_EPI>
 constexpr size_t gemm_smem_bytes() {
-  return (size_t)kStages * stage_bytes<BN>() + 1024;
+  return (size_t)n_stages<TMA_EPI>() * stage_bytes<BN>() + (TMA_EPI ? 2 * kStageWG : 0) + 1024;
+}
+
+// Barriers of one epilogue warpgroup (named barrier 2 + warpgroup, 128 threads).
+__device__ __forceinline__ void wg_bar(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+// Same, returning whether v holds on every thread of the warpgroup; every thread
+// arrives whatever its v, so a warp that gave up on a wait cannot strand the others.
+__device__ __forceinline__ bool wg_all(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, %2, 128, p; selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
 }
 
 // 32 consecutive fp32 accumulators of one output row -> epilogue.
@@ -89,14 +110,22 @@ __device__ __forceinline__ void epi_residual(const GemmEpi& e, int row, int col,
   }
 }
 
-template <int BN>
+// TMA_EPI: the epilogue writes each 128 x 128-byte box of the tile into a swizzled
+// shared-memory buffer and stores it with a TMA store (SiLU split: bf16 boxes of 64
+// columns, tensor map per output segment) or a TMA reduce-add (residual: fp32 boxes
+// of 32 columns into X), two boxes in flight per warpgroup.  Otherwise each thread
+// writes its row of the tile directly.
+template <int BN, bool TMA_EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, GemmArgs p) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const __grid_constant__ CUtensorMap tm_o0, const __grid_constant__ CUtensorMap tm_o1,
+               const __grid_constant__ CUtensorMap tm_o2, const __grid_constant__ CUtensorMap tm_o3, GemmArgs p) {
+  constexpr int kStages = n_stages<TMA_EPI>();
   constexpr uint32_t kStage = stage_bytes<BN>();
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers: 128, 256 or 512 columns
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
+  __shared__ __align__(8) uint64_t bar_full[kStagesDirect], bar_empty[kStagesDirect];
   __shared__ __align__(8) uint64_t bar_acc_full[2], bar_acc_empty[2], bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -219,28 +248,106 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
     const int quad = warp & 3;             // TMEM lanes [32 quad, 32 quad + 32)
     const int half = (warp - 4) >> 2;
     const int r_in = quad * 32 + lane;
+    const int bar_id = 2 + half;
+    const bool issuer = (warp & 3) == 0 && lane == 0;  // first warp of the warpgroup
+    uint8_t* stage = smem + kStages * kStage + half * kStageWG;
+    const uint32_t sstage = sbase + kStages * kStage + half * kStageWG;
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const int a = i & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(b_accf(a), (i >> 1) & 1, abort_flag))) break;
+      bool got = __all_sync(0xffffffffu, mbar_wait(b_accf(a), (i >> 1) & 1, abort_flag));
+      if (TMA_EPI) got = wg_all(bar_id, got);  // uniform over the warpgroup before its barriers
+      if (!got) break;
       tc_fence_after();
-      const int row = (t / nN) * kBM + r_in;
+      const int m0 = (t / nN) * kBM;
+      const int row = m0 + r_in;
       const int col0 = (t % nN) * BN + half * kHalf;
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * BN + half * kHalf);
+      if (!TMA_EPI) {
 #pragma unroll 1
-      for (int c = 0; c < kChunks; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(taddr + c * 32, raw);
-        tmem_ld_wait();
-        if (row < p.M) {
-          if (p.epi.kind == kEpiSiluSplit) epi_silu_split(p.epi, row, col0 + c * 32, raw);
-          else epi_residual(p.epi, row, col0 + c * 32, raw);
+        for (int c = 0; c < kChunks; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(taddr + c * 32, raw);
+          tmem_ld_wait();
+          if (row < p.M) {
+            if (p.epi.kind == kEpiSiluSplit) epi_silu_split(p.epi, row, col0 + c * 32, raw);
+            else epi_residual(p.epi, row, col0 + c * 32, raw);
+          }
+        }
+      } else if (p.epi.kind == kEpiSiluSplit) {
+        // bf16 boxes of 64 columns; kHalf / 64 of them per warpgroup (<= 2: one round)
+        constexpr int kBoxes = kHalf / 64;
+        if (issuer) bulk_wait_read<0>();  // the previous tile's stores have read the staging
+        wg_bar(bar_id);
+#pragma unroll 1
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          uint8_t* rowp = stage + bx * kBoxBytes + r_in * 128;
+#pragma unroll 1
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t raw[32];
+            tmem_ld32(taddr + bx * 64 + h2 * 32, raw);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {  // 16-byte chunk: 8 columns
+              uint4 v;
+              v.x = pack_bf16x2(silu_fast(__uint_as_float(raw[8 * c])), silu_fast(__uint_as_float(raw[8 * c + 1])));
+              v.y = pack_bf16x2(silu_fast(__uint_as_float(raw[8 * c + 2])), silu_fast(__uint_as_float(raw[8 * c + 3])));
+              v.z = pack_bf16x2(silu_fast(__uint_as_float(raw[8 * c + 4])), silu_fast(__uint_as_float(raw[8 * c + 5])));
+              v.w = pack_bf16x2(silu_fast(__uint_as_float(raw[8 * c + 6])), silu_fast(__uint_as_float(raw[8 * c + 7])));
+              const int chunk = h2 * 4 + c;
+              *reinterpret_cast<uint4*>(rowp + ((chunk ^ (r_in & 7)) << 4)) = v;
+            }
+          }
+        }
+        fence_proxy_async();
+        wg_bar(bar_id);
+        if (issuer) {
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            const int col = col0 + bx * 64;
+            const CUtensorMap* om = &tm_o0;
+            int sb = 0;
+#pragma unroll
+            for (int q = 1; q < 4; ++q)
+              if (q < p.epi.n_seg && col >= p.epi.seg_begin[q]) {
+                sb = p.epi.seg_begin[q];
+                om = q == 1 ? &tm_o1 : q == 2 ? &tm_o2 : &tm_o3;
+              }
+            tma_store_2d(om, sstage + bx * kBoxBytes, col - sb, m0);
+          }
+          bulk_commit();
+        }
+      } else {
+        // residual: fp32 boxes of 32 columns reduced into X, two per round
+        constexpr int kBoxes = kHalf / 32;
+#pragma unroll 1
+        for (int b0 = 0; b0 < kBoxes; b0 += 2) {
+          if (issuer) bulk_wait_read<0>();
+          wg_bar(bar_id);
+          const int nb = kBoxes - b0 < 2 ? kBoxes - b0 : 2;
+          for (int bx = 0; bx < nb; ++bx) {
+            uint32_t raw[32];
+            tmem_ld32(taddr + (b0 + bx) * 32, raw);
+            tmem_ld_wait();
+            uint8_t* rowp = stage + bx * kBoxBytes + r_in * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (r_in & 7)) << 4)) =
+                  make_uint4(raw[4 * c], raw[4 * c + 1], raw[4 * c + 2], raw[4 * c + 3]);
+          }
+          fence_proxy_async();
+          wg_bar(bar_id);
+          if (issuer) {
+            for (int bx = 0; bx < nb; ++bx)
+              tma_reduce_add_2d(&tm_o0, sstage + bx * kBoxBytes, col0 + (b0 + bx) * 32, m0);
+            bulk_commit();
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_acce(a));
     }
+    if (TMA_EPI && issuer) bulk_wait<0>();  // every store has completed before the CTA leaves
   }
   __syncthreads();
   if (warp == 1) {
@@ -250,15 +357,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   if (threadIdx.x == 0 && s_abort) atomicOr(&hdr->error, kErrTimeout);
 }
 
-template <int BN>
-cudaError_t gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& args, int n_tiles,
-                        cudaStream_t st) {
-  const size_t smem = gemm_smem_bytes<BN>();
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int BN, bool TMA_EPI>
+cudaError_t gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap (&mo)[4], const GemmArgs& args,
+                        int n_tiles, cudaStream_t st) {
+  const size_t smem = gemm_smem_bytes<BN, TMA_EPI>();
+  cudaError_t e =
+      cudaFuncSetAttribute(gemm_tc_kernel<BN, TMA_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = std::min(n_tiles, sm_count());
-  gemm_tc_kernel<BN><<<grid, kThreads, smem, st>>>(ma, mb, args);
+  gemm_tc_kernel<BN, TMA_EPI><<<grid, kThreads, smem, st>>>(ma, mb, mo[0], mo[1], mo[2], mo[3], args);
   return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t gemm_dispatch(bool tma, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap (&mo)[4],
+                          const GemmArgs& args, int n_tiles, cudaStream_t st) {
+  return tma ? gemm_launch<BN, true>(ma, mb, mo, args, n_tiles, st)
+             : gemm_launch<BN, false>(ma, mb, mo, args, n_tiles, st);
 }
 
 }  // namespace
@@ -271,15 +386,37 @@ cudaError_t launch_gemm_tc(MetaHeader* hdr, const __nv_bfloat16* a, int lda, con
   int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
   const int nM = (M + kBM - 1) / kBM;
   while (bn > 64 && nM * (N / bn) < sm_count() && N % (bn / 2) == 0) bn /= 2;
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mo[4];
+  memset(mo, 0, sizeof(mo));
   if (!make_map_bf16(&ma, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, kBM, kBK) ||
       !make_map_bf16(&mb, b, (uint64_t)N, (uint64_t)K, (uint64_t)K, (uint32_t)bn, kBK))
     return cudaErrorInvalidValue;
+  // TMA epilogue: 64-column bf16 boxes into contiguous segments, or fp32 boxes
+  // reduced into a contiguous X (no row map); otherwise direct stores.
+  bool tma = false;
+  if (epi.kind == kEpiSiluSplit && bn >= 128) {
+    tma = true;
+    for (int sg = 0; sg < epi.n_seg && tma; ++sg) {
+      const int w = epi.seg_begin[sg + 1] - epi.seg_begin[sg];
+      if (w % 64 != 0 || epi.seg_begin[sg] % 64 != 0 || epi.seg_ld[sg] != w ||
+          !make_map_bf16(&mo[sg], epi.seg_ptr[sg], (uint64_t)M, (uint64_t)w, (uint64_t)w, kBM, 64))
+        tma = false;
+    }
+  } else if (epi.kind == kEpiResidual && epi.row_map == nullptr && epi.ldx == N) {
+    EncodeTiledFn fn = encode_fn();
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)kBM};
+    cuuint32_t estr[2] = {1, 1};
+    tma = fn && fn(&mo[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, epi.x, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   GemmArgs args{hdr, M, N, K, epi};
   const int n_tiles = nM * (N / bn);
-  if (bn == 256) return gemm_launch<256>(ma, mb, args, n_tiles, st);
-  if (bn == 128) return gemm_launch<128>(ma, mb, args, n_tiles, st);
-  return gemm_launch<64>(ma, mb, args, n_tiles, st);
+  if (bn == 256) return gemm_dispatch<256>(tma, ma, mb, mo, args, n_tiles, st);
+  if (bn == 128) return gemm_dispatch<128>(tma, ma, mb, mo, args, n_tiles, st);
+  return gemm_dispatch<64>(tma, ma, mb, mo, args, n_tiles, st);
 }
 
 }  // namespace mtfm
