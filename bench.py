@@ -120,23 +120,76 @@ def recorded_traffic():
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled while the timed region runs.
+
+    A thread polls NVML every `interval_ms`; it is created (and NVML initialised) before the timed
+    region, and `begin()` / `stop()` bracket the samples that count.  Without NVML it falls back to
+    an `nvidia-smi --query-gpu ... -lms` subprocess."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h)
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, interval_ms: int = 50):
-        self.proc = None
+    def __init__(self, device, interval_ms: int = 20):
+        import threading
+        self.samples, self.t_begin, self.proc, self.nvml = [], None, None, None
+        self.interval = interval_ms / 1000.0
+        self.stop_flag = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            try:
+                uuid = str(torch.cuda.get_device_properties(device).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(getattr(device, "index", device) or 0))
+            self.nvml, self.handle = pynvml, h
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.nvml = None
+            self._start_smi(int(getattr(device, "index", device) or 0), max(50, interval_ms))
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while not self.stop_flag.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                mask = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((time.monotonic(), mhz, mask))
+            except Exception:
+                pass
+            self.stop_flag.wait(self.interval)
+
+    def _start_smi(self, index, interval_ms):
         self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 f"-lms={interval_ms}", f"-i={device_index}"],
+                 f"-lms={interval_ms}", f"-i={index}"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
 
+    def begin(self):
+        self.t_begin = time.monotonic()
+
     def stop(self):
+        if self.nvml is not None:
+            t_end = time.monotonic()
+            self.stop_flag.set()
+            self.thread.join(timeout=2)
+            t0 = self.t_begin if self.t_begin is not None else 0.0
+            win = [s for s in self.samples if t0 <= s[0] <= t_end] or self.samples[-1:]
+            if not win:
+                return None
+            reasons = sorted(n for n, bit in self.REASON_BITS.items() if any(m & bit for _, _, m in win))
+            return {"sm_mhz": statistics.median(m for _, m, _ in win), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(win), "source": "nvml"}
         if self.proc is None:
             return None
         time.sleep(0.06)
@@ -166,7 +219,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -230,10 +283,12 @@ def run_mtfm(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    sampler = ClockSampler(local_rank) if rank == 0 else None
+    sampler = ClockSampler(dev) if rank == 0 else None
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.begin()
     t0.record(stream)
     for i in range(args.steps):
         step(i, ev[i])
@@ -311,7 +366,12 @@ def run_mtfm(args, rank, world, local_rank):
 
 def run_e2e(args, M, cfg, b, heads, dev, stream, world):
     """Same metric through the public layer calls, with inputs in pinned host memory and the
-    host<->device copies of each step's inputs and outputs inside the timed region."""
+    host<->device copies of each step's inputs and outputs inside the timed region.
+
+    The steps are pipelined the way a data loader would feed the GPU: two sets of device
+    buffers, the inputs of step i+1 copied in (copy-in stream) while step i computes
+    (the bench stream) and step i-1's outputs are copied out (copy-out stream).  The timed
+    region runs from the first copy-in to the last copy-out, on the device clock."""
     import torch
     import torch.distributed as dist
     fi = syn.layer_inputs(b, heads, target=False, seed=11)
@@ -322,40 +382,58 @@ def run_e2e(args, M, cfg, b, heads, dev, stream, world):
             pin(b.t_exp, np.int64), pbf(fi.q), pbf(fi.k), pbf(fi.v), pbf(fi.u),
             pin(fi.gamma, np.float32), pin(fi.beta, np.float32), pbf(ti.q), pbf(ti.k), pbf(ti.v),
             pbf(ti.u), pin(ti.gamma, np.float32), pin(ti.beta, np.float32)]
-    devb = [torch.empty_like(h, device=dev) for h in host]
-    meta = M.alloc_meta(cfg, dev)
     f32 = dict(dtype=torch.float32, device=dev)
-    Y_f, A_f, S_f = (torch.empty(b.total_tokens, heads.dq, **f32), torch.empty(b.total_tokens, heads.dq, **f32),
-                     torch.empty(b.total_tokens, 2, **f32))
-    Y_t, A_t, S_t = (torch.empty(b.total_t, heads.dq, **f32), torch.empty(b.total_t, heads.dq, **f32),
-                     torch.empty(b.total_t, 2, **f32))
-    out_f = torch.empty(Y_f.shape, dtype=torch.float32).pin_memory()
-    out_t = torch.empty(Y_t.shape, dtype=torch.float32).pin_memory()
+    sets = []
+    for _ in range(2):
+        sets.append(dict(
+            inp=[torch.empty_like(h, device=dev) for h in host], meta=M.alloc_meta(cfg, dev),
+            f=(torch.empty(b.total_tokens, heads.dq, **f32), torch.empty(b.total_tokens, heads.dq, **f32),
+               torch.empty(b.total_tokens, 2, **f32)),
+            t=(torch.empty(b.total_t, heads.dq, **f32), torch.empty(b.total_t, heads.dq, **f32),
+               torch.empty(b.total_t, 2, **f32)),
+            out_f=torch.empty(b.total_tokens, heads.dq, dtype=torch.float32).pin_memory(),
+            out_t=torch.empty(b.total_t, heads.dq, dtype=torch.float32).pin_memory(),
+            ev_in=torch.cuda.Event(), ev_comp=torch.cuda.Event(), ev_out=torch.cuda.Event()))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     h2d = sum(h.numel() * h.element_size() for h in host)
-    d2h = out_f.numel() * 4 + out_t.numel() * 4
+    d2h = (b.total_tokens + b.total_t) * heads.dq * 4
 
-    def step():
-        for h, d in zip(host, devb):
-            d.copy_(h, non_blocking=True)
-        lh, lr, lt, rts, tex, q, k, v, u, g, bt, tq, tk, tv, tu, tg, tbt = devb
-        M.pack(cfg, lh, lr, lt, rts, tex, meta, stream)
-        M.attn_full_fwd(cfg, meta, q, k, v, u, g, bt, Y_f, A_f, S_f, stream)
-        M.attn_target_fwd(cfg, meta, tq, tk, tv, tu, tg, tbt, Y_t, A_t, S_t, stream)
-        out_f.copy_(Y_f, non_blocking=True)
-        out_t.copy_(Y_t, non_blocking=True)
+    def step(i):
+        z = sets[i & 1]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(z["ev_comp"])  # step i-2's compute no longer reads this set
+            for h, d in zip(host, z["inp"]):
+                d.copy_(h, non_blocking=True)
+            z["ev_in"].record(s_in)
+        stream.wait_event(z["ev_in"])
+        if i >= 2:
+            stream.wait_event(z["ev_out"])    # step i-2's outputs have been copied out
+        lh, lr, lt, rts, tex, q, k, v, u, g, bt, tq, tk, tv, tu, tg, tbt = z["inp"]
+        M.pack(cfg, lh, lr, lt, rts, tex, z["meta"], stream)
+        M.attn_full_fwd(cfg, z["meta"], q, k, v, u, g, bt, *z["f"], stream)
+        M.attn_target_fwd(cfg, z["meta"], tq, tk, tv, tu, tg, tbt, *z["t"], stream)
+        z["ev_comp"].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(z["ev_comp"])
+            z["out_f"].copy_(z["f"][0], non_blocking=True)
+            z["out_t"].copy_(z["t"][0], non_blocking=True)
+            z["ev_out"].record(s_out)
 
     steps = max(3, min(args.steps, args.e2e_steps))
-    for _ in range(3):
-        step()
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        step()
-    t1.record(stream)
+    t0.record(s_in)
+    for i in range(steps):
+        step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(stream)
+    t1.record(s_out)
     torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1)
     fl = attn_flops(b, heads, False) + attn_flops(b, heads, True)
@@ -367,7 +445,8 @@ def run_e2e(args, M, cfg, b, heads, dev, stream, world):
         ms, fl = float(t[0]), float(w[0])
     return {"value": round(fl / (ms / steps * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": round(ms / steps, 4)}
+            "ms_per_step": round(ms / steps, 4),
+            "pipelining": "two buffer sets; copy-in, compute and copy-out on three streams"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -498,6 +577,8 @@ def run_extra(args):
     out_f = s._fwd_out(N, True)
     out_t = s._fwd_out(T, True)
     steps = max(1, args.steps)
+    clocks = ClockSampler(dev)
+    clocks.begin()
     timed("pack", lambda: s.pack(*lens), steps)
     timed("full_attn", lambda: M.attn_full(cfg, s.meta, F["q"], F["k"], F["v"], out_f[1]), steps)
     timed("full_fwd", lambda: s.full_fwd(F["q"], F["k"], F["v"], F["u"], gam, bet, out=out_f), steps)
@@ -508,6 +589,7 @@ def run_extra(args):
         yt, at, st_ = s.target_fwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet)
         timed("full_bwd", lambda: s.full_bwd(F["q"], F["k"], F["v"], F["u"], gam, bet, af, sf, F["dy"]), steps)
         timed("target_bwd", lambda: s.target_bwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, at, st_, Tg["dy"]), steps)
+    clk = clocks.stop()
     M.pack_check(s.meta)
     peaks, src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -540,7 +622,8 @@ def run_extra(args):
                       "flops_fwd_full": ff, "flops_fwd_target": ft,
                       "peak": f"{src} bf16 {peak_tf} TF/s, HBM {hbm} GB/s"},
            "per_kernel": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
-                          for k, v in layers.items()}}
+                          for k, v in layers.items()},
+           "clocks": clk}
     print(json.dumps(out), flush=True)
 
 
@@ -592,7 +675,8 @@ def run_stack(args):
         res[label] = a.elapsed_time(z) / steps
 
     steps = max(1, args.steps)
-    clocks = ClockSampler(0)
+    clocks = ClockSampler(dev)
+    clocks.begin()
     timed("stack", lambda: M.stack_fwd(cfg, meta, d, layers, x, ws), steps)
     clk = clocks.stop()
     timed("full_layer", lambda: M.layer_fwd(cfg, meta, d, layers[0], x, ws), steps)
