@@ -254,19 +254,19 @@ def run_mtfm(args, rank, world, local_rank):
     A_t = torch.empty(b.total_t, heads.dq, **f32)
     Y_t = torch.empty(b.total_t, heads.dq, **f32)
     S_t = torch.empty(b.total_t, 2, **f32)
-    stream = torch.cuda.current_stream(dev)
+    # graphs cannot be captured on the legacy default stream: every launch goes to `stream`
+    stream = torch.cuda.Stream(dev)
     launches_per_step = 6   # pack (2 kernels), Full attention, Full gate, Target attention, Target gate
 
-    n_ev = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_ev)]
-
-    def step(i, record=None):
+    def step(i, record=None, around_full=None):
         s = sets[i % len(sets)]
         e = record
         if e: e[0].record(stream)
         M.pack(cfg, *lens, meta, stream)
         if e: e[1].record(stream)
+        if around_full: around_full[0].record(stream)
         M.attn_full(cfg, meta, s["q"], s["k"], s["v"], A_f, stream)
+        if around_full: around_full[1].record(stream)
         if e: e[2].record(stream)
         M.gate_fwd(cfg, meta, False, A_f, s["u"], s["g"], s["bt"], Y_f, S_f, stream)
         if e: e[3].record(stream)
@@ -275,12 +275,32 @@ def run_mtfm(args, rank, world, local_rank):
         M.gate_fwd(cfg, meta, True, A_t, s["tu"], s["tg"], s["tbt"], Y_t, S_t, stream)
         if e: e[5].record(stream)
 
-    # correctness gate before timing: the metadata must be valid
-    step(0)
-    M.pack_check(meta, stream)
-    for i in range(args.warmup):
-        step(i)
+    with torch.cuda.stream(stream):
+        # correctness gate before timing: the metadata must be valid
+        step(0)
+        M.pack_check(meta, stream)
+        for i in range(args.warmup):
+            step(i)
     torch.cuda.synchronize(dev)
+    # One CUDA graph per resident input set holds one whole step (the 6 kernel launches and
+    # the Target layer's accumulator clear); the timed loop replays them, step i from set
+    # i mod sets.  Two event-record nodes in each graph time its Full attention launch, so
+    # the kernel's duration is measured inside the timed region (the last launch of each
+    # graph).
+    graphs, full_ev = [], []
+    for r in range(len(sets)):
+        pair = (torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(r, around_full=pair)
+        graphs.append(g)
+        full_ev.append(pair)
+    with torch.cuda.stream(stream):
+        for i in range(max(3, len(sets))):
+            graphs[i % len(sets)].replay()
+    torch.cuda.synchronize(dev)
+    M.pack_check(meta, stream)
     if world > 1:
         dist.barrier()
     sampler = ClockSampler(dev) if rank == 0 else None
@@ -289,21 +309,35 @@ def run_mtfm(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     if sampler:
         sampler.begin()
-    t0.record(stream)
-    for i in range(args.steps):
-        step(i, ev[i])
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(args.steps):
+            graphs[i % len(sets)].replay()
+        t1.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
     if world > 1:
         dist.barrier()
     ms_total = t0.elapsed_time(t1)
+    full_live = [a.elapsed_time(z) for a, z in full_ev[:min(len(sets), args.steps)]]
+    full_ms = sum(full_live) / len(full_live)
+    M.pack_check(meta, stream)
+
+    # Per-part times from a separate eager pass with an event between launches (the events
+    # themselves add a few microseconds per step, so the parts sum to more than a graph step).
+    n_parts = max(1, min(args.steps, 500))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_parts)]
+    with torch.cuda.stream(stream):
+        for i in range(n_parts):
+            step(i, ev[i])
+    torch.cuda.synchronize(dev)
 
     def avg(a, z):
-        return sum(ev[i][a].elapsed_time(ev[i][z]) for i in range(args.steps)) / args.steps
+        return sum(ev[i][a].elapsed_time(ev[i][z]) for i in range(n_parts)) / n_parts
 
     ms_parts = {"pack": avg(0, 1), "full_attn": avg(1, 2), "full_gate": avg(2, 3),
                 "target_attn": avg(3, 4), "target_gate": avg(4, 5)}
+    del graphs
     fl_full = attn_flops(b, heads, False)
     fl_tgt = attn_flops(b, heads, True)
     flops_step = fl_full + fl_tgt
@@ -328,7 +362,7 @@ def run_mtfm(args, rank, world, local_rank):
         peaks, src = load_peaks()
         peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        full_tf = fl_full / (ms_parts["full_attn"] * 1e-3) / 1e12
+        full_tf = fl_full / (full_ms * 1e-3) / 1e12
         tgt_gbs = target_attn_bytes(b, heads) / (ms_parts["target_attn"] * 1e-3) / 1e9
         traffic = recorded_traffic()
         result = {
@@ -340,6 +374,7 @@ def run_mtfm(args, rank, world, local_rank):
                        "total_t": b.total_t, "flops_per_step_per_gpu": flops_step,
                        "l2": f"inputs rotated over {args.sets} resident copies "
                              f"({args.sets * 89} MB of inputs > 126 MB L2)",
+                       "launch": "each step replays a CUDA graph of its launches (one graph per input set)",
                        "parallelism": f"replicas x{world} (users sharded, no collective)"},
             "users_per_s": round(users_all * args.steps / (ms_max * 1e-3), 1),
             "per_layer": {
@@ -351,12 +386,15 @@ def run_mtfm(args, rank, world, local_rank):
                            "attn_gbs": round(tgt_gbs, 1), "attn_hbm_frac": round(tgt_gbs / hbm, 4),
                            "users_per_s": round(b.B / ((ms_parts["target_attn"] + ms_parts["target_gate"]) * 1e-3), 1)},
                 "ms_parts": {k: round(v, 5) for k, v in ms_parts.items()},
+                "ms_parts_note": "eager pass with an event between launches (not the graph-replayed step)",
             },
             "roofline": {"kernel": "Full-layer attention (attn_fwd_tc_kernel, tcgen05)", "bound": "tensor",
                          "achieved": round(full_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(full_tf / peak_tf, 4), "traffic": traffic,
                          "peak_source": f"{src} bf16 dense (burst)",
-                         "flops_per_launch": fl_full, "launch_ms": round(ms_parts["full_attn"], 5)},
+                         "flops_per_launch": fl_full, "launch_ms": round(full_ms, 5),
+                         "launch_ms_source": f"CUDA events around the Full attention launch in each of the "
+                                             f"{len(full_live)} step graphs, their last replays in the timed region"},
             "e2e": e2e,
             "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps,
@@ -674,11 +712,34 @@ def run_stack(args):
         torch.cuda.synchronize()
         res[label] = a.elapsed_time(z) / steps
 
+    def timed_graph(label, fn, steps):
+        # the whole call captured once as a CUDA graph and replayed `steps` times
+        side = torch.cuda.Stream(dev)
+        with torch.cuda.stream(side):
+            for _ in range(max(3, args.warmup)):
+                fn(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn(side)
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            a, z = ev(), ev()
+            a.record(side)
+            for _ in range(steps):
+                g.replay()
+            z.record(side)
+        torch.cuda.synchronize()
+        res[label] = a.elapsed_time(z) / steps
+
     steps = max(1, args.steps)
     clocks = ClockSampler(dev)
     clocks.begin()
-    timed("stack", lambda: M.stack_fwd(cfg, meta, d, layers, x, ws), steps)
+    timed_graph("stack", lambda st: M.stack_fwd(cfg, meta, d, layers, x, ws, st), steps)
     clk = clocks.stop()
+    timed("stack_eager", lambda: M.stack_fwd(cfg, meta, d, layers, x, ws), steps)
     timed("full_layer", lambda: M.layer_fwd(cfg, meta, d, layers[0], x, ws), steps)
     timed("target_layer", lambda: M.layer_fwd(cfg, meta, d, layers[1], x, ws), steps)
     q, kk, vv = rnd(1.0, N, D), rnd(1.0, N, Dkv), rnd(1.0, N, Dkv)
@@ -706,8 +767,10 @@ def run_stack(args):
                       "users": b.B, "total_tokens": N, "total_t": T, "attn_flops": attn_fl,
                       "gemm_flops": gemm_fl,
                       "l2": "per-layer working set (X fp32 + scratch) larger than the 126 MB L2",
+                      "launch": "the stack call captured once as a CUDA graph and replayed per step",
                       "peak": f"{src} bf16 sustained {peak_tf} TF/s"},
            "users_per_s": round(b.B / (ms * 1e-3), 1),
+           "ms_per_step_eager": round(res["stack_eager"], 5),
            "per_layer_users_per_s": round(b.B * len(kinds) / (ms * 1e-3), 1),
            "per_kernel": {
                "full_layer": {"ms": round(res["full_layer"], 5),
