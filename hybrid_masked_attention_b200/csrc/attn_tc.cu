@@ -114,6 +114,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   const MetaView& m = p.m;
   MetaHeader* hdr = m.hdr;
+  pdl_wait();
   if (hdr->error) return;
   // (work item, KV group) pairs, taken from the counter (see the file comment)
   const int n_units = hdr->n_items_full;
@@ -406,6 +407,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     step_base += total;
     ++unit_iter;
   }
+  pdl_trigger();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -440,8 +442,7 @@ cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   grid = std::min(grid, max_items * a.hkv);
-  attn_fwd_tc_kernel<R><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-  return cudaGetLastError();
+  return launch_pdl(attn_fwd_tc_kernel<R>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, a);
 }
 
 }  // namespace

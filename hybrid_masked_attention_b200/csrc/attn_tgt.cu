@@ -142,6 +142,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   const MetaView& m = p.m;
   MetaHeader* hdr = m.hdr;
+  pdl_wait();
   if (hdr->error) return;
   if (hdr->tgt_sub_rows != TR) {  // packed for another head configuration
     if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&hdr->error, kErrConfig);
@@ -461,6 +462,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (n_mine > 0) epilogue(prev);
     if (issuer) bulk_wait<0>();  // every reduce has completed before the CTA leaves
   }
+  pdl_trigger();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -513,8 +515,7 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
   auto launch = [&](auto kern) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e2 != cudaSuccess) return e2;
-    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, ma, args);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, args);
   };
   if (r == 1) return launch(attn_fwd_tgt_kernel<1>);
   if (r == 2) return launch(attn_fwd_tgt_kernel<2>);

@@ -62,6 +62,8 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
                 int D, float eps, const float* __restrict__ a, const __nv_bfloat16* __restrict__ u,
                 const float* __restrict__ gamma, const float* __restrict__ beta,
                 OutT* __restrict__ y, float* __restrict__ stats) {
+  pdl_wait();
+  pdl_trigger();
   if (hdr->error) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
@@ -248,26 +250,24 @@ cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, flo
                             const float* a, const __nv_bfloat16* u, const float* gamma,
                             const float* beta, float* y, float* stats, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  const dim3 grid((rows + 7) / 8), block(256);
   if (D <= 512)
-    gate_fwd_kernel<float, 4><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps, a, u,
-                                                              gamma, beta, y, stats);
-  else
-    gate_fwd_kernel<float, kMaxChunks><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps,
-                                                                       a, u, gamma, beta, y, stats);
-  return cudaGetLastError();
+    return launch_pdl(gate_fwd_kernel<float, 4>, grid, block, 0, st, m.hdr, m.row_type, target, rows, D, eps, a, u,
+                      gamma, beta, y, stats);
+  return launch_pdl(gate_fwd_kernel<float, kMaxChunks>, grid, block, 0, st, m.hdr, m.row_type, target, rows, D, eps,
+                    a, u, gamma, beta, y, stats);
 }
 
 cudaError_t launch_gate_fwd_bf16(const MetaView& m, bool target, int rows, int D, float eps,
                                  const float* a, const __nv_bfloat16* u, const float* gamma,
                                  const float* beta, __nv_bfloat16* y, float* stats, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
+  const dim3 grid((rows + 7) / 8), block(256);
   if (D <= 512)
-    gate_fwd_kernel<__nv_bfloat16, 4><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows, D, eps,
-                                                                      a, u, gamma, beta, y, stats);
-  else
-    gate_fwd_kernel<__nv_bfloat16, kMaxChunks><<<(rows + 7) / 8, 256, 0, st>>>(m.hdr, m.row_type, target, rows,
-                                                                               D, eps, a, u, gamma, beta, y, stats);
-  return cudaGetLastError();
+    return launch_pdl(gate_fwd_kernel<__nv_bfloat16, 4>, grid, block, 0, st, m.hdr, m.row_type, target, rows, D,
+                      eps, a, u, gamma, beta, y, stats);
+  return launch_pdl(gate_fwd_kernel<__nv_bfloat16, kMaxChunks>, grid, block, 0, st, m.hdr, m.row_type, target,
+                    rows, D, eps, a, u, gamma, beta, y, stats);
 }
 
 cudaError_t launch_gate_bwd(const MetaView& m, bool target, int rows, int D, float eps,

@@ -131,6 +131,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
   __shared__ int s_abort;
 
   MetaHeader* hdr = p.hdr;
+  pdl_wait();
   if (hdr->error) return;
   const int nN = p.N / BN, nK = p.K / kBK;
   const int n_tiles = ((p.M + kBM - 1) / kBM) * nN;
@@ -349,6 +350,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
     }
     if (TMA_EPI && issuer) bulk_wait<0>();  // every store has completed before the CTA leaves
   }
+  pdl_trigger();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -365,8 +367,8 @@ cudaError_t gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUte
       cudaFuncSetAttribute(gemm_tc_kernel<BN, TMA_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = std::min(n_tiles, sm_count());
-  gemm_tc_kernel<BN, TMA_EPI><<<grid, kThreads, smem, st>>>(ma, mb, mo[0], mo[1], mo[2], mo[3], args);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN, TMA_EPI>, dim3(grid), dim3(kThreads), smem, st, ma, mb, mo[0], mo[1], mo[2],
+                    mo[3], args);
 }
 
 template <int BN>

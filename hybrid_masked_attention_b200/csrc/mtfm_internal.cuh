@@ -8,6 +8,31 @@
 
 namespace mtfm {
 
+// Programmatic dependent launch.  A kernel started by launch_pdl may begin while the
+// kernel before it on the stream is still running: it calls pdl_wait() before it reads
+// or writes any memory that earlier work on the stream uses (the wait returns once that
+// kernel has completed and its writes are visible), and pdl_trigger() once the kernel
+// after it may be scheduled (which then waits in its own pdl_wait()).  Both are no-ops
+// for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Query rows per work item (one item = one 128-row query tile of one user).
 constexpr int kTileM = 128;
 constexpr int kRowH = 0, kRowR = 1, kRowT = 2;
@@ -128,7 +153,7 @@ inline MetaView meta_view(void* base, const MetaLayout& L) {
 // the item's T rows that the prefix does not cover.  Shared by the packer (to
 // size the Target split) and the kernel (to walk the blocks).
 constexpr int kKeyBlock = 128;
-constexpr int kTargetUnitBlocks = 2;  // smallest key chunk of a Target work unit
+constexpr int kTargetUnitBlocks = 4;  // smallest key chunk of a Target work unit
 constexpr int kTargetUnitsPerSM = 8;  // the packer aims at about this many Target units per SM
 
 // T rows of a Target-layer sub-tile when the r = hq / hkv query heads of a KV group

@@ -64,6 +64,8 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
   extern __shared__ unsigned long long s_keys[];  // [sort_n] (0 when not sorting)
   __shared__ long long s_warp[32];
   __shared__ int s_err;
+  pdl_wait();  // the previous work on the stream may still read this metadata block
+  pdl_trigger();
   const int tid = threadIdx.x;
   if (tid == 0) s_err = 0;
   __syncthreads();
@@ -329,6 +331,8 @@ __device__ void pack_item_rows(MetaView m, bool tgt, int idx, int tgt_sub_rows, 
 __global__ void __launch_bounds__(kTileM)
 pack_rows_kernel(MetaView m, int max_if, int tgt_sub_rows, int hkv, int n_sm, const int64_t* __restrict__ r_ts,
                  const int64_t* __restrict__ t_exp) {
+  pdl_wait();
+  pdl_trigger();
   const MetaHeader* hdr = m.hdr;
   if (hdr->error & kErrBadLengths) return;  // uniform over the grid: nothing to scan either
   const bool tgt = (int)blockIdx.x >= max_if;
@@ -369,18 +373,14 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
   const int tsr = target_sub_rows(cfg.hq, cfg.hkv);
   // one thread per user up to kPackThreads (cheaper block barriers for small batches)
   const int threads = std::min(kPackThreads, std::max(64, (cfg.batch + 31) / 32 * 32));
-  pack_users_kernel<<<1, threads, smem, st>>>(m, cfg.batch, cfg.total_tokens, cfg.total_r,
-                                                   cfg.total_t, cfg.v2_subtokens, tsr,
-                                                   L.max_items_full, L.max_items_target, sort_n,
-                                                   lh, lr, lt);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(pack_users_kernel, dim3(1), dim3(threads), smem, st, m, cfg.batch, cfg.total_tokens,
+                             cfg.total_r, cfg.total_t, cfg.v2_subtokens, tsr, L.max_items_full,
+                             L.max_items_target, sort_n, lh, lr, lt);
   if (e != cudaSuccess) return e;
   const int blocks = L.max_items_full + L.max_items_target;
-  if (blocks > 0) {
-    pack_rows_kernel<<<blocks, kTileM, 0, st>>>(m, L.max_items_full, tsr, cfg.hkv > 0 ? cfg.hkv : 1, sm_count(),
-                                                r_ts, t_exp);
-    e = cudaGetLastError();
-  }
+  if (blocks > 0)
+    e = launch_pdl(pack_rows_kernel, dim3(blocks), dim3(kTileM), 0, st, m, L.max_items_full, tsr,
+                   cfg.hkv > 0 ? cfg.hkv : 1, sm_count(), r_ts, t_exp);
   return e;
 }
 

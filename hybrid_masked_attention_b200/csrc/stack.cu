@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(256)
 rmsnorm_kernel(const MetaHeader* hdr, const float* __restrict__ x, int rows, int d,
                const int32_t* __restrict__ row_map, const float* __restrict__ w, float eps,
                __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   if (hdr->error) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
@@ -59,8 +61,7 @@ cudaError_t launch_rmsnorm(const MetaHeader* hdr, const float* x, int rows, int 
                            cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   if (d <= 0 || d % 4 != 0 || d > 4 * 32 * kMaxChunks) return cudaErrorInvalidValue;
-  rmsnorm_kernel<<<(rows + 7) / 8, 256, 0, st>>>(hdr, x, rows, d, row_map, w, eps, out);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_kernel, dim3((rows + 7) / 8), dim3(256), 0, st, hdr, x, rows, d, row_map, w, eps, out);
 }
 
 }  // namespace mtfm
