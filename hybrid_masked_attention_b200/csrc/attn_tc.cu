@@ -387,6 +387,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
       if (have) {
+        const uint64_t keep_a = l2_evict_last();
         const int sw = warp - 4;  // rows [8 sw, 8 sw + 8) of the tile
 #pragma unroll 1
         for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
@@ -394,7 +395,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
           const float4* src = reinterpret_cast<const float4*>(stage + rr * kStageLd);
           for (int f = lane; f < R * kDH / 4; f += 32) {
-            dst[f] = src[f];
+            st_f4_hint(dst + f, src[f], keep_a);  // the gate reads A next: keep it in L2
           }
         }
       }

@@ -71,14 +71,16 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
   const int nch = D >> 2;  // float4 chunks in the row
   const float* ar = a + (size_t)row * D;
   const __nv_bfloat16* ur = u + (size_t)row * D;
-  // every load of the row (A and U) is issued before the reductions
+  // every load of the row (A and U) is issued before the reductions; A is read for the
+  // last time here (the forward kernel kept it in L2)
+  const uint64_t last_use = l2_evict_first();
   float4 x[NCH];
   uint2 uraw[NCH];
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c = lane + 32 * i;
     if (c < nch) {
-      x[i] = *reinterpret_cast<const float4*>(ar + 4 * c);
+      x[i] = ld_f4_hint(reinterpret_cast<const float4*>(ar + 4 * c), last_use);
       uraw[i] = *reinterpret_cast<const uint2*>(ur + 4 * c);
     }
   }
