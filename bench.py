@@ -117,6 +117,28 @@ def recorded_traffic():
     return float(val.group(1))
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_batch_seed(rank: int) -> int:
+    """Seed of rank `rank`'s batch: every rank packs and runs users of its own (weak scaling,
+    no data-path collective)."""
+    return 1001 + 7919 * rank
+
+
+def reduce_over_ranks(ms: float, work, device):
+    """(max over ranks of `ms`, per-entry sum over ranks of `work`); the identity on one rank.
+    Every rank must call it, in the same order (two all-reduces on the process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms), [float(x) for x in work]
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    w = torch.tensor([float(x) for x in work], dtype=torch.float64, device=device)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t[0]), [float(x) for x in w]
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -232,7 +254,7 @@ def run_mtfm(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     heads = syn.PAIR_HEADS
-    b = syn.pair_batch(args.users, seed=1001 + 7919 * rank)
+    b = syn.pair_batch(args.users, seed=rank_batch_seed(rank))
     cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh)
     to_dev = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
     bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -353,14 +375,7 @@ def run_mtfm(args, rank, world, local_rank):
     flops_step = fl_full + fl_tgt
 
     # aggregate over ranks: time = max, work = sum
-    tot = [ms_total, flops_step, float(b.B)]
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        w = torch.tensor([flops_step, float(b.B)], dtype=torch.float64, device=dev)
-        dist.all_reduce(w, op=dist.ReduceOp.SUM)
-        tot = [float(t[0]), float(w[0]), float(w[1])]
-    ms_max, flops_all, users_all = tot
+    ms_max, (flops_all, users_all) = reduce_over_ranks(ms_total, [flops_step, float(b.B)], dev)
     ms_per_step = ms_max / args.steps
     value = flops_all / (ms_per_step * 1e-3) / 1e12
 
@@ -485,12 +500,7 @@ def run_e2e(args, M, cfg, b, heads, dev, stream, world):
     torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1)
     fl = attn_flops(b, heads, False) + attn_flops(b, heads, True)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        w = torch.tensor([fl], dtype=torch.float64, device=dev)
-        dist.all_reduce(w, op=dist.ReduceOp.SUM)
-        ms, fl = float(t[0]), float(w[0])
+    ms, (fl,) = reduce_over_ranks(ms, [fl], dev)
     return {"value": round(fl / (ms / steps * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 4),
