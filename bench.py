@@ -805,6 +805,93 @@ def run_stack(args):
     print(json.dumps(out), flush=True)
 
 
+def run_infer(args):
+    """Request-level Target attention over a cached key/value prefix: --users requests (default
+    128), each a user whose 2000-token prefix (H 1800, R 200, sorted timestamps) has its
+    keys/values in the cache, scored against 200 candidates with their own exposures.  A step
+    is pack + the cached-prefix Target layer forward (attention + gate), replayed as a CUDA
+    graph; the same layer on the concatenated [prefix; candidates] layout is timed beside it.
+    The prefix cache (128 users: 131 MB) plus the candidates' tensors exceed the 126 MB L2."""
+    import torch
+    import hybrid_masked_attention_b200 as M
+    dev = torch.device("cuda", 0)
+    heads = syn.PAIR_HEADS
+    B = args.users if args.users is not None else 128
+    LH, LR, LT = 1800, 200, 200
+    b = syn.fixed_batch([LH] * B, [LR] * B, [LT] * B, seed=1006)
+    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh)
+    inp = syn.layer_inputs(b, heads, target=True, seed=1006)
+    it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
+    bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    lens = (it(b.L_H, np.int32), it(b.L_R, np.int32), it(b.L_T, np.int32), it(b.r_ts, np.int64),
+            it(b.t_exp, np.int64))
+    rows = np.arange(b.total_tokens).reshape(B, LH + LR + LT)
+    pre_rows, cand_rows = rows[:, :LH + LR].reshape(-1), rows[:, LH + LR:].reshape(-1)
+    q, u, k, v = bf(inp.q), bf(inp.u), bf(inp.k), bf(inp.v)
+    kp, vp, kc, vc = bf(inp.k[pre_rows]), bf(inp.v[pre_rows]), bf(inp.k[cand_rows]), bf(inp.v[cand_rows])
+    g, bt = it(inp.gamma, np.float32), it(inp.beta, np.float32)
+    meta = M.alloc_meta(cfg, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    T, D = b.total_t, heads.dq
+    y, a, st = torch.empty(T, D, **f32), torch.empty(T, D, **f32), torch.empty(T, 2, **f32)
+    side = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def cached(s):
+        M.pack(cfg, *lens, meta, s)
+        M.attn_target_cached_fwd(cfg, meta, q, kp, vp, kc, vc, u, g, bt, y, a, st, s)
+
+    def concat(s):
+        M.pack(cfg, *lens, meta, s)
+        M.attn_target_fwd(cfg, meta, q, k, v, u, g, bt, y, a, st, s)
+
+    def timed_graph(fn, steps):
+        with torch.cuda.stream(side):
+            for _ in range(max(3, args.warmup)):
+                fn(side)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=side):
+            fn(side)
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                gr.replay()
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            e0.record(side)
+            for _ in range(steps):
+                gr.replay()
+            e1.record(side)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    steps = max(1, args.steps)
+    clocks = ClockSampler(dev)
+    clocks.begin()
+    ms = timed_graph(cached, steps)
+    clk = clocks.stop()
+    ms_concat = timed_graph(concat, steps)
+    M.pack_check(meta, side)
+    fl = attn_flops(b, heads, True)
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # bytes a step must move: the prefix K/V, the candidates' Q, K, V, U, and Y (fp32)
+    moved = (kp.numel() + vp.numel() + kc.numel() + vc.numel() + q.numel() + u.numel()) * 2 + T * D * 4
+    out = {"metric": METRIC, "value": round(fl / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
+           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"inference: {B} requests, cached {LH + LR}-token prefix (H {LH}, R {LR}), "
+                                  f"{LT} candidates each; pack + cached-prefix Target layer forward",
+                      "requests": B, "candidates": T, "flops_per_step": fl,
+                      "l2": f"prefix cache + candidate tensors {moved / 1e6:.0f} MB > 126 MB L2",
+                      "launch": "one CUDA graph per step"},
+           "candidates_per_s": round(T / (ms * 1e-3), 1),
+           "gbs": round(moved / (ms * 1e-3) / 1e9, 1), "frac_hbm": round(moved / (ms * 1e-3) / 1e9 / hbm, 4),
+           "concatenated_layout_ms": round(ms_concat, 5),
+           "clocks": clk}
+    print(json.dumps(out), flush=True)
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -813,12 +900,13 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["mtfm", "reference"], default="mtfm")
-    ap.add_argument("--users", type=int, default=None, help="users (default 32; 64 for --workload stack)")
+    ap.add_argument("--users", type=int, default=None,
+                    help="users (default 32; 64 for --workload stack, 128 requests for infer)")
     ap.add_argument("--sets", type=int, default=4, help="resident input copies rotated across steps")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["pair", "sweep", "train", "stack"], default="pair",
-                    help="pair: the headline step; sweep/train/stack: timings of the other configs")
+    ap.add_argument("--workload", choices=["pair", "sweep", "train", "stack", "infer"], default="pair",
+                    help="pair: the headline step; sweep/train/stack/infer: timings of the other configs")
     ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
     ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")
     args = ap.parse_args()
@@ -833,6 +921,9 @@ def main():
 
     if args.workload == "stack":
         run_stack(args)
+        return
+    if args.workload == "infer":
+        run_infer(args)
         return
     if args.users is None:
         args.users = 32

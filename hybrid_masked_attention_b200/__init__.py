@@ -8,6 +8,7 @@ this import fails; build it with ``python hybrid_masked_attention_b200/build.py`
 Function names mirror the C entry points:
     meta_bytes, max_items, pack, pack_check, meta_read,
     attn_full_fwd, attn_target_fwd, attn_full, attn_target, gate_fwd,
+    attn_target_cached_fwd, attn_target_cached,
     bwd_workspace_bytes, attn_full_bwd, attn_target_bwd, attn_target_bwd_static,
     stack_workspace_bytes, layer_fwd, stack_fwd, selftest_wait_timeout
 """
@@ -105,6 +106,8 @@ _sigs = {
     "mtfm_attn_target_fwd": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "mtfm_attn_full": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
     "mtfm_attn_target": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
+    "mtfm_attn_target_cached_fwd": (ctypes.c_int, [_CP] + [_P] * 13),
+    "mtfm_attn_target_cached": (ctypes.c_int, [_CP] + [_P] * 8),
     "mtfm_gate_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]),
     "mtfm_bwd_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int]),
     "mtfm_attn_full_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
@@ -257,6 +260,38 @@ def attn_full(cfg, meta, q, k, v, a, stream=None):
 def attn_target(cfg, meta, q, k, v, a, stream=None):
     """Target-layer attention only (A of the T rows, fp32)."""
     _attn_only(_lib.mtfm_attn_target, "mtfm_attn_target", cfg, meta, q, k, v, a, stream, cfg.total_t)
+
+
+def attn_target_cached_fwd(cfg, meta, q, k_prefix, v_prefix, k_cand, v_cand, u, gamma, beta, y, a, stats,
+                           stream=None):
+    """Target-Attention layer forward over a cached key/value prefix: k_prefix, v_prefix hold
+    the H and R rows of every user [total_tokens - total_t, Dkv], k_cand, v_cand the T rows
+    (the candidates) [total_t, Dkv]; everything else as attn_target_fwd."""
+    c = cfg.c()
+    D, Dkv, T = cfg.D, cfg.Dkv, cfg.total_t
+    P = cfg.total_tokens - T
+    bf, f32 = torch.bfloat16, torch.float32
+    st = _lib.mtfm_attn_target_cached_fwd(
+        ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"), _ptr(q, bf, (T, D), "q"),
+        _ptr(k_prefix, bf, (P, Dkv), "k_prefix"), _ptr(v_prefix, bf, (P, Dkv), "v_prefix"),
+        _ptr(k_cand, bf, (T, Dkv), "k_cand"), _ptr(v_cand, bf, (T, Dkv), "v_cand"),
+        _ptr(u, bf, (T, D), "u"), _ptr(gamma, f32, (3, D), "gamma"), _ptr(beta, f32, (3, D), "beta"),
+        _ptr(y, f32, (T, D), "y"), _ptr(a, f32, (T, D), "a"), _ptr(stats, f32, (T, 2), "stats"), _stream(stream))
+    _check(st, "mtfm_attn_target_cached_fwd")
+
+
+def attn_target_cached(cfg, meta, q, k_prefix, v_prefix, k_cand, v_cand, a, stream=None):
+    """Target attention only over a cached key/value prefix (A of the T rows, fp32)."""
+    c = cfg.c()
+    D, Dkv, T = cfg.D, cfg.Dkv, cfg.total_t
+    P = cfg.total_tokens - T
+    bf = torch.bfloat16
+    st = _lib.mtfm_attn_target_cached(
+        ctypes.byref(c), _ptr(meta, torch.uint8, None, "meta"), _ptr(q, bf, (T, D), "q"),
+        _ptr(k_prefix, bf, (P, Dkv), "k_prefix"), _ptr(v_prefix, bf, (P, Dkv), "v_prefix"),
+        _ptr(k_cand, bf, (T, Dkv), "k_cand"), _ptr(v_cand, bf, (T, Dkv), "v_cand"),
+        _ptr(a, torch.float32, (T, D), "a"), _stream(stream))
+    _check(st, "mtfm_attn_target_cached")
 
 
 def gate_fwd(cfg, meta, target: bool, a, u, gamma, beta, y, stats, stream=None):

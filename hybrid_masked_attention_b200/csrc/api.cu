@@ -141,6 +141,33 @@ mtfm_status attn_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   return gate_fwd(cfg, d_meta, target, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream);
 }
 
+// Target attention over a cached K/V prefix (attention only): the tensor-core Target
+// kernel with the prefix rows from the cache and the T rows' keys/values apart.
+mtfm_status attn_target_cached(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                               const uint16_t* d_kp, const uint16_t* d_vp, const uint16_t* d_kc,
+                               const uint16_t* d_vc, float* d_a, void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, true};
+  const char* force = getenv("MTFM_FWD_KERNEL");
+  if (!attn_fwd_tc_supported(shape) || (force && strcmp(force, "mma") == 0)) return MTFM_ERR_UNSUPPORTED;
+  if (r.total_t == 0 || r.total_tokens == 0) return MTFM_OK;
+  const int prefix_rows = r.total_tokens - r.total_t;
+  if (!d_q || !d_kc || !d_vc || !d_a) return MTFM_ERR_INVALID_ARG;
+  if (prefix_rows > 0 && (!d_kp || !d_vp)) return MTFM_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_kc) || !aligned16(d_vc) || !aligned16(d_a) ||
+      (prefix_rows > 0 && (!aligned16(d_kp) || !aligned16(d_vp))))
+    return MTFM_ERR_INVALID_ARG;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  const MetaView m = meta_view(const_cast<void*>(d_meta), L);
+  auto bf = [](const uint16_t* p) { return reinterpret_cast<const __nv_bfloat16*>(p); };
+  return cuda_status(launch_attn_fwd_tgt(shape, m, L.max_items_target, r.total_t, r.total_tokens, bf(d_q),
+                                         bf(d_kp), bf(d_vp), d_a, static_cast<cudaStream_t>(stream), bf(d_kc),
+                                         bf(d_vc)));
+}
+
 // Scratch of the backward: dA as bf16 hi and lo parts [rows, D] each, then the
 // per-block dgamma/dbeta partials.
 struct BwdWs {
@@ -426,6 +453,35 @@ mtfm_status mtfm_attn_target_fwd(const mtfm_cfg* cfg, const void* d_meta, const 
                                  float* d_a, float* d_stats, void* stream) {
   return attn_fwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_y, d_a, d_stats, stream,
                   true);
+}
+
+mtfm_status mtfm_attn_target_cached_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                        const uint16_t* d_k_prefix, const uint16_t* d_v_prefix,
+                                        const uint16_t* d_k_cand, const uint16_t* d_v_cand,
+                                        const uint16_t* d_u, const float* d_gamma, const float* d_beta,
+                                        float* d_y, float* d_a, float* d_stats, void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  // the gate's arguments are checked before the attention launches
+  if (r.total_t > 0) {
+    if (!d_u || !d_y) return MTFM_ERR_INVALID_ARG;
+    if ((d_gamma == nullptr) != (d_beta == nullptr)) return MTFM_ERR_INVALID_ARG;
+    if (d_gamma && !d_stats) return MTFM_ERR_INVALID_ARG;
+    if (!aligned16(d_u) || !aligned16(d_y) || (d_gamma && (!aligned16(d_gamma) || !aligned16(d_beta))) ||
+        (d_stats && (reinterpret_cast<uintptr_t>(d_stats) & 7u)))
+      return MTFM_ERR_INVALID_ARG;
+  }
+  s = attn_target_cached(cfg, d_meta, d_q, d_k_prefix, d_v_prefix, d_k_cand, d_v_cand, d_a, stream);
+  if (s != MTFM_OK || r.total_t == 0 || r.total_tokens == 0) return s;
+  return gate_fwd(cfg, d_meta, true, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream);
+}
+
+mtfm_status mtfm_attn_target_cached(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                    const uint16_t* d_k_prefix, const uint16_t* d_v_prefix,
+                                    const uint16_t* d_k_cand, const uint16_t* d_v_cand, float* d_a,
+                                    void* stream) {
+  return attn_target_cached(cfg, d_meta, d_q, d_k_prefix, d_v_prefix, d_k_cand, d_v_cand, d_a, stream);
 }
 
 int32_t mtfm_max_items(const mtfm_cfg* cfg, int is_target) {

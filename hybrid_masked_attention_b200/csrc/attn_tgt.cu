@@ -11,6 +11,14 @@
 // of a user fill the tile.  A work unit is one (sub-tile of TR T rows, chunk of
 // kTargetUnitBlocks key blocks, KV group); the CTAs (one per SM) stride over them.
 //
+// Cached-prefix form (request-level inference with shared user K/V, M-Falcon style,
+// Meituan tech blog §3.3.2): the keys/values of a user's H and R rows come from a cache
+// tensor [sum (L_H + L_R), hkv * 64] and those of its T rows (the candidates) from a
+// tensor [sum L_T, hkv * 64].  A sub-tile's key range is then the prefix blocks (read
+// from the cache; a T row sees only the prefix part there) and one block of candidate
+// rows starting at the sub-tile's first T row (the siblings of all its rows: TR and
+// the sibling groups are multiples of the V2 group size).  Same arithmetic otherwise.
+//
 // Roles and the pipeline across units (no block-wide barrier per unit):
 //   warp 0      : TMA producer.  Q tiles into two buffers (the next unit's Q
 //                 loads while this unit computes), K/V blocks through a 3-stage ring.
@@ -64,28 +72,31 @@ struct TgtArgs {
   MetaView m;
   int hq, hkv, v2;
   float alpha;
+  int cached;  // keys/values of the prefix from the cache, of the T rows from the candidates
 };
 
 // One work unit of this kernel, decoded from the metadata.
 struct TgtUnit {
   int u, so, LH, LR, LT, N, g;
+  int kv_row0;  // first K/V row of the user's prefix blocks (cache rows when cached)
   int q_sub0;  // first T row (within the user's T rows) of the sub-tile
   int bi0, nb, kv_min;
   KeyBlocks kb;
 };
 
 template <int R>
-__device__ TgtUnit decode_unit(const MetaView& m, int w, int hkv, int v2) {
+__device__ TgtUnit decode_unit(const MetaView& m, int w, int hkv, int v2, bool cached) {
   constexpr int TR = 128 / R;
   TgtUnit U;
   const int unit = w / hkv;
   U.g = w % hkv;
+  const int32_t* uoff = cached ? m.unit_off_c : m.unit_off;
   int lo = 0, hi = m.hdr->n_items_target - 1;  // last item whose first unit is <= unit
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (m.unit_off[mid] <= unit) lo = mid; else hi = mid - 1;
+    if (uoff[mid] <= unit) lo = mid; else hi = mid - 1;
   }
-  const int local = unit - m.unit_off[lo];
+  const int local = unit - uoff[lo];
   const WorkItem it = m.items_target[lo];
   U.u = it.user;
   U.LH = m.lh[U.u];
@@ -95,6 +106,11 @@ __device__ TgtUnit decode_unit(const MetaView& m, int w, int hkv, int v2) {
   U.so = m.seq_off[U.u];
   const int q0 = it.tile * kTileM;
   U.kb = key_blocks(it.kv_max, U.LH, U.LR, U.LT, U.LH + U.LR, q0, v2);
+  U.kv_row0 = U.so;
+  if (cached) {  // prefix blocks, then one block of candidate rows
+    U.kb.n_blocks = U.kb.nb_pre + 1;
+    U.kv_row0 = U.so - m.t_off[U.u];  // H and R rows of the users before, in the cache
+  }
   const int C = m.hdr->tgt_chunk_blocks;
   const int nchunks = (U.kb.n_blocks + C - 1) / C;
   const int sub = local / nchunks, chunk = local % nchunks;
@@ -130,6 +146,7 @@ template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
                     TgtArgs p) {
   constexpr int TR = 128 / R;
   extern __shared__ uint8_t smem_raw[];
@@ -148,7 +165,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(&hdr->error, kErrConfig);
     return;
   }
-  const int n_work = hdr->n_units_target * p.hkv;
+  const int n_work = (p.cached ? hdr->n_units_target_c : hdr->n_units_target) * p.hkv;
   if ((int)blockIdx.x >= n_work) return;
   const int n_mine = (n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // units of this CTA
   auto unit_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
@@ -195,6 +212,10 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_a);
+    if (p.cached) {
+      tma_prefetch_desc(&tm_kc);
+      tma_prefetch_desc(&tm_vc);
+    }
   }
   __syncthreads();
   tc_fence_after();
@@ -229,10 +250,17 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = false;
             break;
           }
-          const int row = U.so + U.kb.block(U.bi0 + i) * kBN;
           mbar_expect_tx(B(&bar_kvf[s]), 2 * kKVBytes);
-          tma_load_2d(sK + s * kKVBytes, &tm_k, B(&bar_kvf[s]), U.g * kDH, row);
-          tma_load_2d(sV + s * kKVBytes, &tm_v, B(&bar_kvf[s]), U.g * kDH, row);
+          const int bb = U.bi0 + i;
+          if (p.cached && bb >= U.kb.nb_pre) {  // the candidate rows from the sub-tile's first T row
+            const int row = m.t_off[U.u] + U.q_sub0;
+            tma_load_2d(sK + s * kKVBytes, &tm_kc, B(&bar_kvf[s]), U.g * kDH, row);
+            tma_load_2d(sV + s * kKVBytes, &tm_vc, B(&bar_kvf[s]), U.g * kDH, row);
+          } else {
+            const int row = U.kv_row0 + U.kb.block(bb) * kBN;
+            tma_load_2d(sK + s * kKVBytes, &tm_k, B(&bar_kvf[s]), U.g * kDH, row);
+            tma_load_2d(sV + s * kKVBytes, &tm_v, B(&bar_kvf[s]), U.g * kDH, row);
+          }
           ++G;
         }
       }
@@ -338,7 +366,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int k = 0; k < n_mine; ++k) {
         const int j = k % kRing;
         if (k >= kRing && !mbar_wait(B(&bar_de[j]), ((k / kRing) - 1) & 1, abort_flag)) break;
-        s_desc[j] = decode_unit<R>(m, unit_of(k), p.hkv, p.v2);
+        s_desc[j] = decode_unit<R>(m, unit_of(k), p.hkv, p.v2, p.cached != 0);
         mbar_arrive(B(&bar_df[j]));  // release: the descriptor is visible to every waiter
       }
     }
@@ -425,8 +453,15 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!kMasked) {
           silu_chunk<false>(raw, half_alpha, 0u, ph, pl);
         } else {
-          const int j0 = U.kb.block(U.bi0 + i) * kBN + wg * 32;
-          const uint32_t vis = vis_bits(j0, kv_end, sib_lo, sib_hi);
+          const int bb = U.bi0 + i;
+          uint32_t vis;
+          if (!p.cached) {
+            vis = vis_bits(U.kb.block(bb) * kBN + wg * 32, kv_end, sib_lo, sib_hi);
+          } else if (bb < U.kb.nb_pre) {  // cache rows: the prefix rule only
+            vis = vis_bits(bb * kBN + wg * 32, kv_end, 0, 0);
+          } else {  // candidate rows t0pos + q_sub0 + [0, 128): the sibling rule only
+            vis = vis_bits(t0pos + U.q_sub0 + wg * 32, kv_end, sib_lo, sib_hi);
+          }
           if (__all_sync(0xffffffffu, vis == 0u)) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) ph[e] = pl[e] = 0u;
@@ -477,8 +512,12 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 // {64, r, 128 / r} is one stacked tile.  A [total_t, hq * 64] fp32 in boxes of 32 x TR.
 cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_items, int total_t,
                                 int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                const __nv_bfloat16* v, float* a, cudaStream_t st) {
+                                const __nv_bfloat16* v, float* a, cudaStream_t st, const __nv_bfloat16* k_cand,
+                                const __nv_bfloat16* v_cand) {
   if (max_items <= 0 || total_t <= 0 || total_tokens <= 0) return cudaSuccess;
+  const bool cached = k_cand != nullptr;
+  // K/V rows: all rows, or (cached) the H and R rows only, the T rows in k_cand / v_cand
+  const uint64_t kv_rows = cached ? (uint64_t)(total_tokens - total_t) : (uint64_t)total_tokens;
   const int r = s.hq / s.hkv;
   const int TR = 128 / r;
   EncodeTiledFn fn = encode_fn();
@@ -494,9 +533,24 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  if (!make_map_bf16(&mk, k, (uint64_t)total_tokens, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH) ||
-      !make_map_bf16(&mv, v, (uint64_t)total_tokens, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH))
-    return cudaErrorInvalidValue;
+  CUtensorMap mkc, mvc;
+  if (kv_rows > 0) {
+    if (!make_map_bf16(&mk, k, kv_rows, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH) ||
+        !make_map_bf16(&mv, v, kv_rows, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH))
+      return cudaErrorInvalidValue;
+  }
+  if (cached) {
+    if (!make_map_bf16(&mkc, k_cand, (uint64_t)total_t, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH) ||
+        !make_map_bf16(&mvc, v_cand, (uint64_t)total_t, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH))
+      return cudaErrorInvalidValue;
+    if (kv_rows == 0) {  // no prefix rows at all: the prefix maps are never read
+      mk = mkc;
+      mv = mvc;
+    }
+  } else {
+    mkc = mk;  // not read
+    mvc = mv;
+  }
   {
     cuuint64_t dims[2] = {(cuuint64_t)s.hq * kDH, (cuuint64_t)total_t};
     cuuint64_t strides[1] = {(cuuint64_t)s.hq * kDH * 4};
@@ -509,13 +563,13 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
   }
   cudaError_t e = cudaMemsetAsync(a, 0, sizeof(float) * (size_t)total_t * s.hq * kDH, st);  // units add partial sums
   if (e != cudaSuccess) return e;
-  TgtArgs args{m, s.hq, s.hkv, s.v2, s.alpha};
+  TgtArgs args{m, s.hq, s.hkv, s.v2, s.alpha, cached ? 1 : 0};
   const size_t smem = tgt_smem_bytes();
   const int grid = sm_count();
   auto launch = [&](auto kern) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e2 != cudaSuccess) return e2;
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, args);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, mkc, mvc, args);
   };
   if (r == 1) return launch(attn_fwd_tgt_kernel<1>);
   if (r == 2) return launch(attn_fwd_tgt_kernel<2>);

@@ -96,7 +96,10 @@ struct MetaHeader {
   // layer has a few units per SM, splitting long key ranges only as far as needed.
   int32_t tgt_chunk_blocks;
   int32_t pack_done;  // CTAs of the packer's row pass that have finished (the last one scans)
-  int32_t pad[3];
+  // Units of the Target layer with a cached key/value prefix (each sub-tile's key range =
+  // the prefix blocks + one block of candidate rows; same chunk size)
+  int32_t n_units_target_c;
+  int32_t pad[2];
 };
 
 // One work item: a 128-row query tile of one user and the range of prefix
@@ -111,7 +114,7 @@ struct WorkItem {
 
 struct MetaLayout {
   size_t seq_off, r_off, t_off, lh, lr, lt, kv_end, row_type, items_full, items_target, unit_off,
-      t_rows, total;
+      t_rows, unit_off_c, total;
   int32_t max_items_full, max_items_target;
 };
 
@@ -134,6 +137,7 @@ inline MetaLayout meta_layout(int B, int total_tokens, int total_t) {
   L.items_target = o; o = align256(o + sizeof(WorkItem) * (size_t)L.max_items_target);
   L.unit_off = o;     o = align256(o + sizeof(int32_t) * ((size_t)L.max_items_target + 1));
   L.t_rows = o;       o = align256(o + sizeof(int32_t) * (size_t)total_t);
+  L.unit_off_c = o;   o = align256(o + sizeof(int32_t) * ((size_t)L.max_items_target + 1));
   L.total = o;
   return L;
 }
@@ -153,6 +157,7 @@ struct MetaView {
   WorkItem* items_target;
   int32_t* unit_off;  // [max_items_target + 1]: first unit of each Target item (prefix sums)
   int32_t* t_rows;    // [total_t]: global row (in the [sum N] layout) of each T row
+  int32_t* unit_off_c;  // [max_items_target + 1]: as unit_off, for the cached-prefix Target layer
 };
 
 inline MetaView meta_view(void* base, const MetaLayout& L) {
@@ -171,6 +176,7 @@ inline MetaView meta_view(void* base, const MetaLayout& L) {
   v.items_target = reinterpret_cast<WorkItem*>(b + L.items_target);
   v.unit_off = reinterpret_cast<int32_t*>(b + L.unit_off);
   v.t_rows = reinterpret_cast<int32_t*>(b + L.t_rows);
+  v.unit_off_c = reinterpret_cast<int32_t*>(b + L.unit_off_c);
   return v;
 }
 
@@ -232,9 +238,12 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                const __nv_bfloat16* v, float* a, cudaStream_t st);
 // Target layer, heads stacked as MMA rows (head_dim 64, hq / hkv in {1, 2, 4}).
+// With k_cand / v_cand (cached prefix): k, v hold the H and R rows of every user
+// [total_tokens - total_t, hkv * 64], k_cand, v_cand the T rows [total_t, hkv * 64].
 cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_items, int total_t,
                                 int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                const __nv_bfloat16* v, float* a, cudaStream_t st);
+                                const __nv_bfloat16* v, float* a, cudaStream_t st,
+                                const __nv_bfloat16* k_cand = nullptr, const __nv_bfloat16* v_cand = nullptr);
 cudaError_t launch_gate_fwd(const MetaView& m, bool target, int rows, int D, float eps,
                             const float* a, const __nv_bfloat16* u, const float* gamma,
                             const float* beta, float* y, float* stats, cudaStream_t st);

@@ -108,6 +108,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->max_items_full = max_if;
       m.hdr->max_items_target = max_it;
       m.hdr->n_units_target = 0;
+      m.hdr->n_units_target_c = 0;
       m.hdr->sched[0] = m.hdr->sched[1] = 0;
       m.hdr->tgt_sub_rows = tgt_sub_rows;
       m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
@@ -198,6 +199,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->max_items_full = max_if;
     m.hdr->max_items_target = max_it;
     m.hdr->n_units_target = 0;
+    m.hdr->n_units_target_c = 0;
     m.hdr->sched[0] = m.hdr->sched[1] = 0;
     m.hdr->tgt_sub_rows = tgt_sub_rows;
     m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
@@ -243,21 +245,29 @@ __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
   }
   __syncthreads();
   const int C = s_chunk;
-  long long local = 0;
-  for (int i = a; i < b; ++i) {
-    const int v = uo[i + 1];
-    local += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
-  }
-  long long total;
-  long long run = block_exclusive_scan(local, &total, s_warp);
-  for (int i = a; i < b; ++i) {
-    const int v = uo[i + 1];
-    run += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
-    uo[i + 1] = (int)run;
-  }
+  // sub-tiles x ceil(blocks / C) units per item, scanned in place into first-unit offsets
+  auto scan_units = [&](volatile int* arr) -> long long {
+    long long local = 0;
+    for (int i = a; i < b; ++i) {
+      const int v = arr[i + 1];
+      local += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
+    }
+    long long total;
+    long long run = block_exclusive_scan(local, &total, s_warp);
+    for (int i = a; i < b; ++i) {
+      const int v = arr[i + 1];
+      run += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
+      arr[i + 1] = (int)run;
+    }
+    return total;
+  };
+  const long long total = scan_units(uo);
+  const long long total_c = scan_units(m.unit_off_c);
   if (threadIdx.x == 0) {
     uo[0] = 0;
+    m.unit_off_c[0] = 0;
     hdr->n_units_target = (int)total;
+    hdr->n_units_target_c = (int)total_c;
     hdr->tgt_chunk_blocks = C;
   }
 }
@@ -323,7 +333,9 @@ __device__ void pack_item_rows(MetaView m, bool tgt, int idx, int tgt_sub_rows, 
       const int rows = min(kTileM, LT - tile * kTileM);
       const int nsub = (rows + tgt_sub_rows - 1) / tgt_sub_rows;
       m.unit_off[idx + 1] = nsub * 65536 + kb.n_blocks;
-      if (idx == 0) m.unit_off[0] = 0;
+      // with a cached prefix: the prefix blocks, then one block of the sub-tile's candidate rows
+      m.unit_off_c[idx + 1] = nsub * 65536 + kb.nb_pre + 1;
+      if (idx == 0) m.unit_off[0] = m.unit_off_c[0] = 0;
     }
   }
 }

@@ -179,6 +179,34 @@ mtfm_status mtfm_gate_fwd(const mtfm_cfg* cfg, const void* d_meta, int is_target
                           float* d_y, float* d_stats, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Target-Attention forward over a cached key/value prefix: request-level
+ * inference where each user's H and R keys/values were computed once and are
+ * shared by the candidates (T rows) of later requests ([MT] §3.3.2, M-Falcon
+ * style serving).  The result is exactly the Target layer of mtfm_attn_target_fwd
+ * on the sequence [prefix; candidates] of each user (same metadata from mtfm_pack
+ * with the prefix's L_H, L_R and the request's L_T = candidates, exposures in
+ * t_exp); only the K/V layout differs:
+ *   d_k_prefix, d_v_prefix : bf16 [total_tokens - total_t, hkv*head_dim], the H and
+ *                            R rows of every user, users back to back in batch order
+ *                            (user u's rows start at seq_off[u] - t_off[u]);
+ *   d_k_cand, d_v_cand     : bf16 [total_t, hkv*head_dim], the candidates' own keys
+ *                            and values (row t_off[u] + t for candidate t of user u);
+ *   d_q, d_u, d_y, d_a, d_stats, d_gamma, d_beta : as mtfm_attn_target_fwd.
+ * Supported where the tensor-core Target kernel runs (head_dim 64, hq / hkv in
+ * {1, 2, 4}); other shapes return MTFM_ERR_UNSUPPORTED.  mtfm_attn_target_cached
+ * writes A only.
+ * ------------------------------------------------------------------------- */
+mtfm_status mtfm_attn_target_cached_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                        const uint16_t* d_k_prefix, const uint16_t* d_v_prefix,
+                                        const uint16_t* d_k_cand, const uint16_t* d_v_cand,
+                                        const uint16_t* d_u, const float* d_gamma, const float* d_beta,
+                                        float* d_y, float* d_a, float* d_stats, void* stream);
+mtfm_status mtfm_attn_target_cached(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                    const uint16_t* d_k_prefix, const uint16_t* d_v_prefix,
+                                    const uint16_t* d_k_cand, const uint16_t* d_v_cand, float* d_a,
+                                    void* stream);
+
+/* ---------------------------------------------------------------------------
  * Backward passes (training step).  Inputs are the forward's inputs, its saved
  * A (d_a) and stats, and the upstream gradient d_dy (bf16, same shape as Y).
  * Outputs (fp32, fully overwritten):

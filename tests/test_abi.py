@@ -84,6 +84,17 @@ def test_null_and_misaligned_pointers_rejected(lib):
     # gamma without beta
     assert m._lib.mtfm_attn_target_fwd(ctypes.byref(c), 4096, 4096, 4096, 4096, 4096, 4096, None,
                                        4096, 4096, 4096, None) == 1
+    # cached-prefix Target attention: missing candidate keys, misaligned Q, and a head shape
+    # the tensor-core Target kernel does not take
+    c64 = _cfg(head_dim=64)
+    assert m._lib.mtfm_attn_target_cached(ctypes.byref(c64), 4096, 4096, 4096, 4096, None, 4096, 4096, None) == 1
+    assert m._lib.mtfm_attn_target_cached(ctypes.byref(c64), 4096, 4096 + 2, 4096, 4096, 4096, 4096, 4096,
+                                          None) == 1
+    assert m._lib.mtfm_attn_target_cached_fwd(ctypes.byref(c64), 4096, 4096, 4096, 4096, 4096, 4096, 4096,
+                                              4096, None, 4096, 4096, None, None) == 1   # gamma without beta
+    c32 = _cfg(head_dim=32)
+    assert m._lib.mtfm_attn_target_cached(ctypes.byref(c32), 4096, 4096, 4096, 4096, 4096, 4096, 4096,
+                                          None) == 3
     # backward workspace too small
     ws = m._lib.mtfm_bwd_workspace_bytes(ctypes.byref(c), 0)
     assert ws > 0
