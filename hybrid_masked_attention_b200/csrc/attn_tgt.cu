@@ -11,8 +11,8 @@
 // of a user fill the tile.  A work unit is one (sub-tile of TR T rows, chunk of
 // kTargetUnitBlocks key blocks, KV group); the CTAs (one per SM) stride over them.
 //
-// Cached-prefix form (request-level inference with shared user K/V, M-Falcon style,
-// Meituan tech blog §3.3.2): the keys/values of a user's H and R rows come from a cache
+// Cached-prefix form (request-level inference with shared user K/V: M-Falcon micro-
+// batching with a shared KV cache, page "美团推荐大模型 MTFM 深度硬核解析" §5.2.3): the keys/values of a user's H and R rows come from a cache
 // tensor [sum (L_H + L_R), hkv * 64] and those of its T rows (the candidates) from a
 // tensor [sum L_T, hkv * 64].  A sub-tile's key range is then the prefix blocks (read
 // from the cache; a T row sees only the prefix part there) and one block of candidate

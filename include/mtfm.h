@@ -181,8 +181,8 @@ mtfm_status mtfm_gate_fwd(const mtfm_cfg* cfg, const void* d_meta, int is_target
 /* ---------------------------------------------------------------------------
  * Target-Attention forward over a cached key/value prefix: request-level
  * inference where each user's H and R keys/values were computed once and are
- * shared by the candidates (T rows) of later requests ([MT] §3.3.2, M-Falcon
- * style serving).  The result is exactly the Target layer of mtfm_attn_target_fwd
+ * shared by the candidates (T rows) of later requests ([DY] §5.2.3: M-Falcon
+ * micro-batching with a shared KV cache).  The result is exactly the Target layer of mtfm_attn_target_fwd
  * on the sequence [prefix; candidates] of each user (same metadata from mtfm_pack
  * with the prefix's L_H, L_R and the request's L_T = candidates, exposures in
  * t_exp); only the K/V layout differs:
