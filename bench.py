@@ -694,7 +694,7 @@ def run_stack(args):
     import torch
     import hybrid_masked_attention_b200 as M
     dev = torch.device("cuda", 0)
-    heads, d = syn.PAIR_HEADS, 512
+    heads, d = syn.Heads(*(int(x) for x in args.heads.split(","))), args.dmodel
     B = args.users if args.users is not None else 64
     b = syn.pair_batch(B, seed=1002)
     cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh, 1)
@@ -783,7 +783,8 @@ def run_stack(args):
            "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
            "config": {"workload": f"16-layer backbone stack, 4 x (Full, Target, Target, Target): {b.B} users, "
-                                  f"production-shape lengths, d_model {d}, Hq 8 / Hkv 2, head_dim 64",
+                                  f"production-shape lengths, d_model {d}, Hq {heads.hq} / Hkv {heads.hkv}, "
+                                  f"head_dim {heads.dh}",
                       "users": b.B, "total_tokens": N, "total_t": T, "attn_flops": attn_fl,
                       "gemm_flops": gemm_fl,
                       "l2": "per-layer working set (X fp32 + scratch) larger than the 126 MB L2",
@@ -909,6 +910,8 @@ def main():
                     help="pair: the headline step; sweep/train/stack/infer: timings of the other configs")
     ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
     ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")
+    ap.add_argument("--dmodel", type=int, default=512, help="stack: d_model")
+    ap.add_argument("--heads", default="8,2,64", help="stack: Hq,Hkv,head_dim (e.g. 3,1,256 with --dmodel 768)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -24,7 +24,8 @@ mtfm_status resolve(const mtfm_cfg* c, Resolved* r) {
   if (c->hq <= 0 || c->hkv <= 0 || c->head_dim <= 0) return MTFM_ERR_INVALID_ARG;
   if (c->hq % c->hkv != 0) return MTFM_ERR_INVALID_ARG;
   if (c->v2_subtokens != 1 && c->v2_subtokens != 4) return MTFM_ERR_INVALID_ARG;
-  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return MTFM_ERR_UNSUPPORTED;
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256)
+    return MTFM_ERR_UNSUPPORTED;
   if (c->hq / c->hkv > 8) return MTFM_ERR_UNSUPPORTED;
   const long long D = (long long)c->hq * c->head_dim;
   if (D > 1024 || D % 32 != 0) return MTFM_ERR_UNSUPPORTED;
@@ -193,6 +194,7 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   mtfm_status s = resolve(cfg, &r);
   if (s != MTFM_OK) return s;
   if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  if (r.dh == 256) return MTFM_ERR_UNSUPPORTED;  // forward only for head_dim 256
   if (r.total_tokens == 0) return MTFM_OK;
   const int rows = target ? r.total_t : r.total_tokens;
   if (!d_k || !d_v || !d_dk || !d_dv || !d_ws) return MTFM_ERR_INVALID_ARG;

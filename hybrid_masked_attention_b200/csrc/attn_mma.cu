@@ -9,8 +9,10 @@
 // tile's largest kv_end are never loaded (block skipping); blocks below the
 // tile's smallest kv_end skip the per-element mask test.
 //
-// Forward: one CTA = one 128-row query tile of one user x one query head;
-// 8 warps x 16 rows; 64-key blocks double-buffered through cp.async.
+// Forward: one CTA = one 128-row query tile of one user x one query head (x one
+// half of the head's output columns for head_dim 256, where the scores are
+// computed over the whole head in each half); 8 warps x 16 rows; 64-key blocks
+// double-buffered through cp.async.
 // Backward: one CTA = one 64-key block of one user x one KV group; loops over
 // the r query heads of the group and every query tile that can see the block;
 // dK/dV accumulate in registers, dQ is added with fp32 atomics.
@@ -81,9 +83,13 @@ struct FwdSmem {
   static constexpr size_t kBytes = sizeof(__nv_bfloat16) * (size_t)(kQ + 4 * kKV);
 };
 
-template <int DH, bool TARGET>
+// DV: output columns of the head this CTA accumulates (DH, or DH / 2 for head_dim 256:
+// the O registers of a 16-row warp tile hold DV / 8 x 4 floats per thread).
+template <int DH, int DV, bool TARGET>
 __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
+  static_assert(DH % DV == 0, "output split");
   using S = FwdSmem<DH>;
+  const int vcol = blockIdx.z * DV;  // first output column of the head
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   __nv_bfloat16* sK = sQ + S::kQ;       // [2][kBN][stride]
@@ -157,9 +163,9 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
   const RowMask ma = row_mask(m, ui, p.v2, pos0 + ra, ra < nq);
   const RowMask mb = row_mask(m, ui, p.v2, pos0 + rb, rb < nq);
 
-  float o[DH / 8][4];
+  float o[DV / 8][4];
 #pragma unroll
-  for (int i = 0; i < DH / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  for (int i = 0; i < DV / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   uint32_t qa[DH / 16][4];
 
   const float alpha = p.alpha;
@@ -222,11 +228,11 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-      for (int dp = 0; dp < DH / 16; ++dp) {
+      for (int dp = 0; dp < DV / 16; ++dp) {
         uint32_t b0, b1, b2, b3;
         const int mi = lane >> 3;
         const int key = kk * 16 + (lane & 7) + (mi & 1) * 8;
-        const int col = dp * 16 + (mi >> 1) * 8;
+        const int col = vcol + dp * 16 + (mi >> 1) * 8;
         ldsm_x4_t(smem_u32(cV + key * S::kStride + col), b0, b1, b2, b3);
         mma_bf16(o[2 * dp], pa[kk], b0, b1);
         mma_bf16(o[2 * dp + 1], pa[kk], b2, b3);
@@ -241,8 +247,8 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
   // Epilogue: A = O / N_u (fp32)
   const float inv_n = ui.N > 0 ? 1.f / (float)ui.N : 0.f;
 #pragma unroll
-  for (int n = 0; n < DH / 8; ++n) {
-    const int col = h * DH + n * 8 + 2 * (lane & 3);
+  for (int n = 0; n < DV / 8; ++n) {
+    const int col = h * DH + vcol + n * 8 + 2 * (lane & 3);
     if (ra < nq)
       *reinterpret_cast<float2*>(p.a + (size_t)(qrow0 + ra) * ldq + col) =
           make_float2(o[n][0] * inv_n, o[n][1] * inv_n);
@@ -533,11 +539,12 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 
 template <int DH, bool TARGET>
 cudaError_t fwd_dispatch(const FwdArgs& a, int max_items, cudaStream_t st) {
+  constexpr int DV = DH > 128 ? 128 : DH;
   const size_t smem = FwdSmem<DH>::kBytes;
-  cudaError_t e = set_smem(attn_fwd_mma_kernel<DH, TARGET>, smem);
+  cudaError_t e = set_smem(attn_fwd_mma_kernel<DH, DV, TARGET>, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(max_items, a.hq);
-  attn_fwd_mma_kernel<DH, TARGET><<<grid, 256, smem, st>>>(a);
+  dim3 grid(max_items, a.hq, DH / DV);
+  attn_fwd_mma_kernel<DH, DV, TARGET><<<grid, 256, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -562,6 +569,7 @@ cudaError_t launch_attn_fwd_mma(const AttnShape& s, const MetaView& m, int max_i
     case 32: return s.target ? fwd_dispatch<32, true>(args, max_items, st) : fwd_dispatch<32, false>(args, max_items, st);
     case 64: return s.target ? fwd_dispatch<64, true>(args, max_items, st) : fwd_dispatch<64, false>(args, max_items, st);
     case 128: return s.target ? fwd_dispatch<128, true>(args, max_items, st) : fwd_dispatch<128, false>(args, max_items, st);
+    case 256: return s.target ? fwd_dispatch<256, true>(args, max_items, st) : fwd_dispatch<256, false>(args, max_items, st);
     default: return cudaErrorInvalidValue;
   }
 }

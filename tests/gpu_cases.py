@@ -23,4 +23,5 @@ HEADS = {
     "pair": syn.PAIR_HEADS,                 # Hq 8, Hkv 2, dh 64
     "dh128": syn.Heads(4, 1, 128),
     "r8": syn.Heads(8, 1, 32),
+    "dh256": syn.Heads(3, 1, 256),          # the 768-wide shape: Hq 3, Hkv 1, dh 256 (forward only)
 }

@@ -113,6 +113,23 @@ def test_stack_tiny_heads(cuda_ok):
     assert_increment_close(got - X0, ref - X0, "X16 - X0 tiny")
 
 
+def test_stack_d768_dh256(cuda_ok):
+    """The 768-wide shape (d_model 768, Hq 3, Hkv 1, head_dim 256: the mma.sync attention
+    with the output columns in two halves), one Full and one Target layer, 4 users."""
+    import hybrid_masked_attention_b200 as M
+    b, hd, d = syn.pair_batch(4, 1007), syn.Heads(3, 1, 256), 768
+    ws_ = syn.stack_weights(hd, d, 76, kinds=("F", "T"))
+    X0 = _x0(b, d, 76)
+    cfg, meta, ws = _session(b, hd, d)
+    x = torch.from_numpy(X0.astype(np.float32)).cuda()
+    M.stack_fwd(cfg, meta, d, _device_layers(ws_), x, ws)
+    M.pack_check(meta)
+    got = x.cpu().numpy().astype(np.float64)
+    ref = O.stack_fwd(b, hd, ws_, X0)
+    assert_close(got, ref, "X2")
+    assert_increment_close(got - X0, ref - X0, "X2 - X0 (d_model 768)")
+
+
 def _subset(batch, users):
     ro, to = O.offsets(batch.L_R), O.offsets(batch.L_T)
     idx = np.asarray(users)
