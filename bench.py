@@ -595,13 +595,14 @@ def run_extra(args):
     import hybrid_masked_attention_b200 as M
     from hybrid_masked_attention_b200.session import HybridAttention
     dev = torch.device("cuda", 0)
-    heads = syn.PAIR_HEADS
+    heads = syn.Heads(*(int(x) for x in args.heads.split(",")))
     if args.workload == "sweep":
         b = syn.sweep_batch(args.seqlen, v2=args.v2, seed=1003)
         name = f"sweep N={args.seqlen}{' V2' if args.v2 else ''}: {b.B} users x {args.seqlen} tokens"
     else:
         b = syn.pair_batch(args.users, seed=1005)
-        name = f"training step: {b.B} users, production-shape lengths"
+        name = f"training step: {b.B} users, production-shape lengths" + (
+            "" if heads == syn.PAIR_HEADS else f", Hq {heads.hq} / Hkv {heads.hkv}, head_dim {heads.dh}")
     cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh,
                    b.v2_subtokens)
     s = HybridAttention(cfg, dev)
@@ -911,7 +912,8 @@ def main():
     ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
     ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")
     ap.add_argument("--dmodel", type=int, default=512, help="stack: d_model")
-    ap.add_argument("--heads", default="8,2,64", help="stack: Hq,Hkv,head_dim (e.g. 3,1,256 with --dmodel 768)")
+    ap.add_argument("--heads", default="8,2,64",
+                    help="stack/sweep/train: Hq,Hkv,head_dim (e.g. 3,1,256 with --dmodel 768)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -194,7 +194,6 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   mtfm_status s = resolve(cfg, &r);
   if (s != MTFM_OK) return s;
   if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
-  if (r.dh == 256) return MTFM_ERR_UNSUPPORTED;  // forward only for head_dim 256
   if (r.total_tokens == 0) return MTFM_OK;
   const int rows = target ? r.total_t : r.total_tokens;
   if (!d_k || !d_v || !d_dk || !d_dv || !d_ws) return MTFM_ERR_INVALID_ARG;

@@ -291,8 +291,11 @@ struct BwdSmem {
 
 // Every bf16 operand built from an fp32 intermediate (P, dS, dA) is split into
 // hi + lo bf16 parts and multiplied twice, so the products keep ~16 bits.
-template <int DH>
+// DV: output columns of dQ, dK, dV this CTA accumulates (DH, or DH / 2 for head_dim
+// 256, where S^T and dP^T are computed over the whole head in each half).
+template <int DH, int DV>
 __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
+  static_assert(DH % DV == 0, "output split");
   using S = BwdSmem<DH>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem_raw);
@@ -314,7 +317,8 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
   const UserInfo ui = user_info(m, it.user);
   const int j0 = it.tile * kTileM + blockIdx.y * kBwdKeys;
   if (j0 >= ui.N) return;
-  const int g = blockIdx.z, r = p.hq / p.hkv;
+  const int g = blockIdx.z / (DH / DV), r = p.hq / p.hkv;
+  const int vcol = (blockIdx.z % (DH / DV)) * DV;  // first output column of the head
   const int ldq = p.hq * DH, ldk = p.hkv * DH;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0pos = ui.LH + ui.LR;
@@ -353,9 +357,9 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
   const int qi_lo = max(0, p_lo - qpos0);
   const int qi_hi = min(nq, p_hi - qpos0);
 
-  float dk[DH / 8][4], dv[DH / 8][4];
+  float dk[DV / 8][4], dv[DV / 8][4];
 #pragma unroll
-  for (int i = 0; i < DH / 8; ++i)
+  for (int i = 0; i < DV / 8; ++i)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[i][e] = dv[i][e] = 0.f;
 
@@ -452,11 +456,11 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
           *reinterpret_cast<uint32_t*>(sDl + (kr + 8) * S::kDSStride + ql) = dl_[half * 2 + 1];
         }
 #pragma unroll
-        for (int dp = 0; dp < DH / 16; ++dp) {
+        for (int dp = 0; dp < DV / 16; ++dp) {
           uint32_t b0, b1, b2, b3;
           const int mi = lane >> 3;
           const int qq = kk * 16 + (lane & 7) + (mi & 1) * 8;
-          const int col = dp * 16 + (mi >> 1) * 8;
+          const int col = vcol + dp * 16 + (mi >> 1) * 8;
           ldsm_x4_t(smem_u32(sAh + qq * S::kStride + col), b0, b1, b2, b3);
           mma_bf16(dv[2 * dp], ph, b0, b1);
           mma_bf16(dv[2 * dp + 1], ph, b2, b3);
@@ -475,9 +479,9 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
       __syncthreads();
       // dQ[16 queries of this warp] += (dS_hi + dS_lo) K  -> fp32 atomics
       {
-        float dq[DH / 8][4];
+        float dq[DV / 8][4];
 #pragma unroll
-        for (int i = 0; i < DH / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
+        for (int i = 0; i < DV / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < kBwdKeys / 16; ++kk) {
           uint32_t ah[4], al[4];
@@ -487,10 +491,10 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
           ldsm_x4_t(smem_u32(sDh + key * S::kDSStride + qq), ah[0], ah[1], ah[2], ah[3]);
           ldsm_x4_t(smem_u32(sDl + key * S::kDSStride + qq), al[0], al[1], al[2], al[3]);
 #pragma unroll
-          for (int dp = 0; dp < DH / 16; ++dp) {
+          for (int dp = 0; dp < DV / 16; ++dp) {
             uint32_t b0, b1, b2, b3;
             const int key2 = kk * 16 + (lane & 7) + (mi & 1) * 8;
-            const int col = dp * 16 + (mi >> 1) * 8;
+            const int col = vcol + dp * 16 + (mi >> 1) * 8;
             ldsm_x4_t(smem_u32(sK + key2 * S::kStride + col), b0, b1, b2, b3);
             mma_bf16(dq[2 * dp], ah, b0, b1);
             mma_bf16(dq[2 * dp + 1], ah, b2, b3);
@@ -500,8 +504,8 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
         }
         const int qa_ = qt + warp * 16 + (lane >> 2), qb_ = qa_ + 8;
 #pragma unroll
-        for (int n = 0; n < DH / 8; ++n) {
-          const int col = h * DH + n * 8 + 2 * (lane & 3);
+        for (int n = 0; n < DV / 8; ++n) {
+          const int col = h * DH + vcol + n * 8 + 2 * (lane & 3);
           if (qa_ < nq) {
             float* d = p.dq + (size_t)(qrow0 + qa_) * ldq + col;
             atomicAdd(d, dq[n][0]);
@@ -519,8 +523,8 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
   }
   // write dK, dV of this key block (all keys of the block: zero when nothing sees them)
 #pragma unroll
-  for (int n = 0; n < DH / 8; ++n) {
-    const int col = g * DH + n * 8 + 2 * (lane & 3);
+  for (int n = 0; n < DV / 8; ++n) {
+    const int col = g * DH + vcol + n * 8 + 2 * (lane & 3);
     if (ka < ui.N) {
       *reinterpret_cast<float2*>(p.dk + (size_t)(ui.so + ka) * ldk + col) = make_float2(dk[n][0], dk[n][1]);
       *reinterpret_cast<float2*>(p.dv + (size_t)(ui.so + ka) * ldk + col) = make_float2(dv[n][0], dv[n][1]);
@@ -550,11 +554,12 @@ cudaError_t fwd_dispatch(const FwdArgs& a, int max_items, cudaStream_t st) {
 
 template <int DH>
 cudaError_t bwd_dispatch(const BwdArgs& a, int max_items_full, cudaStream_t st) {
+  constexpr int DV = DH > 128 ? 128 : DH;
   const size_t smem = BwdSmem<DH>::kBytes;
-  cudaError_t e = set_smem(attn_bwd_mma_kernel<DH>, smem);
+  cudaError_t e = set_smem(attn_bwd_mma_kernel<DH, DV>, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(max_items_full, kTileM / kBwdKeys, a.hkv);
-  attn_bwd_mma_kernel<DH><<<grid, 128, smem, st>>>(a);
+  dim3 grid(max_items_full, kTileM / kBwdKeys, a.hkv * (DH / DV));
+  attn_bwd_mma_kernel<DH, DV><<<grid, 128, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -585,6 +590,7 @@ cudaError_t launch_attn_bwd_mma(const AttnShape& s, const MetaView& m, int max_i
     case 32: return bwd_dispatch<32>(args, max_items_full, st);
     case 64: return bwd_dispatch<64>(args, max_items_full, st);
     case 128: return bwd_dispatch<128>(args, max_items_full, st);
+    case 256: return bwd_dispatch<256>(args, max_items_full, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -47,9 +47,8 @@
  *     attention kernel draws its work from it and sets it back to zero when it
  *     finishes.  Hence two Full-layer forward calls on one metadata block must
  *     be ordered (same stream, or an event); other calls may overlap.
- *   - Supported: head_dim in {32, 64, 128}, and 256 for the forward calls only
- *     (the backward calls return MTFM_ERR_UNSUPPORTED for it); hq % hkv == 0;
- *     hq/hkv <= 8; hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
+ *   - Supported: head_dim in {32, 64, 128, 256}; hq % hkv == 0; hq/hkv <= 8;
+ *     hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
  *   - No exceptions cross this boundary; no global state is kept.  The
  *     forward attention runs the tcgen05/TMEM kernel for head_dim 64 with

@@ -35,7 +35,7 @@ def _rows(batch, users, target):
 
 CASES = [("tiny", "tiny", True), ("tiny", "tiny", False), ("edge", "pair", True),
          ("edge", "r8", True), ("v2_n512", "pair", True), ("pair", "pair", True),
-         ("pair", "dh128", False)]
+         ("pair", "dh128", False), ("edge", "dh256", True), ("tiny", "dh256", False)]
 
 
 @pytest.mark.parametrize("bname,hname,gln", CASES)
