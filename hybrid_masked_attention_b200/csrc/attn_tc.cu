@@ -208,7 +208,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           ++issued;
         }
         // the next pair, read by every role after this unit's closing barrier
-        s_ticket[(unit_iter + 1) & 1] = (int)atomicAdd(ticket_ctr, 1u);
+        const int w1 = (int)atomicAdd(ticket_ctr, 1u);
+        s_ticket[(unit_iter + 1) & 1] = w1;
+        if (w1 < n_work) {
+          // its Q tiles and first K/V blocks into L2 now, so that its loads after the unit
+          // barrier do not wait for DRAM
+          const int item1 = w1 / p.hkv, g1 = w1 % p.hkv;
+          const WorkItem it1 = m.items_full[item1];
+          const int u1 = it1.user;
+          const int LH1 = m.lh[u1], LR1 = m.lr[u1], N1 = LH1 + LR1 + m.lt[u1], so1 = m.seq_off[u1];
+          for (int hh = 0; hh < R; ++hh) tma_prefetch_l2_2d(&tm_q, (g1 * R + hh) * kDH, so1 + it1.tile * kBM);
+          const KeyBlocks kb1 = key_blocks(it1.kv_max, LH1, LR1, N1, 0, it1.tile * kBM, p.v2);
+          for (int bi = 0; bi < min(kb1.n_blocks, kStages); ++bi) {
+            const int row1 = so1 + kb1.block(bi) * kBN;
+            tma_prefetch_l2_2d(&tm_k, g1 * kDH, row1);
+            tma_prefetch_l2_2d(&tm_v, g1 * kDH, row1);
+          }
+        }
         // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
         // no TMA write may land after this unit's barriers are re-armed or the CTA leaves.
         const long long t0 = clock64();
