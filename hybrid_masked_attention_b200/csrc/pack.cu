@@ -207,6 +207,18 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
   }
 }
 
+constexpr int kTsStage = 512;  // R timestamps of a user staged in shared memory by the row pass (4 KB)
+
+// Number of R timestamps strictly below `x` in the ascending array ts[0, n) (shared memory).
+__device__ __forceinline__ int count_below_shared(const int64_t* ts, int n, int64_t x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (ts[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
 // Number of R timestamps strictly below `x` in the ascending array ts[0, n).
 __device__ __forceinline__ int count_below(const int64_t* __restrict__ ts, int n, int64_t x) {
   int lo = 0, hi = n;
@@ -283,6 +295,17 @@ __device__ void pack_item_rows(MetaView m, bool tgt, int idx, int tgt_sub_rows, 
   const int N = LH + LR + LT, so = m.seq_off[u];
   const int nq = tgt ? LT : N;
   const int r = tile * kTileM + threadIdx.x;
+  // The T rows of this tile search the user's sorted R timestamps: stage them in shared
+  // memory once (one round trip) instead of a chain of dependent global loads per row.
+  __shared__ int64_t s_ts[kTsStage];
+  const int64_t* ts_u = r_ts + m.r_off[u];
+  const int first_row = tgt ? LH + LR + tile * kTileM : tile * kTileM;
+  const bool has_t = first_row + kTileM > LH + LR && tile * kTileM < nq;  // uniform over the CTA
+  const bool staged = has_t && LR <= kTsStage;
+  if (staged) {
+    for (int k = threadIdx.x; k < LR; k += blockDim.x) s_ts[k] = ts_u[k];
+    __syncthreads();
+  }
   int kmin = 0x7fffffff, kmax = 0;
   if (r < nq) {
     const int i = tgt ? LH + LR + r : r;
@@ -298,7 +321,8 @@ __device__ void pack_item_rows(MetaView m, bool tgt, int idx, int tgt_sub_rows, 
         atomicOr(&m.hdr->error, kErrUnsorted);
     } else {
       type = kRowT;
-      kve = LH + count_below(r_ts + m.r_off[u], LR, t_exp[m.t_off[u] + (i - LH - LR)]);
+      const int64_t x = t_exp[m.t_off[u] + (i - LH - LR)];
+      kve = LH + (staged ? count_below_shared(s_ts, LR, x) : count_below(ts_u, LR, x));
     }
     if (!tgt) {
       m.kv_end[so + i] = kve;
