@@ -128,7 +128,8 @@ def _brute_attention(q, k, v, M, hq, hkv, dh, alpha, n_norm):
 
 def check_attention_bruteforce():
     rng = np.random.default_rng(3)
-    for (LH, LR, LT, hq, hkv, dh) in [(3, 2, 2, 2, 1, 4), (2, 3, 3, 4, 2, 3), (0, 2, 1, 2, 2, 2)]:
+    # the last case has r = 3 query heads per KV head (the 768-wide Hq 3 / Hkv 1 shape)
+    for (LH, LR, LT, hq, hkv, dh) in [(3, 2, 2, 2, 1, 4), (2, 3, 3, 4, 2, 3), (0, 2, 1, 2, 2, 2), (2, 2, 3, 3, 1, 5)]:
         N = LH + LR + LT
         r_ts = np.sort(rng.integers(0, 10, LR))
         t_exp = rng.integers(0, 10, LT)
