@@ -2,7 +2,6 @@
 // No allocation, no synchronisation (except mtfm_pack_check / mtfm_meta_read,
 // which synchronise on purpose).  See include/mtfm.h for the contract.
 #include <math.h>
-#include <stdlib.h>
 #include <string.h>
 
 #include "mtfm_internal.cuh"
@@ -58,17 +57,21 @@ mtfm_status check_meta(const void* d_meta, const Resolved& r) {
 
 // tcgen05/TMEM kernels where their TMEM plans fit (head_dim 64, r in {1, 2, 4}; the
 // Target layer stacks the r heads of a group as MMA rows);
-// the mma.sync kernel covers the other head shapes.  MTFM_FWD_KERNEL=mma
-// selects the mma.sync kernel for every shape (for comparisons).
+// the mma.sync kernel covers the other head shapes.  A library compiled with
+// -DMTFM_PORTABLE_KERNELS runs the mma.sync kernels for every shape (a test build
+// for comparing the two; the shipped library has no run-time switch).
+#ifdef MTFM_PORTABLE_KERNELS
+constexpr bool kPortableOnly = true;
+#else
+constexpr bool kPortableOnly = false;
+#endif
 cudaError_t launch_attn(const Resolved& r, const MetaView& m, const MetaLayout& L, bool target,
                         const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                         float* a, cudaStream_t st) {
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
   const int max_items = target ? L.max_items_target : L.max_items_full;
   const int rows = target ? r.total_t : r.total_tokens;
-  const char* force = getenv("MTFM_FWD_KERNEL");
-  const bool force_mma = force && strcmp(force, "mma") == 0;
-  if (!force_mma && attn_fwd_tc_supported(shape)) {
+  if (!kPortableOnly && attn_fwd_tc_supported(shape)) {
     if (target) return launch_attn_fwd_tgt(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
     return launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
   }
@@ -152,8 +155,7 @@ mtfm_status attn_target_cached(const mtfm_cfg* cfg, const void* d_meta, const ui
   if (s != MTFM_OK) return s;
   if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, true};
-  const char* force = getenv("MTFM_FWD_KERNEL");
-  if (!attn_fwd_tc_supported(shape) || (force && strcmp(force, "mma") == 0)) return MTFM_ERR_UNSUPPORTED;
+  if (!attn_fwd_tc_supported(shape) || kPortableOnly) return MTFM_ERR_UNSUPPORTED;
   if (r.total_t == 0 || r.total_tokens == 0) return MTFM_OK;
   const int prefix_rows = r.total_tokens - r.total_t;
   if (!d_q || !d_kc || !d_vc || !d_a) return MTFM_ERR_INVALID_ARG;
@@ -226,9 +228,8 @@ mtfm_status attn_bwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
   if (e != cudaSuccess) return MTFM_ERR_CUDA;
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
   // tcgen05 kernel for head_dim 64; the mma.sync kernel for the other head sizes
-  // (MTFM_BWD_KERNEL=mma selects it for every shape, to compare the two).
-  const char* force = getenv("MTFM_BWD_KERNEL");
-  if (!(force && strcmp(force, "mma") == 0) && attn_bwd_tc_supported(shape)) {
+  // (and for every shape in a -DMTFM_PORTABLE_KERNELS test build).
+  if (!kPortableOnly && attn_bwd_tc_supported(shape)) {
     e = launch_attn_bwd_tc(shape, m, L.max_items_full, rows, r.total_tokens,
                            reinterpret_cast<const __nv_bfloat16*>(d_q), reinterpret_cast<const __nv_bfloat16*>(d_k),
                            reinterpret_cast<const __nv_bfloat16*>(d_v), da_hi, da_lo, d_dq, d_dk, d_dv, st);

@@ -9,39 +9,40 @@
 // the library image itself, so the caller passes only inputs and outputs.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
-// library holds kStaticScratchBytes for the life of the process.  Host code
-// cannot use its name as a device address, so the first call on each device
-// resolves the address with cudaGetSymbolAddress (with that device current)
-// and caches it; that first call should therefore come before any stream
-// capture.  All calls share the one array, so calls whose work overlaps on the
+// library's device code holds kStaticScratchBytes for the life of the process.
+// With CUDA's lazy module loading (the default), that device memory is committed
+// when this file's module is first loaded on a device, which is the first call
+// of this entry point there (its cudaGetSymbolAddress); a caller that reserves
+// the rest of its device memory, or captures streams, afterwards should make one
+// call first.  Later calls allocate nothing.  Host code cannot use the array's
+// name as a device address, so every call looks the address up with
+// cudaGetSymbolAddress on the device of the call's stream, which must be the
+// current device (after a device reset the lookup simply finds the reloaded
+// module).  All calls share the one array, so calls whose work overlaps on the
 // GPU (different streams, or different host threads on one stream without
 // ordering) race on it.  Nothing in it needs to start at zero: every byte the
 // backward reads was written earlier in the same call.
-#include <mutex>
-
 #include "mtfm_internal.cuh"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(24) << 20;  // 24 MiB
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device (resolved once per device).
-mtfm_status static_scratch(void** out) {
+// Device address of g_static_scratch on the current device, which must also be the
+// device of `stream` (NULL: the legacy stream of the current device).
+mtfm_status static_scratch(void* stream, void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTFM_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return MTFM_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MTFM_ERR_CUDA;
+  if (stream) {
+    int sdev = -1;
+    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) return MTFM_ERR_CUDA;
+    if (sdev != dev) return MTFM_ERR_INVALID_ARG;
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return MTFM_ERR_CUDA;
+  *out = p;
   return MTFM_OK;
 }
 
@@ -56,7 +57,7 @@ extern "C" mtfm_status mtfm_attn_target_bwd_static(
   if (need == 0) return MTFM_ERR_INVALID_ARG;
   if (need > kStaticScratchBytes) return MTFM_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
-  const mtfm_status s = static_scratch(&scratch);
+  const mtfm_status s = static_scratch(stream, &scratch);
   if (s != MTFM_OK) return s;
   return mtfm_attn_target_bwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_a, d_stats, d_dy,
                               d_dq, d_dk, d_dv, d_du, d_dgamma, d_dbeta, scratch,

@@ -8,8 +8,10 @@
 // tile holds TR = 128 / r T rows x r heads (row m = t r + h, which is exactly the
 // shared-memory order of a 3-D TMA box {64 dims, r heads, TR rows} of Q), so one
 // QK^T and one PV MMA chain per 128-key block serve all r heads and the few T rows
-// of a user fill the tile.  A work unit is one (sub-tile of TR T rows, chunk of
-// kTargetUnitBlocks key blocks, KV group); the CTAs (one per SM) stride over them.
+// of a user fill the tile.  A work unit is one (sub-tile of TR T rows, chunk of C key
+// blocks, KV group), C = MetaHeader::tgt_chunk_blocks (at least kTargetUnitBlocks),
+// chosen per layer by the packer's Target unit scan; the CTAs (one per SM) stride
+// over the units.
 //
 // Cached-prefix form (request-level inference with shared user K/V: M-Falcon micro-
 // batching with a shared KV cache, page "美团推荐大模型 MTFM 深度硬核解析" §5.2.3): the keys/values of a user's H and R rows come from a cache

@@ -50,11 +50,11 @@
  *   - Supported: head_dim in {32, 64, 128, 256}; hq % hkv == 0; hq/hkv <= 8;
  *     hq*head_dim <= 1024 and a multiple of 32; v2_subtokens in {1, 4}.
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
- *   - No exceptions cross this boundary; no global state is kept.  The
- *     forward attention runs the tcgen05/TMEM kernel for head_dim 64 with
+ *   - No exceptions cross this boundary; no global state is kept (the one
+ *     exception is the fixed scratch array of mtfm_attn_target_bwd_static).
+ *     The forward attention runs the tcgen05/TMEM kernel for head_dim 64 with
  *     hq/hkv in {1, 2, 4} and the portable mma.sync kernel otherwise; the
- *     environment variable MTFM_FWD_KERNEL=mma selects the portable kernel for
- *     every shape (used to compare the two).
+ *     choice depends on the shape only (no run-time switch).
  */
 #ifndef MTFM_H_
 #define MTFM_H_
@@ -207,7 +207,17 @@ mtfm_status mtfm_attn_target_cached(const mtfm_cfg* cfg, const void* d_meta, con
                                     void* stream);
 
 /* ---------------------------------------------------------------------------
- * Backward passes (training step).  Inputs are the forward's inputs, its saved
+ * Backward passes (training step): gradients of the Full-Attention layer
+ * ([DY] §4.1) and Target-Attention layer ([DY] §4.2) forward above, the
+ * backward half of the Full/Target attention kernels the Meituan tech blog
+ * describes in §6.1 (its FA2-derived kernels cover training, forward and
+ * backward, with the dynamic mask read and SiLU fused).  With x = alpha q.k,
+ * sigma = sigmoid(x) and P = SiLU(x) / N_u on visible pairs:
+ *   dU = GLN(A) (*) dY;  dA = GLN backward of dY (*) U;  dgamma, dbeta per type;
+ *   dV_j += sum_i P_ij dA_i;  dS_ij = (dA_i . v_j) sigma (1 + x (1 - sigma)) / N_u;
+ *   dQ_i = alpha sum_j dS_ij k_j;  dK_j = alpha sum_i dS_ij q_i  (over the r heads
+ *   of a KV group for dK, dV).
+ * Inputs are the forward's inputs, its saved
  * A (d_a) and stats, and the upstream gradient d_dy (bf16, same shape as Y).
  * Outputs (fp32, fully overwritten):
  *   d_dq, d_du : same rows as Q/U;   d_dk, d_dv : [total_tokens, hkv*head_dim]
@@ -242,11 +252,16 @@ mtfm_status mtfm_attn_target_bwd(const mtfm_cfg* cfg, const void* d_meta, const 
  * more scratch than that (mtfm_bwd_workspace_bytes(cfg, 1) > 24 MiB; at
  * hq * head_dim = 512 that is about 10,000 T rows).
  *
- * The library allocates nothing here.  The first call on a device looks up the
- * array's device address (make that first call before any stream capture).
- * All calls share the one array: calls whose GPU work can overlap (other
- * streams, or unordered host threads) race on it and must be serialised by
- * the caller.  Its contents are left over from the previous call; none of
+ * Device memory: the array is committed when the library's module holding it
+ * is loaded on a device.  Under CUDA's lazy module loading (the default) that
+ * happens during the first call of this entry point on that device, so a
+ * caller that reserves the rest of its device memory, or starts a stream
+ * capture, afterwards should make one call first; every later call allocates
+ * nothing.  Each call looks up the array's device address on the current
+ * device, which must be the device of `stream` (MTFM_ERR_INVALID_ARG
+ * otherwise).  All calls share the one array: calls whose GPU work can overlap
+ * (other streams, or unordered host threads) race on it and must be serialised
+ * by the caller.  Its contents are left over from the previous call; none of
  * them is read before this call rewrites it.
  * ------------------------------------------------------------------------- */
 mtfm_status mtfm_attn_target_bwd_static(const mtfm_cfg* cfg, const void* d_meta,

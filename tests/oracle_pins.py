@@ -290,13 +290,26 @@ def check_gln_is_layernorm():
     assert m is None and np.array_equal(Y3, A * U)
 
 
-def check_hr_rows_in_target_layer_untouched():
-    """Target layer output covers only T rows ([DY] §4.2 shortcut): the row count is sum L_T."""
+def check_target_rows_ignore_hr_queries():
+    """A row's output depends on its own query and U only ([DY] §4.2: the Target layer
+    drops the H/R queries): changing the Q and U rows of every H and R token leaves
+    the T rows of a Full layer bit-identical, and those rows still equal the Target
+    layer computed without any H/R query, while the H/R rows do change."""
     b = _small_batch()
     hd = syn.Heads(2, 1, 8)
-    tgt = syn.layer_inputs(b, hd, target=True, seed=9)
-    T = O.target_fwd(b, hd, tgt)
-    assert T["Y"].shape[0] == b.total_t and np.isfinite(T["Y"]).all()
+    full = syn.layer_inputs(b, hd, target=False, seed=9)
+    tr = O.t_row_index(b)
+    hr = np.setdiff1d(np.arange(b.total_tokens), tr)
+    base = O.full_fwd(b, hd, full)
+    q, u = full.q.copy(), full.u.copy()
+    q[hr] ^= 0x0041
+    u[hr] ^= 0x0041
+    pert = O.full_fwd(b, hd, syn.LayerInputs(q, full.k, full.v, u, full.gamma, full.beta))
+    assert np.array_equal(pert["Y"][tr], base["Y"][tr])
+    assert np.array_equal(pert["A"][tr], base["A"][tr])
+    assert not np.allclose(pert["Y"][hr], base["Y"][hr])
+    tgt = O.target_fwd(b, hd, syn.LayerInputs(full.q[tr], full.k, full.v, full.u[tr], full.gamma, full.beta))
+    assert np.allclose(tgt["Y"], pert["Y"][tr], rtol=1e-12, atol=1e-12)
 
 
 # ----------------------------------------------------------------------------- backward
@@ -372,7 +385,7 @@ ALL_CHECKS = [
     check_permutation_equivariance,
     check_locality,
     check_gln_is_layernorm,
-    check_hr_rows_in_target_layer_untouched,
+    check_target_rows_ignore_hr_queries,
     check_backward_finite_differences,
     check_dv_closed_form,
 ]

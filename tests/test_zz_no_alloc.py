@@ -7,6 +7,10 @@ results must match mtfm_attn_target_bwd, which runs the same kernels on a
 caller-provided scratch block, on two calls in a row (the second call sees
 the array the first call left behind).
 
+The first call on a device may commit the array (CUDA loads the module that
+holds it lazily); the second call is checked to leave free device memory
+unchanged.
+
 This file is collected last so that a run stopping at the first failure has
 already run every other test.
 """
@@ -42,10 +46,17 @@ def test_static_scratch_backward_matches_workspace_backward(cuda_ok):
         out = {"dq": torch.full((T, D), float("nan"), **f32), "dk": torch.full((N, Dkv), float("nan"), **f32),
                "dv": torch.full((N, Dkv), float("nan"), **f32), "du": torch.full((T, D), float("nan"), **f32),
                "dgamma": torch.full((3, D), float("nan"), **f32), "dbeta": torch.full((3, D), float("nan"), **f32)}
+        torch.cuda.synchronize()
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         attn_target_bwd_static(s.cfg, s.meta, d["q"], d["k"], d["v"], d["u"], d["gamma"], d["beta"], a, st,
                                d["dy"], out["dq"], out["dk"], out["dv"], out["du"], out["dgamma"],
                                out["dbeta"])
         torch.cuda.synchronize()
+        if call == 1:
+            # the first call may load the library module that holds the array; the
+            # second must not take any device memory
+            assert torch.cuda.mem_get_info()[0] == free0, "the second call changed free device memory"
+            assert torch.cuda.memory_allocated() == alloc0
         for name in ("dq", "dk", "dv", "du", "dgamma", "dbeta"):
             assert_close(out[name].cpu().numpy(), ref[name].cpu().numpy(), f"call {call} {name}")
 
