@@ -280,7 +280,7 @@ def run_mtfm(args, rank, world, local_rank):
     stream = torch.cuda.Stream(dev)
     launches_per_step = 6   # pack (2 kernels), Full attention, Full gate, Target attention, Target gate
 
-    def step(i, record=None, around_full=None):
+    def step(i, record=None, around_full=None, around_tgt=None):
         s = sets[i % len(sets)]
         e = record
         if e: e[0].record(stream)
@@ -292,7 +292,9 @@ def run_mtfm(args, rank, world, local_rank):
         if e: e[2].record(stream)
         M.gate_fwd(cfg, meta, False, A_f, s["u"], s["g"], s["bt"], Y_f, S_f, stream)
         if e: e[3].record(stream)
+        if around_tgt: around_tgt[0].record(stream)
         M.attn_target(cfg, meta, s["tq"], s["tk"], s["tv"], A_t, stream)
+        if around_tgt: around_tgt[1].record(stream)
         if e: e[4].record(stream)
         M.gate_fwd(cfg, meta, True, A_t, s["tu"], s["tg"], s["tbt"], Y_t, S_t, stream)
         if e: e[5].record(stream)
@@ -318,41 +320,49 @@ def run_mtfm(args, rank, world, local_rank):
             fn()
         return g
 
-    full_ev = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(nset)]
+    mk = lambda: [(torch.cuda.Event(enable_timing=True, external=True),
+                   torch.cuda.Event(enable_timing=True, external=True)) for _ in range(nset)]
+    full_ev, tgt_ev = mk(), mk()
     g_all = capture(lambda: [step(r) for r in range(nset)])
-    g_ev = capture(lambda: [step(r, around_full=full_ev[r]) for r in range(nset)])
+    g_ev = capture(lambda: [step(r, around_full=full_ev[r], around_tgt=tgt_ev[r]) for r in range(nset)])
     singles = [capture(lambda r=r: step(r)) for r in range(nset)]
-    singles_ev = [capture(lambda r=r: step(r, around_full=full_ev[r])) for r in range(nset)]
+    singles_ev = [capture(lambda r=r: step(r, around_full=full_ev[r], around_tgt=tgt_ev[r])) for r in range(nset)]
     reps, rem = divmod(args.steps, nset)
     with torch.cuda.stream(stream):
         for _ in range(max(1, 3 // nset + 1)):
             g_all.replay()
     torch.cuda.synchronize(dev)
     M.pack_check(meta, stream)
-    if world > 1:
-        dist.barrier()
     sampler = ClockSampler(dev) if rank == 0 else None
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
+    # The K-step region is timed `repeats` times (each bracketed by a barrier and a
+    # synchronize on both sides); the value is the median region, the spread is reported.
+    region_ms, full_runs, tgt_runs = [], [], []
     if sampler:
         sampler.begin()
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for i in range(reps):
-            (g_ev if i == reps - 1 else g_all).replay()
-        for r in range(rem):
-            (singles_ev[r] if reps == 0 else singles[r]).replay()
-        t1.record(stream)
-    torch.cuda.synchronize(dev)
+    for _ in range(max(1, args.repeats)):
+        if world > 1:
+            dist.barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(reps):
+                (g_ev if i == reps - 1 else g_all).replay()
+            for r in range(rem):
+                (singles_ev[r] if reps == 0 else singles[r]).replay()
+            t1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        region_ms.append(t0.elapsed_time(t1))
+        n_timed = nset if reps > 0 else rem
+        full_runs += [a.elapsed_time(z) for a, z in full_ev[:n_timed]]
+        tgt_runs += [a.elapsed_time(z) for a, z in tgt_ev[:n_timed]]
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        dist.barrier()
-    ms_total = t0.elapsed_time(t1)
-    n_timed = nset if reps > 0 else rem
-    full_live = [a.elapsed_time(z) for a, z in full_ev[:n_timed]]
-    full_ms = sum(full_live) / len(full_live)
+    ms_total = statistics.median(region_ms)
+    full_ms = statistics.median(full_runs)
+    tgt_ms = statistics.median(tgt_runs)
     M.pack_check(meta, stream)
 
     # Per-part times from a separate eager pass with an event between launches (the events
@@ -388,11 +398,14 @@ def run_mtfm(args, rank, world, local_rank):
         peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         full_tf = fl_full / (full_ms * 1e-3) / 1e12
-        tgt_gbs = target_attn_bytes(b, heads) / (ms_parts["target_attn"] * 1e-3) / 1e9
+        tgt_gbs = target_attn_bytes(b, heads) / (tgt_ms * 1e-3) / 1e9
         traffic = recorded_traffic()
         result = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "repeats": len(region_ms),
+            "ms_per_step_spread": {"min": round(min(region_ms) / args.steps, 5),
+                                   "max": round(max(region_ms) / args.steps, 5)},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; stands in for the pages' proprietary logs)",
             "config": {"workload": WORKLOAD, "users_per_gpu": b.B, "total_tokens": b.total_tokens,
@@ -407,8 +420,11 @@ def run_mtfm(args, rank, world, local_rank):
                          "attn_tflops": round(full_tf, 2),
                          "users_per_s": round(b.B / ((ms_parts["full_attn"] + ms_parts["full_gate"]) * 1e-3), 1)},
                 "target": {"ms": round(ms_parts["target_attn"] + ms_parts["target_gate"], 5),
-                           "attn_tflops": round(fl_tgt / (ms_parts["target_attn"] * 1e-3) / 1e12, 2),
+                           "attn_ms_in_graph": round(tgt_ms, 5),
+                           "attn_tflops": round(fl_tgt / (tgt_ms * 1e-3) / 1e12, 2),
                            "attn_gbs": round(tgt_gbs, 1), "attn_hbm_frac": round(tgt_gbs / hbm, 4),
+                           "attn_timing": "event-record nodes around the Target attention call (accumulator "
+                                          "clear + kernel) inside the timed region",
                            "users_per_s": round(b.B / ((ms_parts["target_attn"] + ms_parts["target_gate"]) * 1e-3), 1)},
                 "ms_parts": {k: round(v, 5) for k, v in ms_parts.items()},
                 "ms_parts_note": "eager pass with an event between launches (not the graph-replayed step)",
@@ -418,11 +434,11 @@ def run_mtfm(args, rank, world, local_rank):
                          "frac": round(full_tf / peak_tf, 4), "traffic": traffic,
                          "peak_source": f"{src} bf16 dense (burst)",
                          "flops_per_launch": fl_full, "launch_ms": round(full_ms, 5),
-                         "launch_ms_source": f"event-record nodes around the last {len(full_live)} Full attention "
-                                             f"launches of the timed region"},
+                         "launch_ms_source": f"median of event-record nodes around the Full attention launches "
+                                             f"of the last steps of each of the {len(region_ms)} timed regions"},
             "e2e": e2e,
             "clocks": clocks,
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches_per_step * args.steps * len(region_ms),
         }
     return result, b, heads
 
@@ -586,224 +602,281 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------------------- other workloads
 
-def run_extra(args):
-    """Per-kernel timings of the other configurations (one JSON line; not the headline metric):
-    ``sweep``: per-user length N (H:R:T ~ 70:15:15, V2 with --v2), 2^21 / N users;
-    ``train``: forward + backward of one Full and one Target layer, --users users of the
-    production-shape distributions.  Activations are seeded device-side normals (bf16)."""
+class GraphStep:
+    """One step's launches captured as two CUDA graphs: plain, and an instrumented twin with
+    event-record nodes around the named launches.  ``timed`` replays K steps (the last one the
+    twin, so every kernel duration is read inside the timed region without paying for event
+    nodes in every step), ``repeats`` times, each region bracketed by a synchronize."""
+
+    def __init__(self, dev, fn, labels):
+        import torch
+        self.torch, self.dev = torch, dev
+        self.stream = torch.cuda.Stream(dev)
+        self.ev = {l: (torch.cuda.Event(enable_timing=True, external=True),
+                       torch.cuda.Event(enable_timing=True, external=True)) for l in labels}
+        mark = lambda l, i: self.ev[l][i].record(self.stream)
+        with torch.cuda.stream(self.stream):
+            fn(None)                       # eager once (lazy module loads, workspaces)
+        torch.cuda.synchronize(dev)
+        self.g = self._capture(lambda: fn(None))
+        self.gi = self._capture(lambda: fn(mark))
+
+    def _capture(self, f):
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g, stream=self.stream):
+            f()
+        return g
+
+    def timed(self, steps, warmup, repeats, sampler=None):
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            for _ in range(max(3, warmup)):
+                self.g.replay()
+        torch.cuda.synchronize(self.dev)
+        if sampler:
+            sampler.begin()
+        per_step = []
+        for _ in range(repeats):
+            a = torch.cuda.Event(enable_timing=True)
+            z = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(self.dev)
+            with torch.cuda.stream(self.stream):
+                a.record(self.stream)
+                for i in range(steps):
+                    (self.gi if i == steps - 1 else self.g).replay()
+                z.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            per_step.append(a.elapsed_time(z) / steps)
+        clocks = sampler.stop() if sampler else None
+        kernels = {l: a.elapsed_time(z) for l, (a, z) in self.ev.items()}
+        return per_step, kernels, clocks
+
+
+def _spread(per_step):
+    return {"median": round(statistics.median(per_step), 5), "min": round(min(per_step), 5),
+            "max": round(max(per_step), 5), "repeats": len(per_step)}
+
+
+def _dev_inputs(dev, seed):
     import torch
-    import hybrid_masked_attention_b200 as M
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    return lambda std, *shape: (std * torch.randn(*shape, generator=gen, device=dev)).to(torch.bfloat16)
+
+
+def _packed(M, b, heads, dev):
+    import torch
     from hybrid_masked_attention_b200.session import HybridAttention
-    dev = torch.device("cuda", 0)
-    heads = syn.Heads(*(int(x) for x in args.heads.split(",")))
-    if args.workload == "sweep":
-        b = syn.sweep_batch(args.seqlen, v2=args.v2, seed=1003)
-        name = f"sweep N={args.seqlen}{' V2' if args.v2 else ''}: {b.B} users x {args.seqlen} tokens"
-    else:
-        b = syn.pair_batch(args.users, seed=1005)
-        name = f"training step: {b.B} users, production-shape lengths" + (
-            "" if heads == syn.PAIR_HEADS else f", Hq {heads.hq} / Hkv {heads.hkv}, head_dim {heads.dh}")
-    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh,
-                   b.v2_subtokens)
+    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh, b.v2_subtokens)
     s = HybridAttention(cfg, dev)
     it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
     lens = (it(b.L_H, np.int32), it(b.L_R, np.int32), it(b.L_T, np.int32), it(b.r_ts, np.int64),
             it(b.t_exp, np.int64))
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(1234)
-    rnd = lambda *shape: torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    N, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
-    gam = torch.ones(3, D, device=dev)
-    bet = torch.zeros(3, D, device=dev)
-    F = dict(q=rnd(N, D), k=rnd(N, Dkv), v=rnd(N, Dkv), u=rnd(N, D), dy=rnd(N, D))
-    Tg = dict(q=rnd(T, D), k=rnd(N, Dkv), v=rnd(N, Dkv), u=rnd(T, D), dy=rnd(T, D))
     s.pack(*lens, check=True)
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    res = {}
-
-    def timed(label, fn, steps):
-        for _ in range(max(3, args.warmup)):
-            fn()
-        torch.cuda.synchronize()
-        a, z = ev(), ev()
-        a.record()
-        for _ in range(steps):
-            fn()
-        z.record()
-        torch.cuda.synchronize()
-        res[label] = a.elapsed_time(z) / steps
-
-    out_f = s._fwd_out(N, True)
-    out_t = s._fwd_out(T, True)
-    steps = max(1, args.steps)
-    clocks = ClockSampler(dev)
-    clocks.begin()
-    timed("pack", lambda: s.pack(*lens), steps)
-    timed("full_attn", lambda: M.attn_full(cfg, s.meta, F["q"], F["k"], F["v"], out_f[1]), steps)
-    timed("full_fwd", lambda: s.full_fwd(F["q"], F["k"], F["v"], F["u"], gam, bet, out=out_f), steps)
-    timed("target_attn", lambda: M.attn_target(cfg, s.meta, Tg["q"], Tg["k"], Tg["v"], out_t[1]), steps)
-    timed("target_fwd", lambda: s.target_fwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, out=out_t), steps)
-    if args.workload == "train":
-        yf, af, sf = s.full_fwd(F["q"], F["k"], F["v"], F["u"], gam, bet)
-        yt, at, st_ = s.target_fwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet)
-        timed("full_bwd", lambda: s.full_bwd(F["q"], F["k"], F["v"], F["u"], gam, bet, af, sf, F["dy"]), steps)
-        timed("target_bwd", lambda: s.target_bwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, at, st_, Tg["dy"]), steps)
-    clk = clocks.stop()
-    M.pack_check(s.meta)
-    peaks, src = load_peaks()
-    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    ff, ft = attn_flops(b, heads, False), attn_flops(b, heads, True)
-    tf = lambda fl, ms: fl / (ms * 1e-3) / 1e12
-    layers = {
-        "full_attn": {"ms": res["full_attn"], "tflops": tf(ff, res["full_attn"]),
-                      "frac_tensor_peak": tf(ff, res["full_attn"]) / peak_tf},
-        "full_fwd": {"ms": res["full_fwd"], "tflops": tf(ff, res["full_fwd"]),
-                     "users_per_s": b.B / (res["full_fwd"] * 1e-3)},
-        "target_attn": {"ms": res["target_attn"], "tflops": tf(ft, res["target_attn"]),
-                        "gbs": target_attn_bytes(b, heads) / (res["target_attn"] * 1e-3) / 1e9,
-                        "frac_tensor_peak": tf(ft, res["target_attn"]) / peak_tf},
-        "target_fwd": {"ms": res["target_fwd"], "tflops": tf(ft, res["target_fwd"]),
-                       "users_per_s": b.B / (res["target_fwd"] * 1e-3)},
-        "pack": {"ms": res["pack"]},
-    }
-    layers["target_attn"]["frac_hbm"] = layers["target_attn"]["gbs"] / hbm
-    if args.workload == "train":
-        for k, fl in (("full_bwd", ff), ("target_bwd", ft)):
-            layers[k] = {"ms": res[k], "tflops": tf(2.5 * fl, res[k]),
-                         "users_per_s": b.B / (res[k] * 1e-3)}
-    total_ms = res["pack"] + res["full_fwd"] + res["target_fwd"] + res.get("full_bwd", 0) + res.get("target_bwd", 0)
-    total_fl = ff + ft + (2.5 * (ff + ft) if args.workload == "train" else 0.0)
-    out = {"metric": METRIC, "value": round(total_fl / (total_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-           "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(total_ms, 5),
-           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": name, "users": b.B, "total_tokens": N, "total_t": T,
-                      "flops_fwd_full": ff, "flops_fwd_target": ft,
-                      "peak": f"{src} bf16 {peak_tf} TF/s, HBM {hbm} GB/s"},
-           "per_kernel": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
-                          for k, v in layers.items()},
-           "clocks": clk}
-    print(json.dumps(out), flush=True)
+    return cfg, s, lens
 
 
-def run_stack(args):
-    """The 16-layer backbone stack (4 x (Full, Target, Target, Target)) forward on --users
-    users (default 64) of the production-shape distributions, d_model 512, Hq 8 / Hkv 2,
-    head_dim 64; seeded device-side weights N(0, 0.02), output projections N(0, 0.005),
-    X ~ N(0, 1) rounded to bf16.  One JSON line: the stack's time, users/s, and the
-    unmasked attention FLOP plus projection GEMM FLOP rates, with per-layer timings."""
+def sweep_entry(dev, N, v2, steps, warmup, repeats, heads=syn.PAIR_HEADS):
+    """Sequence-length sweep point: 2^21 tokens of users of N tokens each (H:R:T ~ 70:15:15; V2:
+    targets of 4 sub-tokens).  A step is the pair step's path at this shape: pack, Full attention
+    + gate, Target attention + gate.  Activations are seeded device-side N(0, 1) bf16 (GBs, far
+    larger than L2)."""
     import torch
     import hybrid_masked_attention_b200 as M
-    dev = torch.device("cuda", 0)
-    heads, d = syn.Heads(*(int(x) for x in args.heads.split(","))), args.dmodel
-    B = args.users if args.users is not None else 64
-    b = syn.pair_batch(B, seed=1002)
-    cfg = M.Config(b.B, b.total_tokens, b.total_r, b.total_t, heads.hq, heads.hkv, heads.dh, 1)
-    meta = M.alloc_meta(cfg, dev)
-    it = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a, dtype=dt)).to(dev)
-    M.pack(cfg, it(b.L_H, np.int32), it(b.L_R, np.int32), it(b.L_T, np.int32), it(b.r_ts, np.int64),
-           it(b.t_exp, np.int64), meta)
-    M.pack_check(meta)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(1002)
-    rnd = lambda std, *shape: (std * torch.randn(*shape, generator=gen, device=dev)).to(torch.bfloat16)
-    N, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
+    b = syn.sweep_batch(N, v2=v2, seed=1003)
+    cfg, s, lens = _packed(M, b, heads, dev)
+    rnd = _dev_inputs(dev, 1003)
+    Nt, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
+    gam, bet = torch.ones(3, D, device=dev), torch.zeros(3, D, device=dev)
+    F = dict(q=rnd(1, Nt, D), k=rnd(1, Nt, Dkv), v=rnd(1, Nt, Dkv), u=rnd(1, Nt, D))
+    Tg = dict(q=rnd(1, T, D), k=rnd(1, Nt, Dkv), v=rnd(1, Nt, Dkv), u=rnd(1, T, D))
+    out_f, out_t = s._fwd_out(Nt, True), s._fwd_out(T, True)
+
+    def step(mark):
+        s.pack(*lens)
+        if mark: mark("full_attn", 0)
+        M.attn_full(cfg, s.meta, F["q"], F["k"], F["v"], out_f[1])
+        if mark: mark("full_attn", 1)
+        M.gate_fwd(cfg, s.meta, False, out_f[1], F["u"], gam, bet, out_f[0], out_f[2])
+        if mark: mark("target_attn", 0)
+        M.attn_target(cfg, s.meta, Tg["q"], Tg["k"], Tg["v"], out_t[1])
+        if mark: mark("target_attn", 1)
+        M.gate_fwd(cfg, s.meta, True, out_t[1], Tg["u"], gam, bet, out_t[0], out_t[2])
+
+    gs = GraphStep(dev, step, ["full_attn", "target_attn"])
+    per_step, kern, clocks = gs.timed(steps, warmup, repeats, ClockSampler(dev))
+    M.pack_check(s.meta)
+    peaks, src = load_peaks()
+    peak_s = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ff, ft = attn_flops(b, heads, False), attn_flops(b, heads, True)
+    ms = statistics.median(per_step)
+    tf = lambda fl, t: fl / (t * 1e-3) / 1e12
+    tgt_gbs = target_attn_bytes(b, heads) / (kern["target_attn"] * 1e-3) / 1e9
+    tgt_ai = ft / target_attn_bytes(b, heads)
+    ridge = peak_s * 1e12 / (hbm * 1e9)
+    return {
+        "workload": f"sweep N={N}{' V2' if v2 else ''}: {b.B} users x {N} tokens "
+                    f"(L_H {int(b.L_H[0])}, L_R {int(b.L_R[0])}, L_T {int(b.L_T[0])}); Hq {heads.hq} / "
+                    f"Hkv {heads.hkv}, head_dim {heads.dh}",
+        "value": round(tf(ff + ft, ms), 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+        "step_ms": _spread(per_step), "steps": steps, "users_per_s": round(b.B / (ms * 1e-3), 1),
+        "total_tokens": Nt, "total_t": T,
+        "kernels_in_graph_ms": {k: round(v, 5) for k, v in kern.items()},
+        "roofline": {"kernel": "Full-layer attention (attn_fwd_tc_kernel)", "bound": "tensor",
+                     "achieved": round(tf(ff, kern["full_attn"]), 2), "peak": peak_s, "unit": "TFLOP/s",
+                     "frac": round(tf(ff, kern["full_attn"]) / peak_s, 4),
+                     "peak_source": f"{src} bf16 dense (sustained: the step runs for milliseconds)"},
+        "target_roofline": {"kernel": "Target-layer attention call (accumulator clear + attn_fwd_tgt_kernel)",
+                            "bound": "hbm" if tgt_ai < ridge else "tensor",
+                            "achieved_gbs": round(tgt_gbs, 1), "frac_hbm": round(tgt_gbs / hbm, 4),
+                            "achieved_tflops": round(tf(ft, kern["target_attn"]), 2),
+                            "frac_tensor": round(tf(ft, kern["target_attn"]) / peak_s, 4),
+                            "flop_per_byte": round(tgt_ai, 1), "ridge_flop_per_byte": round(ridge, 1)},
+        "clocks": clocks, "l2": "inputs of GBs, far larger than the 126 MB L2",
+    }
+
+
+def train_entry(dev, users, steps, warmup, repeats, heads=syn.PAIR_HEADS):
+    """Training step at the production-shape distributions: pack, forward and backward (dQ, dK,
+    dV, dU, dgamma, dbeta) of one Full and one Target layer; dY ~ N(0, 1) bf16."""
+    import torch
+    import hybrid_masked_attention_b200 as M
+    b = syn.pair_batch(users, seed=1005)
+    cfg, s, lens = _packed(M, b, heads, dev)
+    rnd = _dev_inputs(dev, 1005)
+    Nt, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
+    gam, bet = torch.ones(3, D, device=dev), torch.zeros(3, D, device=dev)
+    F = dict(q=rnd(1, Nt, D), k=rnd(1, Nt, Dkv), v=rnd(1, Nt, Dkv), u=rnd(1, Nt, D), dy=rnd(1, Nt, D))
+    Tg = dict(q=rnd(1, T, D), k=rnd(1, Nt, Dkv), v=rnd(1, Nt, Dkv), u=rnd(1, T, D), dy=rnd(1, T, D))
+    out_f, out_t = s._fwd_out(Nt, True), s._fwd_out(T, True)
+    s.workspace(False), s.workspace(True)
+    gf = s.full_bwd(F["q"], F["k"], F["v"], F["u"], gam, bet, out_f[1], out_f[2], F["dy"])
+    gt = s.target_bwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, out_t[1], out_t[2], Tg["dy"])
+    order = ("dq", "dk", "dv", "du", "dgamma", "dbeta")
+
+    def step(mark):
+        s.pack(*lens)
+        if mark: mark("full_fwd", 0)
+        s.full_fwd(F["q"], F["k"], F["v"], F["u"], gam, bet, out=out_f)
+        if mark: mark("full_fwd", 1)
+        s.target_fwd(Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, out=out_t)
+        if mark: mark("full_bwd", 0)
+        M.attn_full_bwd(cfg, s.meta, F["q"], F["k"], F["v"], F["u"], gam, bet, out_f[1], out_f[2], F["dy"],
+                        *[gf[k] for k in order], s.workspace(False))
+        if mark: mark("full_bwd", 1)
+        if mark: mark("target_bwd", 0)
+        M.attn_target_bwd(cfg, s.meta, Tg["q"], Tg["k"], Tg["v"], Tg["u"], gam, bet, out_t[1], out_t[2],
+                          Tg["dy"], *[gt[k] for k in order], s.workspace(True))
+        if mark: mark("target_bwd", 1)
+
+    gs = GraphStep(dev, step, ["full_fwd", "full_bwd", "target_bwd"])
+    per_step, kern, clocks = gs.timed(steps, warmup, repeats, ClockSampler(dev))
+    M.pack_check(s.meta)
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    ff, ft = attn_flops(b, heads, False), attn_flops(b, heads, True)
+    ms = statistics.median(per_step)
+    tf = lambda fl, t: fl / (t * 1e-3) / 1e12
+    return {
+        "workload": f"training step: {b.B} users, production-shape lengths; fwd + bwd of one Full and one "
+                    f"Target layer; Hq {heads.hq} / Hkv {heads.hkv}, head_dim {heads.dh}",
+        "value": round(tf(3.5 * (ff + ft), ms), 3), "unit": "TFLOP/s",
+        "flop_convention": "forward unmasked FLOPs x 3.5 (backward counted as 2.5x forward)",
+        "ms_per_step": round(ms, 5), "step_ms": _spread(per_step), "steps": steps,
+        "users_per_s": round(b.B / (ms * 1e-3), 1), "total_tokens": Nt, "total_t": T,
+        "kernels_in_graph_ms": {k: round(v, 5) for k, v in kern.items()},
+        "roofline": {"kernel": "Full-layer backward call (gate backward + attn_bwd_tc_kernel)", "bound": "tensor",
+                     "achieved": round(tf(2.5 * ff, kern["full_bwd"]), 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(tf(2.5 * ff, kern["full_bwd"]) / peak, 4),
+                     "peak_source": f"{src} bf16 dense (burst)"},
+        "clocks": clocks, "l2": f"step working set {(Nt * (4 * D + 2 * Dkv) * 2 + Nt * D * 12) / 1e6:.0f} MB > 126 MB L2",
+    }
+
+
+def stack_entry(dev, users, steps, warmup, repeats, heads=syn.PAIR_HEADS, d=512):
+    """The 16-layer backbone stack (4 x (Full, Target, Target, Target)) forward: seeded
+    device-side weights N(0, 0.02), output projections N(0, 0.02 / sqrt(16)), X ~ N(0, 1);
+    the whole mtfm_stack_fwd call replayed as one CUDA graph per step."""
+    import torch
+    import hybrid_masked_attention_b200 as M
+    b = syn.pair_batch(users, seed=1002)
+    cfg, s, lens = _packed(M, b, heads, dev)
+    rnd = _dev_inputs(dev, 1002)
+    Nt, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
     kinds = syn.STACK_KINDS
     layers = []
     for k in kinds:
         w_in = rnd(0.02, 2 * D + 2 * Dkv, d) if k == "F" else rnd(0.02, 2 * D, d)
         w_kv = rnd(0.02, 2 * Dkv, d) if k == "T" else None
-        layers.append(M.LayerWeights(k, torch.ones(d, device=dev), w_in, w_kv,
-                                     rnd(0.02 / np.sqrt(len(kinds)), d, D),
+        layers.append(M.LayerWeights(k, torch.ones(d, device=dev), w_in, w_kv, rnd(0.02 / np.sqrt(len(kinds)), d, D),
                                      torch.ones(3, D, device=dev), torch.zeros(3, D, device=dev)))
-    x = rnd(1.0, N, d).float()
+    x = rnd(1.0, Nt, d).float()
     ws = torch.empty(M.stack_workspace_bytes(cfg, d), dtype=torch.uint8, device=dev)
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    res = {}
 
-    def timed(label, fn, steps):
-        for _ in range(max(3, args.warmup)):
-            fn()
-        torch.cuda.synchronize()
-        a, z = ev(), ev()
-        a.record()
-        for _ in range(steps):
-            fn()
-        z.record()
-        torch.cuda.synchronize()
-        res[label] = a.elapsed_time(z) / steps
+    def step(mark):
+        s.pack(*lens)
+        if mark: mark("stack", 0)
+        M.stack_fwd(cfg, s.meta, d, layers, x, ws)
+        if mark: mark("stack", 1)
 
-    def timed_graph(label, fn, steps):
-        # the whole call captured once as a CUDA graph and replayed `steps` times
-        side = torch.cuda.Stream(dev)
-        with torch.cuda.stream(side):
-            for _ in range(max(3, args.warmup)):
-                fn(side)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=side):
-            fn(side)
-        with torch.cuda.stream(side):
-            for _ in range(3):
-                g.replay()
-            torch.cuda.synchronize()
-            a, z = ev(), ev()
-            a.record(side)
-            for _ in range(steps):
-                g.replay()
-            z.record(side)
-        torch.cuda.synchronize()
-        res[label] = a.elapsed_time(z) / steps
-
-    steps = max(1, args.steps)
-    clocks = ClockSampler(dev)
-    clocks.begin()
-    timed_graph("stack", lambda st: M.stack_fwd(cfg, meta, d, layers, x, ws, st), steps)
-    clk = clocks.stop()
-    timed("stack_eager", lambda: M.stack_fwd(cfg, meta, d, layers, x, ws), steps)
-    timed("full_layer", lambda: M.layer_fwd(cfg, meta, d, layers[0], x, ws), steps)
-    timed("target_layer", lambda: M.layer_fwd(cfg, meta, d, layers[1], x, ws), steps)
-    q, kk, vv = rnd(1.0, N, D), rnd(1.0, N, Dkv), rnd(1.0, N, Dkv)
-    a_buf = torch.empty(N, D, device=dev)
-    timed("full_attn", lambda: M.attn_full(cfg, meta, q, kk, vv, a_buf), steps)
-    timed("target_attn", lambda: M.attn_target(cfg, meta, q[:T], kk, vv, a_buf[:T]), steps)
-    M.pack_check(meta)
+    gs = GraphStep(dev, step, ["stack"])
+    per_step, kern, clocks = gs.timed(steps, warmup, repeats, ClockSampler(dev))
+    M.pack_check(s.meta)
     assert torch.isfinite(x).all().item()
     peaks, src = load_peaks()
-    peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_s = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     ff, ft = attn_flops(b, heads, False), attn_flops(b, heads, True)
-    g_full = 2.0 * N * d * (2 * D + 2 * Dkv) + 2.0 * N * D * d
-    g_tgt = 2.0 * T * d * 2 * D + 2.0 * N * d * 2 * Dkv + 2.0 * T * D * d
+    g_full = 2.0 * Nt * d * (2 * D + 2 * Dkv) + 2.0 * Nt * D * d
+    g_tgt = 2.0 * T * d * 2 * D + 2.0 * Nt * d * 2 * Dkv + 2.0 * T * D * d
     n_f = sum(k == "F" for k in kinds)
     n_t = len(kinds) - n_f
-    attn_fl = n_f * ff + n_t * ft
-    gemm_fl = n_f * g_full + n_t * g_tgt
-    tf = lambda fl, ms: fl / (ms * 1e-3) / 1e12
-    ms = res["stack"]
-    out = {"metric": METRIC, "value": round(tf(attn_fl + gemm_fl, ms), 3), "unit": "TFLOP/s",
-           "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
-           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": f"16-layer backbone stack, 4 x (Full, Target, Target, Target): {b.B} users, "
-                                  f"production-shape lengths, d_model {d}, Hq {heads.hq} / Hkv {heads.hkv}, "
-                                  f"head_dim {heads.dh}",
-                      "users": b.B, "total_tokens": N, "total_t": T, "attn_flops": attn_fl,
-                      "gemm_flops": gemm_fl,
-                      "l2": "per-layer working set (X fp32 + scratch) larger than the 126 MB L2",
-                      "launch": "the stack call captured once as a CUDA graph and replayed per step",
-                      "peak": f"{src} bf16 sustained {peak_tf} TF/s"},
-           "users_per_s": round(b.B / (ms * 1e-3), 1),
-           "ms_per_step_eager": round(res["stack_eager"], 5),
-           "per_layer_users_per_s": round(b.B * len(kinds) / (ms * 1e-3), 1),
-           "per_kernel": {
-               "full_layer": {"ms": round(res["full_layer"], 5),
-                              "tflops": round(tf(ff + g_full, res["full_layer"]), 2)},
-               "target_layer": {"ms": round(res["target_layer"], 5),
-                                "tflops": round(tf(ft + g_tgt, res["target_layer"]), 2)},
-               "full_attn": {"ms": round(res["full_attn"], 5), "tflops": round(tf(ff, res["full_attn"]), 2)},
-               "target_attn": {"ms": round(res["target_attn"], 5), "tflops": round(tf(ft, res["target_attn"]), 2)},
-               "full_gemm_and_rest_ms": round(res["full_layer"] - res["full_attn"], 5),
-               "target_gemm_and_rest_ms": round(res["target_layer"] - res["target_attn"], 5)},
-           "clocks": clk}
+    fl = n_f * (ff + g_full) + n_t * (ft + g_tgt)
+    ms = statistics.median(per_step)
+    tf = lambda f, t: f / (t * 1e-3) / 1e12
+    return {
+        "workload": f"16-layer backbone stack, 4 x (Full, Target, Target, Target): {b.B} users, production-shape "
+                    f"lengths, d_model {d}, Hq {heads.hq} / Hkv {heads.hkv}, head_dim {heads.dh}",
+        "value": round(tf(fl, ms), 3), "unit": "TFLOP/s",
+        "flop_convention": "unmasked attention FLOPs + projection GEMM FLOPs",
+        "ms_per_step": round(ms, 5), "step_ms": _spread(per_step), "steps": steps,
+        "users_per_s": round(b.B / (ms * 1e-3), 1), "per_layer_users_per_s": round(b.B * len(kinds) / (ms * 1e-3), 1),
+        "total_tokens": Nt, "total_t": T, "attn_flops": n_f * ff + n_t * ft, "gemm_flops": n_f * g_full + n_t * g_tgt,
+        "kernels_in_graph_ms": {k: round(v, 5) for k, v in kern.items()},
+        "roofline": {"kernel": "whole stack call (RMSNorm, tcgen05 GEMMs, attention, gates)", "bound": "tensor",
+                     "achieved": round(tf(fl, kern["stack"]), 2), "peak": peak_s, "unit": "TFLOP/s",
+                     "frac": round(tf(fl, kern["stack"]) / peak_s, 4),
+                     "peak_source": f"{src} bf16 dense (sustained)"},
+        "clocks": clocks, "l2": "per-layer working set (X fp32 + scratch) larger than the 126 MB L2",
+    }
+
+
+PER_CONFIG = (
+    ("sweep_n8192", lambda dev, a: sweep_entry(dev, 8192, False, max(2, a.config_steps // 4), a.warmup, 3)),
+    ("sweep_n512", lambda dev, a: sweep_entry(dev, 512, False, a.config_steps, a.warmup, 3)),
+    ("sweep_v2_n2048", lambda dev, a: sweep_entry(dev, 2048, True, max(2, a.config_steps // 2), a.warmup, 3)),
+    ("stack_b64", lambda dev, a: stack_entry(dev, 64, a.config_steps, a.warmup, 5)),
+    ("train_b96", lambda dev, a: train_entry(dev, 96, a.config_steps, a.warmup, 5)),
+    ("train_b160", lambda dev, a: train_entry(dev, 160, a.config_steps, a.warmup, 5)),
+)
+
+
+def run_workload(args):
+    """--workload sweep|train|stack: one JSON line for that configuration alone."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    heads = syn.Heads(*(int(x) for x in args.heads.split(",")))
+    steps = max(1, args.steps)
+    if args.workload == "sweep":
+        e = sweep_entry(dev, args.seqlen, args.v2, steps, args.warmup, args.repeats, heads)
+    elif args.workload == "train":
+        e = train_entry(dev, args.users or 96, steps, args.warmup, args.repeats, heads)
+    else:
+        e = stack_entry(dev, args.users or 64, steps, args.warmup, args.repeats, heads, args.dmodel)
+    out = {"metric": METRIC, "value": e.pop("value"), "unit": e.pop("unit"), "n_gpus": 1, "steps": steps,
+           "warmup": max(3, args.warmup), "ms_per_step": e.pop("ms_per_step"), "higher_is_better": True,
+           "dtype": "bf16", "data": "synthetic", "config": {"workload": e.pop("workload")}, **e}
     print(json.dumps(out), flush=True)
 
 
@@ -899,7 +972,7 @@ def run_infer(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["mtfm", "reference"], default="mtfm")
     ap.add_argument("--users", type=int, default=None,
@@ -914,6 +987,12 @@ def main():
     ap.add_argument("--dmodel", type=int, default=512, help="stack: d_model")
     ap.add_argument("--heads", default="8,2,64",
                     help="stack/sweep/train: Hq,Hkv,head_dim (e.g. 3,1,256 with --dmodel 768)")
+    ap.add_argument("--repeats", type=int, default=10,
+                    help="the K-step timed region is run this many times; value is the median region")
+    ap.add_argument("--config-steps", type=int, default=8,
+                    help="steps per timed region of each per_config entry")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other configurations' entries of the JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -924,17 +1003,14 @@ def main():
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
 
-    if args.workload == "stack":
-        run_stack(args)
-        return
     if args.workload == "infer":
         run_infer(args)
         return
+    if args.workload != "pair":
+        run_workload(args)
+        return
     if args.users is None:
         args.users = 32
-    if args.workload != "pair":
-        run_extra(args)
-        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:
@@ -950,6 +1026,13 @@ def main():
     try:
         res, b, heads = run_mtfm(args, rank, world, local_rank)
         if rank == 0:
+            if world == 1 and not args.no_per_config:
+                # the other configurations, each on this GPU (one process, no collective)
+                dev = torch.device("cuda", local_rank)
+                res["per_config"] = {}
+                for name, fn in PER_CONFIG:
+                    res["per_config"][name] = fn(dev, args)
+                    torch.cuda.empty_cache()
             if world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(b, heads)
             print(json.dumps(res), flush=True)
