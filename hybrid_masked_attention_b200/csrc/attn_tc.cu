@@ -65,7 +65,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
 static_assert(kBN == kKeyBlock, "key blocks of the work lists");
-static_assert(kBM * (4 * kDH + 4) * 4 <= 4 * kQBytes + 2 * kStages * kKVBytes, "O staging fits in the Q + K/V buffers");
+static_assert(kBM * 4 * kDH * 4 <= 4 * kQBytes + 2 * kStages * kKVBytes, "O staging fits in the Q + K/V buffers");
 static_assert(kSiluWG == kWGPerBuf && kChunksPerWG >= 1, "all warpgroups share every step");
 
 struct TcArgs {
@@ -103,7 +103,7 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, TcArgs p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a, TcArgs p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q, bar_o, bar_drain;
   __shared__ __align__(8) uint64_t bar_kv_full[kStages], bar_kv_empty[kStages];
@@ -162,6 +162,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_a);
   }
   __syncthreads();
   tc_fence_after();
@@ -376,14 +377,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
               *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
                   make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      // O / N_u goes through shared memory (the Q and K/V buffers are idle once every
-      // MMA of the unit is done) so that each warp then writes whole rows of A:
-      // coalesced 512-byte stores instead of 16-byte pieces
-      // of 32 different rows.  The named barrier is reached by all 16 SiLU warps,
-      // also after an abort, so it cannot hang.
+      // O / N_u goes through shared memory (the Q and K/V buffers are idle once every MMA
+      // of the unit is done), as 2R boxes of 128 rows x 32 fp32 columns in the layout of
+      // the A tensor map (16-byte chunks XOR-swizzled by row).  A tile whose 128 rows all
+      // belong to its user then goes out as 2R TMA stores issued by one thread: the SiLU
+      // warps only wait until the TMA engine has read the staging tile, not for the
+      // global writes.  A tile that ends past its user's last row is stored row by row
+      // from the staging tile (valid rows only).  The named barrier is reached by all 16
+      // SiLU warps, also after an abort, so it cannot hang.
       const bool have = ok && total > 0;
-      float* stage = reinterpret_cast<float*>(smem);
-      constexpr int kStageLd = R * kDH + 4;  // padded row: conflict-free float4 access
+      uint8_t* stage = smem;
+      constexpr uint32_t kBox = kBM * 128;  // one 32-column box of the tile
       if (have) {
         tc_fence_after();
         const float inv_n = 1.f / (float)N;
@@ -393,25 +397,37 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             uint32_t raw[32];
             tmem_ld32(lane_base + hh * kDH + c * 32, raw);
             tmem_ld_wait();
-            float4* dst = reinterpret_cast<float4*>(stage + row * kStageLd + hh * kDH + c * 32);
+            uint8_t* rowp = stage + (hh * 2 + c) * kBox + row * 128;
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
-                                   __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
+              *reinterpret_cast<float4*>(rowp + ((e ^ (row & 7)) << 4)) =
+                  make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
+                              __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
           }
         }
+        fence_proxy_async();  // the staged tile is read by the TMA engine
       }
       asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
       if (have) {
-        const uint64_t keep_a = l2_evict_last();
-        const int sw = warp - 4;  // rows [8 sw, 8 sw + 8) of the tile
+        const uint64_t keep_a = l2_evict_last();  // the gate reads A next: keep it in L2
+        if (q0 + kBM <= nq) {
+          if (threadIdx.x == 128) {
+            for (int b = 0; b < 2 * R; ++b)
+              tma_store_2d_hint(&tm_a, sQ + b * kBox, g * R * kDH + b * 32, qrow0 + q0, keep_a);
+            bulk_commit();
+            bulk_wait_read<0>();  // the next unit's loads may overwrite the staging area
+          }
+        } else {
+          const int sw = warp - 4;  // rows [8 sw, 8 sw + 8) of the tile
 #pragma unroll 1
-        for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
-          if (q0 + rr >= nq) break;
-          float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
-          const float4* src = reinterpret_cast<const float4*>(stage + rr * kStageLd);
-          for (int f = lane; f < R * kDH / 4; f += 32) {
-            st_f4_hint(dst + f, src[f], keep_a);  // the gate reads A next: keep it in L2
+          for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
+            if (q0 + rr >= nq) break;
+            float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
+            for (int f = lane; f < R * kDH / 4; f += 32) {
+              const float4 v =
+                  *reinterpret_cast<const float4*>(stage + (f / 8) * kBox + rr * 128 + (((f % 8) ^ (rr & 7)) << 4));
+              st_f4_hint(dst + f, v, keep_a);
+            }
           }
         }
       }
@@ -425,6 +441,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     ++unit_iter;
   }
   pdl_trigger();
+  if (threadIdx.x == 128) bulk_wait<0>();  // every TMA store has completed before the CTA leaves
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -452,14 +469,14 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
 // the (work unit, KV group) pairs, whose count the kernel reads from the metadata.
 template <int R>
 cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const TcArgs& a, int max_items, cudaStream_t st) {
+                      const CUtensorMap& ma, const TcArgs& a, int max_items, cudaStream_t st) {
   const size_t smem = tc_smem_bytes<R>();
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   grid = std::min(grid, max_items * a.hkv);
-  return launch_pdl(attn_fwd_tc_kernel<R>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, a);
+  return launch_pdl(attn_fwd_tc_kernel<R>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, a);
 }
 
 }  // namespace
@@ -474,15 +491,26 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
                                const __nv_bfloat16* v, float* a, cudaStream_t st) {
   if (s.target) return cudaErrorInvalidValue;  // the Target layer has its own kernel (attn_tgt.cu)
   if (max_items <= 0 || rows_q <= 0 || total_tokens <= 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, ma;
   if (!make_map(&mq, q, rows_q, s.hq * kDH, kBM) || !make_map(&mk, k, total_tokens, s.hkv * kDH, kBN) ||
       !make_map(&mv, v, total_tokens, s.hkv * kDH, kBN))
     return cudaErrorInvalidValue;
+  {  // A [rows_q, hq * 64] fp32 in boxes of 32 columns x 128 rows (128-byte swizzle)
+    EncodeTiledFn fn = encode_fn();
+    cuuint64_t dims[2] = {(cuuint64_t)s.hq * kDH, (cuuint64_t)rows_q};
+    cuuint64_t strides[1] = {(cuuint64_t)s.hq * kDH * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)kBM};
+    cuuint32_t estr[2] = {1, 1};
+    if (!fn || fn(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   TcArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha};
   const int r = s.hq / s.hkv;
-  if (r == 1) return tc_launch<1>(mq, mk, mv, args, max_items, st);
-  if (r == 2) return tc_launch<2>(mq, mk, mv, args, max_items, st);
-  return tc_launch<4>(mq, mk, mv, args, max_items, st);
+  if (r == 1) return tc_launch<1>(mq, mk, mv, ma, args, max_items, st);
+  if (r == 2) return tc_launch<2>(mq, mk, mv, ma, args, max_items, st);
+  return tc_launch<4>(mq, mk, mv, ma, args, max_items, st);
 }
 
 }  // namespace mtfm
