@@ -266,3 +266,49 @@ def stack_weights(heads: Heads, d_model: int, seed: int, kinds=STACK_KINDS, std:
 def stack_input(batch: JaggedBatch, d_model: int, seed: int) -> np.ndarray:
     """Token matrix X0 [sum N, d_model] ~ N(0, 1), bf16 bit patterns."""
     return normal_bf16(seed, S_X0, (batch.total_tokens, d_model))
+
+
+# ----------------------------------------------------------------------------
+# V2 Target Scale-Up layer (Meituan tech blog §3.3.2): per-sub-token query-side
+# projections and SwiGLU FFNs.
+# ----------------------------------------------------------------------------
+
+S_WUQ4, S_WG4, S_WU4, S_WD4, S_RMS2 = 30, 31, 32, 33, 34
+
+
+@dataclass
+class V2LayerWeights:
+    """Weights of one V2 Target layer: bf16 bit patterns [out, in]; norms float32."""
+    rms_w: np.ndarray              # [d_model] pre-norm of the attention block
+    w_uq: list                     # 4 x [2*dq, d_model]: U then Q rows, one per sub-token position
+    w_kv: np.ndarray               # [2*dkv, d_model]
+    w_o: np.ndarray                # [d_model, dq]
+    gamma: np.ndarray              # [3, dq]
+    beta: np.ndarray               # [3, dq]
+    rms_w2: np.ndarray             # [d_model] pre-norm of the FFN
+    w_gate: list                   # 4 x [d_ff, d_model]
+    w_up: list                     # 4 x [d_ff, d_model]
+    w_down: list                   # 4 x [d_model, d_ff]
+
+
+def v2_layer_weights(heads: Heads, d_model: int, d_ff: int, seed: int, std: float = 0.02,
+                     std_o: float = 0.02, std_ffn: float = 0.02, random_norms: bool = True) -> V2LayerWeights:
+    dq, dkv = heads.dq, heads.dkv
+    w_uq = [normal_bf16(seed * 10 + s, S_WUQ4, (2 * dq, d_model), std) for s in range(4)]
+    w_kv = normal_bf16(seed, S_WKV, (2 * dkv, d_model), std)
+    w_o = normal_bf16(seed, S_WO, (d_model, dq), std_o)
+    w_gate = [normal_bf16(seed * 10 + s, S_WG4, (d_ff, d_model), std_ffn) for s in range(4)]
+    w_up = [normal_bf16(seed * 10 + s, S_WU4, (d_ff, d_model), std_ffn) for s in range(4)]
+    w_down = [normal_bf16(seed * 10 + s, S_WD4, (d_model, d_ff), std_ffn) for s in range(4)]
+    if random_norms:
+        g = rng_for(seed, S_RMS2)
+        rms_w = (1.0 + 0.25 * g.standard_normal(d_model)).astype(np.float32)
+        rms_w2 = (1.0 + 0.25 * g.standard_normal(d_model)).astype(np.float32)
+        gamma = (1.0 + 0.25 * g.standard_normal((3, dq))).astype(np.float32)
+        beta = (0.25 * g.standard_normal((3, dq))).astype(np.float32)
+    else:
+        rms_w = np.ones(d_model, np.float32)
+        rms_w2 = np.ones(d_model, np.float32)
+        gamma = np.ones((3, dq), np.float32)
+        beta = np.zeros((3, dq), np.float32)
+    return V2LayerWeights(rms_w, w_uq, w_kv, w_o, gamma, beta, rms_w2, w_gate, w_up, w_down)

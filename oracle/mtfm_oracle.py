@@ -467,3 +467,78 @@ def stack_fwd(batch, heads, weights, X0, alpha=None, record: bool = False):
         X = (full_layer if lw.kind == "F" else target_layer)(batch, heads, X, lw, alpha)
         xs.append(X)
     return xs if record else X
+
+
+# ----------------------------------------------------------------------------
+# V2 Target Scale-Up layer (Meituan tech blog §3.3.2, items 2-4): every target is
+# 4 sub-tokens; in a Target-Attention layer each sub-token position has its own
+# query-side projection and its own SwiGLU FFN, and the sub-tokens of a target are
+# crossed by a zero-parameter token mixing.
+# ----------------------------------------------------------------------------
+
+V2_SUB = 4
+
+
+def v2_sub_index(batch) -> np.ndarray:
+    """Sub-token position (0..3) of every T row, in the Target layout order: the
+    position of the row among its user's T rows, modulo 4 (each target is 4
+    consecutive T rows, item 1 of §3.3.2)."""
+    out = []
+    for u, LH, LR, LT, s0, _, _ in _users(batch):
+        out.append(np.arange(LT) % V2_SUB)
+    return np.concatenate(out) if out else np.zeros(0, np.int64)
+
+
+def mix_tokens(Xt, n_sub: int = V2_SUB):
+    """Zero-parameter token mixing of the sub-tokens of each target (§3.3.2 item 4,
+    the mixing of RankMixer): every sub-token vector is cut into n_sub equal parts,
+    and new sub-token h is the concatenation of part h of sub-tokens 0, 1, ...,
+    n_sub - 1 of the same target.  Xt: [n_targets * n_sub, d], targets consecutive."""
+    Xt = np.asarray(Xt, dtype=np.float64)
+    n, d = Xt.shape
+    assert n % n_sub == 0 and d % n_sub == 0
+    parts = Xt.reshape(n // n_sub, n_sub, n_sub, d // n_sub)   # [target, sub-token j, part h, :]
+    return parts.transpose(0, 2, 1, 3).reshape(n, d)           # [target, new sub-token h, j, :]
+
+
+def swiglu(X, w_gate, w_up, w_down):
+    """SwiGLU feed-forward network: (SiLU(X W_gate^T) * (X W_up^T)) W_down^T."""
+    return (silu(X @ w_gate.T) * (X @ w_up.T)) @ w_down.T
+
+
+def v2_target_layer(batch, heads, X, lw, alpha=None):
+    """Target-Attention layer of the V2 Target Scale-Up (§3.3.2), on a batch whose
+    targets are 4 sub-tokens (v2_subtokens = 4).  Readings taken where the page is
+    brief: the attention block is the V1 Target layer (§4.2 of the dingyadong.top
+    page) except that sub-token position s projects its [U Q] with its own matrix
+    w_uq[s] (item 2: "different Q projection"; U comes from the same query-side
+    projection); K, V come from the shared w_kv over all rows; the output
+    projection w_o is shared.  Then the 4 sub-tokens of each target are mixed
+    (item 4), and each sub-token position s applies its own pre-normed SwiGLU FFN
+    with a residual (item 2):
+        X_T <- X_T + f2(GLN(A_T) (*) U_T)              (attention, per-s U, Q)
+        X_T <- Mix(X_T)                                (per target)
+        X_T <- X_T + SwiGLU_s(RMSNorm(X_T) * rms_w2)   (per sub-token position s)
+    H / R rows pass through unchanged.  lw: syn.V2LayerWeights."""
+    assert batch.v2_subtokens == V2_SUB
+    dq, dkv = heads.dq, heads.dkv
+    Xn = rmsnorm(X, lw.rms_w)
+    trow = t_row_index(batch)
+    sub = v2_sub_index(batch)
+    ZT = np.zeros((len(trow), 2 * dq))
+    for s in range(V2_SUB):
+        sel = sub == s
+        ZT[sel] = silu(Xn[trow[sel]] @ _f64(lw.w_uq[s]).T)
+    Zkv = silu(Xn @ _f64(lw.w_kv).T)
+    inp = _Proj(ZT[:, dq:], Zkv[:, :dkv], Zkv[:, dkv:], ZT[:, :dq], _f64(lw.gamma), _f64(lw.beta))
+    out = target_fwd(batch, heads, inp, alpha)
+    XT = _f64(X)[trow] + out["Y"] @ _f64(lw.w_o).T
+    XT = mix_tokens(XT)
+    Xn2 = rmsnorm(XT, lw.rms_w2)
+    F = np.zeros_like(XT)
+    for s in range(V2_SUB):
+        sel = sub == s
+        F[sel] = swiglu(Xn2[sel], _f64(lw.w_gate[s]), _f64(lw.w_up[s]), _f64(lw.w_down[s]))
+    Xo = np.array(X, dtype=np.float64, copy=True)
+    Xo[trow] = XT + F
+    return Xo

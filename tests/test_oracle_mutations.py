@@ -8,6 +8,7 @@ import pytest
 
 import oracle_pins as P
 import stack_pins as S
+import v2_pins as V
 from oracle import mtfm_oracle as O
 
 
@@ -159,6 +160,60 @@ def _t_rows_shifted(batch):
     return O.t_row_index.__wrapped__(batch) - 1
 
 
+def _v2_sub_by_target(batch):
+    return (np.arange(batch.total_t) // 4) % 4
+
+
+def _mix_interleaved(Xt, n_sub=O.V2_SUB):
+    n, d = Xt.shape
+    parts = np.asarray(Xt, np.float64).reshape(n // n_sub, n_sub, d // n_sub, n_sub)  # strided parts
+    return parts.transpose(0, 3, 1, 2).reshape(n, d)
+
+
+def _swiglu_gate_up_swapped(X, w_gate, w_up, w_down):
+    return (O.silu(X @ w_up.T) * (X @ w_gate.T)) @ w_down.T
+
+
+def _v2_variant(ffn_residual=True, ffn_per_sub=True, ffn_norm=True):
+    def layer(batch, heads, X, lw, alpha=None):
+        lw2 = syn_copy(lw)
+        if not ffn_per_sub:
+            lw2.w_gate, lw2.w_up, lw2.w_down = [lw.w_gate[0]] * 4, [lw.w_up[0]] * 4, [lw.w_down[0]] * 4
+        if not ffn_norm:
+            lw2.rms_w2 = None
+        Xo = O.v2_target_layer.__wrapped__(batch, heads, X, lw2, alpha) if ffn_norm else _v2_no_norm(batch, heads, X, lw2)
+        if not ffn_residual:
+            trow = O.t_row_index(batch)
+            Xo[trow] = Xo[trow] - _mixed_attn(batch, heads, X, lw2)[trow]
+        return Xo
+    return layer
+
+
+def syn_copy(lw):
+    import copy
+    return copy.copy(lw)
+
+
+def _mixed_attn(batch, heads, X, lw):
+    lw0 = syn_copy(lw)
+    lw0.w_down = [np.zeros_like(x) for x in lw.w_down]
+    return O.v2_target_layer.__wrapped__(batch, heads, X, lw0)
+
+
+def _v2_no_norm(batch, heads, X, lw):
+    orig = O.rmsnorm
+    calls = []
+
+    def rms(Xa, w, eps=O.RMS_EPS):
+        calls.append(1)
+        return orig(Xa, w, eps) if len(calls) == 1 else np.asarray(Xa, np.float64)
+    O.rmsnorm = rms
+    try:
+        return O.v2_target_layer.__wrapped__(batch, heads, X, lw)
+    finally:
+        O.rmsnorm = orig
+
+
 MUTATIONS = {
     "t_rows_do_not_see_self": ("dense_mask_fast", _mask_no_self_t),
     "tie_visible": ("dense_mask_fast", _mask_fast_ties_visible),
@@ -184,6 +239,13 @@ MUTATIONS = {
     "target_kv_from_t_rows": ("target_layer", _target_layer_kv_from_t_rows),
     "target_updates_hr_rows": ("target_layer", _target_layer_updates_all_rows),
     "t_rows_shifted": ("t_row_index", _t_rows_shifted),
+    "v2_sub_by_target_index": ("v2_sub_index", _v2_sub_by_target),
+    "v2_mix_identity": ("mix_tokens", lambda Xt, n_sub=4: np.asarray(Xt, np.float64)),
+    "v2_mix_strided_parts": ("mix_tokens", _mix_interleaved),
+    "v2_swiglu_gate_up_swapped": ("swiglu", _swiglu_gate_up_swapped),
+    "v2_ffn_residual_dropped": ("v2_target_layer", _v2_variant(ffn_residual=False)),
+    "v2_ffn_shared_weights": ("v2_target_layer", _v2_variant(ffn_per_sub=False)),
+    "v2_ffn_prenorm_dropped": ("v2_target_layer", _v2_variant(ffn_norm=False)),
 }
 
 
@@ -199,7 +261,7 @@ def test_pins_catch_mutation(name, monkeypatch):
     fn.__wrapped__ = orig
     monkeypatch.setattr(O, attr, fn)
     caught = []
-    for check in P.ALL_CHECKS + S.STACK_CHECKS:
+    for check in P.ALL_CHECKS + S.STACK_CHECKS + V.V2_CHECKS:
         try:
             check()
         except AssertionError:
