@@ -851,6 +851,55 @@ def stack_entry(dev, users, steps, warmup, repeats, heads=syn.PAIR_HEADS, d=512)
     }
 
 
+def v2_layer_entry(dev, users, seqlen, steps, warmup, repeats, heads=syn.PAIR_HEADS, d=512, dff=1024):
+    """One V2 Target Scale-Up layer (per-sub-token [U Q] projections and SwiGLU FFNs, mixing of
+    each target's 4 sub-tokens; Meituan tech blog §3.3.2) on users of seqlen tokens with V2
+    targets (H:R:T ~ 70:15:15); seeded device-side weights, X ~ N(0, 1)."""
+    import torch
+    import hybrid_masked_attention_b200 as M
+    b = syn.sweep_batch(seqlen, v2=True, B=users, seed=1016)
+    cfg, s, lens = _packed(M, b, heads, dev)
+    rnd = _dev_inputs(dev, 1016)
+    Nt, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
+    ones, zeros = lambda *sh: torch.ones(*sh, device=dev), lambda *sh: torch.zeros(*sh, device=dev)
+    w = M.V2LayerWeights(ones(d), [rnd(0.02, 2 * D, d) for _ in range(4)], rnd(0.02, 2 * Dkv, d), rnd(0.02, d, D),
+                         ones(3, D), zeros(3, D), ones(d), [rnd(0.02, dff, d) for _ in range(4)],
+                         [rnd(0.02, dff, d) for _ in range(4)], [rnd(0.02, d, dff) for _ in range(4)])
+    x = rnd(1.0, Nt, d).float()
+    ws = torch.empty(M.v2_workspace_bytes(cfg, d, dff), dtype=torch.uint8, device=dev)
+
+    def step(mark):
+        s.pack(*lens)
+        if mark: mark("v2_layer", 0)
+        M.v2_target_layer_fwd(cfg, s.meta, d, dff, w, x, ws)
+        if mark: mark("v2_layer", 1)
+
+    gs = GraphStep(dev, step, ["v2_layer"])
+    per_step, kern, clocks = gs.timed(steps, warmup, repeats, ClockSampler(dev))
+    M.pack_check(s.meta)
+    peaks, src = load_peaks()
+    peak_s = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ft = attn_flops(b, heads, True)
+    gemm = 2.0 * Nt * d * 2 * Dkv + 2.0 * T * d * 2 * D + 2.0 * T * D * d + 2.0 * T * d * 2 * dff + 2.0 * T * dff * d
+    ms = statistics.median(per_step)
+    tf = lambda f, t: f / (t * 1e-3) / 1e12
+    return {
+        "workload": f"V2 Target Scale-Up layer: {b.B} users x {seqlen} tokens, {T // 4} targets of 4 sub-tokens; "
+                    f"d_model {d}, d_ff {dff}, Hq {heads.hq} / Hkv {heads.hkv}, head_dim {heads.dh}",
+        "value": round(tf(ft + gemm, ms), 3), "unit": "TFLOP/s",
+        "flop_convention": "unmasked attention FLOPs + projection / FFN GEMM FLOPs",
+        "ms_per_step": round(ms, 5), "step_ms": _spread(per_step), "steps": steps,
+        "users_per_s": round(b.B / (ms * 1e-3), 1), "targets_per_s": round(T / 4 / (ms * 1e-3), 1),
+        "total_tokens": Nt, "total_t": T, "attn_flops": ft, "gemm_flops": gemm,
+        "kernels_in_graph_ms": {k: round(v, 5) for k, v in kern.items()},
+        "roofline": {"kernel": "whole V2 layer call (RMSNorm, tcgen05 GEMMs, Target attention, gate, mixing)",
+                     "bound": "tensor", "achieved": round(tf(ft + gemm, kern["v2_layer"]), 2), "peak": peak_s,
+                     "unit": "TFLOP/s", "frac": round(tf(ft + gemm, kern["v2_layer"]) / peak_s, 4),
+                     "peak_source": f"{src} bf16 dense (sustained)"},
+        "clocks": clocks,
+    }
+
+
 PER_CONFIG = (
     ("sweep_n8192", lambda dev, a: sweep_entry(dev, 8192, False, max(2, a.config_steps // 4), a.warmup, 3)),
     ("sweep_n512", lambda dev, a: sweep_entry(dev, 512, False, a.config_steps, a.warmup, 3)),
@@ -858,6 +907,7 @@ PER_CONFIG = (
     ("stack_b64", lambda dev, a: stack_entry(dev, 64, a.config_steps, a.warmup, 5)),
     ("train_b96", lambda dev, a: train_entry(dev, 96, a.config_steps, a.warmup, 5)),
     ("train_b160", lambda dev, a: train_entry(dev, 160, a.config_steps, a.warmup, 5)),
+    ("v2_layer_n2048", lambda dev, a: v2_layer_entry(dev, 64, 2048, a.config_steps, a.warmup, 5)),
 )
 
 
@@ -872,6 +922,8 @@ def run_workload(args):
         e = sweep_entry(dev, args.seqlen, args.v2, steps, args.warmup, args.repeats, heads)
     elif args.workload == "train":
         e = train_entry(dev, args.users or 96, steps, args.warmup, args.repeats, heads)
+    elif args.workload == "v2layer":
+        e = v2_layer_entry(dev, args.users or 64, args.seqlen, steps, args.warmup, args.repeats, heads, args.dmodel)
     else:
         e = stack_entry(dev, args.users or 64, steps, args.warmup, args.repeats, heads, args.dmodel)
     out = {"metric": METRIC, "value": e.pop("value"), "unit": e.pop("unit"), "n_gpus": 1, "steps": steps,
@@ -980,7 +1032,7 @@ def main():
     ap.add_argument("--sets", type=int, default=4, help="resident input copies rotated across steps")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["pair", "sweep", "train", "stack", "infer"], default="pair",
+    ap.add_argument("--workload", choices=["pair", "sweep", "train", "stack", "infer", "v2layer"], default="pair",
                     help="pair: the headline step; sweep/train/stack/infer: timings of the other configs")
     ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
     ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")

@@ -10,7 +10,8 @@ Function names mirror the C entry points:
     attn_full_fwd, attn_target_fwd, attn_full, attn_target, gate_fwd,
     attn_target_cached_fwd, attn_target_cached,
     bwd_workspace_bytes, attn_full_bwd, attn_target_bwd, attn_target_bwd_static,
-    stack_workspace_bytes, layer_fwd, stack_fwd, selftest_wait_timeout
+    stack_workspace_bytes, layer_fwd, stack_fwd, v2_workspace_bytes, v2_target_layer_fwd,
+    selftest_wait_timeout
 """
 from __future__ import annotations
 
@@ -92,9 +93,17 @@ class CLayerWeights(ctypes.Structure):
                 ("w_o", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
 
 
+class CV2LayerWeights(ctypes.Structure):
+    _fields_ = [("rms_w", ctypes.c_void_p), ("w_uq", ctypes.c_void_p * 4), ("w_kv", ctypes.c_void_p),
+                ("w_o", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("rms_w2", ctypes.c_void_p), ("w_gate", ctypes.c_void_p * 4), ("w_up", ctypes.c_void_p * 4),
+                ("w_down", ctypes.c_void_p * 4)]
+
+
 _P = ctypes.c_void_p
 _CP = ctypes.POINTER(CCfg)
 _LWP = ctypes.POINTER(CLayerWeights)
+_V2P = ctypes.POINTER(CV2LayerWeights)
 _sigs = {
     "mtfm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mtfm_meta_bytes": (ctypes.c_size_t, [_CP]),
@@ -114,6 +123,9 @@ _sigs = {
     "mtfm_attn_target_bwd": (ctypes.c_int, [_CP] + [_P] * 17 + [ctypes.c_size_t, _P]),
     "mtfm_attn_target_bwd_static": (ctypes.c_int, [_CP] + [_P] * 17),
     "mtfm_selftest_wait_timeout": (ctypes.c_int, [_P, ctypes.c_int64, _P]),
+    "mtfm_v2_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int32, ctypes.c_int32]),
+    "mtfm_v2_target_layer_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int32, _V2P, _P, _P,
+                                                ctypes.c_size_t, _P]),
     "mtfm_stack_workspace_bytes": (ctypes.c_size_t, [_CP, ctypes.c_int32]),
     "mtfm_layer_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int, _LWP, _P, _P, ctypes.c_size_t, _P]),
     "mtfm_stack_fwd": (ctypes.c_int, [_CP, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_char_p, _LWP, _P, _P,
@@ -431,6 +443,58 @@ def stack_fwd(cfg: Config, meta: torch.Tensor, d_model: int, layers, x: torch.Te
                                _ptr(x, torch.float32, (cfg.total_tokens, d_model), "x"),
                                _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream)),
            "mtfm_stack_fwd")
+
+
+# ---------------------------------------------------------------------------- V2 Target layer
+
+@dataclass
+class V2LayerWeights:
+    """Device tensors of one V2 Target Scale-Up layer (``mtfm_v2_layer_weights``).
+
+    rms_w, rms_w2 fp32 [d_model]; w_uq: 4 bf16 [2*D, d_model] (U rows, then Q rows), one per
+    sub-token position; w_kv bf16 [2*Dkv, d_model]; w_o bf16 [d_model, D]; gamma, beta fp32
+    [3, D] or None; w_gate, w_up: 4 bf16 [d_ff, d_model]; w_down: 4 bf16 [d_model, d_ff].
+    """
+    rms_w: torch.Tensor
+    w_uq: list
+    w_kv: torch.Tensor
+    w_o: torch.Tensor
+    gamma: Optional[torch.Tensor]
+    beta: Optional[torch.Tensor]
+    rms_w2: torch.Tensor
+    w_gate: list
+    w_up: list
+    w_down: list
+
+
+def v2_workspace_bytes(cfg: Config, d_model: int, d_ff: int) -> int:
+    c = cfg.c()
+    n = _lib.mtfm_v2_workspace_bytes(ctypes.byref(c), int(d_model), int(d_ff))
+    if n == 0:
+        raise MtfmError(3, "mtfm_v2_workspace_bytes")
+    return n
+
+
+def v2_target_layer_fwd(cfg: Config, meta: torch.Tensor, d_model: int, d_ff: int, w: V2LayerWeights,
+                        x: torch.Tensor, ws: torch.Tensor, stream=None):
+    """One V2 Target Scale-Up layer on X (fp32 [total_tokens, d_model], updated in place)."""
+    D, Dkv = cfg.D, cfg.Dkv
+    bf, f32 = torch.bfloat16, torch.float32
+    if len(w.w_uq) != 4 or len(w.w_gate) != 4 or len(w.w_up) != 4 or len(w.w_down) != 4:
+        raise ValueError("w_uq, w_gate, w_up, w_down need one tensor per sub-token position (4)")
+    four = lambda ts, shape, name: (ctypes.c_void_p * 4)(*[_ptr(t, bf, shape, f"{name}[{k}]") for k, t in enumerate(ts)])
+    lw = CV2LayerWeights(
+        _ptr(w.rms_w, f32, (d_model,), "rms_w"), four(w.w_uq, (2 * D, d_model), "w_uq"),
+        _ptr(w.w_kv, bf, (2 * Dkv, d_model), "w_kv"), _ptr(w.w_o, bf, (d_model, D), "w_o"),
+        _ptr(w.gamma, f32, (3, D), "gamma"), _ptr(w.beta, f32, (3, D), "beta"),
+        _ptr(w.rms_w2, f32, (d_model,), "rms_w2"), four(w.w_gate, (d_ff, d_model), "w_gate"),
+        four(w.w_up, (d_ff, d_model), "w_up"), four(w.w_down, (d_model, d_ff), "w_down"))
+    c = cfg.c()
+    _check(_lib.mtfm_v2_target_layer_fwd(ctypes.byref(c), _ptr(meta, torch.uint8, name="meta"), int(d_model),
+                                         int(d_ff), ctypes.byref(lw),
+                                         _ptr(x, f32, (cfg.total_tokens, d_model), "x"),
+                                         _ptr(ws, torch.uint8, name="ws"), ws.numel(), _stream(stream)),
+           "mtfm_v2_target_layer_fwd")
 
 
 def selftest_wait_timeout(meta: torch.Tensor, limit_cycles: int = 2_000_000, stream=None):

@@ -352,6 +352,108 @@ mtfm_status stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int d, int n_laye
   return MTFM_OK;
 }
 
+// ------------------------------------------------------------------ V2 Target layer
+// Scratch: the stack's layer scratch, then the FFN's pre-normed input X~2_T (bf16
+// [T, d]) and hidden layer H (bf16 [T, d_ff]).
+struct V2Ws {
+  StackWs base;
+  size_t xn2, hid, total;
+};
+V2Ws v2_ws(const Resolved& r, int d, int dff) {
+  V2Ws w;
+  w.base = stack_ws(r, d);
+  const size_t T = (size_t)r.total_t;
+  size_t o = w.base.total;
+  w.xn2 = o; o = align256(o + T * d * 2);
+  w.hid = o; o = align256(o + T * dff * 2);
+  w.total = o;
+  return w;
+}
+
+mtfm_status check_v2(const Resolved& r, int d, int dff) {
+  mtfm_status s = check_stack_cfg(r, d);
+  if (s != MTFM_OK) return s;
+  if (r.v2 != 4) return MTFM_ERR_INVALID_ARG;
+  if (dff <= 0 || dff % 64 != 0) return MTFM_ERR_INVALID_ARG;
+  if (r.total_t % 4 != 0) return MTFM_ERR_INVALID_ARG;
+  return MTFM_OK;
+}
+
+mtfm_status v2_layer_fwd(const mtfm_cfg* cfg, const void* d_meta, int d, int dff, const mtfm_v2_layer_weights* w,
+                         float* x, void* d_ws, size_t ws_bytes, void* stream) {
+  Resolved r;
+  mtfm_status s = resolve(cfg, &r);
+  if (s != MTFM_OK) return s;
+  if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
+  if ((s = check_v2(r, d, dff)) != MTFM_OK) return s;
+  if (!w || !w->rms_w || !w->w_kv || !w->w_o || !w->rms_w2) return MTFM_ERR_INVALID_ARG;
+  if ((w->gamma == nullptr) != (w->beta == nullptr)) return MTFM_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->rms_w, w->w_kv, w->w_o, w->rms_w2};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return MTFM_ERR_INVALID_ARG;
+  if (w->gamma && (!aligned16(w->gamma) || !aligned16(w->beta))) return MTFM_ERR_INVALID_ARG;
+  for (int k = 0; k < 4; ++k)
+    if (!w->w_uq[k] || !w->w_gate[k] || !w->w_up[k] || !w->w_down[k] || !aligned16(w->w_uq[k]) ||
+        !aligned16(w->w_gate[k]) || !aligned16(w->w_up[k]) || !aligned16(w->w_down[k]))
+      return MTFM_ERR_INVALID_ARG;
+  if (r.total_tokens == 0 || r.total_t == 0) return MTFM_OK;  // no target: X unchanged
+  if (!x || !aligned16(x)) return MTFM_ERR_INVALID_ARG;
+  if (!d_ws || (reinterpret_cast<uintptr_t>(d_ws) & 255u)) return MTFM_ERR_INVALID_ARG;
+  const V2Ws V = v2_ws(r, d, dff);
+  const StackWs& W = V.base;
+  if (ws_bytes < V.total) return MTFM_ERR_WORKSPACE_TOO_SMALL;
+  const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
+  const MetaView m = meta_view(const_cast<void*>(d_meta), L);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(d_ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  auto wt = [](const uint16_t* q) { return reinterpret_cast<const __nv_bfloat16*>(q); };
+  const int N = r.total_tokens, T = r.total_t, D = r.D, Dkv = r.Dkv, T4 = T / 4;
+  cudaError_t e;
+  // attention block: X~ on all rows (K, V) and on the T rows (the sub-tokens' [U Q])
+  if ((e = launch_rmsnorm(m.hdr, x, N, d, nullptr, w->rms_w, kRmsEps, bf(W.xn), st)) != cudaSuccess) return MTFM_ERR_CUDA;
+  if ((e = launch_rmsnorm(m.hdr, x, T, d, m.t_rows, w->rms_w, kRmsEps, bf(W.xnt), st)) != cudaSuccess)
+    return MTFM_ERR_CUDA;
+  GemmEpi gkv{kEpiSiluSplit, 2, {0, Dkv, 2 * Dkv, 0, 0}, {bf(W.k), bf(W.v), nullptr, nullptr}, {Dkv, Dkv, 0, 0},
+              nullptr, 0, nullptr, 0, nullptr};
+  if ((e = launch_gemm_tc(m.hdr, bf(W.xn), d, wt(w->w_kv), N, 2 * Dkv, d, gkv, st)) != cudaSuccess)
+    return MTFM_ERR_CUDA;
+  // sub-token position s of every target is T row 4 i + s (L_T is a multiple of 4 per user,
+  // so targets start at multiples of 4): strided operands select the rows of one position
+  for (int k = 0; k < 4; ++k) {
+    GemmEpi guq{kEpiSiluSplit, 2, {0, D, 2 * D, 0, 0}, {bf(W.u) + (size_t)k * D, bf(W.q) + (size_t)k * D, nullptr, nullptr},
+                {4 * D, 4 * D, 0, 0}, nullptr, 0, nullptr, 0, nullptr};
+    if ((e = launch_gemm_tc(m.hdr, bf(W.xnt) + (size_t)k * d, 4 * d, wt(w->w_uq[k]), T4, 2 * D, d, guq, st)) !=
+        cudaSuccess)
+      return MTFM_ERR_CUDA;
+  }
+  float* a = reinterpret_cast<float*>(ws + W.a);
+  if ((e = launch_attn(r, m, L, true, bf(W.q), bf(W.k), bf(W.v), a, st)) != cudaSuccess) return MTFM_ERR_CUDA;
+  if ((e = launch_gate_fwd_bf16(m, true, T, D, r.eps, a, bf(W.u), w->gamma, w->beta, bf(W.y),
+                                reinterpret_cast<float*>(ws + W.stats), st)) != cudaSuccess)
+    return MTFM_ERR_CUDA;
+  GemmEpi go{kEpiResidual, 0, {0, 0, 0, 0, 0}, {nullptr, nullptr, nullptr, nullptr}, {0, 0, 0, 0}, x, d, m.t_rows,
+             1, nullptr};
+  if ((e = launch_gemm_tc(m.hdr, bf(W.y), D, wt(w->w_o), T, d, D, go, st)) != cudaSuccess) return MTFM_ERR_CUDA;
+  // mixing of each target's sub-tokens (in place on X), then the FFN's pre-norm
+  if ((e = launch_mix_rmsnorm(m.hdr, x, T4, d, m.t_rows, w->rms_w2, kRmsEps, bf(V.xn2), st)) != cudaSuccess)
+    return MTFM_ERR_CUDA;
+  // per-sub-token SwiGLU FFN with the residual
+  for (int k = 0; k < 4; ++k) {
+    GemmEpi gup{kEpiSwiGLU, 1, {0, 2 * dff, 0, 0, 0}, {bf(V.hid) + (size_t)k * dff, nullptr, nullptr, nullptr},
+                {4 * dff, 0, 0, 0}, nullptr, 0, nullptr, 0, wt(w->w_up[k])};
+    if ((e = launch_gemm_tc(m.hdr, bf(V.xn2) + (size_t)k * d, 4 * d, wt(w->w_gate[k]), T4, 2 * dff, d, gup, st)) !=
+        cudaSuccess)
+      return MTFM_ERR_CUDA;
+    GemmEpi gdn{kEpiResidual, 0, {0, 0, 0, 0, 0}, {nullptr, nullptr, nullptr, nullptr}, {0, 0, 0, 0}, x, d,
+                m.t_rows + k, 4, nullptr};
+    if ((e = launch_gemm_tc(m.hdr, bf(V.hid) + (size_t)k * dff, 4 * dff, wt(w->w_down[k]), T4, d, dff, gdn, st)) !=
+        cudaSuccess)
+      return MTFM_ERR_CUDA;
+  }
+  return MTFM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -552,6 +654,18 @@ mtfm_status mtfm_stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_mo
                            const char* kinds, const mtfm_layer_weights* layers, float* d_x, void* d_ws,
                            size_t ws_bytes, void* stream) {
   return stack_fwd(cfg, d_meta, d_model, n_layers, kinds, layers, d_x, d_ws, ws_bytes, stream);
+}
+
+size_t mtfm_v2_workspace_bytes(const mtfm_cfg* cfg, int32_t d_model, int32_t d_ff) {
+  Resolved r;
+  if (resolve(cfg, &r) != MTFM_OK || check_v2(r, d_model, d_ff) != MTFM_OK) return 0;
+  return v2_ws(r, d_model, d_ff).total;
+}
+
+mtfm_status mtfm_v2_target_layer_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_model, int32_t d_ff,
+                                     const mtfm_v2_layer_weights* weights, float* d_x, void* d_ws, size_t ws_bytes,
+                                     void* stream) {
+  return v2_layer_fwd(cfg, d_meta, d_model, d_ff, weights, d_x, d_ws, ws_bytes, stream);
 }
 
 mtfm_status mtfm_selftest_wait_timeout(void* d_meta, int64_t limit_cycles, void* stream) {

@@ -6,7 +6,11 @@
 //     projection f1 / f_uq / f_kv and activation phi_1 of page "美团推荐大模型
 //     MTFM 深度硬核解析" §4.1, §4.2), or
 //   * the residual X <- X + C (the output projection f2 and the shortcut of
-//     §4.1; for a Target layer the rows are scattered back to the T rows, §4.2).
+//     §4.1; for a Target layer the rows are scattered back to the T rows, §4.2), or
+//   * the SwiGLU hidden layer SiLU(A Bg^T) * (A Bu^T) of the per-sub-token FFN of the
+//     V2 Target layer (Meituan tech blog §3.3.2 item 2): each tile's B rows are BN/2
+//     rows of the gate matrix and the same BN/2 rows of the up matrix, so the gate
+//     and up accumulators of a hidden unit sit in the same TMEM lane.
 //
 // Persistent CTAs (one per SM) stride over 128 x BN output tiles, BN in
 // {64, 128, 256}.  Warp 0 issues the TMA loads of A and B through a 4-stage
@@ -97,7 +101,7 @@ __device__ __forceinline__ void epi_silu_split(const GemmEpi& e, int row, int co
 }
 
 __device__ __forceinline__ void epi_residual(const GemmEpi& e, int row, int col, const uint32_t (&raw)[32]) {
-  const int xr = e.row_map ? e.row_map[row] : row;
+  const int xr = e.row_map ? e.row_map[(size_t)row * (e.row_map_stride > 0 ? e.row_map_stride : 1)] : row;
   float4* p = reinterpret_cast<float4*>(e.x + (size_t)xr * e.ldx + col);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -118,6 +122,7 @@ __device__ __forceinline__ void epi_residual(const GemmEpi& e, int row, int col,
 template <int BN, bool TMA_EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const __grid_constant__ CUtensorMap tm_b2,
                const __grid_constant__ CUtensorMap tm_o0, const __grid_constant__ CUtensorMap tm_o1,
                const __grid_constant__ CUtensorMap tm_o2, const __grid_constant__ CUtensorMap tm_o3, GemmArgs p) {
   constexpr int kStages = n_stages<TMA_EPI>();
@@ -188,7 +193,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
           }
           mbar_expect_tx(b_full(s), kStage);
           tma_load_2d(sbase + s * kStage, &tm_a, b_full(s), kb * kBK, m0);
-          tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0);
+          if (p.epi.kind == kEpiSwiGLU) {  // gate rows, then the same rows of the up matrix
+            tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0 / 2);
+            tma_load_2d(sbase + s * kStage + kABytes + (BN / 2) * 128, &tm_b2, b_full(s), kb * kBK, n0 / 2);
+          } else {
+            tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0);
+          }
           ++G;
         }
       }
@@ -264,7 +274,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
       const int row = m0 + r_in;
       const int col0 = (t % nN) * BN + half * kHalf;
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * BN + half * kHalf);
-      if (!TMA_EPI) {
+      if (!TMA_EPI && p.epi.kind == kEpiSwiGLU) {
+        // warpgroup `half` takes hidden units [half BN/4, (half + 1) BN/4) of the tile: gate
+        // accumulators at tile columns [half BN/4, ...), up at [BN/2 + half BN/4, ...)
+        constexpr int kHid = BN / 4;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * BN + half * kHid);
+        const int h0 = (t % nN) * (BN / 2) + half * kHid;  // first hidden unit of this thread's columns
+#pragma unroll 1
+        for (int c = 0; c < kHid / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tl + c * 32, g);
+          tmem_ld32(tl + BN / 2 + c * 32, u);
+          tmem_ld_wait();
+          if (row < p.M) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[i] = pack_bf16x2(silu_fast(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]),
+                                      silu_fast(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(p.epi.seg_ptr[0] + (size_t)row * p.epi.seg_ld[0] + h0 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
+        }
+      } else if (!TMA_EPI) {
 #pragma unroll 1
         for (int c = 0; c < kChunks; ++c) {
           uint32_t raw[32];
@@ -360,22 +394,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
 }
 
 template <int BN, bool TMA_EPI>
-cudaError_t gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap (&mo)[4], const GemmArgs& args,
-                        int n_tiles, cudaStream_t st) {
+cudaError_t gemm_launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+                        const CUtensorMap (&mo)[4], const GemmArgs& args, int n_tiles, cudaStream_t st) {
   const size_t smem = gemm_smem_bytes<BN, TMA_EPI>();
   cudaError_t e =
       cudaFuncSetAttribute(gemm_tc_kernel<BN, TMA_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = std::min(n_tiles, sm_count());
-  return launch_pdl(gemm_tc_kernel<BN, TMA_EPI>, dim3(grid), dim3(kThreads), smem, st, ma, mb, mo[0], mo[1], mo[2],
-                    mo[3], args);
+  return launch_pdl(gemm_tc_kernel<BN, TMA_EPI>, dim3(grid), dim3(kThreads), smem, st, ma, mb, mb2, mo[0], mo[1],
+                    mo[2], mo[3], args);
 }
 
 template <int BN>
-cudaError_t gemm_dispatch(bool tma, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap (&mo)[4],
-                          const GemmArgs& args, int n_tiles, cudaStream_t st) {
-  return tma ? gemm_launch<BN, true>(ma, mb, mo, args, n_tiles, st)
-             : gemm_launch<BN, false>(ma, mb, mo, args, n_tiles, st);
+cudaError_t gemm_dispatch(bool tma, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+                          const CUtensorMap (&mo)[4], const GemmArgs& args, int n_tiles, cudaStream_t st) {
+  return tma ? gemm_launch<BN, true>(ma, mb, mb2, mo, args, n_tiles, st)
+             : gemm_launch<BN, false>(ma, mb, mb2, mo, args, n_tiles, st);
 }
 
 }  // namespace
@@ -384,15 +418,26 @@ cudaError_t launch_gemm_tc(MetaHeader* hdr, const __nv_bfloat16* a, int lda, con
                            int M, int N, int K, const GemmEpi& epi, cudaStream_t st) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   if (N % 64 != 0 || K <= 0 || K % kBK != 0 || lda % 8 != 0) return cudaErrorInvalidValue;
-  // widest tile that divides N, halved while the grid would leave SMs idle
+  const bool swiglu = epi.kind == kEpiSwiGLU;
+  if (swiglu && (N % 128 != 0 || epi.b_up == nullptr)) return cudaErrorInvalidValue;
+  // widest tile that divides N, halved while the grid would leave SMs idle (SwiGLU: >= 128,
+  // so that each epilogue warpgroup holds whole 32-column chunks of gate and up)
+  const int bn_min = swiglu ? 128 : 64;
   int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
   const int nM = (M + kBM - 1) / kBM;
-  while (bn > 64 && nM * (N / bn) < sm_count() && N % (bn / 2) == 0) bn /= 2;
-  CUtensorMap ma, mb, mo[4];
+  while (bn > bn_min && nM * (N / bn) < sm_count() && N % (bn / 2) == 0) bn /= 2;
+  CUtensorMap ma, mb, mb2, mo[4];
   memset(mo, 0, sizeof(mo));
-  if (!make_map_bf16(&ma, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, kBM, kBK) ||
-      !make_map_bf16(&mb, b, (uint64_t)N, (uint64_t)K, (uint64_t)K, (uint32_t)bn, kBK))
+  if (!make_map_bf16(&ma, a, (uint64_t)M, (uint64_t)K, (uint64_t)lda, kBM, kBK))
     return cudaErrorInvalidValue;
+  if (swiglu) {
+    if (!make_map_bf16(&mb, b, (uint64_t)(N / 2), (uint64_t)K, (uint64_t)K, (uint32_t)(bn / 2), kBK) ||
+        !make_map_bf16(&mb2, epi.b_up, (uint64_t)(N / 2), (uint64_t)K, (uint64_t)K, (uint32_t)(bn / 2), kBK))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map_bf16(&mb, b, (uint64_t)N, (uint64_t)K, (uint64_t)K, (uint32_t)bn, kBK)) return cudaErrorInvalidValue;
+    mb2 = mb;  // not read
+  }
   // TMA epilogue: 64-column bf16 boxes into contiguous segments, or fp32 boxes
   // reduced into a contiguous X (no row map); otherwise direct stores.
   bool tma = false;
@@ -404,7 +449,7 @@ cudaError_t launch_gemm_tc(MetaHeader* hdr, const __nv_bfloat16* a, int lda, con
           !make_map_bf16(&mo[sg], epi.seg_ptr[sg], (uint64_t)M, (uint64_t)w, (uint64_t)w, kBM, 64))
         tma = false;
     }
-  } else if (epi.kind == kEpiResidual && epi.row_map == nullptr && epi.ldx == N) {
+  } else if (epi.kind == kEpiResidual && epi.row_map == nullptr && epi.ldx == N) {  // (SwiGLU: direct stores)
     EncodeTiledFn fn = encode_fn();
     cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
     cuuint64_t strides[1] = {(cuuint64_t)N * 4};
@@ -416,9 +461,9 @@ cudaError_t launch_gemm_tc(MetaHeader* hdr, const __nv_bfloat16* a, int lda, con
   }
   GemmArgs args{hdr, M, N, K, epi};
   const int n_tiles = nM * (N / bn);
-  if (bn == 256) return gemm_dispatch<256>(tma, ma, mb, mo, args, n_tiles, st);
-  if (bn == 128) return gemm_dispatch<128>(tma, ma, mb, mo, args, n_tiles, st);
-  return gemm_dispatch<64>(tma, ma, mb, mo, args, n_tiles, st);
+  if (bn == 256) return gemm_dispatch<256>(tma, ma, mb, mb2, mo, args, n_tiles, st);
+  if (bn == 128) return gemm_dispatch<128>(tma, ma, mb, mb2, mo, args, n_tiles, st);
+  return gemm_dispatch<64>(tma, ma, mb, mb2, mo, args, n_tiles, st);
 }
 
 }  // namespace mtfm

@@ -275,8 +275,12 @@ cudaError_t launch_gate_fwd_bf16(const MetaView& m, bool target, int rows, int D
 //                   segments (e.g. U | Q | K | V), each its own row-major array;
 //   kEpiResidual  : X[row_map[i], :] += C[i, :] in fp32 (row_map NULL: identity).
 constexpr float kRmsEps = 1e-6f;  // RMSNorm epsilon of the pre-norm
+//   kEpiSwiGLU    : the SwiGLU hidden layer H = SiLU(A Bg^T) * (A Bu^T), bf16, into
+//                   seg_ptr[0] (row pitch seg_ld[0]); B = the gate matrix, b_up the up
+//                   matrix (both [N / 2, K]); N counts the gate and up columns together.
 constexpr int kEpiSiluSplit = 0;
 constexpr int kEpiResidual = 1;
+constexpr int kEpiSwiGLU = 2;
 struct GemmEpi {
   int kind;
   int n_seg;
@@ -285,12 +289,19 @@ struct GemmEpi {
   int seg_ld[4];
   float* x;
   int ldx;
-  const int32_t* row_map;
+  const int32_t* row_map;     // residual: X row of output row i = row_map[i * row_map_stride]
+  int row_map_stride;         // 0 reads as 1
+  const __nv_bfloat16* b_up;  // kEpiSwiGLU: the up matrix
 };
-// M >= 0; N a multiple of 64 (and of 32 at segment borders); K a multiple of 64;
-// lda a multiple of 8.  A and B 16-byte aligned.
+// M >= 0; N a multiple of 64 (and of 32 at segment borders; of 128 for kEpiSwiGLU); K a
+// multiple of 64; lda a multiple of 8.  A and B 16-byte aligned.
 cudaError_t launch_gemm_tc(MetaHeader* hdr, const __nv_bfloat16* a, int lda, const __nv_bfloat16* b,
                            int M, int N, int K, const GemmEpi& epi, cudaStream_t st);
+// V2 Target layer: the zero-parameter mixing of each target's 4 sub-tokens, in place on
+// the T rows of X (global rows t_rows[4 i + j] of target i), then out[T row] =
+// bf16(RMSNorm(mixed row) * w).  d a multiple of 16, d <= 1024.
+cudaError_t launch_mix_rmsnorm(const MetaHeader* hdr, float* x, int n_targets, int d, const int32_t* t_rows,
+                               const float* w, float eps, __nv_bfloat16* out, cudaStream_t st);
 // out[i, :] = bf16(RMSNorm(X[row_map ? row_map[i] : i, :]) * w), d a multiple of 4, d <= 1024.
 cudaError_t launch_rmsnorm(const MetaHeader* hdr, const float* x, int rows, int d,
                            const int32_t* row_map, const float* w, float eps, __nv_bfloat16* out,

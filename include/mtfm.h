@@ -321,6 +321,55 @@ mtfm_status mtfm_stack_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_mo
                            float* d_x, void* d_ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * V2 Target Scale-Up layer forward (Meituan tech blog §3.3.2: each target is 4
+ * sub-tokens, items 2-4).  Requires cfg->v2_subtokens = 4 (every user's L_T a
+ * multiple of 4; the 4 sub-tokens of a target are consecutive T rows, position
+ * s = (T row within the user) mod 4).  On X (fp32 [total_tokens, d_model],
+ * updated in place), with X~ = RMSNorm(X) * rms_w (eps 1e-6):
+ *   [U Q]_t = SiLU(X~_t W_uq[s]^T)   for each T row t at sub-token position s
+ *             (item 2: a Q projection per sub-token position; U comes from the
+ *             same query-side projection),
+ *   [K V]   = SiLU(X~ W_kv^T)        on all rows,
+ *   A       = masked SiLU attention of the Target layer with the V2 mask (the 4
+ *             sub-tokens of a target see each other and their shared prefix),
+ *   X_T    <- X_T + (GLN(A) (*) U) W_o^T,
+ *   X_T    <- Mix(X_T): per target, new sub-token h = [part h of sub-token 0 |
+ *             part h of sub-token 1 | ... | part h of sub-token 3], each part
+ *             d_model / 4 wide (item 4: the zero-parameter mixing of RankMixer),
+ *   X_T    <- X_T + SwiGLU_s(RMSNorm(X_T) * rms_w2) for each T row at position s
+ *             (item 2: a SwiGLU FFN per sub-token position):
+ *             SwiGLU_s(z) = (SiLU(z W_gate[s]^T) * (z W_up[s]^T)) W_down[s]^T.
+ * H / R rows are not touched.  The attention block's parameters are this layer's
+ * own, separate from any Full (self-attention) layer's (item 3).
+ * Weights (device pointers; the struct is host memory): rms_w, rms_w2 fp32 [d_model];
+ * w_uq[s] bf16 [2*hq*head_dim, d_model] (U rows, then Q rows); w_kv bf16
+ * [2*hkv*head_dim, d_model]; w_o bf16 [d_model, hq*head_dim]; gamma, beta fp32
+ * [3, hq*head_dim] or both NULL; w_gate[s], w_up[s] bf16 [d_ff, d_model];
+ * w_down[s] bf16 [d_model, d_ff].
+ * Shapes: d_model a multiple of 64, <= 1024; hq*head_dim a multiple of 64; d_ff a
+ * multiple of 64.  d_ws: scratch of at least mtfm_v2_workspace_bytes bytes,
+ * 256-byte aligned (0 for an unsupported configuration).  Precision as the stack:
+ * bf16 tensor-core operands, fp32 accumulation, X fp32.
+ * ------------------------------------------------------------------------- */
+typedef struct mtfm_v2_layer_weights {
+  const float* rms_w;
+  const uint16_t* w_uq[4];
+  const uint16_t* w_kv;
+  const uint16_t* w_o;
+  const float* gamma;
+  const float* beta;
+  const float* rms_w2;
+  const uint16_t* w_gate[4];
+  const uint16_t* w_up[4];
+  const uint16_t* w_down[4];
+} mtfm_v2_layer_weights;
+
+size_t mtfm_v2_workspace_bytes(const mtfm_cfg* cfg, int32_t d_model, int32_t d_ff);
+mtfm_status mtfm_v2_target_layer_fwd(const mtfm_cfg* cfg, const void* d_meta, int32_t d_model, int32_t d_ff,
+                                     const mtfm_v2_layer_weights* weights, float* d_x, void* d_ws,
+                                     size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Self-test of failure detection (no counterpart on the pages).  Launches one
  * CTA that waits, with the bounded mbarrier wait every tensor-core kernel of
  * this library uses, on a barrier nothing arrives on; after limit_cycles SM

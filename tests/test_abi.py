@@ -152,3 +152,19 @@ def test_selftest_arguments(lib):
     assert m._lib.mtfm_selftest_wait_timeout(4096 + 16, 1000, None) == 1
     assert m._lib.mtfm_selftest_wait_timeout(4096, 0, None) == 1
     assert m._lib.mtfm_selftest_wait_timeout(4096, 5_000_000_000, None) == 1
+
+
+def test_v2_layer_host_checks(lib):
+    import hybrid_masked_attention_b200 as m
+    ok = m.Config(batch=2, total_tokens=40, total_r=8, total_t=8, hq=8, hkv=2, head_dim=64, v2_subtokens=4)
+    assert lib.mtfm_v2_workspace_bytes(ctypes.byref(ok.c()), 512, 1024) > 0
+    v1 = m.Config(batch=2, total_tokens=40, total_r=8, total_t=8, hq=8, hkv=2, head_dim=64)
+    assert lib.mtfm_v2_workspace_bytes(ctypes.byref(v1.c()), 512, 1024) == 0     # needs 4 sub-tokens
+    assert lib.mtfm_v2_workspace_bytes(ctypes.byref(ok.c()), 512, 1000) == 0     # d_ff multiple of 64
+    assert lib.mtfm_v2_workspace_bytes(ctypes.byref(ok.c()), 520, 1024) == 0     # d_model multiple of 64
+    odd = m.Config(batch=2, total_tokens=40, total_r=8, total_t=6, hq=8, hkv=2, head_dim=64, v2_subtokens=4)
+    assert lib.mtfm_v2_workspace_bytes(ctypes.byref(odd.c()), 512, 1024) == 0    # T rows in targets of 4
+    # null weights: rejected before any launch
+    st = lib.mtfm_v2_target_layer_fwd(ctypes.byref(ok.c()), ctypes.c_void_p(256), 512, 1024, None, None, None,
+                                      ctypes.c_size_t(0), None)
+    assert st == 1
