@@ -55,9 +55,9 @@ mtfm_status check_meta(const void* d_meta, const Resolved& r) {
   return MTFM_OK;
 }
 
-// tcgen05/TMEM kernels where their TMEM plans fit (head_dim 64, r in {1, 2, 4}; the
-// Target layer stacks the r heads of a group as MMA rows);
-// the mma.sync kernel covers the other head shapes.  A library compiled with
+// tcgen05/TMEM kernels where their TMEM plans fit (head_dim 64, r in {1, 2, 4}: the
+// Target layer stacks the r heads of a group as MMA rows; head_dim 256: one head per
+// unit, Full and Target layers); the mma.sync kernel covers the other head shapes.  A library compiled with
 // -DMTFM_PORTABLE_KERNELS runs the mma.sync kernels for every shape (a test build
 // for comparing the two; the shipped library has no run-time switch).
 #ifdef MTFM_PORTABLE_KERNELS
@@ -75,6 +75,8 @@ cudaError_t launch_attn(const Resolved& r, const MetaView& m, const MetaLayout& 
     if (target) return launch_attn_fwd_tgt(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
     return launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
   }
+  if (!kPortableOnly && attn_fwd_tc256_supported(shape))
+    return launch_attn_fwd_tc256(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
   return launch_attn_fwd_mma(shape, m, max_items, q, k, v, a, st);
 }
 

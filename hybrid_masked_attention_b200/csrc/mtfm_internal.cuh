@@ -237,6 +237,11 @@ bool attn_fwd_tc_supported(const AttnShape& s);
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                const __nv_bfloat16* v, float* a, cudaStream_t st);
+// head_dim 256 (any hq / hkv), Full or Target layer (s.target): tcgen05, one (tile, head) per unit.
+bool attn_fwd_tc256_supported(const AttnShape& s);
+cudaError_t launch_attn_fwd_tc256(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
+                                  int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                  const __nv_bfloat16* v, float* a, cudaStream_t st);
 // Target layer, heads stacked as MMA rows (head_dim 64, hq / hkv in {1, 2, 4}).
 // With k_cand / v_cand (cached prefix): k, v hold the H and R rows of every user
 // [total_tokens - total_t, hkv * 64], k_cand, v_cand the T rows [total_t, hkv * 64].

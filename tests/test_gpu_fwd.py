@@ -15,6 +15,7 @@ CASES = [
     ("pair", "pair", True), ("pair", "pair", False),
     ("edge", "pair", True), ("edge", "dh128", True), ("edge", "r8", True),
     ("edge", "dh256", True), ("v2_n512", "dh256", True), ("tiny", "dh256", False),
+    ("pair", "dh256", True), ("v1_n2048", "dh256", False),
     ("v2_n512", "pair", True), ("v2_n1024", "pair", True), ("v1_n2048", "pair", True),
 ]
 
