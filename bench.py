@@ -278,7 +278,7 @@ def run_mtfm(args, rank, world, local_rank):
     S_t = torch.empty(b.total_t, 2, **f32)
     # graphs cannot be captured on the legacy default stream: every launch goes to `stream`
     stream = torch.cuda.Stream(dev)
-    launches_per_step = 6   # pack (2 kernels), Full attention, Full gate, Target attention, Target gate
+    launches_per_step = 7   # pack (2 kernels), Full attention, Full gate, Target clear, Target attention, Target gate
 
     def step(i, record=None, around_full=None, around_tgt=None):
         s = sets[i % len(sets)]
@@ -306,8 +306,8 @@ def run_mtfm(args, rank, world, local_rank):
         for i in range(args.warmup):
             step(i)
     torch.cuda.synchronize(dev)
-    # The timed steps replay CUDA graphs of the step's launches (the 6 kernels and the Target
-    # layer's accumulator clear): one graph runs a step on each resident input set in turn;
+    # The timed steps replay CUDA graphs of the step's launches (the 7 kernels: 2 pack, Full
+    # attention, gate, the Target layer's conditional accumulator clear, attention, gate): one graph runs a step on each resident input set in turn;
     # its instrumented twin adds two event-record nodes around every Full attention launch
     # and is replayed last, so the kernel's duration is measured inside the timed region
     # without paying for event nodes in every step.  K = nset * reps + rem steps: the last
@@ -423,8 +423,8 @@ def run_mtfm(args, rank, world, local_rank):
                            "attn_ms_in_graph": round(tgt_ms, 5),
                            "attn_tflops": round(fl_tgt / (tgt_ms * 1e-3) / 1e12, 2),
                            "attn_gbs": round(tgt_gbs, 1), "attn_hbm_frac": round(tgt_gbs / hbm, 4),
-                           "attn_timing": "event-record nodes around the Target attention call (accumulator "
-                                          "clear + kernel) inside the timed region",
+                           "attn_timing": "event-record nodes around the Target attention call (conditional "
+                                          "accumulator clear + kernel) inside the timed region",
                            "users_per_s": round(b.B / ((ms_parts["target_attn"] + ms_parts["target_gate"]) * 1e-3), 1)},
                 "ms_parts": {k: round(v, 5) for k, v in ms_parts.items()},
                 "ms_parts_note": "eager pass with an event between launches (not the graph-replayed step)",
@@ -727,7 +727,7 @@ def sweep_entry(dev, N, v2, steps, warmup, repeats, heads=syn.PAIR_HEADS):
                      "achieved": round(tf(ff, kern["full_attn"]), 2), "peak": peak_s, "unit": "TFLOP/s",
                      "frac": round(tf(ff, kern["full_attn"]) / peak_s, 4),
                      "peak_source": f"{src} bf16 dense (sustained: the step runs for milliseconds)"},
-        "target_roofline": {"kernel": "Target-layer attention call (accumulator clear + attn_fwd_tgt_kernel)",
+        "target_roofline": {"kernel": "Target-layer attention call (conditional accumulator clear + attn_fwd_tgt_kernel)",
                             "bound": "hbm" if tgt_ai < ridge else "tensor",
                             "achieved_gbs": round(tgt_gbs, 1), "frac_hbm": round(tgt_gbs / hbm, 4),
                             "achieved_tflops": round(tf(ft, kern["target_attn"]), 2),

@@ -29,10 +29,15 @@
 //                 unit), then O += P_hi V + P_lo V into one of two O buffers.
 //   warps 4..19 : SiLU warpgroups (as in the Full-layer kernel: each warpgroup
 //                 takes 32 of the 128 key columns of a step), then the unit's
-//                 epilogue: O / N_u from TMEM into a swizzled shared-memory tile
-//                 and one TMA reduce-add per 32 columns into A (fp32, zeroed
-//                 first), so chunks of the key range sum without atomics in the
-//                 kernel; rows past the user's last T row are staged as zeros.
+//                 epilogue: O / N_u from TMEM into a swizzled shared-memory tile,
+//                 then into A (fp32).  When every sub-tile's key range is one
+//                 unit (MetaHeader::tgt_single), each row of A gets exactly one
+//                 unit's O: TMA stores, or row stores of the user's rows for a
+//                 sub-tile that runs past its user's last T row.  Otherwise A is
+//                 zeroed first (tgt_zero_kernel, launched just before) and every
+//                 unit adds its partial O with one TMA reduce-add per 32 columns,
+//                 rows past the user's last T row staged as zeros, so the chunks
+//                 sum without atomics.
 // TMEM: O buffers at columns [0, 64) and [64, 128), S buffers at [128 + 128b, +128).
 // Every mbarrier wait is bounded; after a timeout the roles stop issuing work and
 // drain (bounded), the SiLU warps still pass their named barriers the same
@@ -72,6 +77,7 @@ constexpr size_t tgt_smem_bytes() { return 2 * kQBytes + 2 * kStages * kKVBytes 
 
 struct TgtArgs {
   MetaView m;
+  float* a;
   int hq, hkv, v2;
   float alpha;
   int cached;  // keys/values of the prefix from the cache, of the T rows from the candidates
@@ -142,6 +148,18 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half
   }
 }
 
+// Rows [0, rows) of a staged O tile (2R boxes of TR rows x 32 fp32, 16-byte chunks
+// XOR-swizzled by row) to A rows dst + t * ld; 16 warps, warp sw takes rows sw, sw + 16, ...
+template <int R>
+__device__ __noinline__ void store_rows(const uint8_t* stage, float* dst, int ld, int rows, int sw, int lane) {
+  constexpr int TR = 128 / R;
+  for (int tr = sw; tr < rows; tr += 16) {
+    float4* d = reinterpret_cast<float4*>(dst + (size_t)tr * ld);
+    for (int f = lane; f < R * kDH / 4; f += 32)
+      d[f] = *reinterpret_cast<const float4*>(stage + (f >> 3) * (TR * 128) + tr * 128 + (((f & 7) ^ (tr & 7)) << 4));
+  }
+}
+
 __device__ __forceinline__ void silu_bar() { asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory"); }
 
 template <int R>
@@ -170,6 +188,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int n_work = (p.cached ? hdr->n_units_target_c : hdr->n_units_target) * p.hkv;
   if ((int)blockIdx.x >= n_work) return;
   const int n_mine = (n_work - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // units of this CTA
+  const bool single = hdr->tgt_single[p.cached ? 1 : 0] != 0;
   auto unit_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -386,10 +405,10 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // Epilogue of unit e.k: O / N_u -> swizzled staging tile -> TMA reduce-add into A.
     // Each call passes the two named barriers, whatever e.ok says.
     struct Prev {
-      int k, col, y;
+      int k, col, y, rows;
       bool ok;
       float inv_n;
-    } prev{0, 0, 0, false, 0.f};
+    } prev{0, 0, 0, 0, false, 0.f};
     auto epilogue = [&](const Prev& e) {
       const int ob = e.k & 1;
       bool eok = e.ok && ok;
@@ -416,10 +435,21 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
       }
       silu_bar();
-      if (eok && issuer) {
-        for (int b = 0; b < 2 * R; ++b)
-          tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), e.col + (b >> 1) * kDH + (b & 1) * 32, e.y);
-        bulk_commit();
+      if (eok && !single) {
+        if (issuer) {
+          for (int b = 0; b < 2 * R; ++b)
+            tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), e.col + (b >> 1) * kDH + (b & 1) * 32, e.y);
+          bulk_commit();
+        }
+      } else if (eok && e.rows == TR) {
+        if (issuer) {
+          for (int b = 0; b < 2 * R; ++b)
+            tma_store_2d(&tm_a, sO + b * (TR * 128), e.col + (b >> 1) * kDH + (b & 1) * 32, e.y);
+          bulk_commit();
+        }
+      } else if (eok) {
+        // the sub-tile runs past its user's last T row: store the user's rows one by one
+        store_rows<R>(stage, p.a + (size_t)e.y * (p.hq * kDH) + e.col, p.hq * kDH, e.rows, warp - 4, lane);
       }
     };
     // Every SiLU warp walks all n_mine units, also after an abort, so that all of
@@ -495,6 +525,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       prev.inv_n = valid && U.N > 0 ? 1.f / (float)U.N : 0.f;  // rows past the user's T rows add zeros
       prev.col = U.g * R * kDH;
       prev.y = ok ? m.t_off[U.u] + U.q_sub0 : 0;
+      prev.rows = ok ? min(TR, U.LT - U.q_sub0) : 0;
     }
     if (n_mine > 0) epilogue(prev);
     if (issuer) bulk_wait<0>();  // every reduce has completed before the CTA leaves
@@ -506,6 +537,16 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && s_abort) atomicOr(&hdr->error, kErrTimeout);
+}
+
+// Zeroes A when several units of a sub-tile add into its rows (MetaHeader::tgt_single
+// unset); does nothing otherwise.  Launched just before the Target kernel.
+__global__ void __launch_bounds__(256) tgt_zero_kernel(const MetaHeader* hdr, int cached, float4* a, size_t n4) {
+  pdl_wait();
+  pdl_trigger();
+  if (hdr->error || hdr->tgt_single[cached] != 0) return;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x)
+    a[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 }  // namespace
@@ -563,9 +604,14 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaMemsetAsync(a, 0, sizeof(float) * (size_t)total_t * s.hq * kDH, st);  // units add partial sums
-  if (e != cudaSuccess) return e;
-  TgtArgs args{m, s.hq, s.hkv, s.v2, s.alpha, cached ? 1 : 0};
+  {
+    const size_t n4 = (size_t)total_t * s.hq * (kDH / 4);
+    const int zgrid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)sm_count() * 8);
+    cudaError_t e = launch_pdl(tgt_zero_kernel, dim3(zgrid), dim3(256), 0, st, (const MetaHeader*)m.hdr,
+                               cached ? 1 : 0, reinterpret_cast<float4*>(a), n4);
+    if (e != cudaSuccess) return e;
+  }
+  TgtArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha, cached ? 1 : 0};
   const size_t smem = tgt_smem_bytes();
   const int grid = sm_count();
   auto launch = [&](auto kern) -> cudaError_t {

@@ -99,7 +99,10 @@ struct MetaHeader {
   // Units of the Target layer with a cached key/value prefix (each sub-tile's key range =
   // the prefix blocks + one block of candidate rows; same chunk size)
   int32_t n_units_target_c;
-  int32_t pad[2];
+  // 1 when every sub-tile's key range fits in one chunk ([0]: the Target layer, [1]: the
+  // cached-prefix form): each row of A then gets exactly one unit's O, stored directly;
+  // otherwise the chunks' partial O are summed into A (zeroed by a kernel just before).
+  int32_t tgt_single[2];
 };
 
 // One work item: a 128-row query tile of one user and the range of prefix

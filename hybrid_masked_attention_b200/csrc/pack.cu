@@ -110,6 +110,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->n_units_target = 0;
       m.hdr->n_units_target_c = 0;
       m.hdr->sched[0] = m.hdr->sched[1] = 0;
+      m.hdr->tgt_single[0] = m.hdr->tgt_single[1] = 1;
       m.hdr->tgt_sub_rows = tgt_sub_rows;
       m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
       m.hdr->pack_done = 0;
@@ -201,6 +202,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->n_units_target = 0;
     m.hdr->n_units_target_c = 0;
     m.hdr->sched[0] = m.hdr->sched[1] = 0;
+    m.hdr->tgt_single[0] = m.hdr->tgt_single[1] = 1;
     m.hdr->tgt_sub_rows = tgt_sub_rows;
     m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
     m.hdr->pack_done = 0;
@@ -287,6 +289,15 @@ __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
     }
   }
   const int C = s_chunk;
+  // whether every item's key range fits in one chunk (the blocks of a table's items <= C)
+  __shared__ int s_multi[2];
+  if (threadIdx.x < 2) s_multi[threadIdx.x] = 0;
+  __syncthreads();
+  for (int i = a; i < b; ++i) {
+    if ((uo[i + 1] & 0xffff) > C) s_multi[0] = 1;
+    if ((m.unit_off_c[i + 1] & 0xffff) > C) s_multi[1] = 1;
+  }
+  __syncthreads();
   // sub-tiles x ceil(blocks / C) units per item, scanned in place into first-unit offsets
   auto scan_units = [&](volatile int* arr) -> long long {
     long long local = 0;
@@ -311,6 +322,8 @@ __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
     hdr->n_units_target = (int)total;
     hdr->n_units_target_c = (int)total_c;
     hdr->tgt_chunk_blocks = C;
+    hdr->tgt_single[0] = s_multi[0] ? 0 : 1;
+    hdr->tgt_single[1] = s_multi[1] ? 0 : 1;
   }
 }
 
