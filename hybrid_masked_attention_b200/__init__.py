@@ -25,11 +25,13 @@ import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmtfm.so")
+# MTFM_LIBRARY may name another build of the same library (the bounds-checked
+# libmtfm_debug_bounds.so); it changes which file is loaded, not what it runs.
+LIB_PATH = os.environ.get("MTFM_LIBRARY") or os.path.join(_PKG, "libmtfm.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"libmtfm.so not found at {LIB_PATH}; build it with "
+        f"{LIB_PATH} not found; build it with "
         "`python hybrid_masked_attention_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -38,7 +40,7 @@ MTFM_OK = 0
 STATUS_NAMES = {
     0: "MTFM_OK", 1: "MTFM_ERR_INVALID_ARG", 2: "MTFM_ERR_UNSORTED_TS", 3: "MTFM_ERR_UNSUPPORTED",
     4: "MTFM_ERR_WORKSPACE_TOO_SMALL", 5: "MTFM_ERR_CUDA", 6: "MTFM_ERR_TIMEOUT",
-    7: "MTFM_ERR_BAD_LENGTHS",
+    7: "MTFM_ERR_BAD_LENGTHS", 8: "MTFM_ERR_BOUNDS",
 }
 
 
@@ -109,6 +111,8 @@ _sigs = {
     "mtfm_meta_bytes": (ctypes.c_size_t, [_CP]),
     "mtfm_pack": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "mtfm_pack_check": (ctypes.c_int, [_P, _P]),
+    "mtfm_debug_bounds_build": (ctypes.c_int32, []),
+    "mtfm_debug_site": (ctypes.c_int, [_P, _P, _P]),
     "mtfm_meta_read": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "mtfm_max_items": (ctypes.c_int32, [_CP, ctypes.c_int]),
     "mtfm_attn_full_fwd": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -200,6 +204,19 @@ def pack(cfg: Config, lh, lr, lt, r_ts, t_exp, meta: torch.Tensor, stream=None):
 
 def pack_check(meta: torch.Tensor, stream=None):
     _check(_lib.mtfm_pack_check(_ptr(meta, torch.uint8, None, "meta"), _stream(stream)), "mtfm_pack_check")
+
+
+def debug_bounds_build() -> bool:
+    """True when the loaded library is the bounds-checked build (-DMTFM_DEBUG_BOUNDS)."""
+    return bool(_lib.mtfm_debug_bounds_build())
+
+
+def debug_site(meta: torch.Tensor, stream=None) -> int:
+    """Site (file id * 100000 + line) of the first failed check of the bounds-checked build, or 0."""
+    site = ctypes.c_int32()
+    _check(_lib.mtfm_debug_site(_ptr(meta, torch.uint8, None, "meta"), ctypes.byref(site), _stream(stream)),
+           "mtfm_debug_site")
+    return site.value
 
 
 def meta_read(cfg: Config, meta: torch.Tensor, stream=None) -> dict:

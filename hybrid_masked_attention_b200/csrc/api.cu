@@ -470,6 +470,7 @@ const char* mtfm_status_string(mtfm_status s) {
     case MTFM_ERR_CUDA: return "CUDA runtime error";
     case MTFM_ERR_TIMEOUT: return "device wait timed out";
     case MTFM_ERR_BAD_LENGTHS: return "lengths negative, inconsistent with totals, or L_T not a multiple of v2_subtokens";
+    case MTFM_ERR_BOUNDS: return "a bounds check of the bounds-checked build failed";
   }
   return "unknown status";
 }
@@ -507,8 +508,29 @@ mtfm_status mtfm_pack_check(const void* d_meta, void* stream) {
   if (h.magic != kMetaMagic) return MTFM_ERR_INVALID_ARG;
   if (h.error & kErrBadLengths) return MTFM_ERR_BAD_LENGTHS;
   if (h.error & kErrUnsorted) return MTFM_ERR_UNSORTED_TS;
+  if (h.error & kErrBounds) return MTFM_ERR_BOUNDS;
   if (h.error & kErrTimeout) return MTFM_ERR_TIMEOUT;
   if (h.error & kErrConfig) return MTFM_ERR_UNSUPPORTED;
+  return MTFM_OK;
+}
+
+int32_t mtfm_debug_bounds_build(void) {
+#ifdef MTFM_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+mtfm_status mtfm_debug_site(const void* d_meta, int32_t* site, void* stream) {
+  if (!d_meta || !site) return MTFM_ERR_INVALID_ARG;
+  MetaHeader h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, d_meta, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MTFM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MTFM_ERR_CUDA;
+  if (h.magic != kMetaMagic) return MTFM_ERR_INVALID_ARG;
+  *site = h.dbg_site;
   return MTFM_OK;
 }
 

@@ -50,6 +50,8 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kDbgFile = 4;  // site id of this file's bounds checks
+
 constexpr int kDH = 64;
 constexpr int kKB = 128;         // keys per unit (TMEM lanes)
 constexpr int kQS = 64;          // queries per step
@@ -140,7 +142,7 @@ __device__ __forceinline__ ColInfo col_info(const MetaView& m, const BwdUnit& U,
   const int t0pos = U.LH + U.LR;
   const int pos = TARGET ? t0pos + q : q;
   if (q >= 0 && pos < U.N && (!TARGET || q < U.LT)) {
-    c.kve = m.kv_end[U.so + pos];
+    c.kve = MTFM_INBOUNDS(m.hdr, U.so + pos < m.hdr->total_tokens) ? m.kv_end[U.so + pos] : 0;
     if (pos >= t0pos) {
       c.slo = t0pos + ((pos - t0pos) / v2) * v2;
       c.shi = c.slo + v2;
@@ -230,8 +232,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (T == 0) continue;
         if (nkv >= 1 && !mbar_wait(B(&bar_kve), (nkv - 1) & 1, abort_flag)) break;
         mbar_expect_tx(B(&bar_kvf), 2 * kKVTile);
-        tma_load_2d(sKb, &tm_k, B(&bar_kvf), U.g * kDH, U.so + U.j0);
-        tma_load_2d(sVb, &tm_v, B(&bar_kvf), U.g * kDH, U.so + U.j0);
+        if (MTFM_INBOUNDS(hdr, tma_x_ok(U.g * kDH, kDH, p.hkv * kDH, 2) && U.j0 >= 0 && U.j0 < U.N &&
+                                   U.so + U.j0 < hdr->total_tokens)) {
+          tma_load_2d(sKb, &tm_k, B(&bar_kvf), U.g * kDH, U.so + U.j0);
+          tma_load_2d(sVb, &tm_v, B(&bar_kvf), U.g * kDH, U.so + U.j0);
+        }
         ++nkv;
         for (int t = 0; t < T; ++t) {
           const int s = G % kStages;
@@ -242,9 +247,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           const int st = t / (2 * r), h = U.g * r + (t >> 1) % r, hf = t & 1;
           const int row = U.qrow0 + st * 128 + hf * kQS;
           mbar_expect_tx(B(&bar_stf[s]), kStepBytes);
-          tma_load_2d(sQ(s), &tm_q, B(&bar_stf[s]), h * kDH, row);
-          tma_load_2d(sDAh(s), &tm_dah, B(&bar_stf[s]), h * kDH, row);
-          tma_load_2d(sDAl(s), &tm_dal, B(&bar_stf[s]), h * kDH, row);
+          // a half past the unit's last query (its rows are never used) may start past the tensor
+          if (MTFM_INBOUNDS(hdr, tma_x_ok(h * kDH, kDH, p.hq * kDH, 2) && row >= 0 &&
+                                     (st * 128 + hf * kQS >= U.nq ||
+                                      row < (TARGET ? hdr->total_t : hdr->total_tokens)))) {
+            tma_load_2d(sQ(s), &tm_q, B(&bar_stf[s]), h * kDH, row);
+            tma_load_2d(sDAh(s), &tm_dah, B(&bar_stf[s]), h * kDH, row);
+            tma_load_2d(sDAl(s), &tm_dal, B(&bar_stf[s]), h * kDH, row);
+          }
           ++G;
         }
       }
@@ -390,7 +400,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(B(&bar_dqe[db]));
-      if (mrow < e.nvalid) {
+      if (mrow < e.nvalid &&
+          MTFM_INBOUNDS(hdr, e.row0 + mrow < (TARGET ? hdr->total_t : hdr->total_tokens))) {
         float4* dst = reinterpret_cast<float4*>(dq + (size_t)(e.row0 + mrow) * ldq + e.col + wg * 16);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -521,7 +532,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         tc_fence_before();
         mbar_arrive(B(&bar_dkve));
         const float sk = p.alpha * inv_n;
-        if (key_valid)
+        if (key_valid && MTFM_INBOUNDS(hdr, U.so + jrow < hdr->total_tokens))
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             reinterpret_cast<float4*>(dv_row)[j] =

@@ -24,6 +24,8 @@
 namespace mtfm {
 namespace {
 
+constexpr int kDbgFile = 6;  // site id of this file's bounds checks
+
 constexpr int kBN = 64;  // keys per block
 
 struct UserInfo {
@@ -52,7 +54,7 @@ __device__ __forceinline__ RowMask row_mask(const MetaView& m, const UserInfo& u
                                             int pos, bool valid) {
   RowMask rm{0, 0, 0};
   if (!valid) return rm;
-  rm.kv_end = m.kv_end[ui.so + pos];
+  rm.kv_end = MTFM_INBOUNDS(m.hdr, ui.so + pos < m.hdr->total_tokens) ? m.kv_end[ui.so + pos] : 0;
   const int t0 = ui.LH + ui.LR;
   if (pos >= t0) {
     const int lo = t0 + ((pos - t0) / v2) * v2;
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
     for (int c = tid; c < kTileM * kChunks; c += 256) {
       const int r = c / kChunks, cc = c % kChunks;
       const int qi = q0 + r;
-      const bool ok = qi < nq;
+      const bool ok = qi < nq && MTFM_INBOUNDS(hdr, qrow0 + qi < (TARGET ? hdr->total_t : hdr->total_tokens));
       const __nv_bfloat16* src = p.q + (size_t)(qrow0 + (ok ? qi : 0)) * ldq + h * DH + cc * 8;
       cp_async16(smem_u32(sQ + r * S::kStride + cc * 8), src, ok ? 16 : 0);
     }
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(256) attn_fwd_mma_kernel(FwdArgs p) {
       const int rem = c % (kBN * kChunks);
       const int r = rem / kChunks, cc = rem % kChunks;
       const int j = j0 + r;
-      const bool ok = j < ui.N;
+      const bool ok = j < ui.N && MTFM_INBOUNDS(hdr, ui.so + j < hdr->total_tokens);
       const __nv_bfloat16* base = which ? p.v : p.k;
       const __nv_bfloat16* src = base + (size_t)(ui.so + (ok ? j : 0)) * ldk + g * DH + cc * 8;
       __nv_bfloat16* dst = (which ? sV : sK) + stage * S::kKV + r * S::kStride + cc * 8;
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
     const int rem = c % (kBwdKeys * kChunks);
     const int rr = rem / kChunks, cc = rem % kChunks;
     const int j = j0 + rr;
-    const bool ok = j < ui.N;
+    const bool ok = j < ui.N && MTFM_INBOUNDS(hdr, ui.so + j < hdr->total_tokens);
     const __nv_bfloat16* base = which ? p.v : p.k;
     cp_async16(smem_u32((which ? sV : sK) + rr * S::kStride + cc * 8),
                base + (size_t)(ui.so + (ok ? j : 0)) * ldk + g * DH + cc * 8, ok ? 16 : 0);
@@ -379,7 +381,7 @@ __global__ void __launch_bounds__(128) attn_bwd_mma_kernel(BwdArgs p) {
         const int rem = c % (kBwdQ * kChunks);
         const int rr = rem / kChunks, cc = rem % kChunks;
         const int qi = qt + rr;
-        const bool ok = qi < nq;
+        const bool ok = qi < nq && MTFM_INBOUNDS(hdr, qrow0 + qi < (p.target ? hdr->total_t : hdr->total_tokens));
         const __nv_bfloat16* base = which == 0 ? p.q : (which == 1 ? p.da_hi : p.da_lo);
         __nv_bfloat16* dst = which == 0 ? sQ : (which == 1 ? sAh : sAl);
         cp_async16(smem_u32(dst + rr * S::kStride + cc * 8),

@@ -50,10 +50,12 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kDbgFile = 1;  // site id of this file's bounds checks
+
 constexpr int kDH = 64;
 constexpr int kBM = 128;          // query rows per tile (TMEM lanes)
 constexpr int kBN = 128;          // keys per block
-constexpr int kStages = 3;        // K/V ring depth
+constexpr int kStages = 4;        // K/V ring depth
 constexpr int kSBuf = 2;          // S/P buffers in TMEM
 constexpr int kSiluWG = 4;        // SiLU warpgroups
 constexpr int kWGPerBuf = 4;      // warpgroups sharing one step (split by key columns)
@@ -197,15 +199,20 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (lane == 0) {
         mbar_expect_tx(b_q, R * kQBytes);  // Q of the previous unit was consumed before the unit barrier
         for (int hh = 0; hh < R; ++hh)
-          tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
+          if (MTFM_INBOUNDS(hdr, tma_x_ok((g * R + hh) * kDH, kDH, ldq, 2) && q0 < nq && qrow0 + q0 >= 0 &&
+                                     qrow0 + q0 < hdr->total_tokens))
+            tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
         int issued = 0;
         for (int bi = 0; bi < n_blocks; ++bi) {
           const int G = blk_base + bi, s = G % kStages;
           if (G >= kStages && !mbar_wait(b_kve(s), ((G / kStages) - 1) & 1, abort_flag)) break;
           const int row = so + block_of(bi) * kBN;
           mbar_expect_tx(b_kvf(s), 2 * kKVBytes);
-          tma_load_2d(sK + s * kKVBytes, &tm_k, b_kvf(s), g * kDH, row);
-          tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
+          if (MTFM_INBOUNDS(hdr, tma_x_ok(g * kDH, kDH, p.hkv * kDH, 2) && block_of(bi) >= 0 &&
+                                     block_of(bi) * kBN < N && row < hdr->total_tokens)) {
+            tma_load_2d(sK + s * kKVBytes, &tm_k, b_kvf(s), g * kDH, row);
+            tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
+          }
           ++issued;
         }
         // the next pair, read by every role after this unit's closing barrier
@@ -315,7 +322,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int kv_end = 0, sib_lo = 0, sib_hi = 0;
       if (valid) {
         const int pos = pos0 + qi;
-        kv_end = m.kv_end[so + pos];
+        kv_end = MTFM_INBOUNDS(hdr, so + pos < hdr->total_tokens) ? m.kv_end[so + pos] : 0;
         if (pos >= t0pos) {
           sib_lo = t0pos + ((pos - t0pos) / p.v2) * p.v2;
           sib_hi = sib_lo + p.v2;
@@ -370,9 +377,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int n = n_full; ok && n < total; ++n) ok = step(n, std::true_type{});
       // ----------------------------------------------------------- epilogue: A (+)= O / N_u
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_o, unit_iter & 1, abort_flag));
-      if (ok && total == 0) {
+      if (ok && total == 0 && valid && MTFM_INBOUNDS(hdr, qrow0 + qi < hdr->total_tokens)) {
         // no visible key at all (cannot happen for a non-empty Full tile): A = 0
-        for (int hh = wg; hh < R && valid; hh += kSiluWG)
+        for (int hh = wg; hh < R; hh += kSiluWG)
             for (int c = 0; c < kDH; c += 4)
               *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
                   make_float4(0.f, 0.f, 0.f, 0.f);
@@ -413,7 +420,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (q0 + kBM <= nq) {
           if (threadIdx.x == 128) {
             for (int b = 0; b < 2 * R; ++b)
-              tma_store_2d_hint(&tm_a, sQ + b * kBox, g * R * kDH + b * 32, qrow0 + q0, keep_a);
+              if (MTFM_INBOUNDS(hdr, tma_x_ok(g * R * kDH + b * 32, 32, ldq, 4) && qrow0 + q0 >= 0 &&
+                                         qrow0 + q0 + kBM <= hdr->total_tokens))
+                tma_store_2d_hint(&tm_a, sQ + b * kBox, g * R * kDH + b * 32, qrow0 + q0, keep_a);
             bulk_commit();
             bulk_wait_read<0>();  // the next unit's loads may overwrite the staging area
           }
@@ -422,6 +431,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll 1
           for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
             if (q0 + rr >= nq) break;
+            if (!MTFM_INBOUNDS(hdr, qrow0 + q0 + rr < hdr->total_tokens)) break;
             float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
             for (int f = lane; f < R * kDH / 4; f += 32) {
               const float4 v =

@@ -42,6 +42,8 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kDbgFile = 3;  // site id of this file's bounds checks
+
 constexpr int kDH = 256;
 constexpr int kBM = 128;            // query rows per tile
 constexpr int kBN = 64;             // keys per block
@@ -204,7 +206,10 @@ attn_fwd_tc256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // ----------------------------------------------------------- producer
       if (lane == 0) {
         mbar_expect_tx(B(&bar_q), kQBytes);  // Q of the previous unit was consumed before the unit barrier
-        for (int a = 0; a < kAtoms; ++a) tma_load_2d(sQ + a * kQAtom, &tm_q, B(&bar_q), h * kDH + a * 64, qrow0 + q0);
+        for (int a = 0; a < kAtoms; ++a)
+          if (MTFM_INBOUNDS(hdr, tma_x_ok(h * kDH + a * 64, 64, p.hq * kDH, 2) && q0 < nq && qrow0 + q0 >= 0 &&
+                                     qrow0 + q0 < (p.target ? hdr->total_t : hdr->total_tokens)))
+            tma_load_2d(sQ + a * kQAtom, &tm_q, B(&bar_q), h * kDH + a * 64, qrow0 + q0);
         // K runs kKStages - 1 blocks ahead of V: K(0..2), then V(n), K(n + 3) for each n.
         // Global block G = blk_base + n: K stage G % kKStages, V stage G % kVStages.
         bool ok = true;
@@ -224,7 +229,9 @@ attn_fwd_tc256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const int row = so + kb.block(bi) * kBN;
           mbar_expect_tx(B(&bar_kf[s]), kKBytes);
           for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(sK + s * kKBytes + a * kKVAtom, &tm_k, B(&bar_kf[s]), g * kDH + a * 64, row);
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(g * kDH + a * 64, 64, p.hkv * kDH, 2) && kb.block(bi) >= 0 &&
+                                       kb.block(bi) * kBN < N && row < hdr->total_tokens))
+              tma_load_2d(sK + s * kKBytes + a * kKVAtom, &tm_k, B(&bar_kf[s]), g * kDH + a * 64, row);
           return true;
         };
         auto load_v = [&](int bi) -> bool {
@@ -233,7 +240,9 @@ attn_fwd_tc256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const int row = so + kb.block(bi) * kBN;
           mbar_expect_tx(B(&bar_vf[s]), kKBytes);
           for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(sV + s * kKBytes + a * kKVAtom, &tm_v, B(&bar_vf[s]), g * kDH + a * 64, row);
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(g * kDH + a * 64, 64, p.hkv * kDH, 2) && kb.block(bi) >= 0 &&
+                                       kb.block(bi) * kBN < N && row < hdr->total_tokens))
+              tma_load_2d(sV + s * kKBytes + a * kKVAtom, &tm_v, B(&bar_vf[s]), g * kDH + a * 64, row);
           return true;
         };
         for (int bi = 0; bi < 2 * kKStages; ++bi) prefetch(bi);
@@ -348,7 +357,7 @@ attn_fwd_tc256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       int kv_end = 0, sib_lo = 0, sib_hi = 0;
       if (valid) {
         const int pos = pos0 + qi;
-        kv_end = m.kv_end[so + pos];
+        kv_end = MTFM_INBOUNDS(hdr, so + pos < hdr->total_tokens) ? m.kv_end[so + pos] : 0;
         if (pos >= t0pos) {
           sib_lo = t0pos + ((pos - t0pos) / p.v2) * p.v2;
           sib_hi = sib_lo + p.v2;
@@ -424,7 +433,9 @@ attn_fwd_tc256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (q0 + kBM <= nq) {
           if (threadIdx.x == 128) {
             for (int bx = 0; bx < 8; ++bx)
-              tma_store_2d_hint(&tm_a, sQ + bx * kStgBox, h * kDH + bx * 32, qrow0 + q0, keep_a);
+              if (MTFM_INBOUNDS(hdr, tma_x_ok(h * kDH + bx * 32, 32, p.hq * kDH, 4) && qrow0 + q0 >= 0 &&
+                                         qrow0 + q0 + kBM <= (p.target ? hdr->total_t : hdr->total_tokens)))
+                tma_store_2d_hint(&tm_a, sQ + bx * kStgBox, h * kDH + bx * 32, qrow0 + q0, keep_a);
             bulk_commit();
             bulk_wait_read<0>();  // the next unit's loads may overwrite the staging area
           }
@@ -433,6 +444,7 @@ attn_fwd_tc256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll 1
           for (int rr = sw * (kBM / 8); rr < (sw + 1) * (kBM / 8); ++rr) {
             if (q0 + rr >= nq) break;
+            if (!MTFM_INBOUNDS(hdr, qrow0 + q0 + rr < (p.target ? hdr->total_t : hdr->total_tokens))) break;
             float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + h * kDH);
             for (int f = lane; f < kDH / 4; f += 32) {
               const float4 v = *reinterpret_cast<const float4*>(smem + (f / 8) * kStgBox + rr * 128 +

@@ -29,15 +29,18 @@
 //                 unit), then O += P_hi V + P_lo V into one of two O buffers.
 //   warps 4..19 : SiLU warpgroups (as in the Full-layer kernel: each warpgroup
 //                 takes 32 of the 128 key columns of a step), then the unit's
-//                 epilogue: O / N_u from TMEM into a swizzled shared-memory tile,
-//                 then into A (fp32).  When every sub-tile's key range is one
+//                 epilogue: O / N_u from TMEM into a swizzled shared-memory tile.
+//   warp 3      : stores the staged tile into A (fp32), so that no SiLU warp
+//                 waits for a store.  When every sub-tile's key range is one
 //                 unit (MetaHeader::tgt_single), each row of A gets exactly one
 //                 unit's O: TMA stores, or row stores of the user's rows for a
 //                 sub-tile that runs past its user's last T row.  Otherwise A is
 //                 zeroed first (tgt_zero_kernel, launched just before) and every
 //                 unit adds its partial O with one TMA reduce-add per 32 columns,
 //                 rows past the user's last T row staged as zeros, so the chunks
-//                 sum without atomics.
+//                 sum without atomics.  Two mbarriers hand the tile over (every
+//                 SiLU thread arrives, warp 3 waits) and back (warp 3 arrives once
+//                 the copies have read the tile, the SiLU warps wait).
 // TMEM: O buffers at columns [0, 64) and [64, 128), S buffers at [128 + 128b, +128).
 // Every mbarrier wait is bounded; after a timeout the roles stop issuing work and
 // drain (bounded), the SiLU warps still pass their named barriers the same
@@ -57,9 +60,14 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kDbgFile = 2;  // site id of this file's bounds checks
+
 constexpr int kDH = 64;
 constexpr int kBN = 128;     // keys per block
-constexpr int kStages = 3;   // K/V ring
+// K/V ring: the loads of a unit's blocks come from DRAM (~3,000-4,000 clocks under load)
+// while a block takes ~1,700 clocks of MMA and SiLU work, so about three blocks must be in
+// flight beyond the two the MMA warp holds (S two steps ahead): five stages.
+constexpr int kStages = 5;
 constexpr int kSBuf = 3;     // S/P buffers
 constexpr int kSiluWG = 4;
 constexpr int kThreads = 128 + 128 * kSiluWG;
@@ -72,8 +80,10 @@ static_assert(kBN == kKeyBlock, "the packer sizes Target units in blocks of kKey
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "TMEM plan");
 
 constexpr int kRing = 4;                 // decoded-unit descriptors in flight
+constexpr uint16_t kKtNone = 0xffff;
 constexpr int kDescConsumers = 2 + 16;   // producer, MMA warp, 16 SiLU warps
 constexpr size_t tgt_smem_bytes() { return 2 * kQBytes + 2 * kStages * kKVBytes + kStageBytes + 1024; }
+static_assert(tgt_smem_bytes() + 2048 <= 227 * 1024, "dynamic + static shared memory per CTA");
 
 struct TgtArgs {
   MetaView m;
@@ -149,18 +159,19 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half
 }
 
 // Rows [0, rows) of a staged O tile (2R boxes of TR rows x 32 fp32, 16-byte chunks
-// XOR-swizzled by row) to A rows dst + t * ld; 16 warps, warp sw takes rows sw, sw + 16, ...
+// XOR-swizzled by row) to A rows dst + t * ld, by one warp.
 template <int R>
-__device__ __noinline__ void store_rows(const uint8_t* stage, float* dst, int ld, int rows, int sw, int lane) {
+__device__ __noinline__ void store_rows(const uint8_t* stage, float* dst, int ld, int rows, int lane) {
   constexpr int TR = 128 / R;
-  for (int tr = sw; tr < rows; tr += 16) {
-    float4* d = reinterpret_cast<float4*>(dst + (size_t)tr * ld);
-    for (int f = lane; f < R * kDH / 4; f += 32)
-      d[f] = *reinterpret_cast<const float4*>(stage + (f >> 3) * (TR * 128) + tr * 128 + (((f & 7) ^ (tr & 7)) << 4));
+  constexpr int kF = R * kDH / 4;  // float4 per row
+  for (int i = lane; i < rows * kF; i += 32) {
+    const int tr = i / kF, f = i % kF;
+    reinterpret_cast<float4*>(dst + (size_t)tr * ld)[f] =
+        *reinterpret_cast<const float4*>(stage + (f >> 3) * (TR * 128) + tr * 128 + (((f & 7) ^ (tr & 7)) << 4));
   }
 }
 
-__device__ __forceinline__ void silu_bar() { asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory"); }
+
 
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -173,7 +184,13 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __shared__ __align__(8) uint64_t bar_qf[2], bar_qe[2], bar_of[2], bar_oe[2], bar_drain;
   __shared__ __align__(8) uint64_t bar_kvf[kStages], bar_kve[kStages], bar_sf[kSBuf], bar_pf[kSBuf];
   __shared__ __align__(8) uint64_t bar_df[kRing], bar_de[kRing];
+  __shared__ __align__(8) uint64_t bar_stf, bar_ste;  // staging tile full / free
   __shared__ TgtUnit s_desc[kRing];
+  // k_t = kv_end - L_H of the sub-tile's T rows, loaded by the scheduler warp with the
+  // descriptor (kKtNone: the user's L_R does not fit, the SiLU warps load kv_end)
+  __shared__ uint16_t s_kt[kRing][128];
+  // the staged tile's destination, written by warp 4 before it hands the tile over
+  __shared__ int4 s_st[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -221,6 +238,8 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(B(&bar_de[j]), kDescConsumers);
     }
     mbar_init(B(&bar_drain), 1);
+    mbar_init(B(&bar_stf), 128 * kSiluWG);
+    mbar_init(B(&bar_ste), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -263,7 +282,9 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int qb = k & 1;
         if (k >= 2 && !mbar_wait(B(&bar_qe[qb]), ((k - 2) >> 1) & 1, abort_flag)) break;
         mbar_expect_tx(B(&bar_qf[qb]), kQBytes);
-        tma_load_3d(sQ + qb * kQBytes, &tm_q, B(&bar_qf[qb]), 0, U.g * R, m.t_off[U.u] + U.q_sub0);
+        if (MTFM_INBOUNDS(hdr, U.g >= 0 && U.g * R + R <= p.hq && U.q_sub0 >= 0 && U.q_sub0 < U.LT &&
+                                   m.t_off[U.u] + U.q_sub0 < hdr->total_t))
+          tma_load_3d(sQ + qb * kQBytes, &tm_q, B(&bar_qf[qb]), 0, U.g * R, m.t_off[U.u] + U.q_sub0);
         ++nq_loads;
         for (int i = 0; i < U.nb; ++i) {
           const int s = G % kStages;
@@ -275,12 +296,18 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const int bb = U.bi0 + i;
           if (p.cached && bb >= U.kb.nb_pre) {  // the candidate rows from the sub-tile's first T row
             const int row = m.t_off[U.u] + U.q_sub0;
-            tma_load_2d(sK + s * kKVBytes, &tm_kc, B(&bar_kvf[s]), U.g * kDH, row);
-            tma_load_2d(sV + s * kKVBytes, &tm_vc, B(&bar_kvf[s]), U.g * kDH, row);
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(U.g * kDH, kDH, p.hkv * kDH, 2) && row >= 0 && row < hdr->total_t)) {
+              tma_load_2d(sK + s * kKVBytes, &tm_kc, B(&bar_kvf[s]), U.g * kDH, row);
+              tma_load_2d(sV + s * kKVBytes, &tm_vc, B(&bar_kvf[s]), U.g * kDH, row);
+            }
           } else {
             const int row = U.kv_row0 + U.kb.block(bb) * kBN;
-            tma_load_2d(sK + s * kKVBytes, &tm_k, B(&bar_kvf[s]), U.g * kDH, row);
-            tma_load_2d(sV + s * kKVBytes, &tm_v, B(&bar_kvf[s]), U.g * kDH, row);
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(U.g * kDH, kDH, p.hkv * kDH, 2) && U.kb.block(bb) >= 0 &&
+                                       U.kb.block(bb) * kBN < (p.cached ? U.LH + U.LR : U.N) && row >= 0 &&
+                                       row < (p.cached ? hdr->total_tokens - hdr->total_t : hdr->total_tokens))) {
+              tma_load_2d(sK + s * kKVBytes, &tm_k, B(&bar_kvf[s]), U.g * kDH, row);
+              tma_load_2d(sV + s * kKVBytes, &tm_v, B(&bar_kvf[s]), U.g * kDH, row);
+            }
           }
           ++G;
         }
@@ -383,13 +410,24 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------- unit scheduler
-    if (lane == 0) {
-      for (int k = 0; k < n_mine; ++k) {
-        const int j = k % kRing;
-        if (k >= kRing && !mbar_wait(B(&bar_de[j]), ((k / kRing) - 1) & 1, abort_flag)) break;
-        s_desc[j] = decode_unit<R>(m, unit_of(k), p.hkv, p.v2, p.cached != 0);
-        mbar_arrive(B(&bar_df[j]));  // release: the descriptor is visible to every waiter
+    for (int k = 0; k < n_mine; ++k) {
+      const int j = k % kRing;
+      if (k >= kRing && !__all_sync(0xffffffffu, mbar_wait(B(&bar_de[j]), ((k / kRing) - 1) & 1, abort_flag)))
+        break;
+      if (lane == 0) s_desc[j] = decode_unit<R>(m, unit_of(k), p.hkv, p.v2, p.cached != 0);
+      __syncwarp();
+      const TgtUnit& U = s_desc[j];
+      const int t0pos = U.LH + U.LR;
+      for (int i = lane; i < TR; i += 32) {
+        const int qi = U.q_sub0 + i;
+        uint16_t kt = kKtNone;
+        if (U.LR < (int)kKtNone && qi < U.LT &&
+            MTFM_INBOUNDS(hdr, U.so + t0pos + qi < hdr->total_tokens))
+          kt = (uint16_t)(m.kv_end[U.so + t0pos + qi] - U.LH);
+        s_kt[j][i] = kt;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(&bar_df[j]));  // release: descriptor and k_t visible to every waiter
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- SiLU warpgroups + epilogue
@@ -399,11 +437,10 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int t = mrow / R, hh = mrow % R;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const float half_alpha = 0.5f * p.alpha;
-    const bool issuer = threadIdx.x == 128;
     bool ok = true;
     int gp = 0;
-    // Epilogue of unit e.k: O / N_u -> swizzled staging tile -> TMA reduce-add into A.
-    // Each call passes the two named barriers, whatever e.ok says.
+    // Epilogue of unit e.k: O / N_u -> swizzled staging tile, handed to the store warp.
+    // Every call arrives on bar_stf, whatever e.ok says, so the store warp always moves on.
     struct Prev {
       int k, col, y, rows;
       bool ok;
@@ -414,8 +451,9 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       bool eok = e.ok && ok;
       if (eok) eok = __all_sync(0xffffffffu, mbar_wait(B(&bar_of[ob]), (e.k >> 1) & 1, abort_flag));
       if (!eok) ok = false;
-      if (issuer) bulk_wait_read<0>();  // the previous reduces have read the staging tile
-      silu_bar();
+      // the store warp is done reading the staging tile of unit e.k - 1
+      if (eok && e.k > 0) eok = __all_sync(0xffffffffu, mbar_wait(B(&bar_ste), (e.k - 1) & 1, abort_flag));
+      if (!eok) ok = false;
       if (eok) {
         tc_fence_after();
         uint32_t raw[16];
@@ -432,31 +470,17 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               make_float4(__uint_as_float(raw[4 * j]) * e.inv_n, __uint_as_float(raw[4 * j + 1]) * e.inv_n,
                           __uint_as_float(raw[4 * j + 2]) * e.inv_n, __uint_as_float(raw[4 * j + 3]) * e.inv_n);
         }
-        fence_proxy_async();
+        fence_proxy_async();  // the staged tile may be read by the TMA engine
       }
-      silu_bar();
-      if (eok && !single) {
-        if (issuer) {
-          for (int b = 0; b < 2 * R; ++b)
-            tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), e.col + (b >> 1) * kDH + (b & 1) * 32, e.y);
-          bulk_commit();
-        }
-      } else if (eok && e.rows == TR) {
-        if (issuer) {
-          for (int b = 0; b < 2 * R; ++b)
-            tma_store_2d(&tm_a, sO + b * (TR * 128), e.col + (b >> 1) * kDH + (b & 1) * 32, e.y);
-          bulk_commit();
-        }
-      } else if (eok) {
-        // the sub-tile runs past its user's last T row: store the user's rows one by one
-        store_rows<R>(stage, p.a + (size_t)e.y * (p.hq * kDH) + e.col, p.hq * kDH, e.rows, warp - 4, lane);
-      }
+      if (threadIdx.x == 128) s_st[e.k & 1] = make_int4(eok ? 1 : 0, e.col, e.y, e.rows);
+      mbar_arrive(B(&bar_stf));
     };
     // Every SiLU warp walks all n_mine units, also after an abort, so that all of
     // them pass the named barriers of each epilogue the same number of times.
     for (int k = 0; k < n_mine; ++k) {
       TgtUnit U;
       if (ok) ok = __all_sync(0xffffffffu, get_desc(k, U));
+      const uint16_t kt = ok ? s_kt[k % kRing][t] : kKtNone;  // read before the slot is released
       __syncwarp();
       if (ok && lane == 0) release_desc(k);
       if (!ok) U = TgtUnit{};  // after an abort: no work, only the barriers below
@@ -466,7 +490,10 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int t0pos = U.LH + U.LR;
       if (valid) {
         const int pos = t0pos + qi;
-        kv_end = m.kv_end[U.so + pos];
+        if (kt != kKtNone)
+          kv_end = U.LH + kt;
+        else
+          kv_end = MTFM_INBOUNDS(hdr, U.so + pos < hdr->total_tokens) ? m.kv_end[U.so + pos] : 0;
         sib_lo = t0pos + (qi / p.v2) * p.v2;
         sib_hi = sib_lo + p.v2;
       }
@@ -528,7 +555,40 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       prev.rows = ok ? min(TR, U.LT - U.q_sub0) : 0;
     }
     if (n_mine > 0) epilogue(prev);
-    if (issuer) bulk_wait<0>();  // every reduce has completed before the CTA leaves
+  } else if (warp == 3) {
+    // ------------------------------------------------------------- store warp
+    // Takes each staged tile (in unit order) after the SiLU warps have written it, and
+    // hands the staging area back once its copies have read it.
+    for (int k = 0; k < n_mine; ++k) {
+      const bool full = __all_sync(0xffffffffu, mbar_wait(B(&bar_stf), k & 1, abort_flag));
+      int4 st = s_st[k & 1];  // {ok, first column, first row of A, rows}
+      if (!full) st.x = 0;
+      if (st.x && !single) {
+        if (lane == 0) {
+          for (int b = 0; b < 2 * R; ++b)
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(st.y + (b >> 1) * kDH + (b & 1) * 32, 32, p.hq * kDH, 4) &&
+                                       st.z >= 0 && st.z < hdr->total_t))
+              tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), st.y + (b >> 1) * kDH + (b & 1) * 32, st.z);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+      } else if (st.x && st.w == TR) {
+        if (lane == 0) {
+          for (int b = 0; b < 2 * R; ++b)
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(st.y + (b >> 1) * kDH + (b & 1) * 32, 32, p.hq * kDH, 4) &&
+                                       st.z >= 0 && st.z + TR <= hdr->total_t))
+              tma_store_2d(&tm_a, sO + b * (TR * 128), st.y + (b >> 1) * kDH + (b & 1) * 32, st.z);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+      } else if (st.x && MTFM_INBOUNDS(hdr, st.z >= 0 && st.z + st.w <= hdr->total_t)) {
+        // the sub-tile runs past its user's last T row: store the user's rows one by one
+        store_rows<R>(stage, p.a + (size_t)st.z * (p.hq * kDH) + st.y, p.hq * kDH, st.w, lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B(&bar_ste));
+    }
+    if (lane == 0) bulk_wait<0>();  // every copy has completed before the CTA leaves
   }
   pdl_trigger();
   __syncthreads();

@@ -12,6 +12,8 @@
 namespace mtfm {
 namespace {
 
+constexpr int kDbgFile = 7;  // site id of this file's bounds checks
+
 constexpr int kMaxChunks = 8;  // float4 chunks per lane: D <= 32 * 4 * 8 = 1024
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -68,6 +70,7 @@ gate_fwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
   if (row >= rows) return;
+  if (!MTFM_INBOUNDS(hdr, row < (target ? hdr->total_t : hdr->total_tokens))) return;
   const int nch = D >> 2;  // float4 chunks in the row
   const float* ar = a + (size_t)row * D;
   const __nv_bfloat16* ur = u + (size_t)row * D;
@@ -158,6 +161,7 @@ gate_bwd_kernel(const MetaHeader* hdr, const uint8_t* __restrict__ row_type, boo
     __syncthreads();
   }
   for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+    if (!MTFM_INBOUNDS(hdr, row < (target ? hdr->total_t : hdr->total_tokens))) break;
     const float* ar = a + (size_t)row * D;
     const __nv_bfloat16* ur = u + (size_t)row * D;
     const __nv_bfloat16* dyr = dy + (size_t)row * D;

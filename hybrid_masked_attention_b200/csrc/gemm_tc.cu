@@ -35,6 +35,8 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kDbgFile = 5;  // site id of this file's bounds checks
+
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kStagesDirect = 4;  // K-slice ring; 3 when the epilogue stages tiles for TMA
@@ -192,12 +194,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
             break;
           }
           mbar_expect_tx(b_full(s), kStage);
-          tma_load_2d(sbase + s * kStage, &tm_a, b_full(s), kb * kBK, m0);
-          if (p.epi.kind == kEpiSwiGLU) {  // gate rows, then the same rows of the up matrix
-            tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0 / 2);
-            tma_load_2d(sbase + s * kStage + kABytes + (BN / 2) * 128, &tm_b2, b_full(s), kb * kBK, n0 / 2);
-          } else {
-            tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0);
+          // a failed check skips the stage's loads; the consumer's bounded wait gives up on it
+          if (MTFM_INBOUNDS(hdr, tma_x_ok(kb * kBK, kBK, p.K, 2) && m0 >= 0 && m0 < p.M && n0 >= 0 && n0 < p.N)) {
+            tma_load_2d(sbase + s * kStage, &tm_a, b_full(s), kb * kBK, m0);
+            if (p.epi.kind == kEpiSwiGLU) {  // gate rows, then the same rows of the up matrix
+              tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0 / 2);
+              tma_load_2d(sbase + s * kStage + kABytes + (BN / 2) * 128, &tm_b2, b_full(s), kb * kBK, n0 / 2);
+            } else {
+              tma_load_2d(sbase + s * kStage + kABytes, &tm_b, b_full(s), kb * kBK, n0);
+            }
           }
           ++G;
         }
@@ -347,7 +352,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
                 sb = p.epi.seg_begin[q];
                 om = q == 1 ? &tm_o1 : q == 2 ? &tm_o2 : &tm_o3;
               }
-            tma_store_2d(om, sstage + bx * kBoxBytes, col - sb, m0);
+            if (MTFM_INBOUNDS(hdr, col - sb >= 0 && ((col - sb) * 2) % 16 == 0 && m0 >= 0 && m0 < p.M))
+              tma_store_2d(om, sstage + bx * kBoxBytes, col - sb, m0);
           }
           bulk_commit();
         }
@@ -373,7 +379,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__
           wg_bar(bar_id);
           if (issuer) {
             for (int bx = 0; bx < nb; ++bx)
-              tma_reduce_add_2d(&tm_o0, sstage + bx * kBoxBytes, col0 + (b0 + bx) * 32, m0);
+              if (MTFM_INBOUNDS(hdr, tma_x_ok(col0 + (b0 + bx) * 32, 32, p.N, 4) && m0 >= 0 && m0 < p.M))
+                tma_reduce_add_2d(&tm_o0, sstage + bx * kBoxBytes, col0 + (b0 + bx) * 32, m0);
             bulk_commit();
           }
         }

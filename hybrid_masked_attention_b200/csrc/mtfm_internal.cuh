@@ -68,6 +68,7 @@ constexpr int kErrBadLengths = 1;
 constexpr int kErrUnsorted = 2;
 constexpr int kErrTimeout = 4;
 constexpr int kErrConfig = 8;  // a kernel's head configuration differs from the packed one
+constexpr int kErrBounds = 16; // a check of the bounds-checked build failed (MTFM_DEBUG_BOUNDS)
 
 constexpr int kMetaMagic = 0x4d54464d;  // "MTFM"
 
@@ -103,7 +104,37 @@ struct MetaHeader {
   // cached-prefix form): each row of A then gets exactly one unit's O, stored directly;
   // otherwise the chunks' partial O are summed into A (zeroed by a kernel just before).
   int32_t tgt_single[2];
+  // Bounds-checked build only: the site (file id * 100000 + line) of the first failed check.
+  int32_t dbg_site;
 };
+
+// Bounds-checked build.  Compiled with -DMTFM_DEBUG_BOUNDS, the kernels test each TMA
+// coordinate (the inner one 16-byte aligned, the box starting inside its tensor and, for a
+// store, ending inside it) and the global row indices they compute, before using them.  A
+// failed test sets kErrBounds in MetaHeader::error, records its site in
+// MetaHeader::dbg_site and skips the access; a skipped load leaves its mbarrier short of
+// bytes, so the consumer gives up after its bounded wait instead of hanging.  This build
+// stands in for a memory checker; normal builds compile every test to `true`.  Each .cu
+// file that uses MTFM_INBOUNDS defines kDbgFile, its id in the recorded site.
+#ifdef MTFM_DEBUG_BOUNDS
+__device__ __forceinline__ bool dbg_bounds(const MetaHeader* h, bool ok, int site) {
+  if (!ok) {
+    MetaHeader* w = const_cast<MetaHeader*>(h);
+    atomicOr(&w->error, kErrBounds);
+    atomicCAS(&w->dbg_site, 0, site);
+  }
+  return ok;
+}
+#define MTFM_INBOUNDS(h, cond) (::mtfm::dbg_bounds((h), (cond), kDbgFile * 100000 + __LINE__))
+#else
+#define MTFM_INBOUNDS(h, cond) ((void)kDbgFile, true)
+#endif
+
+// Inner TMA coordinate x of a box of w elements of esize bytes in a row of `width`
+// elements: 16-byte aligned start, box inside the row.
+__host__ __device__ __forceinline__ bool tma_x_ok(int x, int w, int width, int esize) {
+  return x >= 0 && (x * esize) % 16 == 0 && x + w <= width;
+}
 
 // One work item: a 128-row query tile of one user and the range of prefix
 // ends (kv_end) over its rows.  Keys at or beyond kv_max are never read for

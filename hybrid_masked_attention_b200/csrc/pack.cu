@@ -111,6 +111,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       m.hdr->n_units_target_c = 0;
       m.hdr->sched[0] = m.hdr->sched[1] = 0;
       m.hdr->tgt_single[0] = m.hdr->tgt_single[1] = 1;
+      m.hdr->dbg_site = 0;
       m.hdr->tgt_sub_rows = tgt_sub_rows;
       m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
       m.hdr->pack_done = 0;
@@ -203,6 +204,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     m.hdr->n_units_target_c = 0;
     m.hdr->sched[0] = m.hdr->sched[1] = 0;
     m.hdr->tgt_single[0] = m.hdr->tgt_single[1] = 1;
+    m.hdr->dbg_site = 0;
     m.hdr->tgt_sub_rows = tgt_sub_rows;
     m.hdr->tgt_chunk_blocks = kTargetUnitBlocks;
     m.hdr->pack_done = 0;

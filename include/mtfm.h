@@ -74,8 +74,10 @@ typedef enum {
   MTFM_ERR_WORKSPACE_TOO_SMALL = 4, /* meta or workspace buffer smaller than the size query */
   MTFM_ERR_CUDA = 5,                /* a CUDA runtime call failed (launch error etc.) */
   MTFM_ERR_TIMEOUT = 6,             /* a bounded device wait gave up (kernel returned early) */
-  MTFM_ERR_BAD_LENGTHS = 7          /* device lengths negative, not summing to the totals, or
+  MTFM_ERR_BAD_LENGTHS = 7,         /* device lengths negative, not summing to the totals, or
                                        L_T not a multiple of v2_subtokens */
+  MTFM_ERR_BOUNDS = 8               /* bounds-checked build only: a kernel found a TMA coordinate
+                                       or a global index out of bounds and skipped the access */
 } mtfm_status;
 
 /* Problem description shared by all calls (host memory, read only). */
@@ -117,10 +119,21 @@ mtfm_status mtfm_pack(const mtfm_cfg* cfg, const int32_t* d_lh, const int32_t* d
                       void* d_meta, size_t meta_bytes, void* stream);
 
 /* Synchronises `stream` and returns the device-side verdict of the last
- * mtfm_pack on d_meta (MTFM_OK, MTFM_ERR_BAD_LENGTHS, MTFM_ERR_UNSORTED_TS)
- * or MTFM_ERR_TIMEOUT if an attention kernel recorded a timeout there.
+ * mtfm_pack on d_meta (MTFM_OK, MTFM_ERR_BAD_LENGTHS, MTFM_ERR_UNSORTED_TS),
+ * MTFM_ERR_BOUNDS if a kernel of the bounds-checked build found an access out
+ * of bounds, or MTFM_ERR_TIMEOUT if a kernel recorded a timeout there.
  * Optional: the hot path never needs it. */
 mtfm_status mtfm_pack_check(const void* d_meta, void* stream);
+
+/* Bounds-checked build (compiled with -DMTFM_DEBUG_BOUNDS; no counterpart on the
+ * pages: it stands in for a device memory checker).  Its kernels test every TMA
+ * coordinate and the global row indices they compute before use; a failed test
+ * records MTFM_ERR_BOUNDS in d_meta's header (see mtfm_pack_check) with its site,
+ * and skips the access.  mtfm_debug_bounds_build returns 1 in that build, else 0.
+ * mtfm_debug_site synchronises `stream` and writes to *site (host) the first failed
+ * test's site, file id * 100000 + source line, or 0; d_meta as for mtfm_pack_check. */
+int32_t mtfm_debug_bounds_build(void);
+mtfm_status mtfm_debug_site(const void* d_meta, int32_t* site, void* stream);
 
 /* Copies the metadata block's arrays into caller host buffers (synchronous;
  * any pointer may be NULL).  seq_off/r_off/t_off are int32 [batch+1],

@@ -105,9 +105,17 @@ def test_null_and_misaligned_pointers_rejected(lib):
 
 def test_status_strings(lib):
     import hybrid_masked_attention_b200 as m
-    for s in range(8):
+    for s in range(9):
         assert m._lib.mtfm_status_string(s)
+        assert b"unknown" not in m._lib.mtfm_status_string(s)
     assert b"unknown" in m._lib.mtfm_status_string(99)
+
+
+def test_debug_bounds_queries(lib):
+    """The shipped library is the normal build; the site query checks its arguments."""
+    import hybrid_masked_attention_b200 as m
+    assert m._lib.mtfm_debug_bounds_build() == 0
+    assert m._lib.mtfm_debug_site(None, None, None) == 1
 
 
 def test_meta_capacity_bounds(lib):
