@@ -98,6 +98,7 @@ struct TgtUnit {
   int u, so, LH, LR, LT, N, g;
   int kv_row0;  // first K/V row of the user's prefix blocks (cache rows when cached)
   int q_sub0;  // first T row (within the user's T rows) of the sub-tile
+  int t_row0;  // its row in Q, A and the candidate K/V: t_off[u] + q_sub0
   int bi0, nb, kv_min;
   KeyBlocks kb;
 };
@@ -133,6 +134,7 @@ __device__ TgtUnit decode_unit(const MetaView& m, int w, int hkv, int v2, bool c
   const int nchunks = (U.kb.n_blocks + C - 1) / C;
   const int sub = local / nchunks, chunk = local % nchunks;
   U.q_sub0 = q0 + sub * TR;
+  U.t_row0 = m.t_off[U.u] + U.q_sub0;
   U.bi0 = chunk * C;
   U.nb = min(U.bi0 + C, U.kb.n_blocks) - U.bi0;
   U.kv_min = it.kv_min;
@@ -283,8 +285,8 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (k >= 2 && !mbar_wait(B(&bar_qe[qb]), ((k - 2) >> 1) & 1, abort_flag)) break;
         mbar_expect_tx(B(&bar_qf[qb]), kQBytes);
         if (MTFM_INBOUNDS(hdr, U.g >= 0 && U.g * R + R <= p.hq && U.q_sub0 >= 0 && U.q_sub0 < U.LT &&
-                                   m.t_off[U.u] + U.q_sub0 < hdr->total_t))
-          tma_load_3d(sQ + qb * kQBytes, &tm_q, B(&bar_qf[qb]), 0, U.g * R, m.t_off[U.u] + U.q_sub0);
+                                   U.t_row0 < hdr->total_t))
+          tma_load_3d(sQ + qb * kQBytes, &tm_q, B(&bar_qf[qb]), 0, U.g * R, U.t_row0);
         ++nq_loads;
         for (int i = 0; i < U.nb; ++i) {
           const int s = G % kStages;
@@ -295,7 +297,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           mbar_expect_tx(B(&bar_kvf[s]), 2 * kKVBytes);
           const int bb = U.bi0 + i;
           if (p.cached && bb >= U.kb.nb_pre) {  // the candidate rows from the sub-tile's first T row
-            const int row = m.t_off[U.u] + U.q_sub0;
+            const int row = U.t_row0;
             if (MTFM_INBOUNDS(hdr, tma_x_ok(U.g * kDH, kDH, p.hkv * kDH, 2) && row >= 0 && row < hdr->total_t)) {
               tma_load_2d(sK + s * kKVBytes, &tm_kc, B(&bar_kvf[s]), U.g * kDH, row);
               tma_load_2d(sV + s * kKVBytes, &tm_vc, B(&bar_kvf[s]), U.g * kDH, row);
@@ -542,7 +544,8 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int i = max(i0, n_full); ok && i < i1; ++i) ok = step(i, std::true_type{});
       };
       // The epilogue of the previous unit runs after this unit's first step, so the
-      // wait for the previous unit's last PV overlaps that step's SiLU.
+      // wait for the previous unit's last PV overlaps that step's SiLU.  (After two steps
+      // measured slower at 512-token users.)
       run_steps(0, 1);
       if (k > 0) epilogue(prev);
       run_steps(1, U.nb);
@@ -551,7 +554,7 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       prev.ok = ok;
       prev.inv_n = valid && U.N > 0 ? 1.f / (float)U.N : 0.f;  // rows past the user's T rows add zeros
       prev.col = U.g * R * kDH;
-      prev.y = ok ? m.t_off[U.u] + U.q_sub0 : 0;
+      prev.y = ok ? U.t_row0 : 0;
       prev.rows = ok ? min(TR, U.LT - U.q_sub0) : 0;
     }
     if (n_mine > 0) epilogue(prev);
