@@ -55,7 +55,7 @@ constexpr int kDbgFile = 1;  // site id of this file's bounds checks
 constexpr int kDH = 64;
 constexpr int kBM = 128;          // query rows per tile (TMEM lanes)
 constexpr int kBN = 128;          // keys per block
-constexpr int kStages = 4;        // K/V ring depth
+constexpr int kStages = 3;        // K/V ring depth
 constexpr int kSBuf = 2;          // S/P buffers in TMEM
 constexpr int kSiluWG = 4;        // SiLU warpgroups
 constexpr int kWGPerBuf = 4;      // warpgroups sharing one step (split by key columns)
@@ -67,7 +67,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
 static_assert(kBN == kKeyBlock, "key blocks of the work lists");
-static_assert(kBM * 4 * kDH * 4 <= 4 * kQBytes + 2 * kStages * kKVBytes, "O staging fits in the Q + K/V buffers");
 static_assert(kSiluWG == kWGPerBuf && kChunksPerWG >= 1, "all warpgroups share every step");
 
 struct TcArgs {
@@ -77,10 +76,18 @@ struct TcArgs {
   float alpha;
 };
 
+// O / N_u leaves through its own staging area (so the next unit's Q and K/V can land while
+// the epilogue runs): at most two heads at a time, each as two boxes of 128 rows x 32 fp32.
+constexpr uint32_t kBox = kBM * 128;  // one 32-column box of the tile
+template <int R>
+constexpr int heads_per_round() { return R < 2 ? R : 2; }
+template <int R>
+constexpr uint32_t stage_off() { return (uint32_t)R * kQBytes + 2 * kStages * kKVBytes; }
 template <int R>
 constexpr size_t tc_smem_bytes() {
-  return (size_t)R * kQBytes + 2 * kStages * kKVBytes + 1024;
+  return stage_off<R>() + (size_t)heads_per_round<R>() * 2 * kBox + 1024;
 }
+static_assert(tc_smem_bytes<4>() + 1024 <= 227 * 1024, "shared memory per CTA");
 
 // SiLU of 32 scores of one row (one TMEM chunk), masked, split into bf16 hi/lo
 // pairs: P = SiLU(alpha s) = h + h tanh(h), h = alpha s / 2.  Scalar fp32 math:
@@ -107,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a, TcArgs p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_o, bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_qe, bar_o, bar_drain;
   __shared__ __align__(8) uint64_t bar_kv_full[kStages], bar_kv_empty[kStages];
   __shared__ __align__(8) uint64_t bar_s_full[kSBuf], bar_p_full[kSBuf];
   __shared__ uint32_t s_tmem;
@@ -134,6 +141,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t sV = sK + kStages * kKVBytes;
 
   const uint32_t b_q = smem_addr(&bar_q), b_o = smem_addr(&bar_o), b_drain = smem_addr(&bar_drain);
+  const uint32_t b_qe = smem_addr(&bar_qe);  // the unit's last S has read the Q tiles
   auto b_kvf = [&](int s) { return smem_addr(&bar_kv_full[s]); };
   auto b_kve = [&](int s) { return smem_addr(&bar_kv_empty[s]); };
   auto b_sf = [&](int b) { return smem_addr(&bar_s_full[b]); };
@@ -145,6 +153,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(b_q, 1);
     mbar_init(b_o, 1);
     mbar_init(b_drain, 1);
+    mbar_init(b_qe, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(b_kvf(s), 1);
       mbar_init(b_kve(s), 1);
@@ -174,6 +183,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // Barrier phases run on across units: K/V stages count key blocks, S/P
   // buffers count steps, Q and O count units, all from the start of the CTA.
   int blk_base = 0, step_base = 0, unit_iter = 0;
+  // producer (warp 0, lane 0): the next unit's Q and first n_pre K/V blocks were loaded
+  // during the current unit; Q loads and K/V blocks issued so far (for the final drain)
+  bool q_pre = false;
+  int n_pre = 0, nq_loads = 0, g_next = 0;  // g_next: 1 + the last K/V block loaded
   for (;;) {
     const int w = s_ticket[unit_iter & 1];  // written before the last block-wide barrier
     if (w >= n_work) break;
@@ -197,13 +210,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp == 0) {
       // ----------------------------------------------------------- producer
       if (lane == 0) {
-        mbar_expect_tx(b_q, R * kQBytes);  // Q of the previous unit was consumed before the unit barrier
-        for (int hh = 0; hh < R; ++hh)
-          if (MTFM_INBOUNDS(hdr, tma_x_ok((g * R + hh) * kDH, kDH, ldq, 2) && q0 < nq && qrow0 + q0 >= 0 &&
-                                     qrow0 + q0 < hdr->total_tokens))
-            tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
-        int issued = 0;
-        for (int bi = 0; bi < n_blocks; ++bi) {
+        if (!q_pre) {
+          mbar_expect_tx(b_q, R * kQBytes);
+          for (int hh = 0; hh < R; ++hh)
+            if (MTFM_INBOUNDS(hdr, tma_x_ok((g * R + hh) * kDH, kDH, ldq, 2) && q0 < nq && qrow0 + q0 >= 0 &&
+                                       qrow0 + q0 < hdr->total_tokens))
+              tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g * R + hh) * kDH, qrow0 + q0);
+          ++nq_loads;
+        }
+        int issued = n_pre;  // blocks [0, n_pre) were loaded during the previous unit
+        for (int bi = n_pre; bi < n_blocks; ++bi) {
           const int G = blk_base + bi, s = G % kStages;
           if (G >= kStages && !mbar_wait(b_kve(s), ((G / kStages) - 1) & 1, abort_flag)) break;
           const int row = so + block_of(bi) * kBN;
@@ -214,35 +230,46 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g * kDH, row);
           }
           ++issued;
+          g_next = G + 1;
         }
         // the next pair, read by every role after this unit's closing barrier
         const int w1 = (int)atomicAdd(ticket_ctr, 1u);
         s_ticket[(unit_iter + 1) & 1] = w1;
-        if (w1 < n_work) {
-          // its Q tiles and first K/V blocks into L2 now, so that its loads after the unit
-          // barrier do not wait for DRAM
+        q_pre = false;
+        n_pre = 0;
+        if (w1 < n_work && issued == n_blocks) {
+          // Its Q tiles and first K/V blocks go into shared memory now, so that they are in
+          // place when this unit's barrier releases: Q once this unit's last S has read the
+          // Q tiles, K/V blocks as this unit's last PVs free the ring's stages.
           const int item1 = w1 / p.hkv, g1 = w1 % p.hkv;
           const WorkItem it1 = m.items_full[item1];
           const int u1 = it1.user;
           const int LH1 = m.lh[u1], LR1 = m.lr[u1], N1 = LH1 + LR1 + m.lt[u1], so1 = m.seq_off[u1];
-          for (int hh = 0; hh < R; ++hh) tma_prefetch_l2_2d(&tm_q, (g1 * R + hh) * kDH, so1 + it1.tile * kBM);
-          const KeyBlocks kb1 = key_blocks(it1.kv_max, LH1, LR1, N1, 0, it1.tile * kBM, p.v2);
-          for (int bi = 0; bi < min(kb1.n_blocks, kStages); ++bi) {
-            const int row1 = so1 + kb1.block(bi) * kBN;
-            tma_prefetch_l2_2d(&tm_k, g1 * kDH, row1);
-            tma_prefetch_l2_2d(&tm_v, g1 * kDH, row1);
+          const int q01 = it1.tile * kBM;
+          const KeyBlocks kb1 = key_blocks(it1.kv_max, LH1, LR1, N1, 0, q01, p.v2);
+          if (mbar_wait(b_qe, unit_iter & 1, abort_flag)) {
+            mbar_expect_tx(b_q, R * kQBytes);
+            for (int hh = 0; hh < R; ++hh)
+              if (MTFM_INBOUNDS(hdr, tma_x_ok((g1 * R + hh) * kDH, kDH, ldq, 2) && q01 < N1 && so1 + q01 >= 0 &&
+                                         so1 + q01 < hdr->total_tokens))
+                tma_load_2d(sQ + hh * kQBytes, &tm_q, b_q, (g1 * R + hh) * kDH, so1 + q01);
+            ++nq_loads;
+            q_pre = true;
+            for (int bi = 0; bi < min(kb1.n_blocks, kStages); ++bi) {
+              const int G = blk_base + n_blocks + bi, s = G % kStages;
+              if (G >= kStages && !mbar_wait(b_kve(s), ((G / kStages) - 1) & 1, abort_flag)) break;
+              const int row1 = so1 + kb1.block(bi) * kBN;
+              mbar_expect_tx(b_kvf(s), 2 * kKVBytes);
+              if (MTFM_INBOUNDS(hdr, tma_x_ok(g1 * kDH, kDH, p.hkv * kDH, 2) && kb1.block(bi) >= 0 &&
+                                         kb1.block(bi) * kBN < N1 && row1 < hdr->total_tokens)) {
+                tma_load_2d(sK + s * kKVBytes, &tm_k, b_kvf(s), g1 * kDH, row1);
+                tma_load_2d(sV + s * kKVBytes, &tm_v, b_kvf(s), g1 * kDH, row1);
+              }
+              ++n_pre;
+              g_next = G + 1;
+            }
           }
         }
-        // Wait (bounded, regardless of abort) for the last copy of every stage and Q:
-        // no TMA write may land after this unit's barriers are re-armed or the CTA leaves.
-        const long long t0 = clock64();
-        auto drain_wait = [&](uint32_t bar, uint32_t par) {
-          while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
-          }
-        };
-        drain_wait(b_q, unit_iter & 1);
-        for (int bi = max(0, issued - kStages); bi < issued; ++bi)
-          drain_wait(b_kvf((blk_base + bi) % kStages), ((blk_base + bi) / kStages) & 1);
       }
     } else if (warp == 1) {
       // ----------------------------------------------------------- MMA issuer
@@ -269,6 +296,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int kk = 0; kk < kDH / 16; ++kk)
             mma_ss2(d, a0 + kk * 2, dhi, b0 + kk * 2, dhi, idesc_qk, kk > 0 ? 1u : 0u);
           mma_commit(b_sf(gb));
+          if (n == total - 1) mma_commit(b_qe);  // the producer may load the next unit's Q
         }
         __syncwarp();
         return true;
@@ -302,6 +330,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncwarp();
       }
       if (elect_one()) {
+        if (ok && total == 0) mma_commit(b_qe);  // (no S at all: Q was never read)
         // on failure, drain every MMA issued so far before TMEM is reused or released
         mma_commit(ok ? b_o : b_drain);
       }
@@ -384,64 +413,66 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
               *reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + qi) * ldq + (g * R + hh) * kDH + c) =
                   make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      // O / N_u goes through shared memory (the Q and K/V buffers are idle once every MMA
-      // of the unit is done), as 2R boxes of 128 rows x 32 fp32 columns in the layout of
-      // the A tensor map (16-byte chunks XOR-swizzled by row).  A tile whose 128 rows all
-      // belong to its user then goes out as 2R TMA stores issued by one thread: the SiLU
-      // warps only wait until the TMA engine has read the staging tile, not for the
-      // global writes.  A tile that ends past its user's last row is stored row by row
-      // from the staging tile (valid rows only).  The named barrier is reached by all 16
-      // SiLU warps, also after an abort, so it cannot hang.
+      // O / N_u goes out through the staging area, heads_per_round heads at a time, as
+      // boxes of 128 rows x 32 fp32 columns in the layout of the A tensor map (16-byte
+      // chunks XOR-swizzled by row).  A tile whose 128 rows all belong to its user goes out
+      // as TMA stores issued by one thread: the SiLU warps only wait until the TMA engine
+      // has read the staging area, not for the global writes.  A tile that ends past its
+      // user's last row is stored row by row from the staging area (valid rows only).
+      // The named barriers are reached by all 16 SiLU warps, also after an abort.
       const bool have = ok && total > 0;
-      uint8_t* stage = smem;
-      constexpr uint32_t kBox = kBM * 128;  // one 32-column box of the tile
-      if (have) {
-        tc_fence_after();
-        const float inv_n = 1.f / (float)N;
-        for (int hh = wg; hh < R; hh += kSiluWG) {
+      constexpr int kHR = heads_per_round<R>();
+      uint8_t* stage = smem + stage_off<R>();
+      const uint32_t s_stage = sQ + stage_off<R>();
+      if (have) tc_fence_after();
+      const float inv_n = 1.f / (float)N;
+      for (int rd = 0; rd < R / kHR; ++rd) {
+        if (threadIdx.x == 128) bulk_wait_read<0>();  // the previous stores have read the area
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
+        const int hh = wg;  // this warpgroup's head (R = 4), or none (wg >= R)
+        if (have && hh < R && hh / kHR == rd) {
 #pragma unroll
           for (int c = 0; c < kDH / 32; ++c) {
             uint32_t raw[32];
             tmem_ld32(lane_base + hh * kDH + c * 32, raw);
             tmem_ld_wait();
-            uint8_t* rowp = stage + (hh * 2 + c) * kBox + row * 128;
+            uint8_t* rowp = stage + ((hh % kHR) * 2 + c) * kBox + row * 128;
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               *reinterpret_cast<float4*>(rowp + ((e ^ (row & 7)) << 4)) =
                   make_float4(__uint_as_float(raw[4 * e]) * inv_n, __uint_as_float(raw[4 * e + 1]) * inv_n,
                               __uint_as_float(raw[4 * e + 2]) * inv_n, __uint_as_float(raw[4 * e + 3]) * inv_n);
           }
+          fence_proxy_async();  // the staged tile is read by the TMA engine
         }
-        fence_proxy_async();  // the staged tile is read by the TMA engine
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
-      if (have) {
-        const uint64_t keep_a = l2_evict_last();  // the gate reads A next: keep it in L2
-        if (q0 + kBM <= nq) {
-          if (threadIdx.x == 128) {
-            for (int b = 0; b < 2 * R; ++b)
-              if (MTFM_INBOUNDS(hdr, tma_x_ok(g * R * kDH + b * 32, 32, ldq, 4) && qrow0 + q0 >= 0 &&
-                                         qrow0 + q0 + kBM <= hdr->total_tokens))
-                tma_store_2d_hint(&tm_a, sQ + b * kBox, g * R * kDH + b * 32, qrow0 + q0, keep_a);
-            bulk_commit();
-            bulk_wait_read<0>();  // the next unit's loads may overwrite the staging area
-          }
-        } else {
-          const int sw = warp - 4;  // rows [8 sw, 8 sw + 8) of the tile
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
+        if (have) {
+          const uint64_t keep_a = l2_evict_last();  // the gate reads A next: keep it in L2
+          const int col0 = (g * R + rd * kHR) * kDH;  // first column of this round's heads
+          if (q0 + kBM <= nq) {
+            if (threadIdx.x == 128) {
+              for (int b = 0; b < 2 * kHR; ++b)
+                if (MTFM_INBOUNDS(hdr, tma_x_ok(col0 + b * 32, 32, ldq, 4) && qrow0 + q0 >= 0 &&
+                                           qrow0 + q0 + kBM <= hdr->total_tokens))
+                  tma_store_2d_hint(&tm_a, s_stage + b * kBox, col0 + b * 32, qrow0 + q0, keep_a);
+              bulk_commit();
+            }
+          } else {
+            const int sw = warp - 4;  // rows [8 sw, 8 sw + 8) of the tile
 #pragma unroll 1
-          for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
-            if (q0 + rr >= nq) break;
-            if (!MTFM_INBOUNDS(hdr, qrow0 + q0 + rr < hdr->total_tokens)) break;
-            float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + g * R * kDH);
-            for (int f = lane; f < R * kDH / 4; f += 32) {
-              const float4 v =
-                  *reinterpret_cast<const float4*>(stage + (f / 8) * kBox + rr * 128 + (((f % 8) ^ (rr & 7)) << 4));
-              st_f4_hint(dst + f, v, keep_a);
+            for (int rr = sw * (kBM / 16); rr < (sw + 1) * (kBM / 16); ++rr) {
+              if (q0 + rr >= nq) break;
+              if (!MTFM_INBOUNDS(hdr, qrow0 + q0 + rr < hdr->total_tokens)) break;
+              float4* dst = reinterpret_cast<float4*>(p.a + (size_t)(qrow0 + q0 + rr) * ldq + col0);
+              for (int f = lane; f < kHR * kDH / 4; f += 32) {
+                const float4 v =
+                    *reinterpret_cast<const float4*>(stage + (f / 8) * kBox + rr * 128 + (((f % 8) ^ (rr & 7)) << 4));
+                st_f4_hint(dst + f, v, keep_a);
+              }
             }
           }
         }
       }
-      fence_proxy_async();  // the next unit's TMA writes overwrite the staged rows
     }
     tc_fence_before();
     __syncthreads();
@@ -451,6 +482,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     ++unit_iter;
   }
   pdl_trigger();
+  if (warp == 0 && lane == 0) {
+    // no TMA write may land after the CTA leaves (loads run ahead across units, and an
+    // abort leaves some unconsumed): wait, bounded, for the last load of Q and of each stage
+    const long long t0 = clock64();
+    auto drain_wait = [&](uint32_t bar, uint32_t par) {
+      while (!mbar_try(bar, par) && clock64() - t0 < kWaitCycles) {
+      }
+    };
+    if (nq_loads > 0) drain_wait(b_q, (nq_loads - 1) & 1);
+    for (int G = max(0, g_next - kStages); G < g_next; ++G) drain_wait(b_kvf(G % kStages), (G / kStages) & 1);
+  }
   if (threadIdx.x == 128) bulk_wait<0>();  // every TMA store has completed before the CTA leaves
   if (warp == 1) {
     __syncwarp();
