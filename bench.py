@@ -280,11 +280,13 @@ def run_mtfm(args, rank, world, local_rank):
     stream = torch.cuda.Stream(dev)
     launches_per_step = 7   # pack (2 kernels), Full attention, Full gate, Target clear, Target attention, Target gate
 
-    def step(i, record=None, around_full=None, around_tgt=None):
+    def step(i, record=None, around_full=None, around_tgt=None, around_pack=None):
         s = sets[i % len(sets)]
         e = record
         if e: e[0].record(stream)
+        if around_pack: around_pack[0].record(stream)
         M.pack(cfg, *lens, meta, stream)
+        if around_pack: around_pack[1].record(stream)
         if e: e[1].record(stream)
         if around_full: around_full[0].record(stream)
         M.attn_full(cfg, meta, s["q"], s["k"], s["v"], A_f, stream)
@@ -322,11 +324,13 @@ def run_mtfm(args, rank, world, local_rank):
 
     mk = lambda: [(torch.cuda.Event(enable_timing=True, external=True),
                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(nset)]
-    full_ev, tgt_ev = mk(), mk()
+    full_ev, tgt_ev, pack_ev = mk(), mk(), mk()
     g_all = capture(lambda: [step(r) for r in range(nset)])
-    g_ev = capture(lambda: [step(r, around_full=full_ev[r], around_tgt=tgt_ev[r]) for r in range(nset)])
+    g_ev = capture(lambda: [step(r, around_full=full_ev[r], around_tgt=tgt_ev[r], around_pack=pack_ev[r])
+                            for r in range(nset)])
     singles = [capture(lambda r=r: step(r)) for r in range(nset)]
-    singles_ev = [capture(lambda r=r: step(r, around_full=full_ev[r], around_tgt=tgt_ev[r])) for r in range(nset)]
+    singles_ev = [capture(lambda r=r: step(r, around_full=full_ev[r], around_tgt=tgt_ev[r], around_pack=pack_ev[r]))
+                  for r in range(nset)]
     reps, rem = divmod(args.steps, nset)
     with torch.cuda.stream(stream):
         for _ in range(max(1, 3 // nset + 1)):
@@ -336,7 +340,7 @@ def run_mtfm(args, rank, world, local_rank):
     sampler = ClockSampler(dev) if rank == 0 else None
     # The K-step region is timed `repeats` times (each bracketed by a barrier and a
     # synchronize on both sides); the value is the median region, the spread is reported.
-    region_ms, full_runs, tgt_runs = [], [], []
+    region_ms, full_runs, tgt_runs, pack_runs = [], [], [], []
     if sampler:
         sampler.begin()
     for _ in range(max(1, args.repeats)):
@@ -359,10 +363,12 @@ def run_mtfm(args, rank, world, local_rank):
         n_timed = nset if reps > 0 else rem
         full_runs += [a.elapsed_time(z) for a, z in full_ev[:n_timed]]
         tgt_runs += [a.elapsed_time(z) for a, z in tgt_ev[:n_timed]]
+        pack_runs += [a.elapsed_time(z) for a, z in pack_ev[:n_timed]]
     clocks = sampler.stop() if sampler else None
     ms_total = statistics.median(region_ms)
     full_ms = statistics.median(full_runs)
     tgt_ms = statistics.median(tgt_runs)
+    pack_ms = statistics.median(pack_runs)
     M.pack_check(meta, stream)
 
     # Per-part times from a separate eager pass with an event between launches (the events
@@ -426,6 +432,7 @@ def run_mtfm(args, rank, world, local_rank):
                            "attn_timing": "event-record nodes around the Target attention call (conditional "
                                           "accumulator clear + kernel) inside the timed region",
                            "users_per_s": round(b.B / ((ms_parts["target_attn"] + ms_parts["target_gate"]) * 1e-3), 1)},
+                "pack_ms_in_graph": round(pack_ms, 5),
                 "ms_parts": {k: round(v, 5) for k, v in ms_parts.items()},
                 "ms_parts_note": "eager pass with an event between launches (not the graph-replayed step)",
             },

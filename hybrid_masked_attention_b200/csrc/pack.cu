@@ -30,31 +30,46 @@ namespace {
 constexpr int kPackThreads = 1024;
 constexpr int kSortMax = 8192;  // users sorted by length when B <= this; natural order beyond
 
-// Block-wide exclusive scan of one int64 value per thread; returns the prefix and the total.
-__device__ long long block_exclusive_scan(long long v, long long* total, long long* s_warp) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  long long x = v;
+// Block-wide exclusive scan of K int64 values per thread at once (one round of
+// barriers for all K); v is replaced by its prefix, total[] receives the totals.
+// s_warp holds 32 * K values.
+template <int K>
+__device__ void block_exclusive_scan_k(long long (&v)[K], long long (&total)[K], long long* s_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  long long x[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) x[k] = v[k];
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    long long y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const long long y = __shfl_up_sync(0xffffffffu, x[k], o);
+      if (lane >= o) x[k] += y;
+    }
   }
-  if (lane == 31) s_warp[warp] = x;
+  if (lane == 31)
+#pragma unroll
+    for (int k = 0; k < K; ++k) s_warp[k * 32 + warp] = x[k];
   __syncthreads();
   if (warp == 0) {
-    long long w = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      long long y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
+    for (int k = 0; k < K; ++k) {
+      long long w = lane < nw ? s_warp[k * 32 + lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_warp[k * 32 + lane] = w;  // inclusive prefix over warps
     }
-    s_warp[lane] = w;  // inclusive prefix over warps
   }
   __syncthreads();
-  long long before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
-  *total = s_warp[(blockDim.x >> 5) - 1];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    total[k] = s_warp[k * 32 + nw - 1];
+    v[k] = (warp > 0 ? s_warp[k * 32 + warp - 1] : 0) + x[k] - v[k];
+  }
   __syncthreads();
-  return before;
 }
 
 __global__ void __launch_bounds__(kPackThreads)
@@ -62,7 +77,7 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
                   int max_if, int max_it, int sort_n, const int32_t* __restrict__ lh,
                   const int32_t* __restrict__ lr, const int32_t* __restrict__ lt) {
   extern __shared__ unsigned long long s_keys[];  // [sort_n] (0 when not sorting)
-  __shared__ long long s_warp[32];
+  __shared__ long long s_warp[32 * 3];
   __shared__ int s_err;
   pdl_wait();  // the previous work on the stream may still read this metadata block
   pdl_trigger();
@@ -87,10 +102,10 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
   if (err) atomicOr(&s_err, kErrBadLengths);
 
   // 2. offsets
-  long long totN, totR, totT;
-  long long pN = block_exclusive_scan(sN, &totN, s_warp);
-  long long pR = block_exclusive_scan(sR, &totR, s_warp);
-  long long pT = block_exclusive_scan(sT, &totT, s_warp);
+  long long off[3] = {sN, sR, sT}, tot[3];
+  block_exclusive_scan_k<3>(off, tot, s_warp);
+  long long pN = off[0], pR = off[1], pT = off[2];
+  const long long totN = tot[0], totR = tot[1], totT = tot[2];
   if (tid == 0 && (totN != total_tokens || totR != total_r || totT != total_t))
     atomicOr(&s_err, kErrBadLengths);
   __syncthreads();
@@ -176,9 +191,10 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
     cF += (n + kTileM - 1) / kTileM;
     cT += (lt[u] + kTileM - 1) / kTileM;
   }
-  long long totF, totTT;
-  long long oF = block_exclusive_scan(cF, &totF, s_warp);
-  long long oT = block_exclusive_scan(cT, &totTT, s_warp);
+  long long oft[2] = {cF, cT}, tot2[2];
+  block_exclusive_scan_k<2>(oft, tot2, s_warp);
+  long long oF = oft[0], oT = oft[1];
+  const long long totF = tot2[0], totTT = tot2[1];
   for (int p = b0; p < b1; ++p) {
     int u = user_at(p);
     int n = lh[u] + lr[u] + lt[u];
@@ -239,7 +255,8 @@ __device__ __forceinline__ int count_below(const int64_t* __restrict__ ts, int n
 // place: unit_off[i] becomes the first unit of item i; n_units_target the total.
 // Run by one whole CTA (the last CTA of pack_rows_kernel to finish).
 __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
-  __shared__ long long s_warp[32];
+  constexpr int kCand = 5;  // chunk sizes kTargetUnitBlocks .. kTargetUnitBlocks + 4
+  __shared__ long long s_warp[32 * (kCand + 1)];
   __shared__ int s_chunk;
   MetaHeader* hdr = m.hdr;
   const int n = hdr->n_items_target;
@@ -247,85 +264,83 @@ __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
   const int per = (n + nthr - 1) / nthr;
   const int a = min(n, (int)threadIdx.x * per), b = min(n, a + per);
   volatile int* uo = m.unit_off;  // written by other CTAs: read past L1
-  long long steps = 0;             // sub-tile key blocks of my items
+  volatile int* uc = m.unit_off_c;
+  __shared__ int s_maxnb[2];      // the most key blocks of an item, per table
+  if (threadIdx.x < 2) s_maxnb[threadIdx.x] = 0;
+  __syncthreads();
+  // one pass over my items: sub-tile key blocks, and units for each candidate chunk
+  long long acc[kCand + 1], tot[kCand + 1];
+#pragma unroll
+  for (int k = 0; k <= kCand; ++k) acc[k] = 0;
+  int maxnb = 0, maxnb_c = 0;
   for (int i = a; i < b; ++i) {
     const int v = uo[i + 1];
-    steps += (long long)(v >> 16) * (v & 0xffff);
+    const int nsub = v >> 16, nb = v & 0xffff;
+    maxnb = max(maxnb, nb);
+    maxnb_c = max(maxnb_c, uc[i + 1] & 0xffff);
+    acc[0] += (long long)nsub * nb;
+#pragma unroll
+    for (int k = 0; k < kCand; ++k) {
+      const int c = kTargetUnitBlocks + k;
+      acc[k + 1] += (long long)nsub * ((nb + c - 1) / c);
+    }
   }
-  long long total_steps;
-  block_exclusive_scan(steps, &total_steps, s_warp);
+  if (maxnb > 0) atomicMax(&s_maxnb[0], maxnb);
+  if (maxnb_c > 0) atomicMax(&s_maxnb[1], maxnb_c);
+  block_exclusive_scan_k<kCand + 1>(acc, tot, s_warp);  // (its barriers also publish s_maxnb)
   if (threadIdx.x == 0) {
+    const long long total_steps = tot[0];
     const long long target_units = (long long)kTargetUnitsPerSM * n_sm;
     const long long c = (total_steps * hkv + target_units - 1) / target_units;
-    s_chunk = (int)max((long long)kTargetUnitBlocks, min(c, (long long)1 << 20));
-  }
-  __syncthreads();
-  auto units_for = [&](int c) -> long long {  // whole CTA
-    long long local = 0;
-    for (int i = a; i < b; ++i) {
-      const int v = uo[i + 1];
-      local += (long long)(v >> 16) * (((v & 0xffff) + c - 1) / c);
-    }
-    long long total;
-    block_exclusive_scan(local, &total, s_warp);
-    return total;
-  };
-  if (s_chunk == kTargetUnitBlocks) {  // uniform: a short layer
-    // The CTAs (one per SM) take the units in rounds.  With three rounds or fewer a sparse
-    // last round is a large share of the launch: take the C in [kTargetUnitBlocks,
-    // kTargetUnitBlocks + 4] with the fewest rounds x (C - 1) block-steps (a unit's first
-    // block overlaps the previous unit's epilogue; measured on the pair batch: 26.8 -> 22.8 us).
-    const long long r0 = (units_for(kTargetUnitBlocks) * hkv + n_sm - 1) / n_sm;
-    if (r0 <= 3) {
-      long long best = r0 * (kTargetUnitBlocks - 1);
-      int best_c = kTargetUnitBlocks;
-      for (int c = kTargetUnitBlocks + 1; c <= kTargetUnitBlocks + 4; ++c) {
-        const long long cost = (units_for(c) * hkv + n_sm - 1) / n_sm * (c - 1);
-        if (cost < best) {
-          best = cost;
-          best_c = c;
+    int chunk = (int)max((long long)kTargetUnitBlocks, min(c, (long long)1 << 20));
+    if (chunk == kTargetUnitBlocks) {  // a short layer
+      // The CTAs (one per SM) take the units in rounds.  With three rounds or fewer a
+      // sparse last round is a large share of the launch: take the C in [kTargetUnitBlocks,
+      // kTargetUnitBlocks + 4] with the fewest rounds x (C - 1) block-steps (a unit's first
+      // block overlaps the previous unit's epilogue; measured on the pair batch: 26.8 -> 22.8 us).
+      const long long r0 = (tot[1] * hkv + n_sm - 1) / n_sm;
+      if (r0 <= 3) {
+        long long best = r0 * (kTargetUnitBlocks - 1);
+        for (int k = 1; k < kCand; ++k) {
+          const int cc = kTargetUnitBlocks + k;
+          const long long cost = (tot[k + 1] * hkv + n_sm - 1) / n_sm * (cc - 1);
+          if (cost < best) {
+            best = cost;
+            chunk = cc;
+          }
         }
       }
-      if (threadIdx.x == 0) s_chunk = best_c;
-      __syncthreads();
     }
+    s_chunk = chunk;
   }
+  __syncthreads();
   const int C = s_chunk;
   // whether every item's key range fits in one chunk (the blocks of a table's items <= C)
-  __shared__ int s_multi[2];
-  if (threadIdx.x < 2) s_multi[threadIdx.x] = 0;
-  __syncthreads();
+  const bool multi = s_maxnb[0] > C, multi_c = s_maxnb[1] > C;
+  // sub-tiles x ceil(blocks / C) units per item, both tables scanned in place (one
+  // round) into first-unit offsets
+  auto units_of = [&](int v) { return (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C); };
+  long long run[2] = {0, 0}, tot2[2];
   for (int i = a; i < b; ++i) {
-    if ((uo[i + 1] & 0xffff) > C) s_multi[0] = 1;
-    if ((m.unit_off_c[i + 1] & 0xffff) > C) s_multi[1] = 1;
+    run[0] += units_of(uo[i + 1]);
+    run[1] += units_of(uc[i + 1]);
   }
-  __syncthreads();
-  // sub-tiles x ceil(blocks / C) units per item, scanned in place into first-unit offsets
-  auto scan_units = [&](volatile int* arr) -> long long {
-    long long local = 0;
-    for (int i = a; i < b; ++i) {
-      const int v = arr[i + 1];
-      local += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
-    }
-    long long total;
-    long long run = block_exclusive_scan(local, &total, s_warp);
-    for (int i = a; i < b; ++i) {
-      const int v = arr[i + 1];
-      run += (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C);
-      arr[i + 1] = (int)run;
-    }
-    return total;
-  };
-  const long long total = scan_units(uo);
-  const long long total_c = scan_units(m.unit_off_c);
+  block_exclusive_scan_k<2>(run, tot2, s_warp);
+  for (int i = a; i < b; ++i) {
+    run[0] += units_of(uo[i + 1]);
+    uo[i + 1] = (int)run[0];
+    run[1] += units_of(uc[i + 1]);
+    uc[i + 1] = (int)run[1];
+  }
+  const long long total = tot2[0], total_c = tot2[1];
   if (threadIdx.x == 0) {
     uo[0] = 0;
     m.unit_off_c[0] = 0;
     hdr->n_units_target = (int)total;
     hdr->n_units_target_c = (int)total_c;
     hdr->tgt_chunk_blocks = C;
-    hdr->tgt_single[0] = s_multi[0] ? 0 : 1;
-    hdr->tgt_single[1] = s_multi[1] ? 0 : 1;
+    hdr->tgt_single[0] = multi ? 0 : 1;
+    hdr->tgt_single[1] = multi_c ? 0 : 1;
   }
 }
 
