@@ -162,20 +162,45 @@ pack_users_kernel(MetaView m, int B, int total_tokens, int total_r, int total_t,
       s_keys[i] = key;
     }
     __syncthreads();
-    for (int size = 2; size <= sort_n; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < sort_n; i += nthr) {
-          int j = i ^ stride;
-          if (j > i) {
-            bool desc = (i & size) == 0;
-            unsigned long long a = s_keys[i], b = s_keys[j];
-            if ((a < b) == desc) {
-              s_keys[i] = b;
-              s_keys[j] = a;
+    if (sort_n <= nthr) {
+      // one key per thread, held in a register: partners closer than a warp swap through
+      // shuffles, farther ones through shared memory (one barrier pair per such round)
+      unsigned long long x = tid < sort_n ? s_keys[tid] : 0;
+      for (int size = 2; size <= sort_n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          unsigned long long y;
+          if (stride >= 32) {
+            __syncthreads();
+            if (tid < sort_n) s_keys[tid] = x;
+            __syncthreads();
+            y = tid < sort_n ? s_keys[tid ^ stride] : 0;
+          } else {
+            y = __shfl_xor_sync(0xffffffffu, x, stride);
+          }
+          // the lower index of a pair keeps the larger key where the run descends
+          const bool keep_max = ((tid & size) == 0) == ((tid & stride) == 0);
+          x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+        }
+      }
+      __syncthreads();
+      if (tid < sort_n) s_keys[tid] = x;
+      __syncthreads();
+    } else {
+      for (int size = 2; size <= sort_n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          for (int i = tid; i < sort_n; i += nthr) {
+            int j = i ^ stride;
+            if (j > i) {
+              bool desc = (i & size) == 0;
+              unsigned long long a = s_keys[i], b = s_keys[j];
+              if ((a < b) == desc) {
+                s_keys[i] = b;
+                s_keys[j] = a;
+              }
             }
           }
+          __syncthreads();
         }
-        __syncthreads();
       }
     }
   }
@@ -273,11 +298,33 @@ __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
 #pragma unroll
   for (int k = 0; k <= kCand; ++k) acc[k] = 0;
   int maxnb = 0, maxnb_c = 0;
+  // my first kCache items' entries stay in registers for the later passes
+  constexpr int kCache = 4;
+  int c0[kCache], c1[kCache];
+#pragma unroll
+  for (int j = 0; j < kCache; ++j) {
+    c0[j] = a + j < b ? uo[a + j + 1] : 0;
+    c1[j] = a + j < b ? uc[a + j + 1] : 0;
+  }
+  auto ent0 = [&](int i) -> int {  // uo[i + 1], from registers where cached
+    int v = 0;
+#pragma unroll
+    for (int j = 0; j < kCache; ++j)
+      if (i == a + j) v = c0[j];
+    return i < a + kCache ? v : uo[i + 1];
+  };
+  auto ent1 = [&](int i) -> int {
+    int v = 0;
+#pragma unroll
+    for (int j = 0; j < kCache; ++j)
+      if (i == a + j) v = c1[j];
+    return i < a + kCache ? v : uc[i + 1];
+  };
   for (int i = a; i < b; ++i) {
-    const int v = uo[i + 1];
+    const int v = ent0(i);
     const int nsub = v >> 16, nb = v & 0xffff;
     maxnb = max(maxnb, nb);
-    maxnb_c = max(maxnb_c, uc[i + 1] & 0xffff);
+    maxnb_c = max(maxnb_c, ent1(i) & 0xffff);
     acc[0] += (long long)nsub * nb;
 #pragma unroll
     for (int k = 0; k < kCand; ++k) {
@@ -322,14 +369,14 @@ __device__ void scan_target_units(MetaView m, int hkv, int n_sm) {
   auto units_of = [&](int v) { return (long long)(v >> 16) * (((v & 0xffff) + C - 1) / C); };
   long long run[2] = {0, 0}, tot2[2];
   for (int i = a; i < b; ++i) {
-    run[0] += units_of(uo[i + 1]);
-    run[1] += units_of(uc[i + 1]);
+    run[0] += units_of(ent0(i));
+    run[1] += units_of(ent1(i));
   }
   block_exclusive_scan_k<2>(run, tot2, s_warp);
   for (int i = a; i < b; ++i) {
-    run[0] += units_of(uo[i + 1]);
-    uo[i + 1] = (int)run[0];
-    run[1] += units_of(uc[i + 1]);
+    run[0] += units_of(ent0(i));
+    run[1] += units_of(ent1(i));
+    uo[i + 1] = (int)run[0];  // (item i's entry was read above: in place is safe)
     uc[i + 1] = (int)run[1];
   }
   const long long total = tot2[0], total_c = tot2[1];
@@ -467,8 +514,9 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
     attr_set = true;
   }
   const int tsr = target_sub_rows(cfg.hq, cfg.hkv);
-  // one thread per user up to kPackThreads (cheaper block barriers for small batches)
-  const int threads = std::min(kPackThreads, std::max(64, (cfg.batch + 31) / 32 * 32));
+  // one thread per user (and per sort key) up to kPackThreads (cheaper block barriers for
+  // small batches)
+  const int threads = std::min(kPackThreads, std::max(std::max(64, sort_n), (cfg.batch + 31) / 32 * 32));
   cudaError_t e = launch_pdl(pack_users_kernel, dim3(1), dim3(threads), smem, st, m, cfg.batch, cfg.total_tokens,
                              cfg.total_r, cfg.total_t, cfg.v2_subtokens, tsr, L.max_items_full,
                              L.max_items_target, sort_n, lh, lr, lt);
