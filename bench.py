@@ -683,14 +683,14 @@ def _packed(M, b, heads, dev):
     return cfg, s, lens
 
 
-def sweep_entry(dev, N, v2, steps, warmup, repeats, heads=syn.PAIR_HEADS):
-    """Sequence-length sweep point: 2^21 tokens of users of N tokens each (H:R:T ~ 70:15:15; V2:
-    targets of 4 sub-tokens).  A step is the pair step's path at this shape: pack, Full attention
+def sweep_entry(dev, N, v2, steps, warmup, repeats, heads=syn.PAIR_HEADS, total_tokens=1 << 21):
+    """Sequence-length sweep point: 2^21 tokens (or total_tokens, for smaller profiling runs) of
+    users of N tokens each (H:R:T ~ 70:15:15; V2: targets of 4 sub-tokens).  A step is the pair step's path at this shape: pack, Full attention
     + gate, Target attention + gate.  Activations are seeded device-side N(0, 1) bf16 (GBs, far
     larger than L2)."""
     import torch
     import hybrid_masked_attention_b200 as M
-    b = syn.sweep_batch(N, v2=v2, seed=1003)
+    b = syn.sweep_batch(N, v2=v2, total_tokens=total_tokens, seed=1003)
     cfg, s, lens = _packed(M, b, heads, dev)
     rnd = _dev_inputs(dev, 1003)
     Nt, T, D, Dkv = b.total_tokens, b.total_t, heads.dq, heads.dkv
@@ -926,7 +926,7 @@ def run_workload(args):
     heads = syn.Heads(*(int(x) for x in args.heads.split(",")))
     steps = max(1, args.steps)
     if args.workload == "sweep":
-        e = sweep_entry(dev, args.seqlen, args.v2, steps, args.warmup, args.repeats, heads)
+        e = sweep_entry(dev, args.seqlen, args.v2, steps, args.warmup, args.repeats, heads, args.tokens)
     elif args.workload == "train":
         e = train_entry(dev, args.users or 96, steps, args.warmup, args.repeats, heads)
     elif args.workload == "v2layer":
@@ -1042,6 +1042,8 @@ def main():
     ap.add_argument("--workload", choices=["pair", "sweep", "train", "stack", "infer", "v2layer"], default="pair",
                     help="pair: the headline step; sweep/train/stack/infer: timings of the other configs")
     ap.add_argument("--seqlen", type=int, default=2048, help="sweep: tokens per user")
+    ap.add_argument("--tokens", type=int, default=1 << 21,
+                    help="sweep: total tokens (default 2^21; smaller for profiler captures)")
     ap.add_argument("--v2", action="store_true", help="sweep: V2 targets (4 sub-tokens each)")
     ap.add_argument("--dmodel", type=int, default=512, help="stack: d_model")
     ap.add_argument("--heads", default="8,2,64",
