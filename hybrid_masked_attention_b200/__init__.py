@@ -117,6 +117,8 @@ _sigs = {
     "mtfm_max_items": (ctypes.c_int32, [_CP, ctypes.c_int]),
     "mtfm_attn_full_fwd": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "mtfm_attn_target_fwd": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "mtfm_attn_full_fwd_bf16y": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "mtfm_attn_target_fwd_bf16y": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "mtfm_attn_full": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
     "mtfm_attn_target": (ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P]),
     "mtfm_attn_target_cached_fwd": (ctypes.c_int, [_CP] + [_P] * 13),
@@ -246,7 +248,7 @@ def meta_read(cfg: Config, meta: torch.Tensor, stream=None) -> dict:
     return out
 
 
-def _fwd(fn, where, cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream, rows):
+def _fwd(fn, where, cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream, rows, y_dtype=torch.float32):
     c = cfg.c()
     D, Dkv, N = cfg.D, cfg.Dkv, cfg.total_tokens
     bf = torch.bfloat16
@@ -254,7 +256,7 @@ def _fwd(fn, where, cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream, row
             _ptr(q, bf, (rows, D), "q"), _ptr(k, bf, (N, Dkv), "k"), _ptr(v, bf, (N, Dkv), "v"),
             _ptr(u, bf, (rows, D), "u"),
             _ptr(gamma, torch.float32, (3, D), "gamma"), _ptr(beta, torch.float32, (3, D), "beta"),
-            _ptr(y, torch.float32, (rows, D), "y"), _ptr(a, torch.float32, (rows, D), "a"),
+            _ptr(y, y_dtype, (rows, D), "y"), _ptr(a, torch.float32, (rows, D), "a"),
             _ptr(stats, torch.float32, (rows, 2), "stats"), _stream(stream))
     _check(st, where)
 
@@ -269,6 +271,18 @@ def attn_target_fwd(cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream=None
     """Target-Attention layer forward (T rows only)."""
     _fwd(_lib.mtfm_attn_target_fwd, "mtfm_attn_target_fwd", cfg, meta, q, k, v, u, gamma, beta, y,
          a, stats, stream, cfg.total_t)
+
+
+def attn_full_fwd_bf16y(cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream=None):
+    """attn_full_fwd with y as bf16 (the fp32 value rounded to nearest)."""
+    _fwd(_lib.mtfm_attn_full_fwd_bf16y, "mtfm_attn_full_fwd_bf16y", cfg, meta, q, k, v, u, gamma, beta, y, a,
+         stats, stream, cfg.total_tokens, torch.bfloat16)
+
+
+def attn_target_fwd_bf16y(cfg, meta, q, k, v, u, gamma, beta, y, a, stats, stream=None):
+    """attn_target_fwd with y as bf16 (the fp32 value rounded to nearest)."""
+    _fwd(_lib.mtfm_attn_target_fwd_bf16y, "mtfm_attn_target_fwd_bf16y", cfg, meta, q, k, v, u, gamma, beta, y,
+         a, stats, stream, cfg.total_t, torch.bfloat16)
 
 
 def _attn_only(fn, where, cfg, meta, q, k, v, a, stream, rows):

@@ -102,9 +102,10 @@ mtfm_status attn_only(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d
                                  static_cast<cudaStream_t>(stream)));
 }
 
+// d_y: fp32, or bf16 (round to nearest) when y_bf16.
 mtfm_status gate_fwd(const mtfm_cfg* cfg, const void* d_meta, bool target, const float* d_a,
-                     const uint16_t* d_u, const float* d_gamma, const float* d_beta, float* d_y,
-                     float* d_stats, void* stream) {
+                     const uint16_t* d_u, const float* d_gamma, const float* d_beta, void* d_y,
+                     float* d_stats, void* stream, bool y_bf16 = false) {
   Resolved r;
   mtfm_status s = resolve(cfg, &r);
   if (s != MTFM_OK) return s;
@@ -120,15 +121,19 @@ mtfm_status gate_fwd(const mtfm_cfg* cfg, const void* d_meta, bool target, const
     return MTFM_ERR_INVALID_ARG;
   const MetaLayout L = meta_layout(r.B, r.total_tokens, r.total_t);
   const MetaView m = meta_view(const_cast<void*>(d_meta), L);
-  return cuda_status(launch_gate_fwd(m, target, rows, r.D, r.eps, d_a,
-                                     reinterpret_cast<const __nv_bfloat16*>(d_u), d_gamma, d_beta,
-                                     d_y, d_stats, static_cast<cudaStream_t>(stream)));
+  const __nv_bfloat16* u = reinterpret_cast<const __nv_bfloat16*>(d_u);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (y_bf16)
+    return cuda_status(launch_gate_fwd_bf16(m, target, rows, r.D, r.eps, d_a, u, d_gamma, d_beta,
+                                            static_cast<__nv_bfloat16*>(d_y), d_stats, st));
+  return cuda_status(launch_gate_fwd(m, target, rows, r.D, r.eps, d_a, u, d_gamma, d_beta,
+                                     static_cast<float*>(d_y), d_stats, st));
 }
 
 mtfm_status attn_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
                      const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
-                     const float* d_gamma, const float* d_beta, float* d_y, float* d_a,
-                     float* d_stats, void* stream, bool target) {
+                     const float* d_gamma, const float* d_beta, void* d_y, float* d_a,
+                     float* d_stats, void* stream, bool target, bool y_bf16 = false) {
   Resolved r;
   mtfm_status s = resolve(cfg, &r);
   if (s != MTFM_OK) return s;
@@ -144,7 +149,7 @@ mtfm_status attn_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_
     return MTFM_ERR_INVALID_ARG;
   s = attn_only(cfg, d_meta, d_q, d_k, d_v, d_a, stream, target);
   if (s != MTFM_OK) return s;
-  return gate_fwd(cfg, d_meta, target, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream);
+  return gate_fwd(cfg, d_meta, target, d_a, d_u, d_gamma, d_beta, d_y, d_stats, stream, y_bf16);
 }
 
 // Target attention over a cached K/V prefix (attention only): the tensor-core Target
@@ -581,6 +586,22 @@ mtfm_status mtfm_attn_target_fwd(const mtfm_cfg* cfg, const void* d_meta, const 
                                  float* d_a, float* d_stats, void* stream) {
   return attn_fwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_y, d_a, d_stats, stream,
                   true);
+}
+
+mtfm_status mtfm_attn_full_fwd_bf16y(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                     const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                     const float* d_gamma, const float* d_beta, uint16_t* d_y, float* d_a,
+                                     float* d_stats, void* stream) {
+  return attn_fwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_y, d_a, d_stats, stream,
+                  false, true);
+}
+
+mtfm_status mtfm_attn_target_fwd_bf16y(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                       const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                       const float* d_gamma, const float* d_beta, uint16_t* d_y,
+                                       float* d_a, float* d_stats, void* stream) {
+  return attn_fwd(cfg, d_meta, d_q, d_k, d_v, d_u, d_gamma, d_beta, d_y, d_a, d_stats, stream,
+                  true, true);
 }
 
 mtfm_status mtfm_attn_target_cached_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,

@@ -176,6 +176,23 @@ mtfm_status mtfm_attn_target_fwd(const mtfm_cfg* cfg, const void* d_meta, const 
                                  const float* d_gamma, const float* d_beta, float* d_y,
                                  float* d_a, float* d_stats, void* stream);
 
+/* The same two layer forwards with Y = GLN(A) (*) U ([DY] §4.1, §4.2) stored as bf16
+ * (uint16 bit patterns, [rows, hq*head_dim], 16-byte aligned): each element is the
+ * fp32 value the fp32 entry point computes, rounded to nearest even.  For a caller whose
+ * next step takes Y as a bf16 operand (the output projection f2), at half the bytes; A
+ * and d_stats stay fp32 (the backward's saved inputs).  Same arguments, checks and
+ * errors as mtfm_attn_full_fwd / mtfm_attn_target_fwd otherwise.  (Storing Y in bf16
+ * adds up to half a bf16 ulp per element: against an exact reference, max-abs
+ * errors then track the largest |Y| of the batch.) */
+mtfm_status mtfm_attn_full_fwd_bf16y(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                     const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                     const float* d_gamma, const float* d_beta, uint16_t* d_y, float* d_a,
+                                     float* d_stats, void* stream);
+mtfm_status mtfm_attn_target_fwd_bf16y(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,
+                                       const uint16_t* d_k, const uint16_t* d_v, const uint16_t* d_u,
+                                       const float* d_gamma, const float* d_beta, uint16_t* d_y,
+                                       float* d_a, float* d_stats, void* stream);
+
 /* The two halves of a layer forward, for callers that schedule them apart
  * (the layer calls above are exactly attention followed by the gate).
  *   mtfm_attn_full / mtfm_attn_target : writes A only (fp32, shapes as above).

@@ -84,6 +84,13 @@ def test_null_and_misaligned_pointers_rejected(lib):
     # gamma without beta
     assert m._lib.mtfm_attn_target_fwd(ctypes.byref(c), 4096, 4096, 4096, 4096, 4096, 4096, None,
                                        4096, 4096, 4096, None) == 1
+    # the bf16-Y forwards check the same arguments: missing K, misaligned Y, gamma without beta
+    assert m._lib.mtfm_attn_full_fwd_bf16y(ctypes.byref(c), 4096, 4096, None, 4096, 4096, None, None,
+                                           4096, 4096, None, None) == 1
+    assert m._lib.mtfm_attn_full_fwd_bf16y(ctypes.byref(c), 4096, 4096, 4096, 4096, 4096, None, None,
+                                           4096 + 2, 4096, None, None) == 1
+    assert m._lib.mtfm_attn_target_fwd_bf16y(ctypes.byref(c), 4096, 4096, 4096, 4096, 4096, 4096, None,
+                                             4096, 4096, 4096, None) == 1
     # cached-prefix Target attention: missing candidate keys, misaligned Q, and a head shape
     # the tensor-core Target kernel does not take
     c64 = _cfg(head_dim=64)

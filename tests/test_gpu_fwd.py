@@ -96,3 +96,35 @@ def test_work_counters_rewind(cuda_ok):
     for (yf, af, _), (yt, at, _) in outs:
         assert_close(af.cpu().numpy(), ref_f["A"], "A full")
         assert_close(at.cpu().numpy(), ref_t["A"], "A target")
+
+
+@pytest.mark.parametrize("bname,hname", [("pair", "pair"), ("edge", "pair"), ("tiny", "tiny")])
+@pytest.mark.parametrize("target", [False, True], ids=["full", "target"])
+def test_bf16y_is_rounded_fp32_y(bname, hname, target, cuda_ok):
+    """The bf16-Y entry points store exactly the fp32 entry points' Y rounded to nearest bf16,
+    with the same A and row statistics; the fp32 Y is checked against the oracle above."""
+    import hybrid_masked_attention_b200 as M
+    b, hd = BATCHES[bname](), HEADS[hname]
+    inp = syn.layer_inputs(b, hd, target=target, seed=13, gln=True)
+    s = packed(b, hd)
+    d = upload_layer(inp)
+    rows = b.total_t if target else b.total_tokens
+    f32 = dict(dtype=torch.float32, device="cuda")
+    y, a, st = (torch.empty(rows, hd.dq, **f32), torch.empty(rows, hd.dq, **f32), torch.empty(rows, 2, **f32))
+    yb = torch.empty(rows, hd.dq, dtype=torch.bfloat16, device="cuda")
+    ab, stb = torch.empty_like(a), torch.empty_like(st)
+    f, fb = (M.attn_target_fwd, M.attn_target_fwd_bf16y) if target else (M.attn_full_fwd, M.attn_full_fwd_bf16y)
+    f(s.cfg, s.meta, d["q"], d["k"], d["v"], d["u"], d["gamma"], d["beta"], y, a, st)
+    fb(s.cfg, s.meta, d["q"], d["k"], d["v"], d["u"], d["gamma"], d["beta"], yb, ab, stb)
+    M.pack_check(s.meta)
+    torch.cuda.synchronize()
+    if not target:  # one unit writes each row of A: both calls compute the same bits
+        assert torch.equal(ab, a) and torch.equal(stb, st)
+        assert torch.equal(yb, y.to(torch.bfloat16)), "bf16 Y differs from the rounded fp32 Y"
+    else:  # key chunks may add into A in either order: Y within half a bf16 ulp (+ that noise)
+        assert torch.allclose(ab, a, rtol=1e-5, atol=1e-6)
+        yf = yb.float()
+        bound = y.abs() * 2.0 ** -8 + 1e-5 * y.pow(2).mean().sqrt()
+        assert bool(((yf - y).abs() <= bound).all()), "bf16 Y is not the rounded fp32 Y"
+    ref = (O.target_fwd if target else O.full_fwd)(b, hd, inp)
+    assert_close(y.cpu().numpy(), ref["Y"], "Y (fp32 entry)")
