@@ -113,7 +113,7 @@ struct MetaHeader {
 // store, ending inside it) and the global row indices they compute, before using them.  A
 // failed test sets kErrBounds in MetaHeader::error, records its site in
 // MetaHeader::dbg_site and skips the access; a skipped load leaves its mbarrier short of
-// bytes, so the consumer gives up after its bounded wait instead of hanging.  This build
+// bytes, so the consumer gives up after its bounded wait instead of hanging.  The checked build
 // stands in for a memory checker; normal builds compile every test to `true`.  Each .cu
 // file that uses MTFM_INBOUNDS defines kDbgFile, its id in the recorded site.
 #ifdef MTFM_DEBUG_BOUNDS
