@@ -16,7 +16,9 @@
 // (user, 128-row query tile) with all its key blocks.  A step is one (128-key
 // block, query head) pair:
 //   warp 0      : TMA producer (Q tiles of the r heads once per item, then K/V
-//                 blocks of 128 keys through a 3-stage ring);
+//                 blocks of 128 keys through a 3-stage ring; once the item's last
+//                 S has read Q, the next item's Q and first K/V blocks, so they are
+//                 in place when the item's closing barrier releases);
 //   warp 1      : TMEM allocation and the MMA issue (whole warp runs the
 //                 control flow, one elected lane issues);
 //   warps 4..19 : four "SiLU" warpgroups that share every step, each on 32 of
@@ -24,8 +26,9 @@
 //                 mask + SiLU, write P as two bf16 parts P_hi + P_lo (~16
 //                 significant bits) back into the same TMEM columns, and signal
 //                 the MMA warp, which issues O_h += P_hi V + P_lo V with P read
-//                 from TMEM; at the end of the item they write O / N_u to A
-//                 through shared memory (whole rows per warp).
+//                 from TMEM; at the end of the item they stage O / N_u in a
+//                 shared-memory area of its own (two heads per round) that leaves
+//                 for A as TMA stores (row stores for a user's ragged last tile).
 // TMEM (512 columns): O_h at columns [64h, 64h+64) for h < r (<= 4), S buffers
 // b = 0, 1 at [256 + 128b, 384 + 128b).  While the warpgroups run the SiLU of
 // step n, the tensor pipe runs O += P(n-1) V and S(n+1) = Q K^T.

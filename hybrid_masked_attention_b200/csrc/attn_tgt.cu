@@ -23,13 +23,17 @@
 //
 // Roles and the pipeline across units (no block-wide barrier per unit):
 //   warp 0      : TMA producer.  Q tiles into two buffers (the next unit's Q
-//                 loads while this unit computes), K/V blocks through a 3-stage ring.
+//                 loads while this unit computes), K/V blocks through a 5-stage ring
+//                 (a block's DRAM load outlasts a step: see kStages).
 //   warp 1      : TMEM allocation and MMA issue.  S = Q K^T into one of three
 //                 S buffers, issued up to two steps ahead (also into the next
 //                 unit), then O += P_hi V + P_lo V into one of two O buffers.
+//   warp 2      : decodes the units into a 4-slot descriptor ring, with each
+//                 sub-tile's k_t = kv_end - L_H of its T rows (uint16, shared memory).
 //   warps 4..19 : SiLU warpgroups (as in the Full-layer kernel: each warpgroup
 //                 takes 32 of the 128 key columns of a step), then the unit's
-//                 epilogue: O / N_u from TMEM into a swizzled shared-memory tile.
+//                 epilogue (after the next unit's first step): O / N_u from TMEM
+//                 into a swizzled shared-memory tile.
 //   warp 3      : stores the staged tile into A (fp32), so that no SiLU warp
 //                 waits for a store.  When every sub-tile's key range is one
 //                 unit (MetaHeader::tgt_single), each row of A gets exactly one
