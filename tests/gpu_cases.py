@@ -21,6 +21,8 @@ BATCHES = {
 HEADS = {
     "tiny": syn.TINY_HEADS,                 # Hq 2, Hkv 1, dh 32
     "pair": syn.PAIR_HEADS,                 # Hq 8, Hkv 2, dh 64
+    "r1": syn.Heads(2, 2, 64),              # one query head per KV group (tcgen05 kernels at r = 1)
+    "r2": syn.Heads(4, 2, 64),              # two query heads per KV group (r = 2)
     "dh128": syn.Heads(4, 1, 128),
     "r8": syn.Heads(8, 1, 32),
     "dh256": syn.Heads(3, 1, 256),          # the 768-wide shape: Hq 3, Hkv 1, dh 256 (forward only)

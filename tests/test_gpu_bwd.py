@@ -35,7 +35,8 @@ def _rows(batch, users, target):
 
 CASES = [("tiny", "tiny", True), ("tiny", "tiny", False), ("edge", "pair", True),
          ("edge", "r8", True), ("v2_n512", "pair", True), ("pair", "pair", True),
-         ("pair", "dh128", False), ("edge", "dh256", True), ("tiny", "dh256", False)]
+         ("pair", "dh128", False), ("edge", "dh256", True), ("tiny", "dh256", False),
+         ("edge", "r1", True), ("edge", "r2", True), ("v2_n512", "r2", True)]
 
 
 @pytest.mark.parametrize("bname,hname,gln", CASES)

@@ -17,6 +17,8 @@ CASES = [
     ("edge", "dh256", True), ("v2_n512", "dh256", True), ("tiny", "dh256", False),
     ("pair", "dh256", True), ("v1_n2048", "dh256", False),
     ("v2_n512", "pair", True), ("v2_n1024", "pair", True), ("v1_n2048", "pair", True),
+    ("pair", "r1", True), ("edge", "r1", True), ("pair", "r2", True), ("edge", "r2", True),
+    ("v2_n512", "r2", True), ("v1_n2048", "r1", False),
 ]
 
 
