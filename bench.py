@@ -793,7 +793,8 @@ def train_entry(dev, users, steps, warmup, repeats, heads=syn.PAIR_HEADS):
         "ms_per_step": round(ms, 5), "step_ms": _spread(per_step), "steps": steps,
         "users_per_s": round(b.B / (ms * 1e-3), 1), "total_tokens": Nt, "total_t": T,
         "kernels_in_graph_ms": {k: round(v, 5) for k, v in kern.items()},
-        "roofline": {"kernel": "Full-layer backward call (gate backward + attn_bwd_tc_kernel)", "bound": "tensor",
+        "roofline": {"kernel": "Full-layer backward call (gate backward + "
+                               f"{'attn_bwd_tc_kernel' if heads.dh == 64 else 'attn_bwd_mma_kernel'})", "bound": "tensor",
                      "achieved": round(tf(2.5 * ff, kern["full_bwd"]), 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(tf(2.5 * ff, kern["full_bwd"]) / peak, 4),
                      "peak_source": f"{src} bf16 dense (burst)"},
@@ -910,11 +911,18 @@ def v2_layer_entry(dev, users, seqlen, steps, warmup, repeats, heads=syn.PAIR_HE
 PER_CONFIG = (
     ("sweep_n8192", lambda dev, a: sweep_entry(dev, 8192, False, max(2, a.config_steps // 4), a.warmup, 3)),
     ("sweep_n512", lambda dev, a: sweep_entry(dev, 512, False, a.config_steps, a.warmup, 3)),
+    ("sweep_n1024", lambda dev, a: sweep_entry(dev, 1024, False, a.config_steps, a.warmup, 3)),
+    ("sweep_n2048", lambda dev, a: sweep_entry(dev, 2048, False, max(2, a.config_steps // 2), a.warmup, 3)),
+    ("sweep_n4096", lambda dev, a: sweep_entry(dev, 4096, False, max(2, a.config_steps // 4), a.warmup, 3)),
     ("sweep_v2_n2048", lambda dev, a: sweep_entry(dev, 2048, True, max(2, a.config_steps // 2), a.warmup, 3)),
     ("stack_b64", lambda dev, a: stack_entry(dev, 64, a.config_steps, a.warmup, 5)),
     ("train_b96", lambda dev, a: train_entry(dev, 96, a.config_steps, a.warmup, 5)),
     ("train_b160", lambda dev, a: train_entry(dev, 160, a.config_steps, a.warmup, 5)),
     ("v2_layer_n2048", lambda dev, a: v2_layer_entry(dev, 64, 2048, a.config_steps, a.warmup, 5)),
+    ("stack_b64_d768_dh256", lambda dev, a: stack_entry(dev, 64, a.config_steps, a.warmup, 5,
+                                                        heads=syn.Heads(3, 1, 256), d=768)),
+    ("train_b96_dh256", lambda dev, a: train_entry(dev, 96, a.config_steps, a.warmup, 5,
+                                                   heads=syn.Heads(3, 1, 256))),
 )
 
 
