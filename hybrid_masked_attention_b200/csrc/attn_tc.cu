@@ -55,7 +55,6 @@ using namespace sm100;
 
 constexpr int kDbgFile = 1;  // site id of this file's bounds checks
 
-constexpr int kDH = 64;
 constexpr int kBM = 128;          // query rows per tile (TMEM lanes)
 constexpr int kBN = 128;          // keys per block
 constexpr int kStages = 3;        // K/V ring depth
@@ -64,8 +63,11 @@ constexpr int kSiluWG = 4;        // SiLU warpgroups
 constexpr int kWGPerBuf = 4;      // warpgroups sharing one step (split by key columns)
 constexpr int kChunksPerWG = kBN / 32 / kWGPerBuf;  // 32-key chunks per warpgroup and step
 constexpr int kThreads = 128 + 128 * kSiluWG;
-constexpr uint32_t kQBytes = kBM * kDH * 2;   // 16 KB
-constexpr uint32_t kKVBytes = kBN * kDH * 2;
+// head_dim DH (64, or 32): a Q tile and a K or V block are 128 rows of DH bf16
+template <int DH>
+constexpr uint32_t q_bytes() { return kBM * DH * 2; }
+template <int DH>
+constexpr uint32_t kv_bytes() { return kBN * DH * 2; }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 256;              // S buffer b at columns [256 + kBN b, 256 + kBN (b + 1))
 static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "S buffers exceed TMEM");
@@ -80,17 +82,17 @@ struct TcArgs {
 };
 
 // O / N_u leaves through its own staging area (so the next unit's Q and K/V can land while
-// the epilogue runs): at most two heads at a time, each as two boxes of 128 rows x 32 fp32.
+// the epilogue runs): at most two heads at a time, each as DH / 32 boxes of 128 rows x 32 fp32.
 constexpr uint32_t kBox = kBM * 128;  // one 32-column box of the tile
 template <int R>
 constexpr int heads_per_round() { return R < 2 ? R : 2; }
-template <int R>
-constexpr uint32_t stage_off() { return (uint32_t)R * kQBytes + 2 * kStages * kKVBytes; }
-template <int R>
+template <int R, int DH>
+constexpr uint32_t stage_off() { return (uint32_t)R * q_bytes<DH>() + 2 * kStages * kv_bytes<DH>(); }
+template <int R, int DH>
 constexpr size_t tc_smem_bytes() {
-  return stage_off<R>() + (size_t)heads_per_round<R>() * 2 * kBox + 1024;
+  return stage_off<R, DH>() + (size_t)heads_per_round<R>() * (DH / 32) * kBox + 1024;
 }
-static_assert(tc_smem_bytes<4>() + 1024 <= 227 * 1024, "shared memory per CTA");
+static_assert(tc_smem_bytes<4, 64>() + 1024 <= 227 * 1024, "shared memory per CTA");
 
 // SiLU of 32 scores of one row (one TMEM chunk), masked, split into bf16 hi/lo
 // pairs: P = SiLU(alpha s) = h + h tanh(h), h = alpha s / 2.  Scalar fp32 math:
@@ -112,10 +114,13 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half
   }
 }
 
-template <int R>
+template <int R, int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a, TcArgs p) {
+  static_assert(DH == 64 || DH == 32, "head_dim 64 (128-byte swizzle) or 32 (64-byte swizzle)");
+  constexpr int kDH = DH;
+  constexpr uint32_t kQBytes = q_bytes<DH>(), kKVBytes = kv_bytes<DH>();
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q, bar_qe, bar_o, bar_drain;
   __shared__ __align__(8) uint64_t bar_kv_full[kStages], bar_kv_empty[kStages];
@@ -283,7 +288,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, kDH, true);
       // descriptor words: the high word is shared; low words step by (bytes >> 4)
-      const uint32_t dhi = sw128_desc_hi(1024);
+      const uint32_t dhi = bf16_rows_desc_hi<DH>();
       const uint32_t q_lo = sw128_desc_lo(sQ, 16), k_lo = sw128_desc_lo(sK, 16), v_lo = sw128_desc_lo(sV, 16);
       bool ok = __all_sync(0xffffffffu, mbar_wait(b_q, unit_iter & 1, abort_flag));
       auto issue_s = [&](int n) -> bool {
@@ -319,14 +324,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int bi = n / R, hh = n % R, s = (blk_base + bi) % kStages;
         const uint32_t pt = tmem + kSCol0 + b * kBN;  // P = P_hi + P_lo, bf16 pairs
         const uint32_t o = tmem + hh * kDH;
-        const uint32_t vb = v_lo + s * (kKVBytes >> 4);  // V rows (keys): 16 per k-step = 2048 B
+        const uint32_t vb = v_lo + s * (kKVBytes >> 4);  // V rows (keys): 16 per k-step
+        constexpr uint32_t kVStep = (16 * kDH * 2) >> 4;   // 16 rows of V, in 16-byte units
         const uint32_t acc0 = bi > 0 ? 1u : 0u;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
-            mma_ts2(o, pt + col, vb + kk * (2048 >> 4), dhi, idesc_pv, kk > 0 ? 1u : acc0);
-            mma_ts2(o, pt + col + 16, vb + kk * (2048 >> 4), dhi, idesc_pv, 1u);
+            mma_ts2(o, pt + col, vb + kk * kVStep, dhi, idesc_pv, kk > 0 ? 1u : acc0);
+            mma_ts2(o, pt + col + 16, vb + kk * kVStep, dhi, idesc_pv, 1u);
           }
           if (hh == R - 1) mma_commit(b_kve(s));
         }
@@ -425,8 +431,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // The named barriers are reached by all 16 SiLU warps, also after an abort.
       const bool have = ok && total > 0;
       constexpr int kHR = heads_per_round<R>();
-      uint8_t* stage = smem + stage_off<R>();
-      const uint32_t s_stage = sQ + stage_off<R>();
+      uint8_t* stage = smem + stage_off<R, DH>();
+      const uint32_t s_stage = sQ + stage_off<R, DH>();
       if (have) tc_fence_after();
       const float inv_n = 1.f / (float)N;
       for (int rd = 0; rd < R / kHR; ++rd) {
@@ -439,7 +445,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             uint32_t raw[32];
             tmem_ld32(lane_base + hh * kDH + c * 32, raw);
             tmem_ld_wait();
-            uint8_t* rowp = stage + ((hh % kHR) * 2 + c) * kBox + row * 128;
+            uint8_t* rowp = stage + ((hh % kHR) * (kDH / 32) + c) * kBox + row * 128;
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               *reinterpret_cast<float4*>(rowp + ((e ^ (row & 7)) << 4)) =
@@ -454,7 +460,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const int col0 = (g * R + rd * kHR) * kDH;  // first column of this round's heads
           if (q0 + kBM <= nq) {
             if (threadIdx.x == 128) {
-              for (int b = 0; b < 2 * kHR; ++b)
+              for (int b = 0; b < (kDH / 32) * kHR; ++b)
                 if (MTFM_INBOUNDS(hdr, tma_x_ok(col0 + b * 32, 32, ldq, 4) && qrow0 + q0 >= 0 &&
                                            qrow0 + q0 + kBM <= hdr->total_tokens))
                   tma_store_2d_hint(&tm_a, s_stage + b * kBox, col0 + b * 32, qrow0 + q0, keep_a);
@@ -515,30 +521,31 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // ------------------------------------------------------------------ host side
-// Row-major bf16 matrix [rows, cols]; box_rows x 64 boxes with the 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-  return make_map_bf16(map, base, (uint64_t)rows, (uint64_t)cols, (uint64_t)cols, (uint32_t)box_rows, kDH);
+// Row-major bf16 matrix [rows, cols]; boxes of box_rows x dh (the 128-byte swizzle for
+// dh 64, the 64-byte swizzle for dh 32).
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows, int dh) {
+  return make_map_bf16(map, base, (uint64_t)rows, (uint64_t)cols, (uint64_t)cols, (uint32_t)box_rows, (uint32_t)dh);
 }
 
 // One CTA per SM (TMEM and shared memory allow no more); the CTAs stride over
 // the (work unit, KV group) pairs, whose count the kernel reads from the metadata.
-template <int R>
+template <int R, int DH>
 cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& ma, const TcArgs& a, int max_items, cudaStream_t st) {
-  const size_t smem = tc_smem_bytes<R>();
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R>,
+  const size_t smem = tc_smem_bytes<R, DH>();
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<R, DH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = sm_count();
   grid = std::min(grid, max_items * a.hkv);
-  return launch_pdl(attn_fwd_tc_kernel<R>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, a);
+  return launch_pdl(attn_fwd_tc_kernel<R, DH>, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, a);
 }
 
 }  // namespace
 
 bool attn_fwd_tc_supported(const AttnShape& s) {
   const int r = s.hq / s.hkv;
-  return s.dh == kDH && (r == 1 || r == 2 || r == 4);
+  return (s.dh == 64 || s.dh == 32) && (r == 1 || r == 2 || r == 4);
 }
 
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
@@ -547,13 +554,15 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
   if (s.target) return cudaErrorInvalidValue;  // the Target layer has its own kernel (attn_tgt.cu)
   if (max_items <= 0 || rows_q <= 0 || total_tokens <= 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, ma;
-  if (!make_map(&mq, q, rows_q, s.hq * kDH, kBM) || !make_map(&mk, k, total_tokens, s.hkv * kDH, kBN) ||
-      !make_map(&mv, v, total_tokens, s.hkv * kDH, kBN))
+  if (!attn_fwd_tc_supported(s)) return cudaErrorInvalidValue;
+  const int dh = s.dh;
+  if (!make_map(&mq, q, rows_q, s.hq * dh, kBM, dh) || !make_map(&mk, k, total_tokens, s.hkv * dh, kBN, dh) ||
+      !make_map(&mv, v, total_tokens, s.hkv * dh, kBN, dh))
     return cudaErrorInvalidValue;
-  {  // A [rows_q, hq * 64] fp32 in boxes of 32 columns x 128 rows (128-byte swizzle)
+  {  // A [rows_q, hq * dh] fp32 in boxes of 32 columns x 128 rows (128-byte swizzle)
     EncodeTiledFn fn = encode_fn();
-    cuuint64_t dims[2] = {(cuuint64_t)s.hq * kDH, (cuuint64_t)rows_q};
-    cuuint64_t strides[1] = {(cuuint64_t)s.hq * kDH * 4};
+    cuuint64_t dims[2] = {(cuuint64_t)s.hq * dh, (cuuint64_t)rows_q};
+    cuuint64_t strides[1] = {(cuuint64_t)s.hq * dh * 4};
     cuuint32_t box[2] = {32, (cuuint32_t)kBM};
     cuuint32_t estr[2] = {1, 1};
     if (!fn || fn(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -563,9 +572,14 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
   }
   TcArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha};
   const int r = s.hq / s.hkv;
-  if (r == 1) return tc_launch<1>(mq, mk, mv, ma, args, max_items, st);
-  if (r == 2) return tc_launch<2>(mq, mk, mv, ma, args, max_items, st);
-  return tc_launch<4>(mq, mk, mv, ma, args, max_items, st);
+  if (dh == 32) {
+    if (r == 1) return tc_launch<1, 32>(mq, mk, mv, ma, args, max_items, st);
+    if (r == 2) return tc_launch<2, 32>(mq, mk, mv, ma, args, max_items, st);
+    return tc_launch<4, 32>(mq, mk, mv, ma, args, max_items, st);
+  }
+  if (r == 1) return tc_launch<1, 64>(mq, mk, mv, ma, args, max_items, st);
+  if (r == 2) return tc_launch<2, 64>(mq, mk, mv, ma, args, max_items, st);
+  return tc_launch<4, 64>(mq, mk, mv, ma, args, max_items, st);
 }
 
 }  // namespace mtfm

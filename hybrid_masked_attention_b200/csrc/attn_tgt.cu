@@ -66,7 +66,6 @@ using namespace sm100;
 
 constexpr int kDbgFile = 2;  // site id of this file's bounds checks
 
-constexpr int kDH = 64;
 constexpr int kBN = 128;     // keys per block
 // K/V ring: the loads of a unit's blocks come from DRAM (~3,000-4,000 clocks under load)
 // while a block takes ~1,700 clocks of MMA and SiLU work, so about three blocks must be in
@@ -75,9 +74,14 @@ constexpr int kStages = 5;
 constexpr int kSBuf = 3;     // S/P buffers
 constexpr int kSiluWG = 4;
 constexpr int kThreads = 128 + 128 * kSiluWG;
-constexpr uint32_t kQBytes = 128 * kDH * 2;   // one stacked Q tile
-constexpr uint32_t kKVBytes = kBN * kDH * 2;
-constexpr uint32_t kStageBytes = 128 * kDH * 4;  // O tile in fp32: 2r boxes of TR x 32
+// head_dim DH (64, or 32): one stacked Q tile, one K or V block, one staged O tile
+// (fp32: DH / 32 boxes of TR rows x 32 columns per head)
+template <int DH>
+constexpr uint32_t q_bytes() { return 128 * DH * 2; }
+template <int DH>
+constexpr uint32_t kv_bytes() { return kBN * DH * 2; }
+template <int DH>
+constexpr uint32_t stage_bytes() { return 128 * DH * 4; }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 128;
 static_assert(kBN == kKeyBlock, "the packer sizes Target units in blocks of kKeyBlock keys");
@@ -86,8 +90,11 @@ static_assert(kSCol0 + kSBuf * kBN <= kTmemCols, "TMEM plan");
 constexpr int kRing = 4;                 // decoded-unit descriptors in flight
 constexpr uint16_t kKtNone = 0xffff;
 constexpr int kDescConsumers = 2 + 16;   // producer, MMA warp, 16 SiLU warps
-constexpr size_t tgt_smem_bytes() { return 2 * kQBytes + 2 * kStages * kKVBytes + kStageBytes + 1024; }
-static_assert(tgt_smem_bytes() + 2048 <= 227 * 1024, "dynamic + static shared memory per CTA");
+template <int DH>
+constexpr size_t tgt_smem_bytes() {
+  return 2 * q_bytes<DH>() + 2 * kStages * kv_bytes<DH>() + stage_bytes<DH>() + 1024;
+}
+static_assert(tgt_smem_bytes<64>() + 2048 <= 227 * 1024, "dynamic + static shared memory per CTA");
 
 struct TgtArgs {
   MetaView m;
@@ -164,12 +171,12 @@ __device__ __forceinline__ void silu_chunk(const uint32_t (&raw)[32], float half
   }
 }
 
-// Rows [0, rows) of a staged O tile (2R boxes of TR rows x 32 fp32, 16-byte chunks
-// XOR-swizzled by row) to A rows dst + t * ld, by one warp.
-template <int R>
+// Rows [0, rows) of a staged O tile (R * DH / 32 boxes of TR rows x 32 fp32, 16-byte
+// chunks XOR-swizzled by row) to A rows dst + t * ld, by one warp.
+template <int R, int DH>
 __device__ __noinline__ void store_rows(const uint8_t* stage, float* dst, int ld, int rows, int lane) {
   constexpr int TR = 128 / R;
-  constexpr int kF = R * kDH / 4;  // float4 per row
+  constexpr int kF = R * DH / 4;  // float4 per row
   for (int i = lane; i < rows * kF; i += 32) {
     const int tr = i / kF, f = i % kF;
     reinterpret_cast<float4*>(dst + (size_t)tr * ld)[f] =
@@ -179,13 +186,17 @@ __device__ __noinline__ void store_rows(const uint8_t* stage, float* dst, int ld
 
 
 
-template <int R>
+template <int R, int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
                     TgtArgs p) {
+  static_assert(DH == 64 || DH == 32, "head_dim 64 (128-byte swizzle) or 32 (64-byte swizzle)");
   constexpr int TR = 128 / R;
+  constexpr int kDH = DH;
+  constexpr int kBoxes = DH / 32;  // 32-column boxes of one head's O
+  constexpr uint32_t kQBytes = q_bytes<DH>(), kKVBytes = kv_bytes<DH>();
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_qf[2], bar_qe[2], bar_of[2], bar_oe[2], bar_drain;
   __shared__ __align__(8) uint64_t bar_kvf[kStages], bar_kve[kStages], bar_sf[kSBuf], bar_pf[kSBuf];
@@ -331,8 +342,9 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ------------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBN, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kDH, true);
-    const uint32_t dhi = sw128_desc_hi(1024);
+    const uint32_t dhi = bf16_rows_desc_hi<DH>();
     const uint32_t q_lo = sw128_desc_lo(sQ, 16), k_lo = sw128_desc_lo(sK, 16), v_lo = sw128_desc_lo(sV, 16);
+    constexpr uint32_t kVStep = (16 * kDH * 2) >> 4;  // 16 rows (keys) of V, in 16-byte units
     bool ok = true;
     // S cursor: unit ks, step is within it, global step gs
     int ks = 0, is = 0, gs = 0, nb_s = 0;
@@ -395,8 +407,8 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             const uint32_t col = 32 * (kk >> 1) + 8 * (kk & 1);
-            mma_ts2(o, pt + col, vb + kk * (2048 >> 4), dhi, idesc_pv, (kk > 0 || i > 0) ? 1u : 0u);
-            mma_ts2(o, pt + col + 16, vb + kk * (2048 >> 4), dhi, idesc_pv, 1u);
+            mma_ts2(o, pt + col, vb + kk * kVStep, dhi, idesc_pv, (kk > 0 || i > 0) ? 1u : 0u);
+            mma_ts2(o, pt + col + 16, vb + kk * kVStep, dhi, idesc_pv, 1u);
           }
           mma_commit(B(&bar_kve[gp % kStages]));
           if (i == nb - 1) mma_commit(B(&bar_of[ob]));
@@ -461,22 +473,28 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (eok && e.k > 0) eok = __all_sync(0xffffffffu, mbar_wait(B(&bar_ste), (e.k - 1) & 1, abort_flag));
       if (!eok) ok = false;
       if (eok) {
+        // O columns [16 wg, 16 wg + 16) (the warpgroups past DH / 16 have none)
+        const bool mine = wg * 16 < kDH;
         tc_fence_after();
         uint32_t raw[16];
-        tmem_ld16(lane_base + ob * kDH + wg * 16, raw);  // O columns [16 wg, 16 wg + 16)
-        tmem_ld_wait();
+        if (mine) {
+          tmem_ld16(lane_base + ob * kDH + wg * 16, raw);
+          tmem_ld_wait();
+        }
         tc_fence_before();
         mbar_arrive(B(&bar_oe[ob]));
-        const int box = hh * 2 + (wg >> 1);  // 32-column box of this head
-        uint8_t* rowp = stage + box * (TR * 128) + t * 128;
+        if (mine) {
+          const int box = hh * kBoxes + (wg >> 1);  // 32-column box of this head
+          uint8_t* rowp = stage + box * (TR * 128) + t * 128;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int chunk = (wg & 1) * 4 + j;  // 16-byte chunk within the 128-byte row
-          *reinterpret_cast<float4*>(rowp + ((chunk ^ (t & 7)) << 4)) =
-              make_float4(__uint_as_float(raw[4 * j]) * e.inv_n, __uint_as_float(raw[4 * j + 1]) * e.inv_n,
-                          __uint_as_float(raw[4 * j + 2]) * e.inv_n, __uint_as_float(raw[4 * j + 3]) * e.inv_n);
+          for (int j = 0; j < 4; ++j) {
+            const int chunk = (wg & 1) * 4 + j;  // 16-byte chunk within the 128-byte row
+            *reinterpret_cast<float4*>(rowp + ((chunk ^ (t & 7)) << 4)) =
+                make_float4(__uint_as_float(raw[4 * j]) * e.inv_n, __uint_as_float(raw[4 * j + 1]) * e.inv_n,
+                            __uint_as_float(raw[4 * j + 2]) * e.inv_n, __uint_as_float(raw[4 * j + 3]) * e.inv_n);
+          }
+          fence_proxy_async();  // the staged tile may be read by the TMA engine
         }
-        fence_proxy_async();  // the staged tile may be read by the TMA engine
       }
       if (threadIdx.x == 128) s_st[e.k & 1] = make_int4(eok ? 1 : 0, e.col, e.y, e.rows);
       mbar_arrive(B(&bar_stf));
@@ -572,25 +590,25 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (!full) st.x = 0;
       if (st.x && !single) {
         if (lane == 0) {
-          for (int b = 0; b < 2 * R; ++b)
-            if (MTFM_INBOUNDS(hdr, tma_x_ok(st.y + (b >> 1) * kDH + (b & 1) * 32, 32, p.hq * kDH, 4) &&
+          for (int b = 0; b < kBoxes * R; ++b)
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(st.y + (b / kBoxes) * kDH + (b % kBoxes) * 32, 32, p.hq * kDH, 4) &&
                                        st.z >= 0 && st.z < hdr->total_t))
-              tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), st.y + (b >> 1) * kDH + (b & 1) * 32, st.z);
+              tma_reduce_add_2d(&tm_a, sO + b * (TR * 128), st.y + (b / kBoxes) * kDH + (b % kBoxes) * 32, st.z);
           bulk_commit();
           bulk_wait_read<0>();
         }
       } else if (st.x && st.w == TR) {
         if (lane == 0) {
-          for (int b = 0; b < 2 * R; ++b)
-            if (MTFM_INBOUNDS(hdr, tma_x_ok(st.y + (b >> 1) * kDH + (b & 1) * 32, 32, p.hq * kDH, 4) &&
+          for (int b = 0; b < kBoxes * R; ++b)
+            if (MTFM_INBOUNDS(hdr, tma_x_ok(st.y + (b / kBoxes) * kDH + (b % kBoxes) * 32, 32, p.hq * kDH, 4) &&
                                        st.z >= 0 && st.z + TR <= hdr->total_t))
-              tma_store_2d(&tm_a, sO + b * (TR * 128), st.y + (b >> 1) * kDH + (b & 1) * 32, st.z);
+              tma_store_2d(&tm_a, sO + b * (TR * 128), st.y + (b / kBoxes) * kDH + (b % kBoxes) * 32, st.z);
           bulk_commit();
           bulk_wait_read<0>();
         }
       } else if (st.x && MTFM_INBOUNDS(hdr, st.z >= 0 && st.z + st.w <= hdr->total_t)) {
         // the sub-tile runs past its user's last T row: store the user's rows one by one
-        store_rows<R>(stage, p.a + (size_t)st.z * (p.hq * kDH) + st.y, p.hq * kDH, st.w, lane);
+        store_rows<R, DH>(stage, p.a + (size_t)st.z * (p.hq * kDH) + st.y, p.hq * kDH, st.w, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(B(&bar_ste));
@@ -618,8 +636,9 @@ __global__ void __launch_bounds__(256) tgt_zero_kernel(const MetaHeader* hdr, in
 
 }  // namespace
 
-// Q [total_t, hq * 64] as a 3-D tensor {64 dims, hq heads, total_t rows}: a box of
-// {64, r, 128 / r} is one stacked tile.  A [total_t, hq * 64] fp32 in boxes of 32 x TR.
+// Q [total_t, hq * dh] as a 3-D tensor {dh dims, hq heads, total_t rows}: a box of
+// {dh, r, 128 / r} is one stacked tile (rows of 128 bytes for dh 64, of 64 bytes with the
+// 64-byte swizzle for dh 32).  A [total_t, hq * dh] fp32 in boxes of 32 x TR.
 cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_items, int total_t,
                                 int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                 const __nv_bfloat16* v, float* a, cudaStream_t st, const __nv_bfloat16* k_cand,
@@ -630,28 +649,30 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
   const uint64_t kv_rows = cached ? (uint64_t)(total_tokens - total_t) : (uint64_t)total_tokens;
   const int r = s.hq / s.hkv;
   const int TR = 128 / r;
+  const int dh = s.dh;
+  if (!attn_fwd_tc_supported(s)) return cudaErrorInvalidValue;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv, ma;
   {
-    cuuint64_t dims[3] = {(cuuint64_t)kDH, (cuuint64_t)s.hq, (cuuint64_t)total_t};
-    cuuint64_t strides[2] = {(cuuint64_t)kDH * 2, (cuuint64_t)s.hq * kDH * 2};
-    cuuint32_t box[3] = {(cuuint32_t)kDH, (cuuint32_t)r, (cuuint32_t)TR};
+    cuuint64_t dims[3] = {(cuuint64_t)dh, (cuuint64_t)s.hq, (cuuint64_t)total_t};
+    cuuint64_t strides[2] = {(cuuint64_t)dh * 2, (cuuint64_t)s.hq * dh * 2};
+    cuuint32_t box[3] = {(cuuint32_t)dh, (cuuint32_t)r, (cuuint32_t)TR};
     cuuint32_t estr[3] = {1, 1, 1};
     if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(q), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, bf16_row_swizzle((uint32_t)dh), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   CUtensorMap mkc, mvc;
   if (kv_rows > 0) {
-    if (!make_map_bf16(&mk, k, kv_rows, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH) ||
-        !make_map_bf16(&mv, v, kv_rows, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH))
+    if (!make_map_bf16(&mk, k, kv_rows, (uint64_t)s.hkv * dh, (uint64_t)s.hkv * dh, kBN, dh) ||
+        !make_map_bf16(&mv, v, kv_rows, (uint64_t)s.hkv * dh, (uint64_t)s.hkv * dh, kBN, dh))
       return cudaErrorInvalidValue;
   }
   if (cached) {
-    if (!make_map_bf16(&mkc, k_cand, (uint64_t)total_t, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH) ||
-        !make_map_bf16(&mvc, v_cand, (uint64_t)total_t, (uint64_t)s.hkv * kDH, (uint64_t)s.hkv * kDH, kBN, kDH))
+    if (!make_map_bf16(&mkc, k_cand, (uint64_t)total_t, (uint64_t)s.hkv * dh, (uint64_t)s.hkv * dh, kBN, dh) ||
+        !make_map_bf16(&mvc, v_cand, (uint64_t)total_t, (uint64_t)s.hkv * dh, (uint64_t)s.hkv * dh, kBN, dh))
       return cudaErrorInvalidValue;
     if (kv_rows == 0) {  // no prefix rows at all: the prefix maps are never read
       mk = mkc;
@@ -662,8 +683,8 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
     mvc = mv;
   }
   {
-    cuuint64_t dims[2] = {(cuuint64_t)s.hq * kDH, (cuuint64_t)total_t};
-    cuuint64_t strides[1] = {(cuuint64_t)s.hq * kDH * 4};
+    cuuint64_t dims[2] = {(cuuint64_t)s.hq * dh, (cuuint64_t)total_t};
+    cuuint64_t strides[1] = {(cuuint64_t)s.hq * dh * 4};
     cuuint32_t box[2] = {32, (cuuint32_t)TR};
     cuuint32_t estr[2] = {1, 1};
     if (fn(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -672,23 +693,28 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
       return cudaErrorInvalidValue;
   }
   {
-    const size_t n4 = (size_t)total_t * s.hq * (kDH / 4);
+    const size_t n4 = (size_t)total_t * s.hq * (dh / 4);
     const int zgrid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)sm_count() * 8);
     cudaError_t e = launch_pdl(tgt_zero_kernel, dim3(zgrid), dim3(256), 0, st, (const MetaHeader*)m.hdr,
                                cached ? 1 : 0, reinterpret_cast<float4*>(a), n4);
     if (e != cudaSuccess) return e;
   }
   TgtArgs args{m, a, s.hq, s.hkv, s.v2, s.alpha, cached ? 1 : 0};
-  const size_t smem = tgt_smem_bytes();
+  const size_t smem = dh == 32 ? tgt_smem_bytes<32>() : tgt_smem_bytes<64>();
   const int grid = sm_count();
   auto launch = [&](auto kern) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e2 != cudaSuccess) return e2;
     return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, mq, mk, mv, ma, mkc, mvc, args);
   };
-  if (r == 1) return launch(attn_fwd_tgt_kernel<1>);
-  if (r == 2) return launch(attn_fwd_tgt_kernel<2>);
-  return launch(attn_fwd_tgt_kernel<4>);
+  if (dh == 32) {
+    if (r == 1) return launch(attn_fwd_tgt_kernel<1, 32>);
+    if (r == 2) return launch(attn_fwd_tgt_kernel<2, 32>);
+    return launch(attn_fwd_tgt_kernel<4, 32>);
+  }
+  if (r == 1) return launch(attn_fwd_tgt_kernel<1, 64>);
+  if (r == 2) return launch(attn_fwd_tgt_kernel<2, 64>);
+  return launch(attn_fwd_tgt_kernel<4, 64>);
 }
 
 }  // namespace mtfm

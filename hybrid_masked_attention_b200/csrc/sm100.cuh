@@ -261,6 +261,19 @@ __device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo) 
 __device__ __forceinline__ uint32_t sw128_desc_hi(uint32_t sbo) {
   return ((sbo >> 4) & 0x3FFF) | (1u << 14) | (2u << 29);
 }
+// High word of the 64-byte-swizzle descriptor (layout type 4): rows of 64 bytes
+// (32 bf16), 8-row atoms of 512 bytes.  K-major: sbo = stride of 8-row groups;
+// MN-major with the MN extent inside one atom: sbo = stride of 8-row groups along K.
+__device__ __forceinline__ uint32_t sw64_desc_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFF) | (1u << 14) | (4u << 29);
+}
+// The high word for bf16 tiles whose rows are dh elements: the 128-byte swizzle
+// for dh 64, the 64-byte swizzle for dh 32 (8-row groups of 8 * 2 * dh bytes).
+template <int DH>
+__device__ __forceinline__ uint32_t bf16_rows_desc_hi() {
+  static_assert(DH == 32 || DH == 64, "rows of 64 or 128 bytes");
+  return DH == 64 ? sw128_desc_hi(1024) : sw64_desc_hi(512);
+}
 // D[tmem] (+)= A[smem desc] * B[smem desc], descriptors given as (lo, hi) words
 __device__ __forceinline__ void mma_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
                                         uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {

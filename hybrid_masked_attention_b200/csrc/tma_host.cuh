@@ -25,19 +25,24 @@ inline EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// The swizzle whose span is one box row of box_cols bf16 (128 or 64 bytes).
+inline CUtensorMapSwizzle bf16_row_swizzle(uint32_t box_cols) {
+  return box_cols * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+}
+
 // Row-major bf16 matrix [rows, cols] (row pitch ld_elems); boxes of box_rows x
-// box_cols with the 128-byte swizzle (box_cols * 2 bytes must be 128).  Rows
-// past `rows` read as zeros.
+// box_cols with the swizzle of one box row: 128 bytes (box_cols 64) or 64 bytes
+// (box_cols 32).  Rows past `rows` read as zeros.
 inline bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                           uint64_t ld_elems, uint32_t box_rows, uint32_t box_cols) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
+  if (!fn || (box_cols != 64 && box_cols != 32)) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld_elems * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, bf16_row_swizzle(box_cols),
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -52,9 +52,11 @@
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
  *   - No exceptions cross this boundary; no global state is kept (the one
  *     exception is the fixed scratch array of mtfm_attn_target_bwd_static).
- *     The forward attention runs the tcgen05/TMEM kernel for head_dim 64 with
- *     hq/hkv in {1, 2, 4} and the portable mma.sync kernel otherwise; the
- *     choice depends on the shape only (no run-time switch).
+ *     The forward attention runs tcgen05/TMEM kernels for head_dim 64 and 32
+ *     with hq/hkv in {1, 2, 4} and for head_dim 256, the backward for head_dim
+ *     64; other shapes (head_dim 128, or hq/hkv of 3 or 5..8 at head_dim 32 or
+ *     64, and the backward at head_dim 32, 128, 256) run the portable mma.sync
+ *     kernels.  The choice depends on the shape only (no run-time switch).
  */
 #ifndef MTFM_H_
 #define MTFM_H_
@@ -222,8 +224,8 @@ mtfm_status mtfm_gate_fwd(const mtfm_cfg* cfg, const void* d_meta, int is_target
  *   d_k_cand, d_v_cand     : bf16 [total_t, hkv*head_dim], the candidates' own keys
  *                            and values (row t_off[u] + t for candidate t of user u);
  *   d_q, d_u, d_y, d_a, d_stats, d_gamma, d_beta : as mtfm_attn_target_fwd.
- * Supported where the tensor-core Target kernel runs (head_dim 64, hq / hkv in
- * {1, 2, 4}); other shapes return MTFM_ERR_UNSUPPORTED.  mtfm_attn_target_cached
+ * Supported where the tensor-core Target kernel runs (head_dim 64 or 32, hq / hkv
+ * in {1, 2, 4}); other shapes return MTFM_ERR_UNSUPPORTED.  mtfm_attn_target_cached
  * writes A only.
  * ------------------------------------------------------------------------- */
 mtfm_status mtfm_attn_target_cached_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,

@@ -25,5 +25,7 @@ HEADS = {
     "r2": syn.Heads(4, 2, 64),              # two query heads per KV group (r = 2)
     "dh128": syn.Heads(4, 1, 128),
     "r8": syn.Heads(8, 1, 32),
+    "dh32_r1": syn.Heads(2, 2, 32),         # head_dim 32 on the tcgen05 kernels (64-byte swizzle), r = 1
+    "dh32_r4": syn.Heads(4, 1, 32),         # head_dim 32, r = 4
     "dh256": syn.Heads(3, 1, 256),          # the 768-wide shape: Hq 3, Hkv 1, dh 256 (forward only)
 }

@@ -19,6 +19,10 @@ CASES = [
     ("v2_n512", "pair", True), ("v2_n1024", "pair", True), ("v1_n2048", "pair", True),
     ("pair", "r1", True), ("edge", "r1", True), ("pair", "r2", True), ("edge", "r2", True),
     ("v2_n512", "r2", True), ("v1_n2048", "r1", False),
+    # head_dim 32 on the tcgen05 kernels: the tiny heads (r = 2) on larger batches, r = 1 and 4
+    ("pair", "tiny", True), ("edge", "tiny", True), ("v1_n2048", "tiny", False),
+    ("pair", "dh32_r1", True), ("edge", "dh32_r1", False), ("pair", "dh32_r4", True),
+    ("edge", "dh32_r4", True), ("v2_n512", "dh32_r4", True),
 ]
 
 
