@@ -52,29 +52,35 @@ using namespace sm100;
 
 constexpr int kDbgFile = 4;  // site id of this file's bounds checks
 
-constexpr int kDH = 64;
 constexpr int kKB = 128;         // keys per unit (TMEM lanes)
 constexpr int kQS = 64;          // queries per step
 constexpr int kSiluWG = 4;
 constexpr int kThreads = 128 + 128 * kSiluWG;
-constexpr uint32_t kKVTile = kKB * kDH * 2;   // 16 KB: one K or V block
-constexpr uint32_t kQTile = kQS * kDH * 2;    // 8 KB: Q, dA_hi or dA_lo tile of a step
-constexpr uint32_t kStepBytes = 3 * kQTile;   // one stage of the Q/dA ring
 constexpr uint32_t kDSHalf = kKB * kQS * 2;   // 16 KB: dS^T for 64 queries, one part
 constexpr uint32_t kTmemCols = 512;
+// TMEM columns (head_dim 64; at head_dim 32 each accumulator uses the first half of its range)
 constexpr uint32_t kColDV = 0, kColDK = 64, kColDQ = 128, kColSP = 256;
-
-// shared memory map (offsets from the 1024-aligned base)
-constexpr int kStages = 4;                                  // Q / dA ring: loads run 3 steps ahead
-constexpr uint32_t kOffKV = 0;                              // K, V of the unit
-constexpr uint32_t kOffStage = kOffKV + 2 * kKVTile;        // kStages x (Q, dA_hi, dA_lo)
+constexpr int kStages = 4;       // Q / dA ring: loads run 3 steps ahead
 // dS^T of a super-tile: hi (2 query halves), then lo (2 halves).  The dQ MMA that
 // reads it is issued as soon as the second half is written, ahead of that step's
 // dV/dK MMAs, so it has finished before the next super-tile's first half is written.
 constexpr uint32_t kDSBuf = 4 * kDSHalf;
-constexpr uint32_t kOffDS = kOffStage + kStages * kStepBytes;
-constexpr size_t kSmemBytes = kOffDS + kDSBuf + 1024;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+// Shared memory map for head_dim DH (64: rows of 128 bytes, 128-byte swizzle; 32: rows of
+// 64 bytes, 64-byte swizzle), offsets from the 1024-aligned base.
+template <int DH>
+struct BwdLayout {
+  static constexpr uint32_t kKVTile = kKB * DH * 2;   // one K or V block (16 KB at DH 64)
+  static constexpr uint32_t kQTile = kQS * DH * 2;    // Q, dA_hi or dA_lo tile of a step (8 KB at DH 64)
+  static constexpr uint32_t kStepBytes = 3 * kQTile;  // one stage of the Q/dA ring
+  static constexpr uint32_t kOffKV = 0;                                // K, V of the unit
+  static constexpr uint32_t kOffStage = kOffKV + 2 * kKVTile;          // kStages x (Q, dA_hi, dA_lo)
+  static constexpr uint32_t kOffDS = kOffStage + kStages * kStepBytes;  // dS^T (128-byte rows)
+  static constexpr size_t kSmemBytes = kOffDS + kDSBuf + 1024;
+  // 16 rows of a K, Q or dA tile read MN-major (one k-step of 16 keys or queries), in 16-byte units
+  static constexpr uint32_t kRows16 = (16 * DH * 2) >> 4;
+};
+static_assert(BwdLayout<64>::kSmemBytes <= 227 * 1024, "shared memory");
 
 struct BwdTcArgs {
   MetaView m;
@@ -151,12 +157,17 @@ __device__ __forceinline__ ColInfo col_info(const MetaView& m, const BwdUnit& U,
   return c;
 }
 
-template <bool TARGET>
+template <bool TARGET, int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_dah,
                    const __grid_constant__ CUtensorMap tm_dal, float* __restrict__ dq,
                    float* __restrict__ dk, float* __restrict__ dv, BwdTcArgs p) {
+  static_assert(DH == 64 || DH == 32, "head_dim 64 (128-byte swizzle) or 32 (64-byte swizzle)");
+  using L = BwdLayout<DH>;
+  constexpr int kDH = DH;
+  constexpr uint32_t kKVTile = L::kKVTile, kQTile = L::kQTile, kStepBytes = L::kStepBytes;
+  constexpr uint32_t kOffKV = L::kOffKV, kOffStage = L::kOffStage, kOffDS = L::kOffDS;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_kvf, bar_kve, bar_stf[kStages], bar_ste[kStages], bar_sdp[2], bar_pds[2];
   __shared__ __align__(8) uint64_t bar_dqf[2], bar_dqe[2], bar_dsfree, bar_dkvf, bar_dkve, bar_drain;
@@ -272,9 +283,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     constexpr uint32_t id_sdp = idesc_bf16_f32(128, kQS, false);          // S^T, dP^T: A, B K-major
     constexpr uint32_t id_acc = idesc_bf16_f32(128, kDH, true);           // dV, dK: A in TMEM, B MN-major
     constexpr uint32_t id_dq = idesc_bf16_f32_ab(128, kDH, true, true);   // dQ: A, B MN-major
-    const uint32_t dhi = sw128_desc_hi(1024);
+    const uint32_t dhi = bf16_rows_desc_hi<DH>();  // K, V, Q, dA tiles (rows of DH bf16)
+    const uint32_t ds_hi = sw128_desc_hi(1024);     // the dS^T tile (rows of 64 queries)
     auto lo = [](uint32_t addr) { return sw128_desc_lo(addr, 16); };
     const uint32_t ds_lo = sw128_desc_lo(sDS, kDSHalf);  // MN-major A: query halves kDSHalf apart
+    constexpr uint32_t kRows16 = L::kRows16;
     bool ok = true;
     int G = 0, ST = 0, kd = 0;
     auto issue_sdp = [&](int gs) -> bool {
@@ -329,9 +342,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < kKB / 16; ++kk) {
-              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + kk * 128, dhi, lo(sKb) + kk * 128, dhi, id_dq, kk > 0 ? 1u : 0u);
-              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + ((2 * kDSHalf) >> 4) + kk * 128, dhi, lo(sKb) + kk * 128, dhi,
-                      id_dq, 1u);
+              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + kk * 128, ds_hi, lo(sKb) + kk * kRows16, dhi, id_dq,
+                      kk > 0 ? 1u : 0u);
+              mma_ss2(tmem + kColDQ + db * kDH, ds_lo + ((2 * kDSHalf) >> 4) + kk * 128, ds_hi,
+                      lo(sKb) + kk * kRows16, dhi, id_dq, 1u);
             }
             mma_commit(B(&bar_dqf[db]));
             mma_commit(B(&bar_dsfree));
@@ -343,7 +357,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (elect_one()) {
 #pragma unroll
           for (int c = 0; c < kQS / 16; ++c) {  // 16 queries per MMA: TMEM columns [16c, 16c + 8) hi, [+8, +16) lo
-            const uint32_t bq = lo(sQ(s)) + c * 128, bh = lo(sDAh(s)) + c * 128, bl = lo(sDAl(s)) + c * 128;
+            const uint32_t bq = lo(sQ(s)) + c * kRows16, bh = lo(sDAh(s)) + c * kRows16, bl = lo(sDAl(s)) + c * kRows16;
             const uint32_t acc0 = (t > 0 || c > 0) ? 1u : 0u;
             mma_ts2(tmem + kColDV, pT + 16 * c, bh, dhi, id_acc, acc0);      // P_hi dA_hi
             mma_ts2(tmem + kColDV, pT + 16 * c + 8, bh, dhi, id_acc, 1u);    // P_lo dA_hi
@@ -374,6 +388,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   } else if (warp >= 4) {
     // ------------------------------------------------------------- elementwise + epilogues
     const int wg = (warp - 4) >> 2;  // query columns [16 wg, 16 wg + 16) of each step
+    // output columns [16 wg, 16 wg + 16) of dQ, dK, dV (none for wg >= DH / 16: those
+    // warpgroups read the columns of warpgroup wg % (DH / 16) from TMEM and store nothing)
+    const bool mine = wg * 16 < kDH;
+    const uint32_t ocol = (uint32_t)((kDH == 64 ? wg : (wg & 1)) * 16);
     const int quad = warp & 3;
     const int mrow = quad * 32 + lane;  // TMEM lane: key row (steps) or query row (dQ)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -396,11 +414,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       }
       tc_fence_after();
       uint32_t raw[16];
-      tmem_ld16(lane_base + kColDQ + db * kDH + wg * 16, raw);
+      tmem_ld16(lane_base + kColDQ + db * kDH + ocol, raw);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(B(&bar_dqe[db]));
-      if (mrow < e.nvalid &&
+      if (mine && mrow < e.nvalid &&
           MTFM_INBOUNDS(hdr, e.row0 + mrow < (TARGET ? hdr->total_t : hdr->total_tokens))) {
         float4* dst = reinterpret_cast<float4*>(dq + (size_t)(e.row0 + mrow) * ldq + e.col + wg * 16);
 #pragma unroll
@@ -417,7 +435,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       float* dk_row = dk + (size_t)(U.so + jrow) * ldkv + U.g * kDH + wg * 16;
       float* dv_row = dv + (size_t)(U.so + jrow) * ldkv + U.g * kDH + wg * 16;
       if (T == 0) {  // no query sees this key block: dK = dV = 0
-        if (key_valid)
+        if (key_valid && mine)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             reinterpret_cast<float4*>(dk_row)[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -526,13 +544,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       if (eok) {
         tc_fence_after();
         uint32_t rv[16], rk[16];
-        tmem_ld16(lane_base + kColDV + wg * 16, rv);
-        tmem_ld16(lane_base + kColDK + wg * 16, rk);
+        tmem_ld16(lane_base + kColDV + ocol, rv);
+        tmem_ld16(lane_base + kColDK + ocol, rk);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(B(&bar_dkve));
         const float sk = p.alpha * inv_n;
-        if (key_valid && MTFM_INBOUNDS(hdr, U.so + jrow < hdr->total_tokens))
+        if (mine && key_valid && MTFM_INBOUNDS(hdr, U.so + jrow < hdr->total_tokens))
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             reinterpret_cast<float4*>(dv_row)[j] =
@@ -557,29 +575,36 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
 }  // namespace
 
-bool attn_bwd_tc_supported(const AttnShape& s) { return s.dh == kDH && s.hq % s.hkv == 0; }
+bool attn_bwd_tc_supported(const AttnShape& s) { return (s.dh == 64 || s.dh == 32) && s.hq % s.hkv == 0; }
 
 cudaError_t launch_attn_bwd_tc(const AttnShape& s, const MetaView& m, int max_items_full, int rows_q,
                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                const __nv_bfloat16* v, const __nv_bfloat16* da_hi, const __nv_bfloat16* da_lo,
                                float* dq, float* dk, float* dv, cudaStream_t st) {
   if (max_items_full <= 0 || total_tokens <= 0) return cudaSuccess;
-  const uint64_t Dq = (uint64_t)s.hq * kDH, Dkv = (uint64_t)s.hkv * kDH;
+  if (!attn_bwd_tc_supported(s)) return cudaErrorInvalidValue;
+  const int dh = s.dh;
+  const uint64_t Dq = (uint64_t)s.hq * dh, Dkv = (uint64_t)s.hkv * dh;
   const uint64_t rq = rows_q > 0 ? (uint64_t)rows_q : 1;  // a valid map even without query rows
   CUtensorMap mk, mv, mq, mdah, mdal;
-  if (!make_map_bf16(&mk, k, total_tokens, Dkv, Dkv, kKB, kDH) || !make_map_bf16(&mv, v, total_tokens, Dkv, Dkv, kKB, kDH) ||
-      !make_map_bf16(&mq, q, rq, Dq, Dq, kQS, kDH) || !make_map_bf16(&mdah, da_hi, rq, Dq, Dq, kQS, kDH) ||
-      !make_map_bf16(&mdal, da_lo, rq, Dq, Dq, kQS, kDH))
+  if (!make_map_bf16(&mk, k, total_tokens, Dkv, Dkv, kKB, dh) || !make_map_bf16(&mv, v, total_tokens, Dkv, Dkv, kKB, dh) ||
+      !make_map_bf16(&mq, q, rq, Dq, Dq, kQS, dh) || !make_map_bf16(&mdah, da_hi, rq, Dq, Dq, kQS, dh) ||
+      !make_map_bf16(&mdal, da_lo, rq, Dq, Dq, kQS, dh))
     return cudaErrorInvalidValue;
   BwdTcArgs args{m, s.hq, s.hkv, s.v2, s.alpha};
   const int grid = std::min(sm_count(), max_items_full * s.hkv);
-  auto launch = [&](auto kern) -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  auto launch = [&](auto kern, size_t smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, kSmemBytes, st>>>(mk, mv, mq, mdah, mdal, dq, dk, dv, args);
+    kern<<<grid, kThreads, smem, st>>>(mk, mv, mq, mdah, mdal, dq, dk, dv, args);
     return cudaGetLastError();
   };
-  return s.target ? launch(attn_bwd_tc_kernel<true>) : launch(attn_bwd_tc_kernel<false>);
+  if (dh == 32) {
+    constexpr size_t sm32 = BwdLayout<32>::kSmemBytes;
+    return s.target ? launch(attn_bwd_tc_kernel<true, 32>, sm32) : launch(attn_bwd_tc_kernel<false, 32>, sm32);
+  }
+  constexpr size_t sm64 = BwdLayout<64>::kSmemBytes;
+  return s.target ? launch(attn_bwd_tc_kernel<true, 64>, sm64) : launch(attn_bwd_tc_kernel<false, 64>, sm64);
 }
 
 }  // namespace mtfm

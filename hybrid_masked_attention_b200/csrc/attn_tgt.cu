@@ -473,14 +473,13 @@ attn_fwd_tgt_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (eok && e.k > 0) eok = __all_sync(0xffffffffu, mbar_wait(B(&bar_ste), (e.k - 1) & 1, abort_flag));
       if (!eok) ok = false;
       if (eok) {
-        // O columns [16 wg, 16 wg + 16) (the warpgroups past DH / 16 have none)
+        // O columns [16 wg, 16 wg + 16) (the warpgroups past DH / 16 have none: they read
+        // the columns of warpgroup wg % (DH / 16) and stage nothing)
         const bool mine = wg * 16 < kDH;
         tc_fence_after();
         uint32_t raw[16];
-        if (mine) {
-          tmem_ld16(lane_base + ob * kDH + wg * 16, raw);
-          tmem_ld_wait();
-        }
+        tmem_ld16(lane_base + ob * kDH + (kDH == 64 ? wg : (wg & 1)) * 16, raw);
+        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(B(&bar_oe[ob]));
         if (mine) {

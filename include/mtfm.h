@@ -54,9 +54,10 @@
  *     exception is the fixed scratch array of mtfm_attn_target_bwd_static).
  *     The forward attention runs tcgen05/TMEM kernels for head_dim 64 and 32
  *     with hq/hkv in {1, 2, 4} and for head_dim 256, the backward for head_dim
- *     64; other shapes (head_dim 128, or hq/hkv of 3 or 5..8 at head_dim 32 or
- *     64, and the backward at head_dim 32, 128, 256) run the portable mma.sync
- *     kernels.  The choice depends on the shape only (no run-time switch).
+ *     64 and 32; other shapes (head_dim 128, hq/hkv of 3 or 5..8 in the
+ *     forward at head_dim 32 or 64, the backward at head_dim 128 and 256) run
+ *     the portable mma.sync kernels.  The choice depends on the shape only (no
+ *     run-time switch).
  */
 #ifndef MTFM_H_
 #define MTFM_H_

@@ -36,7 +36,10 @@ def _rows(batch, users, target):
 CASES = [("tiny", "tiny", True), ("tiny", "tiny", False), ("edge", "pair", True),
          ("edge", "r8", True), ("v2_n512", "pair", True), ("pair", "pair", True),
          ("pair", "dh128", False), ("edge", "dh256", True), ("tiny", "dh256", False),
-         ("edge", "r1", True), ("edge", "r2", True), ("v2_n512", "r2", True)]
+         ("edge", "r1", True), ("edge", "r2", True), ("v2_n512", "r2", True),
+         # head_dim 32 on the tcgen05 backward (64-byte swizzle): r = 2, 1, 4 (and 8 above)
+         ("edge", "tiny", True), ("pair", "tiny", False), ("v2_n512", "dh32_r1", True),
+         ("edge", "dh32_r4", True)]
 
 
 @pytest.mark.parametrize("bname,hname,gln", CASES)
