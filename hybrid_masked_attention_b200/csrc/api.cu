@@ -71,10 +71,10 @@ cudaError_t launch_attn(const Resolved& r, const MetaView& m, const MetaLayout& 
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, target};
   const int max_items = target ? L.max_items_target : L.max_items_full;
   const int rows = target ? r.total_t : r.total_tokens;
-  if (!kPortableOnly && attn_fwd_tc_supported(shape)) {
-    if (target) return launch_attn_fwd_tgt(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
+  if (!kPortableOnly && target && attn_fwd_tgt_supported(shape))
+    return launch_attn_fwd_tgt(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
+  if (!kPortableOnly && !target && attn_fwd_tc_supported(shape))
     return launch_attn_fwd_tc(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
-  }
   if (!kPortableOnly && attn_fwd_tc256_supported(shape))
     return launch_attn_fwd_tc256(shape, m, max_items, rows, r.total_tokens, q, k, v, a, st);
   return launch_attn_fwd_mma(shape, m, max_items, q, k, v, a, st);
@@ -162,7 +162,7 @@ mtfm_status attn_target_cached(const mtfm_cfg* cfg, const void* d_meta, const ui
   if (s != MTFM_OK) return s;
   if ((s = check_meta(d_meta, r)) != MTFM_OK) return s;
   AttnShape shape{r.hq, r.hkv, r.dh, r.v2, r.alpha, true};
-  if (!attn_fwd_tc_supported(shape) || kPortableOnly) return MTFM_ERR_UNSUPPORTED;
+  if (!attn_fwd_tgt_supported(shape) || kPortableOnly) return MTFM_ERR_UNSUPPORTED;
   if (r.total_t == 0 || r.total_tokens == 0) return MTFM_OK;
   const int prefix_rows = r.total_tokens - r.total_t;
   if (!d_q || !d_kc || !d_vc || !d_a) return MTFM_ERR_INVALID_ARG;

@@ -29,7 +29,9 @@
 //                 from TMEM; at the end of the item they stage O / N_u in a
 //                 shared-memory area of its own (two heads per round) that leaves
 //                 for A as TMA stores (row stores for a user's ragged last tile).
-// TMEM (512 columns): O_h at columns [64h, 64h+64) for h < r (<= 4), S buffers
+// Head widths: dh 64 (rows of 128 bytes, 128-byte swizzle; r <= 4) and dh 32 (rows of
+// 64 bytes, 64-byte swizzle; r <= 8).
+// TMEM (512 columns): O_h at columns [dh h, dh (h+1)) for h < r (r dh <= 256), S buffers
 // b = 0, 1 at [256 + 128b, 384 + 128b).  While the warpgroups run the SiLU of
 // step n, the tensor pipe runs O += P(n-1) V and S(n+1) = Q K^T.
 // Key blocks above the tile's largest kv_end are never loaded; blocks entirely
@@ -93,6 +95,7 @@ constexpr size_t tc_smem_bytes() {
   return stage_off<R, DH>() + (size_t)heads_per_round<R>() * (DH / 32) * kBox + 1024;
 }
 static_assert(tc_smem_bytes<4, 64>() + 1024 <= 227 * 1024, "shared memory per CTA");
+static_assert(tc_smem_bytes<8, 32>() + 1024 <= 227 * 1024, "shared memory per CTA");
 
 // SiLU of 32 scores of one row (one TMEM chunk), masked, split into bf16 hi/lo
 // pairs: P = SiLU(alpha s) = h + h tanh(h), h = alpha s / 2.  Scalar fp32 math:
@@ -438,7 +441,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int rd = 0; rd < R / kHR; ++rd) {
         if (threadIdx.x == 128) bulk_wait_read<0>();  // the previous stores have read the area
         asm volatile("bar.sync 1, %0;" ::"n"(128 * kSiluWG) : "memory");
-        const int hh = wg;  // this warpgroup's head (R = 4), or none (wg >= R)
+        // this warpgroup's head: R <= 4: head wg (none for wg >= R), in the round of its pair;
+        // R = 8: in round rd, warpgroups 0 and 1 take heads 2 rd and 2 rd + 1
+        const int hh = R <= kSiluWG ? wg : rd * kHR + wg;
         if (have && hh < R && hh / kHR == rd) {
 #pragma unroll
           for (int c = 0; c < kDH / 32; ++c) {
@@ -545,7 +550,9 @@ cudaError_t tc_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
 
 bool attn_fwd_tc_supported(const AttnShape& s) {
   const int r = s.hq / s.hkv;
-  return (s.dh == 64 || s.dh == 32) && (r == 1 || r == 2 || r == 4);
+  // O takes r * head_dim of the 256 TMEM columns beside the two S buffers
+  return s.hq % s.hkv == 0 && ((s.dh == 64 && (r == 1 || r == 2 || r == 4)) ||
+                               (s.dh == 32 && (r == 1 || r == 2 || r == 4 || r == 8)));
 }
 
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
@@ -575,7 +582,8 @@ cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_it
   if (dh == 32) {
     if (r == 1) return tc_launch<1, 32>(mq, mk, mv, ma, args, max_items, st);
     if (r == 2) return tc_launch<2, 32>(mq, mk, mv, ma, args, max_items, st);
-    return tc_launch<4, 32>(mq, mk, mv, ma, args, max_items, st);
+    if (r == 4) return tc_launch<4, 32>(mq, mk, mv, ma, args, max_items, st);
+    return tc_launch<8, 32>(mq, mk, mv, ma, args, max_items, st);
   }
   if (r == 1) return tc_launch<1, 64>(mq, mk, mv, ma, args, max_items, st);
   if (r == 2) return tc_launch<2, 64>(mq, mk, mv, ma, args, max_items, st);

@@ -5,8 +5,8 @@
 // blog §3.2: the H keys, the R keys with ts < exposure, the sibling block).
 //
 // The r = hq / hkv query heads of a KV group are stacked as MMA rows: a 128-row
-// tile holds TR = 128 / r T rows x r heads (row m = t r + h, which is exactly the
-// shared-memory order of a 3-D TMA box {64 dims, r heads, TR rows} of Q), so one
+// tile holds TR = 128 / r T rows x r heads, r in {1, 2, 4, 8} (row m = t r + h, which is
+// exactly the shared-memory order of a 3-D TMA box {dh, r heads, TR rows} of Q), so one
 // QK^T and one PV MMA chain per 128-key block serve all r heads and the few T rows
 // of a user fill the tile.  A work unit is one (sub-tile of TR T rows, chunk of C key
 // blocks, KV group), C = MetaHeader::tgt_chunk_blocks (at least kTargetUnitBlocks),
@@ -635,6 +635,12 @@ __global__ void __launch_bounds__(256) tgt_zero_kernel(const MetaHeader* hdr, in
 
 }  // namespace
 
+// The r heads of a group stacked as 128 / r T rows each: r in {1, 2, 4, 8}; head_dim 64 or 32.
+bool attn_fwd_tgt_supported(const AttnShape& s) {
+  const int r = s.hkv > 0 ? s.hq / s.hkv : 0;
+  return (s.dh == 64 || s.dh == 32) && s.hq % s.hkv == 0 && (r == 1 || r == 2 || r == 4 || r == 8);
+}
+
 // Q [total_t, hq * dh] as a 3-D tensor {dh dims, hq heads, total_t rows}: a box of
 // {dh, r, 128 / r} is one stacked tile (rows of 128 bytes for dh 64, of 64 bytes with the
 // 64-byte swizzle for dh 32).  A [total_t, hq * dh] fp32 in boxes of 32 x TR.
@@ -649,7 +655,7 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
   const int r = s.hq / s.hkv;
   const int TR = 128 / r;
   const int dh = s.dh;
-  if (!attn_fwd_tc_supported(s)) return cudaErrorInvalidValue;
+  if (!attn_fwd_tgt_supported(s)) return cudaErrorInvalidValue;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv, ma;
@@ -709,11 +715,13 @@ cudaError_t launch_attn_fwd_tgt(const AttnShape& s, const MetaView& m, int max_i
   if (dh == 32) {
     if (r == 1) return launch(attn_fwd_tgt_kernel<1, 32>);
     if (r == 2) return launch(attn_fwd_tgt_kernel<2, 32>);
-    return launch(attn_fwd_tgt_kernel<4, 32>);
+    if (r == 4) return launch(attn_fwd_tgt_kernel<4, 32>);
+    return launch(attn_fwd_tgt_kernel<8, 32>);
   }
   if (r == 1) return launch(attn_fwd_tgt_kernel<1, 64>);
   if (r == 2) return launch(attn_fwd_tgt_kernel<2, 64>);
-  return launch(attn_fwd_tgt_kernel<4, 64>);
+  if (r == 4) return launch(attn_fwd_tgt_kernel<4, 64>);
+  return launch(attn_fwd_tgt_kernel<8, 64>);
 }
 
 }  // namespace mtfm

@@ -226,7 +226,7 @@ constexpr int kTargetUnitsPerSM = 8;  // the packer aims at about this many Targ
 // are stacked as MMA rows (128 = rows x r); 128 when that kernel does not apply.
 __host__ __device__ inline int target_sub_rows(int hq, int hkv) {
   const int r = hkv > 0 ? hq / hkv : 1;
-  return (r == 1 || r == 2 || r == 4) ? 128 / r : 128;
+  return (r == 1 || r == 2 || r == 4 || r == 8) ? 128 / r : 128;
 }
 
 struct KeyBlocks {
@@ -267,7 +267,8 @@ cudaError_t launch_pack(const mtfm_cfg& cfg, const MetaView& m, const int32_t* l
 cudaError_t launch_attn_fwd_mma(const AttnShape& s, const MetaView& m, int max_items,
                                 const __nv_bfloat16* q, const __nv_bfloat16* k,
                                 const __nv_bfloat16* v, float* a, cudaStream_t st);
-bool attn_fwd_tc_supported(const AttnShape& s);
+bool attn_fwd_tc_supported(const AttnShape& s);   // Full layer (attn_tc.cu)
+bool attn_fwd_tgt_supported(const AttnShape& s);  // Target layer (attn_tgt.cu)
 cudaError_t launch_attn_fwd_tc(const AttnShape& s, const MetaView& m, int max_items, int rows_q,
                                int total_tokens, const __nv_bfloat16* q, const __nv_bfloat16* k,
                                const __nv_bfloat16* v, float* a, cudaStream_t st);

@@ -52,11 +52,13 @@
  *   - Outputs are fp32 (bf16 inputs, fp32 accumulation throughout).
  *   - No exceptions cross this boundary; no global state is kept (the one
  *     exception is the fixed scratch array of mtfm_attn_target_bwd_static).
- *     The forward attention runs tcgen05/TMEM kernels for head_dim 64 and 32
- *     with hq/hkv in {1, 2, 4} and for head_dim 256, the backward for head_dim
- *     64 and 32; other shapes (head_dim 128, hq/hkv of 3 or 5..8 in the
- *     forward at head_dim 32 or 64, the backward at head_dim 128 and 256) run
- *     the portable mma.sync kernels.  The choice depends on the shape only (no
+ *     tcgen05/TMEM kernels run: the Full-layer forward at head_dim 64 with
+ *     hq/hkv in {1, 2, 4} and at head_dim 32 with hq/hkv in {1, 2, 4, 8}; the
+ *     Target-layer forward at head_dim 64 and 32 with hq/hkv in {1, 2, 4, 8};
+ *     both forwards at head_dim 256; the backward at head_dim 64 and 32.  The
+ *     other shapes (head_dim 128; hq/hkv of 3, 5, 6, 7; hq/hkv 8 in the Full
+ *     forward at head_dim 64; the backward at head_dim 128 and 256) run the
+ *     portable mma.sync kernels.  The choice depends on the shape only (no
  *     run-time switch).
  */
 #ifndef MTFM_H_
@@ -226,7 +228,7 @@ mtfm_status mtfm_gate_fwd(const mtfm_cfg* cfg, const void* d_meta, int is_target
  *                            and values (row t_off[u] + t for candidate t of user u);
  *   d_q, d_u, d_y, d_a, d_stats, d_gamma, d_beta : as mtfm_attn_target_fwd.
  * Supported where the tensor-core Target kernel runs (head_dim 64 or 32, hq / hkv
- * in {1, 2, 4}); other shapes return MTFM_ERR_UNSUPPORTED.  mtfm_attn_target_cached
+ * in {1, 2, 4, 8}); other shapes return MTFM_ERR_UNSUPPORTED.  mtfm_attn_target_cached
  * writes A only.
  * ------------------------------------------------------------------------- */
 mtfm_status mtfm_attn_target_cached_fwd(const mtfm_cfg* cfg, const void* d_meta, const uint16_t* d_q,

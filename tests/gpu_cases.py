@@ -27,5 +27,6 @@ HEADS = {
     "r8": syn.Heads(8, 1, 32),
     "dh32_r1": syn.Heads(2, 2, 32),         # head_dim 32 on the tcgen05 kernels (64-byte swizzle), r = 1
     "dh32_r4": syn.Heads(4, 1, 32),         # head_dim 32, r = 4
+    "r8_dh64": syn.Heads(8, 1, 64),         # r = 8 at head_dim 64: tcgen05 Target kernel, mma.sync Full kernel
     "dh256": syn.Heads(3, 1, 256),          # the 768-wide shape: Hq 3, Hkv 1, dh 256 (forward only)
 }

@@ -55,7 +55,9 @@ def _run(batch, heads, gln=True, seed=111):
 CASES = [("pair", syn.PAIR_HEADS), ("edge", syn.PAIR_HEADS), ("v2_n512", syn.PAIR_HEADS),
          ("v1_n2048", syn.Heads(4, 2, 64)), ("pair", syn.Heads(2, 2, 64)),
          # head_dim 32 (64-byte swizzle) at r = 2, 1, 4
-         ("tiny", syn.TINY_HEADS), ("pair", syn.Heads(2, 2, 32)), ("v2_n512", syn.Heads(4, 1, 32))]
+         ("tiny", syn.TINY_HEADS), ("pair", syn.Heads(2, 2, 32)), ("v2_n512", syn.Heads(4, 1, 32)),
+         # r = 8 (16 T rows per sub-tile) at head_dim 32 and 64
+         ("pair", syn.Heads(8, 1, 32)), ("edge", syn.Heads(8, 1, 64))]
 
 
 @pytest.mark.parametrize("bname,heads", CASES, ids=[f"{b}-{h.hq}x{h.hkv}" for b, h in CASES])
@@ -95,7 +97,7 @@ def test_cached_prefix_plain_gate_and_attention_only(cuda_ok):
 
 
 def test_cached_prefix_unsupported_shape(cuda_ok):
-    batch, heads = BATCHES["tiny"](), syn.Heads(8, 1, 32)   # r = 8: no tensor-core Target kernel
+    batch, heads = BATCHES["tiny"](), syn.Heads(4, 1, 128)   # head_dim 128: no tensor-core Target kernel
     cfg = config_for(batch, heads)
     meta = M.alloc_meta(cfg)
     M.pack(cfg, *upload_batch(batch), meta)

@@ -23,6 +23,8 @@ CASES = [
     ("pair", "tiny", True), ("edge", "tiny", True), ("v1_n2048", "tiny", False),
     ("pair", "dh32_r1", True), ("edge", "dh32_r1", False), ("pair", "dh32_r4", True),
     ("edge", "dh32_r4", True), ("v2_n512", "dh32_r4", True),
+    # r = 8: both tcgen05 kernels at head_dim 32 (16 T rows per Target sub-tile), the Target one at 64
+    ("pair", "r8", True), ("v2_n512", "r8", True), ("pair", "r8_dh64", True), ("edge", "r8_dh64", False),
 ]
 
 
