@@ -102,6 +102,9 @@ def test_null_and_misaligned_pointers_rejected(lib):
     c128 = _cfg(head_dim=128)   # head_dim 128: no tensor-core Target kernel
     assert m._lib.mtfm_attn_target_cached(ctypes.byref(c128), 4096, 4096, 4096, 4096, 4096, 4096, 4096,
                                           None) == 3
+    c8 = _cfg(hq=8, hkv=1, head_dim=32)   # r = 8 at head_dim 32 is taken: the missing candidate V is the error
+    assert m._lib.mtfm_attn_target_cached(ctypes.byref(c8), 4096, 4096, 4096, 4096, 4096, None, 4096,
+                                          None) == 1
     c3 = _cfg(hq=6, hkv=2, head_dim=64)   # r = 3: none either
     assert m._lib.mtfm_attn_target_cached(ctypes.byref(c3), 4096, 4096, 4096, 4096, 4096, 4096, 4096,
                                           None) == 3
