@@ -15,6 +15,7 @@ This file is collected last so that a run stopping at the first failure has
 already run every other test.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -47,16 +48,24 @@ def test_static_scratch_backward_matches_workspace_backward(cuda_ok):
                "dv": torch.full((N, Dkv), float("nan"), **f32), "du": torch.full((T, D), float("nan"), **f32),
                "dgamma": torch.full((3, D), float("nan"), **f32), "dbeta": torch.full((3, D), float("nan"), **f32)}
         torch.cuda.synchronize()
-        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
-        attn_target_bwd_static(s.cfg, s.meta, d["q"], d["k"], d["v"], d["u"], d["gamma"], d["beta"], a, st,
-                               d["dy"], out["dq"], out["dk"], out["dv"], out["du"], out["dgamma"],
-                               out["dbeta"])
-        torch.cuda.synchronize()
+        # Python's cycle collector would otherwise free tensors left by earlier tests in the
+        # middle of the measured call (torch's allocated-bytes counter then drops)
+        gc.collect()
+        gc.disable()
+        try:
+            free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+            attn_target_bwd_static(s.cfg, s.meta, d["q"], d["k"], d["v"], d["u"], d["gamma"], d["beta"], a, st,
+                                   d["dy"], out["dq"], out["dk"], out["dv"], out["du"], out["dgamma"],
+                                   out["dbeta"])
+            torch.cuda.synchronize()
+            free1, alloc1 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+        finally:
+            gc.enable()
         if call == 1:
             # the first call may load the library module that holds the array; the
             # second must not take any device memory
-            assert torch.cuda.mem_get_info()[0] == free0, "the second call changed free device memory"
-            assert torch.cuda.memory_allocated() == alloc0
+            assert free1 == free0, "the second call changed free device memory"
+            assert alloc1 == alloc0, "the second call allocated through torch"
         for name in ("dq", "dk", "dv", "du", "dgamma", "dbeta"):
             assert_close(out[name].cpu().numpy(), ref[name].cpu().numpy(), f"call {call} {name}")
 
